@@ -1,0 +1,197 @@
+"""ctypes front end of the fp64 CPU oracle (``retention_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  The product path never imports this module; only
+the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` do.  Arrays go in as anything numpy can turn into float64 and
+come back as float64 numpy arrays.  The arithmetic lives in the C file; this
+module only marshals arguments.
+
+Layouts: Q, K ``[B, H, L, dk]``; V, O ``[B, H, L, dv]``; G, Y ``[B, L, H*dv]``;
+state ``[B, H, dk, dv]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "retention_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
+        ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+        ("gamma", ctypes.POINTER(ctypes.c_double)),
+        ("rotate", ctypes.c_int), ("theta_base", ctypes.c_double),
+        ("pos_offset", ctypes.c_longlong), ("nthreads", ctypes.c_int),
+    ]
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH, extra_flags=()) -> str:
+    """Compile the oracle with gcc (IEEE arithmetic: no fast-math)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+           *extra_flags, src, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return out
+
+
+def _stale() -> bool:
+    return (not os.path.exists(_LIB_PATH)
+            or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+
+
+def load(path: str | None = None):
+    """Load (building first if missing or older than the source)."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if _stale():
+                build()
+            _lib = _bind(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _bind(lib):
+    P = ctypes.POINTER(_Problem)
+    d = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_msr_gammas.argtypes = [ctypes.c_int, d]
+    lib.oracle_xpos_rotate.argtypes = [d, ctypes.c_int, ctypes.c_double,
+                                       ctypes.c_double, d]
+    lib.oracle_retention_parallel.argtypes = [P, d, d, d, d]
+    lib.oracle_retention_recurrent.argtypes = [P, d, d, d, d, d, d]
+    lib.oracle_retention_chunkwise.argtypes = [P, ctypes.c_int, d, d, d, d, d, d]
+    lib.oracle_retention_rows.argtypes = [
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, d, d, d, ctypes.c_double,
+        ctypes.c_int, ctypes.c_double, ctypes.c_longlong, d, ctypes.c_int,
+        ctypes.POINTER(ctypes.c_longlong), d]
+    lib.oracle_gate_groupnorm.argtypes = [ctypes.c_int] * 4 + [
+        d, d, ctypes.c_double, d]
+    for f in ("oracle_retention_parallel", "oracle_retention_recurrent",
+              "oracle_retention_chunkwise", "oracle_retention_rows",
+              "oracle_gate_groupnorm"):
+        getattr(lib, f).restype = ctypes.c_int
+    return lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a torch tensor: exact upcast on the host
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _problem(Q, V, gamma, rotate, theta_base, pos_offset, nthreads):
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    g = _f64(gamma).reshape(-1)
+    if g.shape[0] != H:
+        raise ValueError("gamma must have one entry per head")
+    p = _Problem(B, H, L, dk, dv, _ptr(g), int(bool(rotate)), float(theta_base),
+                 int(pos_offset), int(nthreads))
+    return p, g  # keep g alive
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def gammas(H: int, lib=None) -> np.ndarray:
+    lib = lib or load()
+    g = np.zeros(H, dtype=np.float64)
+    lib.oracle_msr_gammas(H, _ptr(g))
+    return g
+
+
+def xpos_rotate(x, pos: float, theta_base: float = 10000.0, lib=None) -> np.ndarray:
+    lib = lib or load()
+    x = _f64(x).reshape(-1)
+    out = np.zeros_like(x)
+    lib.oracle_xpos_rotate(_ptr(x), x.shape[0], float(pos), float(theta_base), _ptr(out))
+    return out
+
+
+def parallel(Q, K, V, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
+             nthreads=0, lib=None) -> np.ndarray:
+    lib = lib or load()
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    p, _g = _problem(Q, V, gamma, rotate, theta_base, pos_offset, nthreads)
+    O = np.zeros(Q.shape[:3] + (V.shape[-1],))
+    _check(lib.oracle_retention_parallel(ctypes.byref(p), _ptr(Q), _ptr(K),
+                                         _ptr(V), _ptr(O)), "parallel")
+    return O
+
+
+def recurrent(Q, K, V, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
+              state_in=None, nthreads=0, lib=None):
+    """Returns (O, state_out)."""
+    lib = lib or load()
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    p, _g = _problem(Q, V, gamma, rotate, theta_base, pos_offset, nthreads)
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    S_in = None if state_in is None else _f64(state_in)
+    S_out = np.zeros((B, H, dk, dv))
+    O = np.zeros((B, H, L, dv))
+    _check(lib.oracle_retention_recurrent(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V),
+                                          _ptr(S_in), _ptr(S_out), _ptr(O)),
+           "recurrent")
+    return O, S_out
+
+
+def chunkwise(Q, K, V, gamma, chunk, rotate=False, theta_base=10000.0,
+              pos_offset=0, state_in=None, nthreads=0, lib=None):
+    """Returns (O, state_out)."""
+    lib = lib or load()
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    p, _g = _problem(Q, V, gamma, rotate, theta_base, pos_offset, nthreads)
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    S_in = None if state_in is None else _f64(state_in)
+    S_out = np.zeros((B, H, dk, dv))
+    O = np.zeros((B, H, L, dv))
+    _check(lib.oracle_retention_chunkwise(ctypes.byref(p), int(chunk), _ptr(Q), _ptr(K),
+                                          _ptr(V), _ptr(S_in), _ptr(S_out), _ptr(O)),
+           "chunkwise")
+    return O, S_out
+
+
+def rows(q, k, v, gamma: float, rows, rotate=False, theta_base=10000.0,
+         pos_offset=0, state0=None, lib=None) -> np.ndarray:
+    """Outputs of selected rows of ONE (b,h) slice: q, k [L, dk], v [L, dv]."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    L, dk = q.shape
+    dv = v.shape[-1]
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+    out = np.zeros((r.shape[0], dv))
+    s0 = None if state0 is None else _f64(state0)
+    _check(lib.oracle_retention_rows(
+        L, dk, dv, _ptr(q), _ptr(k), _ptr(v), float(gamma), int(bool(rotate)),
+        float(theta_base), int(pos_offset), _ptr(s0), r.shape[0],
+        r.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), _ptr(out)), "rows")
+    return out
+
+
+def gate_groupnorm(O, G, eps=1e-5, lib=None) -> np.ndarray:
+    """O [B, H, L, dv], G [B, L, H*dv] -> Y [B, L, H*dv]."""
+    lib = lib or load()
+    O, G = _f64(O), _f64(G)
+    B, H, L, dv = O.shape
+    Y = np.zeros((B, L, H * dv))
+    _check(lib.oracle_gate_groupnorm(B, L, H, dv, _ptr(O), _ptr(G), float(eps), _ptr(Y)),
+           "gate_groupnorm")
+    return Y
