@@ -1,0 +1,412 @@
+"""Benchmark of the multi-scale retention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one chunkwise retention forward with the fused per-head
+GroupNorm + swish gate over the RetNet-1.3B-shaped MSR workload (B=8, H=8,
+L=4096, d_k=256, d_v=512, chunk 128, xPos rotation, bf16 in/out, fp32
+accumulate): Q, K, V, G in, Y out, all resident in HBM.  Throughput is
+tokens (B*L) per second over the whole job.  The same JSON line carries the
+roofline of the dominant kernel, an end-to-end figure through host buffers,
+the recurrent decode measurement (B=64, H=16, d_k=256, d_v=512, fp32 state,
+256 steps in a CUDA graph after a chunkwise prefill of 8192 tokens), the
+parallel form on the MSR workload, the CPU oracle baseline and the SM clocks
+seen during the timed region.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
+the workload (independent sequences, no data exchange): weak scaling, value =
+all ranks' tokens / max over ranks of the timed device time.
+
+``--impl reference`` times the fp64 CPU oracle instead (the only other
+implementation of the method here), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from retentive_network_scale_b200.synth import WORKLOADS, make_decode_inputs, make_inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2**20
+
+
+# --------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def chunkwise_flops_per_token_head(C, dk, dv):
+    """Algorithmic flops of the chunkwise form per token and head: causal
+    pairs only inside a chunk ((C+1)/2 keys on average, 2 flops per
+    multiply-add for q.k and for p.v) plus the carried-state read and the
+    state update (2 dk dv each)."""
+    return (C + 1) * (dk + dv) + 4 * dk * dv
+
+
+def parallel_flops_per_token_head(L, dk, dv):
+    return (L + 1) * (dk + dv)
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": seen, "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample(w, max_seconds=20.0):
+    """Time the fp64 oracle (recurrent form, then GroupNorm + gate) on whole
+    (b, h) slices of the workload, adding slices until ~max_seconds of work.
+    Returns (tokens/s equivalent, cores, description)."""
+    from oracle import oracle as orc
+    x = make_inputs(w, B=1)
+    cores = os.cpu_count() or 1
+    gam = orc.gammas(w.H)
+    q, k, v = (x[n].double().numpy() for n in ("Q", "K", "V"))
+    g = x["G"].double().numpy() if "G" in x else None
+    slices, elapsed = 0, 0.0
+    batch = min(w.H, cores)
+    while elapsed < max_seconds / 2 and slices < w.B * w.H:
+        hs = [(slices + i) % w.H for i in range(batch)]
+        t0 = time.perf_counter()
+        O, _ = orc.recurrent(q[:, hs], k[:, hs], v[:, hs], gam[hs], rotate=w.rotate,
+                             theta_base=w.theta_base, nthreads=cores)
+        if g is not None:
+            gg = np.concatenate([g[:, :, h * w.d_v:(h + 1) * w.d_v] for h in hs], axis=-1)
+            orc.gate_groupnorm(O, gg)
+        elapsed += time.perf_counter() - t0
+        slices += batch
+    tokens = slices * w.L / w.H  # a token needs all H head slices
+    desc = (f"{slices} (b,h) slices of L={w.L} (recurrent form"
+            f"{' + GroupNorm/gate' if g is not None else ''}), fp64, {cores} threads")
+    return tokens / elapsed, cores, desc, elapsed
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS["msr_1p3b"]
+    if world > 1 and rank != 0:
+        return
+    values = []
+    cores, desc = os.cpu_count(), ""
+    for i in range(args.warmup + args.steps):
+        v, cores, desc, _ = oracle_sample(w, max_seconds=max(2.0, 60.0 / (args.steps + args.warmup)))
+        if i >= args.warmup:
+            values.append(v)
+    val = statistics.median(values)
+    line = {"impl": "reference", "metric": "retention fwd tokens/s (RetNet-1.3B MSR chunkwise + GN/gate)",
+            "value": val, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: RetNet-1.3B-shaped MSR chunkwise forward + GroupNorm/swish gate, "
+                        f"B={w.B} H={w.H} L={w.L} d_k={w.d_k} d_v={w.d_v} chunk={w.chunk}, "
+                        f"xPos on, bf16 in/out",
+            "global_batch": w.B, "seq_len": w.L, "heads": w.H, "d_k": w.d_k, "d_v": w.d_v,
+            "chunk": w.chunk, "parallelism": "replicas",
+            "l2": "inputs (805 MB) larger than L2; no flush"}
+
+
+# ----------------------------------------------------------------- GPU timing
+def time_launches(fn, n, stream):
+    """Device time per call (ms) over n back-to-back calls, CUDA events on
+    the launching stream."""
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(n):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / n
+
+
+def bench_decode(R, pk, warm=2, reps=3):
+    w = WORKLOADS["decode"]
+    x = make_inputs(w, device="cuda")
+    steps = make_decode_inputs(w, device="cuda")
+    g = R.msr_gammas(w.H)
+    S = torch.empty(w.B, w.H, w.d_k, w.d_v, device="cuda")
+    O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream()
+    prefill = lambda: R.ret_chunkwise(x["Q"], x["K"], x["V"], g, w.chunk, O=O, state_out=S,  # noqa: E731
+                                      rotate=w.rotate)
+    prefill()
+    t_prefill = time_launches(prefill, 2, stream)
+    del O, x
+    o = torch.empty(w.decode_steps, w.B, w.H, w.d_v, device="cuda", dtype=torch.bfloat16)
+    state = S.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        # one eager pass first (lazy module loading), then capture
+        for t in range(2):
+            R.ret_recurrent_step(steps["q"][t], steps["k"][t], steps["v"][t], state, o[t], g,
+                                 pos=w.L + t, rotate=w.rotate, stream=side)
+        side.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            for t in range(w.decode_steps):
+                R.ret_recurrent_step(steps["q"][t], steps["k"][t], steps["v"][t], state, o[t], g,
+                                     pos=w.L + t, rotate=w.rotate, stream=side)
+    stream.wait_stream(side)
+    for _ in range(warm):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = time_launches(graph.replay, reps, stream) / w.decode_steps
+    graph.reset()
+    bytes_step = (2 * w.B * w.H * w.d_k * w.d_v * 4            # state read + write
+                  + w.B * w.H * (2 * w.d_k + w.d_v) * 2       # q, k, v (bf16)
+                  + w.B * w.H * w.d_v * 2)                    # o (bf16)
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    flop_prefill = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
+    return {
+        "workload": f"decode: B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v}, fp32 state, bf16 q/k/v/o, "
+                    f"{w.decode_steps} steps in one CUDA graph after a {w.L}-token chunkwise prefill",
+        "tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / pk["hbm_gbs"], "bytes_per_step": bytes_step},
+        "prefill": {"ms": t_prefill, "tokens_per_s": w.B * w.L / (t_prefill * 1e-3),
+                    "tflops": flop_prefill / (t_prefill * 1e-3) / 1e12},
+        "gpu_launches_per_step": 1,
+    }
+
+
+def bench_parallel(R, w, d, pk, reps=3):
+    g = R.msr_gammas(w.H)
+    O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
+    fn = lambda: R.ret_parallel(d["Q"], d["K"], d["V"], O, g, rotate=w.rotate)  # noqa: E731
+    fn()
+    ms = time_launches(fn, reps, torch.cuda.current_stream())
+    fl = w.B * w.H * w.L * parallel_flops_per_token_head(w.L, w.d_k, w.d_v)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": f"parallel form on {w.name} (O bf16, no gate)", "ms": ms,
+            "tokens_per_s": w.B * w.L / (ms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"]}}
+
+
+def run_ours(args, world, rank, local):
+    from retentive_network_scale_b200 import build as rbuild
+    from retentive_network_scale_b200 import retention as R
+    if rank == 0:
+        rbuild.build()
+    barrier(world)
+    R.load_library()
+    pk, pk_src = peaks()
+    w = WORKLOADS["msr_1p3b"]
+    host = make_inputs(w)
+    host = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.cuda(non_blocking=True) for k, v in host.items()}
+    g = R.msr_gammas(w.H)
+    Y = torch.empty(w.B, w.L, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, G=d["G"], Y=Y, rotate=w.rotate)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n0 = R.ret_kernel_launches()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = R.ret_kernel_launches() - n0
+    ms_local = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    tokens_step = w.B * w.L
+    value = world * tokens_step / (ms * 1e-3)
+
+    # dominant kernel: the whole step is the chunkwise call
+    flops = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
+    bytes_alg = sum(t.numel() * t.element_size() for t in d.values()) + Y.numel() * Y.element_size()
+    tf = flops / (ms_local * 1e-3) / 1e12
+    gbs = bytes_alg / (ms_local * 1e-3) / 1e9
+    roofline = {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tf / pk["bf16_tflops"], "traffic": None,
+                "peak_source": f"{pk_src} (bf16 burst)",
+                "flops_per_launch": flops, "bytes_per_launch": bytes_alg,
+                "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / pk["hbm_gbs"]}}
+
+    # end to end: pinned host buffers in, Y back to pinned host memory
+    Y_host = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+    n_e2e = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for k in d:
+            d[k].copy_(host[k], non_blocking=True)
+        step()
+        Y_host.copy_(Y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(time_launches(e2e_step, n_e2e, stream), world)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = Y.numel() * Y.element_size()
+
+    extra = {}
+    if not args.skip_extra:
+        extra["parallel"] = bench_parallel(R, w, d, pk)
+        del d
+        torch.cuda.empty_cache()
+        extra["decode"] = bench_decode(R, pk)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        v, cores, desc, _ = oracle_sample(w, max_seconds=args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": "retention fwd tokens/s (RetNet-1.3B MSR chunkwise + GN/gate)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w),
+            "roofline": roofline,
+            "e2e": {"value": world * tokens_step / (ms_e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+            **extra,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-extra", action="store_true", help="only the main step")
+    ap.add_argument("--skip-cpu", action="store_true", help="no CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * retention.h -- C ABI of the B200 multi-scale retention forward library
+ * (libretention.so, hand-written CUDA for sm_100a).
+ *
+ * What is computed.  Per batch b and head h with scalar decay gamma_h, every
+ * form returns
+ *     o_n = sum_{m <= n} gamma_h^{n-m} (q^_n . k^_m) v_m ,
+ * the scalar-gamma retention of "Retentive Network: A Successor to
+ * Transformer for Large Language Models" (paper summary, blog.csdn.net
+ * 132817411, section 2.1), where q^_n, k^_m are the rows turned by the xPos
+ * factor e^{i n theta}: a row of even width d_k is read as d_k/2 complex
+ * numbers (x[2j], x[2j+1]) and pair j is turned by the angle
+ * pos * theta_j, theta_j = theta_base^(-2j/d_k), for Q and K alike, so the
+ * score is the real part of (Q_n e^{in theta})(K_m e^{im theta})^dagger.
+ * There is no 1/sqrt(d_k) score scale (the pages give none).
+ *
+ * Conventions shared by every entry point.
+ *  - Pointers named as device pointers must be device memory of the current
+ *    device (or managed memory); every one must be 16-byte aligned.  Pointers
+ *    named as host pointers are read during the call only.
+ *  - The caller owns every buffer and the stream.  The library allocates no
+ *    device memory, keeps no per-call state, and never synchronises unless a
+ *    function says so.  `stream` is a cudaStream_t passed as void*; NULL is
+ *    the legacy default stream.
+ *  - Arguments are checked before any launch.  A call that returns an error
+ *    launched nothing and wrote nothing.  A call that returns RET_OK has only
+ *    queued work: kernel faults surface on the stream, and a bounded device
+ *    wait that gave up is reported by ret_last_device_status().
+ *  - Layouts are dense and row-major:
+ *        Q, K    [B][H][L][d_k]     V, O   [B][H][L][d_v]
+ *        G, Y    [B][L][H*d_v]      state  [B][H][d_k][d_v]  (always fp32)
+ *    Row t of a (b,h) slice sits at absolute position pos_offset + t.  A
+ *    state is S after absorbing every token before the first row of the
+ *    call, so prefill and decode must use continuous positions.
+ *  - Limits: 1 <= H <= RET_MAX_HEADS, 1 <= d_k <= 256, 1 <= d_v <= 512,
+ *    d_v a multiple of 4, d_k even when rotating; B, L >= 0 (zero sizes are
+ *    accepted and do nothing); 0 <= gamma_h <= 1.
+ *  - Only sm_100 devices are supported: elsewhere every compute entry point
+ *    returns RET_ERR_UNSUPPORTED.  There is no fallback of any kind.
+ */
+#ifndef RETENTION_H
+#define RETENTION_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RET_MAX_HEADS 128
+
+typedef enum {
+    RET_OK = 0,
+    RET_ERR_NULL = 1,        /* a required pointer is NULL                    */
+    RET_ERR_SHAPE = 2,       /* a size is negative or beyond the limits above */
+    RET_ERR_DTYPE = 3,       /* dtype code not RET_F32 / RET_BF16             */
+    RET_ERR_ALIGN = 4,       /* a device pointer is not 16-byte aligned       */
+    RET_ERR_ARG = 5,         /* gamma outside [0,1] or not finite, chunk < 1,
+                                odd d_k with rotation, eps < 0, bad base      */
+    RET_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required       */
+    RET_ERR_UNSUPPORTED = 7, /* not an sm_100 device                          */
+    RET_ERR_CUDA = 8,        /* a CUDA runtime call or launch failed          */
+    RET_ERR_TIMEOUT = 9      /* a bounded device wait gave up (see
+                                ret_last_device_status)                        */
+} ret_status;
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+/* Problem description.  The struct is read during the call only. */
+typedef struct {
+    int B, H, L, d_k, d_v;   /* L must be 1 for ret_recurrent_step          */
+    int in_dtype;            /* ret_dtype of Q, K, V (and G)                */
+    int out_dtype;           /* ret_dtype of O (and Y)                      */
+    const double *gamma;     /* HOST array [H]: decay of each head          */
+    int rotate;              /* 0: no xPos rotation; 1: rotate Q and K      */
+    double theta_base;       /* theta_j = theta_base^(-2j/d_k), e.g. 10000  */
+    long long pos_offset;    /* absolute position of row 0 (>= 0)           */
+} ret_desc;
+
+/*
+ * ret_parallel -- the parallel representation (section 2.1, form (1)):
+ *     Retention(X) = (Q K^T (.) D) V,  D_nm = gamma^{n-m} (n >= m), else 0,
+ * with Q, K rotated as above.  Q, K, V: device, in_dtype.  O: device,
+ * out_dtype, fully overwritten.  No state in or out.
+ * Errors: RET_ERR_NULL, _SHAPE, _DTYPE, _ALIGN, _ARG, _UNSUPPORTED, _CUDA.
+ */
+ret_status ret_parallel(const ret_desc *desc, const void *Q, const void *K,
+                        const void *V, void *O, void *stream);
+
+/*
+ * ret_chunkwise -- the chunkwise recurrent representation (section 2.1,
+ * form (3): parallel inside a chunk of `chunk` rows, a decayed state carried
+ * between chunks).  For the chunk of n rows after state R:
+ *     o_j = sum_{j'<=j} gamma^{j-j'} (q^_j.k^_{j'}) v_{j'} + gamma^{j+1} q^_j R
+ *     R  <- gamma^n R + sum_{j'} gamma^{n-1-j'} k^_{j'}^T v_{j'}
+ * (the recurrent form unrolled over the chunk; the last chunk may be short).
+ * The result equals ret_parallel's up to rounding for every chunk size.
+ *   state_in  device fp32 [B][H][d_k][d_v] or NULL (zeros).
+ *   state_out device fp32, or NULL; may alias state_in.
+ *   O         device out_dtype [B][H][L][d_v], or NULL when only Y is wanted.
+ *   G, Y      both NULL, or both device: G in_dtype, Y out_dtype
+ *             [B][L][H*d_v]; then Y = swish(G) (.) GroupNorm_h(O) (as in
+ *             ret_gate_norm) is written as well, with epsilon gn_eps.
+ *   workspace device scratch of workspace_bytes; required only when
+ *             ret_workspace_size() returns a non-zero size for this call.
+ * At least one of O and Y must be requested.
+ * Errors: those of ret_parallel, plus RET_ERR_WORKSPACE.
+ */
+ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q,
+                         const void *K, const void *V, const float *state_in,
+                         float *state_out, void *O, const void *G, float gn_eps,
+                         void *Y, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* Bytes of workspace ret_chunkwise needs for this description and chunk
+ * (0 when none).  Depends only on the arguments; never fails (returns 0
+ * for descriptions that ret_chunkwise would reject). */
+size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O,
+                          int want_Y);
+
+/*
+ * ret_recurrent_step -- one step of the recurrent representation (section
+ * 2.1, form (2)): S_n = gamma S_{n-1} + k^_n^T v_n, then o_n = q^_n S_n
+ * (update first, then read).  desc->L must be 1 and desc->pos_offset is the
+ * absolute position n of this token.
+ *   q, k   device in_dtype [B][H][d_k];  v device in_dtype [B][H][d_v]
+ *   state  device fp32 [B][H][d_k][d_v], updated in place
+ *   o      device out_dtype [B][H][d_v]
+ * Errors: those of ret_parallel.
+ */
+ret_status ret_recurrent_step(const ret_desc *desc, const void *q,
+                              const void *k, const void *v, float *state,
+                              void *o, void *stream);
+
+/*
+ * ret_gate_norm -- section 2.2: Y = swish(G) (.) GroupNorm_h(O), one group
+ * per head taken per token over its d_v channels, population variance, no
+ * affine parameters, swish(x) = x sigmoid(x):
+ *     Y[b,t,h*d_v+c] = swish(G[b,t,h*d_v+c]) (O[b,h,t,c] - mu) / sqrt(var + eps)
+ *   O  device o_dtype [B][H][L][d_v];  G device g_dtype [B][L][H*d_v]
+ *   Y  device y_dtype [B][L][H*d_v], fully overwritten
+ * Errors: RET_ERR_NULL, _SHAPE, _DTYPE, _ALIGN, _ARG (eps < 0), _UNSUPPORTED,
+ * _CUDA.
+ */
+ret_status ret_gate_norm(int B, int L, int H, int d_v, int o_dtype,
+                         const void *O, int g_dtype, const void *G, float eps,
+                         int y_dtype, void *Y, void *stream);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * that bounded waits in the kernels latch (RET_ERR_TIMEOUT), or
+ * RET_ERR_CUDA when the stream reports an error. */
+ret_status ret_last_device_status(void *stream);
+
+/* Number of kernels this library has launched in this process so far, over
+ * all devices and threads (benchmarks count their launches with it). */
+unsigned long long ret_kernel_launches(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char *ret_status_string(ret_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_H */

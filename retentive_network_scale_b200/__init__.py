@@ -9,7 +9,8 @@ from importlib import import_module
 
 _BINDING_NAMES = (
     "ret_parallel", "ret_chunkwise", "ret_recurrent_step", "ret_gate_norm",
-    "ret_workspace_size", "ret_last_device_status", "ret_status_string",
+    "ret_workspace_size", "ret_last_device_status", "ret_kernel_launches",
+    "ret_status_string",
     "RetentionError", "msr_gammas", "load_library",
 )
 

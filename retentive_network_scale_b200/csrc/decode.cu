@@ -1,0 +1,152 @@
+// decode.cu -- one recurrent retention step over the fp32 state:
+//   S <- gamma S + k^^T v   (in place),   o = q^ S   (update, then read).
+// "Retentive Network" paper summary, section 2.1, recurrent form (2).
+//
+// Bound by HBM: each step reads and writes the whole d_k x d_v fp32 state
+// once (8 d_k d_v bytes per head) and does 4 flops per element.  One CTA
+// owns COLS contiguous columns of one (b,h) state, all d_k rows: threads
+// move 16-byte float4 pieces, TPR = COLS/4 threads cover a row segment, so a
+// warp touches 32/TPR rows with fully used 128-byte lines.  Each thread keeps
+// eight rows of loads in flight.  The column sums of q^ S are reduced
+// through shared memory.  State traffic uses streaming (evict-first) hints:
+// the state is larger than L2 and is not read again within the step.
+#include "common.cuh"
+#include "launch.h"
+
+namespace ret {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowsInFlight = 8;
+
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    uint2 u = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+template <typename TI, typename TO, int COLS>
+__global__ void __launch_bounds__(kThreads)
+recurrent_step_kernel(Params p, int ncol_tiles, const TI *q, const TI *k,
+                      const TI *v, float *state, TO *o) {
+    constexpr int TPR = COLS / 4;
+    constexpr int RG = kThreads / TPR;
+    __shared__ float qs[kMaxDk], ks[kMaxDk];
+    __shared__ float red[kThreads * 4];
+
+    const int bh = blockIdx.x / ncol_tiles, ct = blockIdx.x - bh * ncol_tiles;
+    const int h = bh % p.H;
+    const size_t qk_off = (size_t)bh * p.dk;
+
+    // q^, k^ for this head into shared memory
+    if (p.rotate) {
+        for (int j = threadIdx.x; j < p.dk / 2; j += kThreads) {
+            float c, s;
+            rot_cs(p.pos_offset, p.theta[j], &c, &s);
+            float q0 = ld(q, qk_off + 2 * j), q1 = ld(q, qk_off + 2 * j + 1);
+            float k0 = ld(k, qk_off + 2 * j), k1 = ld(k, qk_off + 2 * j + 1);
+            rot_pair(q0, q1, c, s);
+            rot_pair(k0, k1, c, s);
+            qs[2 * j] = q0; qs[2 * j + 1] = q1;
+            ks[2 * j] = k0; ks[2 * j + 1] = k1;
+        }
+    } else {
+        for (int i = threadIdx.x; i < p.dk; i += kThreads) {
+            qs[i] = ld(q, qk_off + i);
+            ks[i] = ld(k, qk_off + i);
+        }
+    }
+    __syncthreads();
+
+    const int tpr = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+    const int c = ct * COLS + 4 * tpr;
+    const float4 vv = load4(v + (size_t)bh * p.dv + c);
+    const float g = exp2f(p.log2g[h]);  // gamma (0 when log2 gamma = -inf)
+    float *S = state + (size_t)bh * p.dk * p.dv + c;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    for (int i0 = rg; i0 < p.dk; i0 += RG * kRowsInFlight) {
+        float4 s[kRowsInFlight];
+#pragma unroll
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            int i = i0 + u * RG;
+            if (i < p.dk) s[u] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)i * p.dv));
+        }
+#pragma unroll
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            int i = i0 + u * RG;
+            if (i < p.dk) {
+                const float ki = ks[i], qi = qs[i];
+                s[u].x = fmaf(g, s[u].x, ki * vv.x);
+                s[u].y = fmaf(g, s[u].y, ki * vv.y);
+                s[u].z = fmaf(g, s[u].z, ki * vv.z);
+                s[u].w = fmaf(g, s[u].w, ki * vv.w);
+                __stcs(reinterpret_cast<float4 *>(S + (size_t)i * p.dv), s[u]);
+                acc.x = fmaf(qi, s[u].x, acc.x);
+                acc.y = fmaf(qi, s[u].y, acc.y);
+                acc.z = fmaf(qi, s[u].z, acc.z);
+                acc.w = fmaf(qi, s[u].w, acc.w);
+            }
+        }
+    }
+
+    // o[c'] = sum over row groups; red is [RG][COLS]
+    red[rg * COLS + 4 * tpr + 0] = acc.x;
+    red[rg * COLS + 4 * tpr + 1] = acc.y;
+    red[rg * COLS + 4 * tpr + 2] = acc.z;
+    red[rg * COLS + 4 * tpr + 3] = acc.w;
+    __syncthreads();
+    // level 1: thread t sums 4 row groups of column t % COLS
+    constexpr int PARTS = kThreads / COLS;   // == RG / 4
+    {
+        const int cc = threadIdx.x % COLS, part = threadIdx.x / COLS;
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sum += red[(part * 4 + r) * COLS + cc];
+        __syncthreads();
+        red[part * COLS + cc] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x < COLS) {
+        float sum = 0.f;
+        for (int part = 0; part < PARTS; ++part) sum += red[part * COLS + threadIdx.x];
+        st(o, (size_t)bh * p.dv + ct * COLS + threadIdx.x, sum);
+    }
+}
+
+template <typename TI, typename TO>
+cudaError_t launch_t(const Params &p, const void *q, const void *k, const void *v,
+                     float *state, void *o, cudaStream_t st) {
+    int cols = (p.dv % 32 == 0) ? 32 : (p.dv % 16 == 0) ? 16 : (p.dv % 8 == 0) ? 8 : 4;
+    int tiles = p.dv / cols;
+    long long blocks = (long long)p.B * p.H * tiles;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const TI *qq = (const TI *)q, *kk = (const TI *)k, *vv = (const TI *)v;
+    TO *oo = (TO *)o;
+    switch (cols) {
+        case 32: recurrent_step_kernel<TI, TO, 32><<<(unsigned)blocks, kThreads, 0, st>>>(p, tiles, qq, kk, vv, state, oo); break;
+        case 16: recurrent_step_kernel<TI, TO, 16><<<(unsigned)blocks, kThreads, 0, st>>>(p, tiles, qq, kk, vv, state, oo); break;
+        case 8: recurrent_step_kernel<TI, TO, 8><<<(unsigned)blocks, kThreads, 0, st>>>(p, tiles, qq, kk, vv, state, oo); break;
+        default: recurrent_step_kernel<TI, TO, 4><<<(unsigned)blocks, kThreads, 0, st>>>(p, tiles, qq, kk, vv, state, oo); break;
+    }
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+}  // namespace
+
+cudaError_t launch_recurrent_step(const Params &p, bool in_bf16, bool out_bf16,
+                                  const void *q, const void *k, const void *v,
+                                  float *state, void *o, cudaStream_t st) {
+    if (in_bf16)
+        return out_bf16 ? launch_t<__nv_bfloat16, __nv_bfloat16>(p, q, k, v, state, o, st)
+                        : launch_t<__nv_bfloat16, float>(p, q, k, v, state, o, st);
+    return out_bf16 ? launch_t<float, __nv_bfloat16>(p, q, k, v, state, o, st)
+                    : launch_t<float, float>(p, q, k, v, state, o, st);
+}
+
+}  // namespace ret

@@ -1,0 +1,30 @@
+// launch.h -- internal launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ret {
+
+// Adds n to the process-wide launch counter (ret_kernel_launches).
+void note_launches(int n);
+
+cudaError_t launch_parallel_simt(const Params &p, bool in_bf16, bool out_bf16,
+                                 const void *Q, const void *K, const void *V,
+                                 void *O, cudaStream_t st);
+
+cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
+                                  bool out_bf16, const void *Q, const void *K,
+                                  const void *V, const float *s_in,
+                                  float *s_out, void *O, cudaStream_t st);
+
+cudaError_t launch_recurrent_step(const Params &p, bool in_bf16, bool out_bf16,
+                                  const void *q, const void *k, const void *v,
+                                  float *state, void *o, cudaStream_t st);
+
+cudaError_t launch_gate_norm(int B, int L, int H, int dv, bool o_bf16,
+                             const void *O, bool g_bf16, const void *G,
+                             float eps, bool y_bf16, void *Y, cudaStream_t st);
+
+}  // namespace ret

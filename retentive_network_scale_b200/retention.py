@@ -1,0 +1,246 @@
+"""ctypes binding of ``libretention.so`` (declared in ``include/retention.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  The functions take torch CUDA tensors (torch provides device
+memory and streams), check that they are contiguous CUDA tensors of the
+expected shapes -- a host pointer handed to a kernel would fault -- build the
+``ret_desc``, call the C entry point of the same name on the current (or
+given) stream and raise ``RetentionError`` on any non-zero status.
+
+The library is required: if it is missing or cannot be loaded, every call
+raises; nothing falls back to another implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libretention.so")
+
+RET_F32, RET_BF16 = 0, 1
+RET_MAX_HEADS = 128
+STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET_ERR_ALIGN",
+                "RET_ERR_ARG", "RET_ERR_WORKSPACE", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA",
+                "RET_ERR_TIMEOUT"]
+
+# every symbol include/retention.h declares
+EXPORTS = ("ret_parallel", "ret_chunkwise", "ret_workspace_size", "ret_recurrent_step",
+           "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches", "ret_status_string")
+
+
+class RetentionError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else str(status)
+        super().__init__(f"{what}: {name} ({_status_text(status)})")
+
+
+class RetDesc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
+        ("d_k", ctypes.c_int), ("d_v", ctypes.c_int),
+        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("gamma", ctypes.POINTER(ctypes.c_double)),
+        ("rotate", ctypes.c_int), ("theta_base", ctypes.c_double),
+        ("pos_offset", ctypes.c_longlong),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m retentive_network_scale_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    vp, st, D = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(RetDesc)
+    lib.ret_parallel.argtypes = [D, vp, vp, vp, vp, vp]
+    lib.ret_chunkwise.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                  ctypes.c_float, vp, vp, st, vp]
+    lib.ret_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.ret_workspace_size.restype = st
+    lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
+    lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
+                                                       ctypes.c_int, vp, vp]
+    lib.ret_last_device_status.argtypes = [vp]
+    lib.ret_kernel_launches.argtypes = []
+    lib.ret_kernel_launches.restype = ctypes.c_ulonglong
+    lib.ret_status_string.argtypes = [ctypes.c_int]
+    lib.ret_status_string.restype = ctypes.c_char_p
+    for f in ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "ret_gate_norm",
+              "ret_last_device_status"):
+        getattr(lib, f).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _status_text(status: int) -> str:
+    try:
+        return load_library().ret_status_string(status).decode()
+    except Exception:  # the library itself failed to load
+        return "?"
+
+
+def msr_gammas(H: int) -> list:
+    """Decay schedule gamma_h = 1 - 2^(-5-h) of the multi-scale retention
+    layer ("Retentive Network" paper summary, section 2.2)."""
+    return [1.0 - 2.0 ** (-5 - h) for h in range(H)]
+
+
+# ---------------------------------------------------------------- marshalling
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RET_F32
+    if t.dtype == torch.bfloat16:
+        return RET_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t, name, shape=None, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate=False,
+              theta_base=10000.0, pos_offset=0):
+    if len(gamma) != H:
+        raise ValueError("gamma needs one value per head")
+    g = (ctypes.c_double * H)(*[float(x) for x in gamma])
+    d = RetDesc(B, H, L, d_k, d_v, in_dtype, out_dtype,
+                ctypes.cast(g, ctypes.POINTER(ctypes.c_double)), int(bool(rotate)),
+                float(theta_base), int(pos_offset))
+    d._keep = g  # keep the host gamma array alive with the struct
+    return d
+
+
+def _check(status, what):
+    if status != 0:
+        raise RetentionError(status, what)
+
+
+# ---------------------------------------------------------------- entry points
+def ret_parallel(Q, K, V, O, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
+                 stream=None):
+    """Parallel form: O = (Q^ K^^T (.) D) V.  Q, K [B,H,L,dk], V, O [B,H,L,dv]."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _dev(Q, "Q"); _dev(K, "K", Q.shape, Q.dtype); _dev(V, "V", (B, H, L, dv), Q.dtype)
+    _dev(O, "O", (B, H, L, dv))
+    d = make_desc(B, H, L, dk, dv, _dtype_code(Q), _dtype_code(O), gamma, rotate,
+                  theta_base, pos_offset)
+    _check(lib.ret_parallel(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                            _stream(stream)), "ret_parallel")
+    return O
+
+
+def ret_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk,
+                       want_O=True, want_Y=False, rotate=False, theta_base=10000.0,
+                       pos_offset=0) -> int:
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
+    return int(lib.ret_workspace_size(ctypes.byref(d), int(chunk), int(bool(want_O)),
+                                      int(bool(want_Y))))
+
+
+def ret_chunkwise(Q, K, V, gamma, chunk, O=None, state_in=None, state_out=None, G=None,
+                  Y=None, gn_eps=1e-5, rotate=False, theta_base=10000.0, pos_offset=0,
+                  workspace=None, stream=None):
+    """Chunkwise recurrent form with optional state in/out and the fused
+    GroupNorm + swish gate (Y).  Allocates the workspace with torch when the
+    call needs one and none is given.  Returns (O, Y, state_out)."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _dev(Q, "Q"); _dev(K, "K", Q.shape, Q.dtype); _dev(V, "V", (B, H, L, dv), Q.dtype)
+    _dev(O, "O", (B, H, L, dv))
+    _dev(state_in, "state_in", (B, H, dk, dv), torch.float32)
+    _dev(state_out, "state_out", (B, H, dk, dv), torch.float32)
+    _dev(G, "G", (B, L, H * dv), Q.dtype)
+    _dev(Y, "Y", (B, L, H * dv))
+    if O is not None and Y is not None and O.dtype != Y.dtype:
+        raise TypeError("O and Y must share a dtype")
+    out_t = O if O is not None else Y
+    if out_t is None:
+        raise ValueError("request O, Y or both")
+    d = make_desc(B, H, L, dk, dv, _dtype_code(Q), _dtype_code(out_t), gamma, rotate,
+                  theta_base, pos_offset)
+    need = int(lib.ret_workspace_size(ctypes.byref(d), int(chunk), int(O is not None),
+                                      int(Y is not None)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_chunkwise(ctypes.byref(d), int(chunk), _ptr(Q), _ptr(K), _ptr(V),
+                             _ptr(state_in), _ptr(state_out), _ptr(O), _ptr(G),
+                             float(gn_eps), _ptr(Y), _ptr(workspace), ws_bytes,
+                             _stream(stream)), "ret_chunkwise")
+    return O, Y, state_out
+
+
+def ret_recurrent_step(q, k, v, state, o, gamma, pos, rotate=False, theta_base=10000.0,
+                       stream=None):
+    """One recurrent step at absolute position ``pos``: q, k [B,H,dk],
+    v, o [B,H,dv], state [B,H,dk,dv] fp32 updated in place."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _dev(q, "q"); _dev(k, "k", q.shape, q.dtype); _dev(v, "v", (B, H, dv), q.dtype)
+    _dev(state, "state", (B, H, dk, dv), torch.float32); _dev(o, "o", (B, H, dv))
+    d = make_desc(B, H, 1, dk, dv, _dtype_code(q), _dtype_code(o), gamma, rotate,
+                  theta_base, pos)
+    _check(lib.ret_recurrent_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(state),
+                                  _ptr(o), _stream(stream)), "ret_recurrent_step")
+    return o
+
+
+def ret_gate_norm(O, G, Y, eps=1e-5, stream=None):
+    """Y = swish(G) (.) GroupNorm_h(O): O [B,H,L,dv]; G, Y [B,L,H*dv]."""
+    lib = load_library()
+    B, H, L, dv = O.shape
+    _dev(O, "O"); _dev(G, "G", (B, L, H * dv)); _dev(Y, "Y", (B, L, H * dv))
+    _check(lib.ret_gate_norm(B, L, H, dv, _dtype_code(O), _ptr(O), _dtype_code(G), _ptr(G),
+                             float(eps), _dtype_code(Y), _ptr(Y), _stream(stream)),
+           "ret_gate_norm")
+    return Y
+
+
+def ret_last_device_status(stream=None) -> int:
+    return int(load_library().ret_last_device_status(_stream(stream)))
+
+
+def ret_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(load_library().ret_kernel_launches())
+
+
+def ret_status_string(status: int) -> str:
+    return load_library().ret_status_string(int(status)).decode()

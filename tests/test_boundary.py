@@ -1,0 +1,147 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol ``include/retention.h`` declares, and rejects invalid arguments with
+the documented status before any device work.  Only invalid calls are made
+here (they return before the library touches CUDA), plus one valid call on a
+machine without an sm_100 device, which must refuse rather than fall back."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from retentive_network_scale_b200 import build as rbuild
+from retentive_network_scale_b200 import retention as R
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retention.h")
+
+# A 16-byte aligned address that is never dereferenced: every call below is
+# rejected by argument checks that run before any pointer is used.
+FAKE = 0x10000
+MISALIGNED = 0x10008
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rbuild.build()
+    return R.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ret_[a-z_]+)\s*\(", text)))
+
+
+def test_header_lists_the_entry_points():
+    assert declared_functions() == sorted(R.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(len(R.STATUS_NAMES)):
+        s = lib.ret_status_string(code)
+        assert s and len(s) >= 2
+    assert lib.ret_status_string(0) == b"ok"
+
+
+def desc(**kw):
+    base = dict(B=2, H=2, L=8, d_k=16, d_v=16, in_dtype=R.RET_BF16, out_dtype=R.RET_BF16,
+                gamma=[0.9, 0.99], rotate=True)
+    base.update(kw)
+    return R.make_desc(**base)
+
+
+def call_parallel(lib, d, Q=FAKE, K=FAKE, V=FAKE, O=FAKE):
+    return lib.ret_parallel(ctypes.byref(d), Q, K, V, O, None)
+
+
+def call_chunkwise(lib, d, chunk=4, Q=FAKE, K=FAKE, V=FAKE, s_in=None, s_out=None, O=FAKE,
+                   G=None, eps=1e-5, Y=None, ws=None, ws_bytes=0):
+    return lib.ret_chunkwise(ctypes.byref(d), chunk, Q, K, V, s_in, s_out, O, G, eps, Y, ws,
+                             ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), "RET_ERR_SHAPE"), (dict(L=-2), "RET_ERR_SHAPE"), (dict(H=0, gamma=[]), "RET_ERR_SHAPE"),
+    (dict(H=R.RET_MAX_HEADS + 1, gamma=[0.5] * (R.RET_MAX_HEADS + 1)), "RET_ERR_SHAPE"),
+    (dict(d_k=258), "RET_ERR_SHAPE"), (dict(d_v=516), "RET_ERR_SHAPE"),
+    (dict(d_v=18), "RET_ERR_SHAPE"), (dict(d_k=0), "RET_ERR_SHAPE"),
+    (dict(in_dtype=7), "RET_ERR_DTYPE"), (dict(out_dtype=-1), "RET_ERR_DTYPE"),
+    (dict(gamma=[1.5, 0.9]), "RET_ERR_ARG"), (dict(gamma=[-0.1, 0.9]), "RET_ERR_ARG"),
+    (dict(gamma=[float("nan"), 0.9]), "RET_ERR_ARG"),
+    (dict(d_k=15), "RET_ERR_ARG"), (dict(theta_base=0.0), "RET_ERR_ARG"),
+    (dict(pos_offset=-1), "RET_ERR_ARG"), (dict(raw_rotate=2), "RET_ERR_ARG"),
+])
+def test_bad_descriptions(lib, kw, status):
+    raw_rotate = kw.pop("raw_rotate", None)
+    d = desc(**kw)
+    if raw_rotate is not None:
+        d.rotate = raw_rotate
+    want = R.STATUS_NAMES.index(status)
+    assert call_parallel(lib, d) == want
+    assert call_chunkwise(lib, d) == want
+    assert lib.ret_workspace_size(ctypes.byref(d), 4, 0, 1) == 0
+
+
+def test_null_description(lib):
+    assert lib.ret_parallel(None, FAKE, FAKE, FAKE, FAKE, None) == R.STATUS_NAMES.index("RET_ERR_NULL")
+
+
+def test_bad_pointers(lib):
+    d = desc()
+    NULL, ALIGN = R.STATUS_NAMES.index("RET_ERR_NULL"), R.STATUS_NAMES.index("RET_ERR_ALIGN")
+    assert call_parallel(lib, d, Q=None) == NULL
+    assert call_parallel(lib, d, O=None) == NULL
+    assert call_parallel(lib, d, V=MISALIGNED) == ALIGN
+    assert call_chunkwise(lib, d, O=None) == NULL                      # nothing requested
+    assert call_chunkwise(lib, d, G=FAKE, Y=None) == NULL              # G without Y
+    assert call_chunkwise(lib, d, s_out=MISALIGNED) == ALIGN
+    assert call_chunkwise(lib, d, chunk=0) == R.STATUS_NAMES.index("RET_ERR_ARG")
+    assert call_chunkwise(lib, d, G=FAKE, Y=FAKE, eps=-1.0) == R.STATUS_NAMES.index("RET_ERR_ARG")
+    # Y without O needs workspace for the fp32 O it normalises
+    need = lib.ret_workspace_size(ctypes.byref(d), 4, 0, 1)
+    assert need == 4 * 2 * 2 * 8 * 16
+    assert call_chunkwise(lib, d, O=None, G=FAKE, Y=FAKE) == R.STATUS_NAMES.index("RET_ERR_WORKSPACE")
+    assert call_chunkwise(lib, d, O=None, G=FAKE, Y=FAKE, ws=FAKE, ws_bytes=need - 1) == \
+        R.STATUS_NAMES.index("RET_ERR_WORKSPACE")
+
+
+def test_recurrent_step_arguments(lib):
+    d = desc(L=2)
+    assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_SHAPE")
+    d = desc(L=1)
+    assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_NULL")
+    assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, FAKE, MISALIGNED, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_ALIGN")
+
+
+def test_gate_norm_arguments(lib):
+    SHAPE, DT = R.STATUS_NAMES.index("RET_ERR_SHAPE"), R.STATUS_NAMES.index("RET_ERR_DTYPE")
+    assert lib.ret_gate_norm(1, 4, 2, 18, 0, FAKE, 0, FAKE, 1e-5, 0, FAKE, None) == SHAPE
+    assert lib.ret_gate_norm(1, 4, 0, 16, 0, FAKE, 0, FAKE, 1e-5, 0, FAKE, None) == SHAPE
+    assert lib.ret_gate_norm(1, 4, 2, 16, 3, FAKE, 0, FAKE, 1e-5, 0, FAKE, None) == DT
+    assert lib.ret_gate_norm(1, 4, 2, 16, 0, FAKE, 0, FAKE, -1.0, 0, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_ARG")
+    assert lib.ret_gate_norm(1, 4, 2, 16, 0, None, 0, FAKE, 1e-5, 0, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_NULL")
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the refusal on a machine without sm_100")
+def test_valid_call_without_sm100_refuses(lib):
+    # zero-length problem: valid arguments, nothing would be read
+    d = desc(L=0)
+    assert call_parallel(lib, d) == R.STATUS_NAMES.index("RET_ERR_UNSUPPORTED")
+
+
+def test_binding_rejects_host_tensors():
+    q = torch.zeros(1, 1, 4, 8)
+    with pytest.raises(TypeError):
+        R.ret_parallel(q, q, q, q, [0.5])
