@@ -131,12 +131,15 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     ret_status s = check_desc(desc);
     if (s != RET_OK) return s;
     if (chunk < 1) return RET_ERR_ARG;
-    if ((G == nullptr) != (Y == nullptr)) return RET_ERR_NULL;
-    const bool want_Y = Y != nullptr, want_O = O != nullptr;
-    if (!want_Y && !want_O) return RET_ERR_NULL;
-    if (want_Y && !(gn_eps >= 0.0f && std::isfinite(gn_eps))) return RET_ERR_ARG;
     const bool empty = (long long)desc->B * desc->L == 0;
-    if (!empty && (!Q || !K || !V)) return RET_ERR_NULL;
+    const bool want_Y = Y != nullptr, want_O = O != nullptr;
+    if (!empty) {
+        // (an empty problem may come with NULL buffers: nothing is read or written)
+        if ((G == nullptr) != (Y == nullptr)) return RET_ERR_NULL;
+        if (!want_Y && !want_O) return RET_ERR_NULL;
+        if (!Q || !K || !V) return RET_ERR_NULL;
+    }
+    if (want_Y && !(gn_eps >= 0.0f && std::isfinite(gn_eps))) return RET_ERR_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(G) ||
         !aligned16(Y) || !aligned16(state_in) || !aligned16(state_out) || !aligned16(workspace))
         return RET_ERR_ALIGN;
@@ -161,8 +164,15 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     const bool in_bf16 = desc->in_dtype == RET_BF16, out_bf16 = desc->out_dtype == RET_BF16;
     void *o_buf = want_O ? O : workspace;
     const bool o_bf16 = want_O ? out_bf16 : false;
-    cudaError_t e = launch_chunkwise_simt(p, chunk, in_bf16, o_bf16, Q, K, V, state_in,
-                                          state_out, o_buf, st);
+    cudaError_t e;
+    if (chunkwise_tc_supported(p, chunk, in_bf16)) {
+        int *status = device_status_word();
+        if (!status) return RET_ERR_CUDA;
+        e = launch_chunkwise_tc(p, o_bf16, Q, K, V, state_in, state_out, o_buf, status, st);
+    } else {
+        e = launch_chunkwise_simt(p, chunk, in_bf16, o_bf16, Q, K, V, state_in, state_out, o_buf,
+                                  st);
+    }
     if (e == cudaSuccess && want_Y)
         e = launch_gate_norm(desc->B, desc->L, desc->H, desc->d_v, o_bf16, o_buf, in_bf16, G,
                              gn_eps, out_bf16, Y, st);

@@ -19,6 +19,16 @@ cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
                                   const void *V, const float *s_in,
                                   float *s_out, void *O, cudaStream_t st);
 
+// Tensor-core chunkwise kernel: bf16 inputs, chunk 128, d_k 128 or 256,
+// d_v a multiple of 128.
+bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16);
+cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
+                                const void *V, const float *s_in, float *s_out, void *O,
+                                int *status, cudaStream_t st);
+
+// Address of the device status word bounded waits latch errors into.
+int *device_status_word();
+
 cudaError_t launch_recurrent_step(const Params &p, bool in_bf16, bool out_bf16,
                                   const void *q, const void *k, const void *v,
                                   float *state, void *o, cudaStream_t st);

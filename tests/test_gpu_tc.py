@@ -1,0 +1,88 @@
+"""Parity of the tensor-core chunkwise path (bf16 inputs, chunk 128, d_k 128
+or 256, d_v a multiple of 128) against the fp64 oracle: ragged tails, a
+single row, state in/out (aliased), rotation at large positions, gamma = 0
+and gamma = 1 heads, fp32 and bf16 outputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from parity import rel_l2, TOL_BF16
+from retentive_network_scale_b200 import retention as R
+from retentive_network_scale_b200.synth import random_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from retentive_network_scale_b200 import build
+    build.build()
+    R.load_library()
+    yield
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+
+
+def _inputs(B, H, L, dk, dv, seed):
+    Q = random_tensor((B, H, L, dk), seed, dk ** -0.5).bfloat16()
+    K = random_tensor((B, H, L, dk), seed + 1, dk ** -0.5).bfloat16()
+    V = random_tensor((B, H, L, dv), seed + 2).bfloat16()
+    return Q, K, V
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,out", [
+    (1, 2, 128, 128, 128, torch.float32),
+    (1, 2, 300, 128, 128, torch.float32),
+    (2, 1, 1, 256, 128, torch.float32),
+    (1, 3, 257, 256, 256, torch.bfloat16),
+    (2, 2, 640, 256, 512, torch.bfloat16),
+])
+def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out):
+    Q, K, V = _inputs(B, H, L, dk, dv, 100 + L)
+    g = ([0.0, 0.96875, 1.0] * 2)[:H] if H > 1 else [0.96875]
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=5)
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=out)
+    S = torch.empty(B, H, dk, dv, device="cuda")
+    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, state_out=S, rotate=True,
+                    pos_offset=5)
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
+            assert rel_l2(S[b, h], S_ref[b, h]) <= TOL_BF16, (b, h)
+
+
+def test_tc_state_chaining_and_large_positions():
+    """Two calls joined through an aliased state equal one oracle run; the
+    second starts near position 60000."""
+    B, H, L1, L2, dk, dv = 1, 2, 200, 190, 128, 128
+    Q, K, V = _inputs(B, H, L1 + L2, dk, dv, 7)
+    g = [0.96875, 0.999]
+    p0 = 60000
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=p0)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    S = torch.empty(B, H, dk, dv, device="cuda")
+    O1 = torch.empty(B, H, L1, dv, device="cuda")
+    O2 = torch.empty(B, H, L2, dv, device="cuda")
+    R.ret_chunkwise(Qd[:, :, :L1].contiguous(), Kd[:, :, :L1].contiguous(), Vd[:, :, :L1].contiguous(),
+                    g, 128, O=O1, state_out=S, rotate=True, pos_offset=p0)
+    R.ret_chunkwise(Qd[:, :, L1:].contiguous(), Kd[:, :, L1:].contiguous(), Vd[:, :, L1:].contiguous(),
+                    g, 128, O=O2, state_in=S, state_out=S, rotate=True, pos_offset=p0 + L1)
+    got = torch.cat([O1, O2], 2)
+    for h in range(H):
+        assert rel_l2(got[0, h], O_ref[0, h]) <= TOL_BF16
+        assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16
+
+
+def test_tc_without_rotation_and_gate():
+    B, H, L, dk, dv = 2, 2, 384, 256, 256
+    Q, K, V = _inputs(B, H, L, dk, dv, 21)
+    G = random_tensor((B, L, H * dv), 24).bfloat16()
+    g = [0.9, 0.995]
+    O_ref, _ = orc.recurrent(Q, K, V, g)
+    Y_ref = orc.gate_groupnorm(O_ref, G)
+    Y = torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16)
+    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, G=G.cuda(), Y=Y)
+    assert rel_l2(Y, Y_ref) <= TOL_BF16
