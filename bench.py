@@ -23,6 +23,7 @@ implementation of the method here), on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -204,7 +205,7 @@ def config_of(w):
                         f"xPos on, bf16 in/out",
             "global_batch": w.B, "seq_len": w.L, "heads": w.H, "d_k": w.d_k, "d_v": w.d_v,
             "chunk": w.chunk, "parallelism": "replicas",
-            "l2": "inputs (805 MB) larger than L2; no flush"}
+            "l2": f"inputs ({w.B * w.H * w.L * (2 * w.d_k + 2 * w.d_v) * 2 / 1e6:.0f} MB) larger than L2; no flush"}
 
 
 # ----------------------------------------------------------------- GPU timing
@@ -296,6 +297,8 @@ def run_ours(args, world, rank, local):
     R.load_library()
     pk, pk_src = peaks()
     w = WORKLOADS["msr_1p3b"]
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch)
     host = make_inputs(w)
     host = {k: v.pin_memory() for k, v in host.items()}
     d = {k: v.cuda(non_blocking=True) for k, v in host.items()}
@@ -395,6 +398,8 @@ def main():
     ap.add_argument("--skip-extra", action="store_true", help="only the main step")
     ap.add_argument("--skip-cpu", action="store_true", help="no CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the MSR workload's batch (small cases for profiler captures)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:

@@ -117,9 +117,11 @@ ret_status ret_parallel(const ret_desc *desc, const void *Q, const void *K, cons
 
 size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_Y) {
     if (check_desc(desc) != RET_OK || chunk < 1) return 0;
-    // The CUDA-core chunkwise path needs an fp32 O to normalise when only Y
-    // is requested.
-    if (want_Y && !want_O)
+    // The tensor-core kernel normalises in its epilogue.  The CUDA-core
+    // chunkwise path needs an fp32 O to normalise when only Y is requested.
+    Params p;
+    make_params(desc, &p);
+    if (want_Y && !want_O && !chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16))
         return sizeof(float) * (size_t)desc->B * desc->H * desc->L * desc->d_v;
     return 0;
 }
@@ -164,15 +166,14 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     const bool in_bf16 = desc->in_dtype == RET_BF16, out_bf16 = desc->out_dtype == RET_BF16;
     void *o_buf = want_O ? O : workspace;
     const bool o_bf16 = want_O ? out_bf16 : false;
-    cudaError_t e;
     if (chunkwise_tc_supported(p, chunk, in_bf16)) {
         int *status = device_status_word();
         if (!status) return RET_ERR_CUDA;
-        e = launch_chunkwise_tc(p, o_bf16, Q, K, V, state_in, state_out, o_buf, status, st);
-    } else {
-        e = launch_chunkwise_simt(p, chunk, in_bf16, o_bf16, Q, K, V, state_in, state_out, o_buf,
-                                  st);
+        return from_cuda(launch_chunkwise_tc(p, out_bf16, Q, K, V, state_in, state_out, O, G, Y,
+                                             gn_eps, status, st));
     }
+    cudaError_t e = launch_chunkwise_simt(p, chunk, in_bf16, o_bf16, Q, K, V, state_in, state_out,
+                                          o_buf, st);
     if (e == cudaSuccess && want_Y)
         e = launch_gate_norm(desc->B, desc->L, desc->H, desc->d_v, o_bf16, o_buf, in_bf16, G,
                              gn_eps, out_bf16, Y, st);

@@ -20,11 +20,13 @@ cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
                                   float *s_out, void *O, cudaStream_t st);
 
 // Tensor-core chunkwise kernel: bf16 inputs, chunk 128, d_k 128 or 256,
-// d_v a multiple of 128.
+// d_v a multiple of 128 (at most 512), every gamma_h^128 >= 2^-60.  With Y
+// (and G) given it also writes Y = swish(G) (.) GroupNorm_h(O); O may then
+// be NULL.
 bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16);
 cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
                                 const void *V, const float *s_in, float *s_out, void *O,
-                                int *status, cudaStream_t st);
+                                const void *G, void *Y, float eps, int *status, cudaStream_t st);
 
 // Address of the device status word bounded waits latch errors into.
 int *device_status_word();

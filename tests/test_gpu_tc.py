@@ -1,7 +1,8 @@
 """Parity of the tensor-core chunkwise path (bf16 inputs, chunk 128, d_k 128
-or 256, d_v a multiple of 128) against the fp64 oracle: ragged tails, a
-single row, state in/out (aliased), rotation at large positions, gamma = 0
-and gamma = 1 heads, fp32 and bf16 outputs."""
+or 256, d_v a multiple of 128, gamma^128 >= 2^-60) against the fp64 oracle:
+ragged tails, a single row, state in/out (aliased), rotation at large
+positions, gamma = 1 heads, fp32 and bf16 outputs, and the fused GroupNorm +
+swish gate epilogue at cluster sizes 1, 2 and 4 (one launch per call)."""
 import numpy as np
 import pytest
 import torch
@@ -40,7 +41,7 @@ def _inputs(B, H, L, dk, dv, seed):
 ])
 def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out):
     Q, K, V = _inputs(B, H, L, dk, dv, 100 + L)
-    g = ([0.0, 0.96875, 1.0] * 2)[:H] if H > 1 else [0.96875]
+    g = ([0.75, 0.96875, 1.0] * 2)[:H] if H > 1 else [0.96875]
     O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=5)
     O = torch.empty(B, H, L, dv, device="cuda", dtype=out)
     S = torch.empty(B, H, dk, dv, device="cuda")
@@ -76,13 +77,44 @@ def test_tc_state_chaining_and_large_positions():
         assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16
 
 
-def test_tc_without_rotation_and_gate():
-    B, H, L, dk, dv = 2, 2, 384, 256, 256
-    Q, K, V = _inputs(B, H, L, dk, dv, 21)
+@pytest.mark.parametrize("dk,dv,rotate,with_O,with_state", [
+    (256, 256, False, False, False),
+    (256, 512, True, True, False),
+    (128, 128, True, False, True),
+    (128, 384, False, True, True),
+])
+def test_tc_fused_gate_groupnorm(dk, dv, rotate, with_O, with_state):
+    """Y = swish(G) (.) GroupNorm_h(O) from the one fused launch."""
+    B, H, L = 2, 2, 300
+    Q, K, V = _inputs(B, H, L, dk, dv, 21 + dv)
     G = random_tensor((B, L, H * dv), 24).bfloat16()
+    S0 = random_tensor((B, H, dk, dv), 25, 0.3) if with_state else None
     g = [0.9, 0.995]
-    O_ref, _ = orc.recurrent(Q, K, V, g)
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=17, state_in=S0)
     Y_ref = orc.gate_groupnorm(O_ref, G)
     Y = torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16)
-    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, G=G.cuda(), Y=Y)
-    assert rel_l2(Y, Y_ref) <= TOL_BF16
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16) if with_O else None
+    S = torch.empty(B, H, dk, dv, device="cuda")
+    n0 = R.ret_kernel_launches()
+    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, G=G.cuda(), Y=Y, rotate=rotate,
+                    pos_offset=17, state_in=None if S0 is None else S0.cuda(), state_out=S)
+    assert R.ret_kernel_launches() - n0 == 1
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(Y[b, :, h * dv:(h + 1) * dv], Y_ref[b, :, h * dv:(h + 1) * dv]) <= TOL_BF16
+            assert rel_l2(S[b, h], S_ref[b, h]) <= TOL_BF16
+            if with_O:
+                assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16
+
+
+def test_small_gamma_uses_cuda_core_path():
+    """gamma below the tensor-core range (gamma^128 < 2^-60) still matches."""
+    B, H, L, dk, dv = 1, 2, 200, 128, 128
+    Q, K, V = _inputs(B, H, L, dk, dv, 31)
+    g = [0.0, 0.5]
+    O_ref, _ = orc.recurrent(Q, K, V, g, rotate=True)
+    O = torch.empty(B, H, L, dv, device="cuda")
+    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, rotate=True)
+    assert rel_l2(O, O_ref) <= TOL_BF16
