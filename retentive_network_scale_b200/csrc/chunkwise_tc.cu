@@ -8,11 +8,11 @@
 //   R  <- gamma^n R + sum_j' gamma^{n-1-j'} k^_j'^T v_j'
 // The kernel evaluates it in a rescaled form that leaves the tensor cores
 // nothing but plain products:
-//   V'   = diag(zeta) V,            zeta_j  = gamma^{n-1-j}
+//   K~   = diag(zeta) K^,           zeta_j  = gamma^{n-1-j}   (fused into the turn of K)
 //   Rbar = bf16(gamma^n R)          (the decayed state, kept that way in TMEM)
-//   O''  = Q^ Rbar + mask(Q^ K^^T) V'        (mask: keep j' <= j)
+//   O''  = Q^ Rbar + mask(Q^ K~^T) V         (mask: keep j' <= j)
 //   o_j  = alpha_j O''_j,           alpha_j = gamma^{j+1-n}
-//   R    <- gamma^n R + K^^T V'
+//   R    <- gamma^n R + K~^T V
 // which is the same sum term by term (gamma^{j+1-n} gamma^{n-1-j'} =
 // gamma^{j-j'}, gamma^{j+1-n} gamma^n = gamma^{j+1}).  All factors stay in
 // range while gamma^128 >= 2^-60; other decays use the CUDA-core kernel.
@@ -20,12 +20,14 @@
 // One CTA owns one (b, h) and a 128-column slice of V and walks the chunks
 // in order.  Tensor memory (512 columns): S [128 x 128] (P, the bf16 mask
 // of S, overwrites half of it and feeds the P V' product as the A operand),
-// O'' [128 x 128], and the fp32 state slice R [d_k x 128] as d_k/128 halves
-// of 128 lanes.  Shared memory: TMA-loaded Q, K, V tiles (128-byte swizzle)
-// and Rbar in the MN-major layout read as a B operand.  Loads of Q, K and V
-// complete on separate barriers and are issued as soon as the MMAs that
-// read the previous tile finish, so the next chunk's Q streams in while
-// this chunk's state update runs.
+// O'' [128 x 128] (the two together are one 128 x 256 accumulator), and the
+// fp32 state slice transposed, R^T [128 x d_k] (lanes are V columns).
+// Shared memory: TMA-loaded Q, K, V tiles (128-byte swizzle), with K^ and
+// Rbar^T interleaved per 64-column block so that [K~ ; Rbar^T] is the single
+// 256-row B operand of the [S | O''] product.  Loads of Q, K and V complete
+// on separate barriers and are issued as soon as the MMAs that read the
+// previous tile finish; V needs no preparation, so its load overlaps the
+// next [S | O''] product.
 //
 // Fused epilogue (Y = swish(G) (.) GroupNorm_h(O)): the CTAs of one head
 // form a cluster along d_v; each reduces its 128 columns of a row to a mean
@@ -40,6 +42,8 @@
 // and TMEM is freed.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc_util.cuh"
@@ -51,39 +55,42 @@ using namespace tc;
 
 constexpr int kC = 128;       // chunk rows (MMA M)
 constexpr int kTV = 128;      // value columns per CTA (MMA N)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kMaxCluster = kMaxDv / kTV;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 constexpr float kMinLog2GammaTimesC = -60.f;        // gamma^C >= 2^-60
 
-enum { BQ = 0, BK, BV, BS, BX, BU, BPV, kNumBars };
+enum { BQ = 0, BK, BV, BS, BU, BPV, kNumBars };
 
 template <int DK>
 struct Layout {
     static constexpr uint32_t kQ = 0;                    // Q^: DK/64 blocks of 16 KB
     static constexpr uint32_t kQBytes = kC * DK * 2;
-    static constexpr uint32_t kK = kQ + kQBytes;         // K^
-    static constexpr uint32_t kV = kK + kQBytes;         // V (then V'): 2 blocks of 16 KB
+    // K^ and the bf16 state copy Rbar^T interleaved per 64-column block, so
+    // that [K^ ; Rbar^T] is one 256-row K-major B operand of the S|X product:
+    // block kb = [K^ rows 0..127 | Rbar^T rows (v columns) 0..127], 32 KB.
+    static constexpr uint32_t kKR = kQ + kQBytes;
+    static constexpr uint32_t kKRBytes = 2 * kC * DK * 2;
+    static constexpr uint32_t kV = kKR + kKRBytes;       // V (then V'): 2 blocks of 16 KB
     static constexpr uint32_t kVBytes = kC * kTV * 2;
-    static constexpr uint32_t kR = kV + kVBytes;         // Rbar: 2 column blocks of DK*128 B
-    static constexpr uint32_t kRBytes = DK * kTV * 2;
-    static constexpr uint32_t kSmall = kR + kRBytes;
+    static constexpr uint32_t kSmall = kV + kVBytes;
     static constexpr uint32_t kBar = kSmall;             // kNumBars mbarriers
     static constexpr uint32_t kTmemSlot = kSmall + 64;
     static constexpr uint32_t kAbort = kSmall + 68;
-    static constexpr uint32_t kRotStep = kSmall + 128;   // DK/2 float2
-    static constexpr uint32_t kBytes = kRotStep + DK * 4;
+    static constexpr uint32_t kBytes = kSmall + 128;
     // GroupNorm scratch inside the V tile, which is dead between the P V'
     // product and the next V load.
-    static constexpr uint32_t kGnPart = kV;              // [128] float2: second warpgroup's partials
-    static constexpr uint32_t kGnStat = kV + 1024;       // [128] float2: per-row mean and scale
-    static constexpr uint32_t kGnXchg = kV + 2048;       // [cluster rank][128] float2
+    static constexpr uint32_t kGnPart = kV;              // [4 warpgroups][128] row sums
+    static constexpr uint32_t kGnPart2 = kV + 2048;      // [4 warpgroups][128] centred squares
+    static constexpr uint32_t kGnXchg = kV + 4096;       // [cluster rank][128] (mean, M2)
+    static __device__ __forceinline__ uint32_t k_blk(int kb) { return kKR + kb * 32768; }
+    static __device__ __forceinline__ uint32_t rbar_blk(int kb) { return kKR + kb * 32768 + 16384; }
 };
 
-constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);   // Q^ (K-major) x K^ (K-major)
-constexpr uint32_t kIdescX = idesc_bf16(128, kTV, 0, 1);   // Q^ x Rbar (MN-major)
-constexpr uint32_t kIdescPV = idesc_bf16(128, kTV, 0, 1);  // P (tmem) x V' (MN-major)
-constexpr uint32_t kIdescU = idesc_bf16(128, kTV, 1, 1);   // K^^T (MN-major) x V' (MN-major)
+// [S | O''] = Q^ [K^ ; Rbar^T]^T : A Q^ (K-major), B 256 rows (K-major)
+constexpr uint32_t kIdescSX = idesc_bf16(128, 256, 0, 0);
+// O'' += P V' : A P from tensor memory, B V' (MN-major)
+constexpr uint32_t kIdescPV = idesc_bf16(128, kTV, 0, 1);
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                          int *status) {
@@ -108,12 +115,12 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
 }
 
-// Row d of Rbar (MN-major B operand: blocks of 64 columns, each DK rows of
-// 128 bytes, 128-byte swizzle): 32 values from column col0.
+// Row c of Rbar^T (K-major, 128-byte swizzle, inside the interleaved K^ /
+// Rbar^T blocks): the 32 values of d-columns [d0, d0+32).
 template <int DK>
-__device__ __forceinline__ void st_rbar_row32(uint8_t *rbar, int d, int col0, const float *v) {
-    const int blk = col0 >> 6;
-    const int ch0 = (col0 & 63) >> 3;
+__device__ __forceinline__ void st_rbarT_row32(uint8_t *smem, int c, int d0, const float *v) {
+    uint8_t *blk = smem + Layout<DK>::rbar_blk(d0 >> 6) + c * 128;
+    const int ch0 = (d0 & 63) >> 3;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 w;
@@ -121,45 +128,16 @@ __device__ __forceinline__ void st_rbar_row32(uint8_t *rbar, int d, int col0, co
         w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
         w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
         w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        const int phys = (ch0 + q) ^ (d & 7);
-        *reinterpret_cast<uint4 *>(rbar + blk * (DK * 128) + d * 128 + phys * 16) = w;
+        *reinterpret_cast<uint4 *>(blk + (((ch0 + q) ^ (c & 7)) << 4)) = w;
     }
 }
 
-// xPos turn of one [128 x DK] K-major swizzled tile in place.  Thread ->
-// (16-byte column chunk = 4 pairs, starting row r0); it walks rows r0,
-// r0+RS, ... and advances its four angles by RS*theta_j per step.
-template <int DK>
-__device__ void rotate_tile(uint8_t *tile, const float2 *rotstep, const Params &p, int t0, int n,
-                            int tid) {
-    constexpr int NCH = DK / 8;
-    constexpr int RS = kThreads / NCH;
-    const int c16 = tid % NCH;
-    const int r0 = tid / NCH;
-    const int blk = c16 >> 3, cw = c16 & 7;
-    float c[4], s[4], sc[4], ss[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int j = c16 * 4 + e;
-        rot_cs(p.pos_offset + t0 + r0, p.theta[j], &c[e], &s[e]);
-        sc[e] = rotstep[j].x;
-        ss[e] = rotstep[j].y;
-    }
-#pragma unroll 2
-    for (int r = r0; r < n; r += RS) {
-        uint4 *ptr = reinterpret_cast<uint4 *>(tile + blk * 16384 + r * 128 + ((cw ^ (r & 7)) << 4));
-        uint4 w = *ptr;
-        uint32_t *u = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_bf16(u[e]);
-            u[e] = pack_bf16(x.x * c[e] - x.y * s[e], x.x * s[e] + x.y * c[e]);
-            const float cn = c[e] * sc[e] - s[e] * ss[e];
-            s[e] = c[e] * ss[e] + s[e] * sc[e];
-            c[e] = cn;
-        }
-        *ptr = w;
-    }
+// cos and sin of pos * theta: the product and its reduction to [-pi, pi]
+// in fp64, then the fast sine/cosine (absolute error near 2^-21 there).
+__device__ __forceinline__ void rot_cs_fast(long long pos, double theta, float *c, float *s) {
+    const double a = (double)pos * theta;
+    const double k = rint(a * 0.15915494309189533577);
+    __sincosf((float)fma(-k, 6.283185307179586477, a), s, c);
 }
 
 template <typename T>
@@ -183,21 +161,29 @@ __device__ __forceinline__ void st_row32<__nv_bfloat16>(__nv_bfloat16 *dst, cons
     }
 }
 
+// swish(g) = g * sigmoid(g) with the fast exponential and division.
+__device__ __forceinline__ float swish_fast(float g) { return __fdividef(g, 1.f + __expf(-g)); }
+
 template <int DK, typename TO, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const Params p,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmY, const Params p,
                     const float *__restrict__ state_in, float *__restrict__ state_out,
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, TO *__restrict__ Y,
                     float gn_eps, int *status) {
     using Ly = Layout<DK>;
-    constexpr int NH = DK / 128;   // state halves of 128 rows
-    constexpr int KB = DK / 64;    // 64-column blocks of Q^, K^
+    constexpr int KB = DK / 64;        // 64-column blocks of Q^, K^, Rbar^T
+    constexpr int NCH = DK / 8;        // 16-byte chunks per Q/K row
+    constexpr int RS = kThreads / NCH; // rows rotated in parallel
+    constexpr int RG = DK / 128;       // 32-column groups per thread in the state passes
+    constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V^T K~ (both MN-major)
+    constexpr bool kStage = sizeof(TO) == 2;  // bf16 tiles leave by TMA store
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int wg = tid >> 7;        // warpgroup
-    const int row = tid & 127;      // TMEM lane of this thread
+    const int wg = tid >> 7;        // warpgroup 0..3; each covers all 128 TMEM lanes
+    const int row = tid & 127;      // TMEM lane: chunk row for S/O, V column for R^T
     const int bh = blockIdx.y, h = bh % p.H;
     const int v0 = blockIdx.x * kTV;
     const float lg = p.log2g[h];
@@ -210,7 +196,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     auto bar = [&](int i) { return sbase + Ly::kBar + 8u * i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::kAbort);
-    float2 *rotstep = reinterpret_cast<float2 *>(smem + Ly::kRotStep);
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
@@ -222,27 +207,26 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_alloc(sbase + Ly::kTmemSlot, 512);
         tmem_relinquish();
     }
-    constexpr int kRS = kThreads / (DK / 8);
+    // rotation: this thread's column chunk, first row and per-step turn
+    const int rc16 = tid % NCH, rr0 = tid / NCH;
+    float rsc[4] = {1.f, 1.f, 1.f, 1.f}, rss[4] = {0.f, 0.f, 0.f, 0.f};
+    float rc0[4], rs0[4];
     if (p.rotate)
-        for (int j = tid; j < DK / 2; j += kThreads) {
-            float c, s;
-            rot_cs(kRS, p.theta[j], &c, &s);
-            rotstep[j] = make_float2(c, s);
-        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rot_cs_fast(RS, p.theta[rc16 * 4 + e], &rsc[e], &rss[e]);
+    auto prep_angles = [&](int c) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            rot_cs_fast(p.pos_offset + (long long)c * kC + rr0, p.theta[rc16 * 4 + e], &rc0[e], &rs0[e]);
+    };
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + Ly::kTmemSlot);
     const uint32_t tS = tmem, tO = tmem + 128, tR = tmem + 256;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    // Ownership of the state columns in the R passes: with two halves each
-    // warpgroup takes one half; with one half they split its 128 columns.
-    const int r_half = (NH == 2) ? wg : 0;
-    const int r_col0 = (NH == 2) ? 0 : wg * 64;
-    const int r_groups = (NH == 2) ? 4 : 2;
-    const int r_d = r_half * 128 + row;
-    // O / P: each warpgroup owns 64 columns of a row.
-    const int o_col0 = wg * 64;
+    const int r_d0 = wg * (DK / 4);  // d-columns of R^T this thread moves
+    const int o_col0 = wg * 32;      // S / O columns of this thread
 
     auto load_q = [&](int c) {
         mbar_expect_tx(bar(BQ), Ly::kQBytes);
@@ -252,102 +236,26 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     auto load_k = [&](int c) {
         mbar_expect_tx(bar(BK), Ly::kQBytes);
         for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(sbase + Ly::kK + kb * 16384, &tmK, bar(BK), kb * 64, c * kC, bh);
+            tma_load_3d(sbase + Ly::k_blk(kb), &tmK, bar(BK), kb * 64, c * kC, bh);
     };
     auto load_v = [&](int c) {
         mbar_expect_tx(bar(BV), Ly::kVBytes);
         for (int nb = 0; nb < 2; ++nb)
             tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, c * kC, bh);
     };
-    auto vdesc = [&](int ks) { return sdesc_sw128(sbase + Ly::kV + ks * 2048, 16384, 1024); };
     auto sync_alive = [&]() {
         __syncthreads();
         return *abort_flag == 0;
     };
-
-    if (tid == 0) {
-        load_q(0);
-        load_k(0);
-        load_v(0);
-    }
-
-    // starting state: TMEM R = gamma^{n_0} S_in and Rbar = bf16 of the same
-    const bool has_in = state_in != nullptr;
-    if (has_in) {
-        const float g0 = decay_pow(lg, min(kC, L));
-        const float *src = state_in + ((size_t)bh * DK + r_d) * dv + v0;
-        for (int g = 0; g < r_groups; ++g) {
-            const int col = r_col0 + 32 * g;
-            float v[32];
-            uint32_t r[32];
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                const float4 x = *reinterpret_cast<const float4 *>(src + col + i);
-                v[i] = x.x * g0; v[i + 1] = x.y * g0; v[i + 2] = x.z * g0; v[i + 3] = x.w * g0;
-            }
-            st_rbar_row32<DK>(smem + Ly::kR, r_d, col, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-            tmem_st32(tR + r_half * 128 + lane_base + col, r);
-        }
-        tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    bool alive = sync_alive();
-
+    // K~ = diag(zeta) K^ without rotation: zeta_j = gamma^{n-1-j}
+    auto scale_k = [&](int n) {
+        const float zeta = row < n ? decay_pow(lg, n - 1 - row) : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < nchunks; ++c) {
-        const uint32_t par = c & 1;  // every barrier completes once per chunk
-        const int t0 = c * kC;
-        const int n = min(kC, L - t0);
-        const bool has_state = has_in || c > 0;
-        const bool last = c + 1 == nchunks;
-
-        // ---- rotate Q and K of this chunk in place
-        if (alive) {
-            wait_bar(bar(BQ), par, abort_flag, status);
-            wait_bar(bar(BK), par, abort_flag, status);
-        }
-        alive = sync_alive();
-        if (alive && p.rotate) {
-            rotate_tile<DK>(smem + Ly::kQ, rotstep, p, t0, n, tid);
-            rotate_tile<DK>(smem + Ly::kK, rotstep, p, t0, n, tid);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- S = Q^ K^^T ; O'' = Q^ Rbar
-        if (alive && tid == 0) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int ks = 0; ks < DK / 16; ++ks) {
-                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                mma_ss(tS, sdesc_sw128(sbase + Ly::kQ + off, 16, 1024),
-                       sdesc_sw128(sbase + Ly::kK + off, 16, 1024), kIdescS, ks > 0);
-            }
-            mma_commit(bar(BS));
-            if (has_state) {
-#pragma unroll 1
-                for (int ks = 0; ks < DK / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_ss(tO, sdesc_sw128(sbase + Ly::kQ + off, 16, 1024),
-                           sdesc_sw128(sbase + Ly::kR + ks * 2048, DK * 128, 1024), kIdescX, ks > 0);
-                }
-            }
-            mma_commit(bar(BX));
-        }
-
-        // ---- V' = diag(zeta) V in place, while the MMAs run
-        if (alive) wait_bar(bar(BV), par, abort_flag, status);
-        alive = sync_alive();
-        if (alive) {
-            const float zeta = row < n ? decay_pow(lg, n - 1 - row) : 0.f;
-            uint8_t *vrow = smem + Ly::kV + wg * 16384 + row * 128;
+        for (int kb = wg; kb < KB; kb += 4) {
+            uint8_t *krow = smem + Ly::k_blk(kb) + row * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(vrow + (((q + row) & 7) << 4));
+                uint4 *ptr = reinterpret_cast<uint4 *>(krow + (((q + row) & 7) << 4));
                 uint4 w = *ptr;
                 uint32_t *u = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
@@ -358,183 +266,344 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 *ptr = w;
             }
         }
-        fence_proxy_async_smem();
+    };
+    // this thread's slice of the rotation of one tile (rows r0, r0+RS, ...),
+    // rows scaled by gamma^{n-1-r} when `zeta` is set (K~)
+    auto rotate = [&](uint32_t blk0, uint32_t blk_stride, int n, bool zeta) {
+        const int blk = rc16 >> 3, cw = rc16 & 7;
+        uint8_t *base = smem + blk0 + blk * blk_stride;
+        float c[4], sn[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            c[e] = rc0[e];
+            sn[e] = rs0[e];
+        }
+#pragma unroll 2
+        for (int r = rr0; r < n; r += RS) {
+            const float z = zeta ? decay_pow(lg, n - 1 - r) : 1.f;
+            uint4 *ptr = reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4));
+            uint4 w = *ptr;
+            uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = unpack_bf16(u[e]);
+                const float zc = z * c[e], zs = z * sn[e];
+                u[e] = pack_bf16(x.x * zc - x.y * zs, x.x * zs + x.y * zc);
+                const float cn = c[e] * rsc[e] - sn[e] * rss[e];
+                sn[e] = c[e] * rss[e] + sn[e] * rsc[e];
+                c[e] = cn;
+            }
+            *ptr = w;
+        }
+    };
+    // K~ of a chunk: turned and scaled, or scaled only
+    auto prep_k = [&](int n) {
+        if (p.rotate)
+            rotate(Ly::kKR, 32768, n, true);
+        else
+            scale_k(n);
+    };
+    // MMA descriptors: fixed buffers, so only the start address moves
+    const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);          // A of [S|O''], K-major
+    const uint64_t dKR = sdesc_sw128(sbase + Ly::kKR, 16, 1024);        // B of [S|O''], K-major
+    const uint64_t dVa = sdesc_sw128(sbase + Ly::kV, 16384, 1024);      // A of R^T update, MN-major
+    const uint64_t dKb = sdesc_sw128(sbase + Ly::kKR, 32768, 1024);     // B of R^T update, MN-major
+    const uint64_t dVb = dVa;                                           // B of P V, MN-major
+
+    if (tid == 0) {
+        load_q(0);
+        load_k(0);
+        load_v(0);
+    }
+    // Starting state: TMEM R^T = gamma^{n_0} S_in^T and Rbar^T = bf16 of the
+    // same; zeros without a state (the S|X product then gives O'' = 0).
+    const bool has_in = state_in != nullptr;
+    {
+        const float g0 = decay_pow(lg, min(kC, L));
+#pragma unroll 1
+        for (int g = 0; g < RG; ++g) {
+            const int d0 = r_d0 + 32 * g;
+            float v[32];
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = has_in ? state_in[((size_t)bh * DK + d0 + i) * dv + v0 + row] * g0 : 0.f;
+            st_rbarT_row32<DK>(smem, row, d0, v);
+            if (has_in) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+                tmem_st32(tR + lane_base + d0, r);
+            }
+        }
+        if (has_in) tmem_wait_st();
+    }
+    // chunk 0: turn Q and K, scale K
+    bool alive = true;
+    {
+        const int n0 = min(kC, L);
+        if (tid == 0) {
+            wait_bar(bar(BQ), 0, abort_flag, status);
+            wait_bar(bar(BK), 0, abort_flag, status);
+        }
+        alive = sync_alive();
+        if (alive) {
+            if (p.rotate) {
+                prep_angles(0);
+                rotate(Ly::kQ, 16384, n0, false);
+            }
+            prep_k(n0);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    alive = sync_alive();
+
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+        const uint32_t par = c & 1;  // every barrier completes once per chunk
+        const int t0 = c * kC;
+        const int n = min(kC, L - t0);
+        const bool has_state = has_in || c > 0;
+        const bool last = c + 1 == nchunks;
+        const int n_next = last ? 0 : min(kC, L - t0 - kC);
+
+        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T  (thread 0)
+        if (alive && tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < DK / 16; ++ks) {
+                const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                const uint64_t offkr = (uint64_t)(((ks >> 2) * 32768 + (ks & 3) * 32) >> 4);
+                mma_ss(tS, dQ + off, dKR + offkr, kIdescSX, ks > 0);
+            }
+            mma_commit(bar(BS));
+        }
+        // ---- R^T += V^T K~ as soon as V is in (thread 32; no data shared with
+        // the products thread 0 issues, so the two need no ordering)
+        if (alive && tid == 32) {
+            tc_fence_after();
+            if (wait_bar(bar(BV), par, abort_flag, status)) {
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks) {
+                    const uint64_t off = (uint64_t)((ks * 2048) >> 4);
+                    mma_ss(tR, dVa + off, dKb + off, kIdescU, (ks > 0 || has_state) ? 1u : 0u);
+                }
+            }
+            mma_commit(bar(BU));
+        }
 
         // ---- P = bf16(S) on j' <= j, else 0, into tensor memory
-        if (alive) wait_bar(bar(BS), par, abort_flag, status);
+        if (alive && tid == 0) {
+            wait_bar(bar(BS), par, abort_flag, status);
+            if (!last) load_q(c + 1);  // Q^ is no longer read
+        }
         alive = sync_alive();
         tc_fence_after();
         if (alive) {
-            uint32_t a[32], bb[32], pk[32];
+            uint32_t a[32], pk[16];
             tmem_ld32(tS + lane_base + o_col0, a);
-            tmem_ld32(tS + lane_base + o_col0 + 32, bb);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int k0 = o_col0 + 2 * i, k1 = o_col0 + 32 + 2 * i;
+                const int k0 = o_col0 + 2 * i;
                 pk[i] = pack_bf16(k0 <= row ? __uint_as_float(a[2 * i]) : 0.f,
                                   k0 + 1 <= row ? __uint_as_float(a[2 * i + 1]) : 0.f);
-                pk[16 + i] = pack_bf16(k1 <= row ? __uint_as_float(bb[2 * i]) : 0.f,
-                                       k1 + 1 <= row ? __uint_as_float(bb[2 * i + 1]) : 0.f);
             }
-            // keys [0,64) -> columns [0,32), keys [64,128) -> columns [64,96)
-            tmem_st32(tS + lane_base + o_col0, pk);
+            // keys [32w, 32w+32) -> columns [32w, 32w+16)
+            tmem_st16(tS + lane_base + o_col0, pk);
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- R += K^^T V' ; O'' += P V'
-        if (alive && tid == 0) {
+        // ---- O'' += P V
+        if (alive && tid == 0 && wait_bar(bar(BV), par, abort_flag, status)) {
             tc_fence_after();
-#pragma unroll 1
-            for (int hh = 0; hh < NH; ++hh)
-#pragma unroll 1
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ss(tR + hh * 128, sdesc_sw128(sbase + Ly::kK + hh * 32768 + ks * 2048, 16384, 1024),
-                           vdesc(ks), kIdescU, (ks > 0 || has_state) ? 1u : 0u);
-            mma_commit(bar(BU));
-#pragma unroll 1
+#pragma unroll
             for (int ks = 0; ks < kC / 16; ++ks)
-                mma_ts(tO, tS + (ks >> 2) * 64 + (ks & 3) * 8, vdesc(ks), kIdescPV,
-                       (ks > 0 || has_state) ? 1u : 0u);
+                mma_ts(tO, tS + (ks >> 1) * 32 + (ks & 1) * 8, dVb + (uint64_t)((ks * 2048) >> 4),
+                       kIdescPV, 1u);
             mma_commit(bar(BPV));
-            // Q^ is dead once S and O'' = Q^ Rbar are done: fetch the next Q
-            if (!last && wait_bar(bar(BX), par, abort_flag, status)) load_q(c + 1);
         }
 
-        // ---- state: R -> gamma^{n'} R in TMEM and Rbar; or state_out
-        if (alive) wait_bar(bar(BU), par, abort_flag, status);
+        // ---- state: R^T -> gamma^{n'} R^T in TMEM and Rbar^T; or state_out
+        if (alive && tid == 0) {
+            wait_bar(bar(BU), par, abort_flag, status);
+            if (!last) load_k(c + 1);  // K^ is no longer read
+        }
         alive = sync_alive();
         tc_fence_after();
-        if (alive && tid == 0 && !last) load_k(c + 1);
         if (alive) {
-            const float gnext = last ? 1.f : decay_pow(lg, min(kC, L - t0 - kC));
+            const float gnext = last ? 1.f : decay_pow(lg, n_next);
 #pragma unroll 1
-            for (int g = 0; g < r_groups; ++g) {
-                const int col = r_col0 + 32 * g;
+            for (int g = 0; g < RG; ++g) {
+                const int d0 = r_d0 + 32 * g;
                 uint32_t r[32];
                 float v[32];
-                tmem_ld32(tR + r_half * 128 + lane_base + col, r);
+                tmem_ld32(tR + lane_base + d0, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gnext;
                 if (last) {
-                    if (state_out) st_row32<float>(state_out + ((size_t)bh * DK + r_d) * dv + v0 + col, v);
+                    if (state_out) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            state_out[((size_t)bh * DK + d0 + i) * dv + v0 + row] = v[i];
+                    }
                 } else {
-                    st_rbar_row32<DK>(smem + Ly::kR, r_d, col, v);
+                    st_rbarT_row32<DK>(smem, row, d0, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-                    tmem_st32(tR + r_half * 128 + lane_base + col, r);
+                    tmem_st32(tR + lane_base + d0, r);
                 }
             }
             tmem_wait_st();
         }
 
+        // ---- next chunk's Q^ while P V' runs
+        if (alive && !last && tid == 0) wait_bar(bar(BQ), par ^ 1, abort_flag, status);
+        alive = sync_alive();
+        if (alive && !last && p.rotate) {
+            prep_angles(c + 1);
+            rotate(Ly::kQ, 16384, n_next, false);
+        }
+
         // ---- epilogue: o_j = alpha_j O''_j (and the fused GroupNorm + gate)
-        if (alive) wait_bar(bar(BPV), par, abort_flag, status);
+        if (alive && tid == 0) wait_bar(bar(BPV), par, abort_flag, status);
         alive = sync_alive();
         tc_fence_after();
-        const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}, lg finite here
-        float x[64];
+        const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite here
+        float x[32];
         if (alive) {
-            uint32_t a[32], bb[32];
+            uint32_t a[32];
             tmem_ld32(tO + lane_base + o_col0, a);
-            tmem_ld32(tO + lane_base + o_col0 + 32, bb);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                x[i] = __uint_as_float(a[i]);
-                x[32 + i] = __uint_as_float(bb[i]);
-            }
+            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
         }
         const size_t orow = ((size_t)bh * L + t0 + row) * dv + v0 + o_col0;
-        if constexpr (!FUSE) {
-            if (alive && row < n) {
-                float y[64];
+        // bf16 tiles leave through shared memory (the V tile, dead now) and a
+        // TMA store; rows past the sequence end are clipped by the store.
+        auto stage_store = [&](const float *vals, const CUtensorMap *map, int x0, int y0, int z0) {
+            uint8_t *dst = smem + Ly::kV + (wg >> 1) * 16384 + row * 128;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) y[i] = x[i] * alpha;
-                st_row32<TO>(O + orow, y);
-                st_row32<TO>(O + orow + 32, y + 32);
+            for (int q = 0; q < 4; ++q) {
+                uint4 w;
+                w.x = pack_bf16(vals[8 * q + 0], vals[8 * q + 1]);
+                w.y = pack_bf16(vals[8 * q + 2], vals[8 * q + 3]);
+                w.z = pack_bf16(vals[8 * q + 4], vals[8 * q + 5]);
+                w.w = pack_bf16(vals[8 * q + 6], vals[8 * q + 7]);
+                *reinterpret_cast<uint4 *>(dst + ((((wg & 1) * 4 + q) ^ (row & 7)) << 4)) = w;
             }
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tma_store_3d(map, sbase + Ly::kV, x0, y0, z0);
+                tma_store_3d(map, sbase + Ly::kV + 16384, x0 + 64, y0, z0);
+                bulk_commit();
+                bulk_wait_read();
+            }
+            __syncthreads();
+        };
+        if constexpr (!FUSE) {
+            if (alive) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] *= alpha;
+            }
+            if constexpr (kStage) {
+                if (alive) stage_store(x, &tmO, v0, t0, bh);
+            } else if (alive && row < n) {
+                st_row32<TO>(O + orow, x);
+            }
+            if (alive && tid == 0 && !last) load_v(c + 1);  // V is no longer read
         } else {
             const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
             const uint32_t rank = cluster_rank();
             const int b = bh / p.H;
-            const size_t grow = ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o_col0;
-            uint4 gv[8];
+            const size_t grow =
+                ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o_col0;
+            uint4 gv[4];
             if (alive && row < n) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) gv[q] = *reinterpret_cast<const uint4 *>(G + grow + 8 * q);
+                for (int q = 0; q < 4; ++q) gv[q] = *reinterpret_cast<const uint4 *>(G + grow + 8 * q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) gv[q] = make_uint4(0u, 0u, 0u, 0u);
             }
-            float2 *part = reinterpret_cast<float2 *>(smem + Ly::kGnPart);
-            float2 *stat = reinterpret_cast<float2 *>(smem + Ly::kGnStat);
+            float *part = reinterpret_cast<float *>(smem + Ly::kGnPart);    // [4][128] sums
+            float *part2 = reinterpret_cast<float *>(smem + Ly::kGnPart2);  // [4][128] centred squares
             const float2 *xchg = reinterpret_cast<const float2 *>(smem + Ly::kGnXchg);
             // CTA-local mean and centred sum of squares of the row's 128 columns
             float s = 0.f;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) s += x[i];
-            if (wg == 1) part[row].x = s;
+            for (int i = 0; i < 32; ++i) s += x[i];
+            part[wg * 128 + row] = s;
             __syncthreads();
-            if (wg == 0) stat[row].x = (s + part[row].x) * (1.f / kTV);
-            __syncthreads();
-            const float mc = stat[row].x;
+            const float mc =
+                ((part[row] + part[128 + row]) + (part[256 + row] + part[384 + row])) * (1.f / kTV);
             float q2 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
-            if (wg == 1) part[row].y = q2;
-            // every CTA of the head is past its P V' product: V tiles are free
+            for (int i = 0; i < 32; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
+            part2[wg * 128 + row] = q2;
+            // every CTA of the head is past its P V product: V tiles are free
             cluster_sync();
             if (alive && wg == 0) {
-                const float m2c = q2 + part[row].y;
+                const float m2c = (part2[row] + part2[128 + row]) + (part2[256 + row] + part2[384 + row]);
                 const uint32_t slot = sbase + Ly::kGnXchg + (rank * 128 + row) * 8;
                 for (int r = 0; r < nr; ++r) st_cluster_f32x2(map_to_rank(slot, r), mc, m2c);
             }
             cluster_sync();
-            if (alive && wg == 0) {
-                float mean = 0.f;
-                for (int r = 0; r < nr; ++r) mean += xchg[r * 128 + row].x;
-                mean /= (float)nr;
-                float m2 = 0.f;
-                for (int r = 0; r < nr; ++r) {
-                    const float2 e = xchg[r * 128 + row];
-                    m2 += e.y + (float)kTV * (e.x - mean) * (e.x - mean);
-                }
-                const float var = m2 / (float)(nr * kTV);   // of O'' ; O = alpha O''
-                stat[row] = make_float2(mean, alpha * rsqrtf(alpha * alpha * var + gn_eps));
+            float mean = 0.f;
+            for (int r = 0; r < nr; ++r) mean += xchg[r * 128 + row].x;
+            mean /= (float)nr;
+            float m2 = 0.f;
+            for (int r = 0; r < nr; ++r) {
+                const float2 e = xchg[r * 128 + row];
+                m2 += e.y + (float)kTV * (e.x - mean) * (e.x - mean);
             }
-            __syncthreads();
-            if (alive && row < n) {
-                const float2 ms = stat[row];
-                float y[64];
+            const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
+            const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
+            __syncthreads();                           // the scratch in the V tile is read
+            float y[32];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t *u = reinterpret_cast<const uint32_t *>(&gv[q]);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t *u = reinterpret_cast<const uint32_t *>(&gv[q]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 g2 = unpack_bf16(u[e]);
-                        const int i = 8 * q + 2 * e;
-                        y[i] = g2.x / (1.f + expf(-g2.x)) * ((x[i] - ms.x) * ms.y);
-                        y[i + 1] = g2.y / (1.f + expf(-g2.y)) * ((x[i + 1] - ms.x) * ms.y);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 g2 = unpack_bf16(u[e]);
+                    const int i = 8 * q + 2 * e;
+                    y[i] = swish_fast(g2.x) * ((x[i] - mean) * scale);
+                    y[i + 1] = swish_fast(g2.y) * ((x[i + 1] - mean) * scale);
                 }
+            }
+            if constexpr (kStage) {
+                if (alive) stage_store(y, &tmY, h * dv + v0, t0, b);
+                if (alive && O) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) y[i] = x[i] * alpha;
+                    stage_store(y, &tmO, v0, t0, bh);
+                }
+            } else if (alive && row < n) {
                 st_row32<TO>(Y + grow, y);
-                st_row32<TO>(Y + grow + 32, y + 32);
                 if (O) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) y[i] = x[i] * alpha;
+                    for (int i = 0; i < 32; ++i) y[i] = x[i] * alpha;
                     st_row32<TO>(O + orow, y);
-                    st_row32<TO>(O + orow + 32, y + 32);
                 }
             }
+            if (alive && tid == 0 && !last) load_v(c + 1);
         }
+
+        // ---- next chunk's K~
+        if (alive && !last && tid == 0) wait_bar(bar(BK), par ^ 1, abort_flag, status);
+        alive = sync_alive();
+        if (alive && !last) prep_k(n_next);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        // the V tile (and the GroupNorm scratch in it) is free: next V
-        if (alive && tid == 0 && !last) load_v(c + 1);
     }
 
+    if (tid == 0) bulk_wait_all();       // output stores in flight
     if constexpr (FUSE) cluster_sync();  // peers may still write into this CTA's smem before it
     // After an abort, copies and MMAs still in flight get a bounded time to
     // land before the shared and tensor memory are released.
@@ -586,6 +655,13 @@ template <int DK, typename TO, bool FUSE>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                      const void *G, void *Y, float eps, int *status, cudaStream_t st) {
+    CUtensorMap mo, my;
+    std::memset(&mo, 0, sizeof(mo));
+    std::memset(&my, 0, sizeof(my));
+    if (sizeof(TO) == 2) {
+        if (O && !make_map(&mo, O, p.dv, p.L, p.B * p.H)) return cudaErrorInvalidValue;
+        if (Y && !make_map(&my, Y, p.H * p.dv, p.L, p.B)) return cudaErrorInvalidValue;
+    }
     auto kern = chunkwise_tc_kernel<DK, TO, FUSE>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -602,7 +678,7 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p, s_in, s_out, (TO *)O,
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, my, p, s_in, s_out, (TO *)O,
                            (const __nv_bfloat16 *)G, (TO *)Y, eps, status);
     if (e == cudaSuccess) note_launches(1);
     return e;
