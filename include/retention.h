@@ -112,6 +112,33 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q,
                          void *Y, void *workspace, size_t workspace_bytes,
                          void *stream);
 
+/*
+ * ret_chunkwise_gate_static -- no counterpart in the paper.  The same call as
+ * ret_chunkwise with G and Y given and O = NULL, for callers that must not
+ * allocate device memory while they run: for instance a service whose
+ * device memory is reserved up front by a host framework, or one held to a
+ * fixed memory budget once serving starts.  Such callers cannot provide the
+ * workspace ret_chunkwise takes for shapes the tensor-core kernel does not
+ * cover (an fp32 O of B*H*L*d_v floats, normalised into Y afterwards).
+ * Here that scratch is a fixed array of RET_STATIC_SCRATCH_FLOATS floats
+ * (16 MiB) inside the library; every device that loads the library holds
+ * it until the process exits.  Nothing is allocated by this call.
+ *   - Problems whose scratch would exceed the array return
+ *     RET_ERR_WORKSPACE before anything runs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; calls that overlap on the GPU (other streams or threads)
+ *     race on it.
+ * Arguments, layouts and other errors are those of ret_chunkwise.
+ */
+#define RET_STATIC_SCRATCH_FLOATS (4u << 20)
+ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk, const void *Q,
+                                     const void *K, const void *V, const float *state_in,
+                                     float *state_out, const void *G, float gn_eps,
+                                     void *Y, void *stream);
+
 /* Bytes of workspace ret_chunkwise needs for this description and chunk
  * (0 when none).  Depends only on the arguments; never fails (returns 0
  * for descriptions that ret_chunkwise would reject). */

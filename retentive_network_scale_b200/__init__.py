@@ -8,7 +8,8 @@ the input generator (``synth``) can be used without the library.
 from importlib import import_module
 
 _BINDING_NAMES = (
-    "ret_parallel", "ret_chunkwise", "ret_recurrent_step", "ret_gate_norm",
+    "ret_parallel", "ret_chunkwise", "ret_chunkwise_gate_static", "ret_recurrent_step",
+    "ret_gate_norm",
     "ret_workspace_size", "ret_last_device_status", "ret_kernel_launches",
     "ret_status_string",
     "RetentionError", "msr_gammas", "load_library",

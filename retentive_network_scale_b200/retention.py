@@ -27,8 +27,10 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
                 "RET_ERR_TIMEOUT"]
 
 # every symbol include/retention.h declares
-EXPORTS = ("ret_parallel", "ret_chunkwise", "ret_workspace_size", "ret_recurrent_step",
-           "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches", "ret_status_string")
+EXPORTS = ("ret_parallel", "ret_chunkwise", "ret_chunkwise_gate_static", "ret_workspace_size",
+           "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
+           "ret_status_string")
+RET_STATIC_SCRATCH_FLOATS = 4 << 20
 
 
 class RetentionError(RuntimeError):
@@ -66,6 +68,8 @@ def load_library(path: str = LIB_PATH):
     lib.ret_parallel.argtypes = [D, vp, vp, vp, vp, vp]
     lib.ret_chunkwise.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
                                   ctypes.c_float, vp, vp, st, vp]
+    lib.ret_chunkwise_gate_static.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp,
+                                              ctypes.c_float, vp, vp]
     lib.ret_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.ret_workspace_size.restype = st
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
@@ -76,8 +80,8 @@ def load_library(path: str = LIB_PATH):
     lib.ret_kernel_launches.restype = ctypes.c_ulonglong
     lib.ret_status_string.argtypes = [ctypes.c_int]
     lib.ret_status_string.restype = ctypes.c_char_p
-    for f in ("ret_parallel", "ret_chunkwise", "ret_recurrent_step", "ret_gate_norm",
-              "ret_last_device_status"):
+    for f in ("ret_parallel", "ret_chunkwise", "ret_chunkwise_gate_static", "ret_recurrent_step",
+              "ret_gate_norm", "ret_last_device_status"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -204,6 +208,26 @@ def ret_chunkwise(Q, K, V, gamma, chunk, O=None, state_in=None, state_out=None, 
                              float(gn_eps), _ptr(Y), _ptr(workspace), ws_bytes,
                              _stream(stream)), "ret_chunkwise")
     return O, Y, state_out
+
+
+def ret_chunkwise_gate_static(Q, K, V, gamma, chunk, G, Y, state_in=None, state_out=None,
+                              gn_eps=1e-5, rotate=False, theta_base=10000.0, pos_offset=0,
+                              stream=None):
+    """Chunkwise form with the fused GroupNorm + swish gate (Y only) whose
+    scratch is the library's fixed device array: nothing is allocated."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _dev(Q, "Q"); _dev(K, "K", Q.shape, Q.dtype); _dev(V, "V", (B, H, L, dv), Q.dtype)
+    _dev(G, "G", (B, L, H * dv), Q.dtype); _dev(Y, "Y", (B, L, H * dv))
+    _dev(state_in, "state_in", (B, H, dk, dv), torch.float32)
+    _dev(state_out, "state_out", (B, H, dk, dv), torch.float32)
+    d = make_desc(B, H, L, dk, dv, _dtype_code(Q), _dtype_code(Y), gamma, rotate, theta_base,
+                  pos_offset)
+    _check(lib.ret_chunkwise_gate_static(ctypes.byref(d), int(chunk), _ptr(Q), _ptr(K), _ptr(V),
+                                         _ptr(state_in), _ptr(state_out), _ptr(G), float(gn_eps),
+                                         _ptr(Y), _stream(stream)), "ret_chunkwise_gate_static")
+    return Y
 
 
 def ret_recurrent_step(q, k, v, state, o, gamma, pos, rotate=False, theta_base=10000.0,
