@@ -56,6 +56,7 @@ using namespace tc;
 constexpr int kC = 128;       // chunk rows (MMA M)
 constexpr int kTV = 128;      // value columns per CTA (MMA N)
 constexpr int kThreads = 512;
+constexpr int kGroup = 256;   // two groups of two warpgroups
 constexpr int kMaxCluster = kMaxDv / kTV;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 constexpr float kMinLog2GammaTimesC = -60.f;        // gamma^C >= 2^-60
@@ -80,9 +81,9 @@ struct Layout {
     static constexpr uint32_t kBytes = kSmall + 128;
     // GroupNorm scratch inside the V tile, which is dead between the P V'
     // product and the next V load.
-    static constexpr uint32_t kGnPart = kV;              // [4 warpgroups][128] row sums
-    static constexpr uint32_t kGnPart2 = kV + 2048;      // [4 warpgroups][128] centred squares
-    static constexpr uint32_t kGnXchg = kV + 4096;       // [cluster rank][128] (mean, M2)
+    static constexpr uint32_t kGnPart = kV;              // [2 warpgroups][128] row sums
+    static constexpr uint32_t kGnPart2 = kV + 1024;      // [2 warpgroups][128] centred squares
+    static constexpr uint32_t kGnXchg = kV + 2048;       // [cluster rank][128] (mean, M2)
     static __device__ __forceinline__ uint32_t k_blk(int kb) { return kKR + kb * 32768; }
     static __device__ __forceinline__ uint32_t rbar_blk(int kb) { return kKR + kb * 32768 + 16384; }
 };
@@ -173,10 +174,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, TO *__restrict__ Y,
                     float gn_eps, int *status) {
     using Ly = Layout<DK>;
-    constexpr int KB = DK / 64;        // 64-column blocks of Q^, K^, Rbar^T
-    constexpr int NCH = DK / 8;        // 16-byte chunks per Q/K row
-    constexpr int RS = kThreads / NCH; // rows rotated in parallel
-    constexpr int RG = DK / 128;       // 32-column groups per thread in the state passes
+    constexpr int KB = DK / 64;         // 64-column blocks of Q^, K~, Rbar^T
+    constexpr int NCH = DK / 8;         // 16-byte chunks per Q/K row
+    constexpr int RSG = kGroup / NCH;   // rows one group turns in parallel
+    constexpr int RGA = DK / 64;        // 32-column groups per thread in the state pass (group A)
     constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V^T K~ (both MN-major)
     constexpr bool kStage = sizeof(TO) == 2;  // bf16 tiles leave by TMA store
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -184,6 +185,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5;
     const int wg = tid >> 7;        // warpgroup 0..3; each covers all 128 TMEM lanes
     const int row = tid & 127;      // TMEM lane: chunk row for S/O, V column for R^T
+    const int grp = tid >> 8;       // 0: state pass and Q (warpgroups 0,1); 1: output and K (2,3)
+    const int gtid = tid & 255;     // thread index within the group
+    const int gwg = wg & 1;         // warpgroup within the group
     const int bh = blockIdx.y, h = bh % p.H;
     const int v0 = blockIdx.x * kTV;
     const float lg = p.log2g[h];
@@ -207,26 +211,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_alloc(sbase + Ly::kTmemSlot, 512);
         tmem_relinquish();
     }
-    // rotation: this thread's column chunk, first row and per-step turn
-    const int rc16 = tid % NCH, rr0 = tid / NCH;
-    float rsc[4] = {1.f, 1.f, 1.f, 1.f}, rss[4] = {0.f, 0.f, 0.f, 0.f};
-    float rc0[4], rs0[4];
-    if (p.rotate)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) rot_cs_fast(RS, p.theta[rc16 * 4 + e], &rsc[e], &rss[e]);
-    auto prep_angles = [&](int c) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            rot_cs_fast(p.pos_offset + (long long)c * kC + rr0, p.theta[rc16 * 4 + e], &rc0[e], &rs0[e]);
-    };
+    // rotation (per group): column chunk and first row of this thread
+    const int rc16 = gtid % NCH, rr0 = gtid / NCH;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + Ly::kTmemSlot);
     const uint32_t tS = tmem, tO = tmem + 128, tR = tmem + 256;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int r_d0 = wg * (DK / 4);  // d-columns of R^T this thread moves
-    const int o_col0 = wg * 32;      // S / O columns of this thread
 
     auto load_q = [&](int c) {
         mbar_expect_tx(bar(BQ), Ly::kQBytes);
@@ -247,11 +239,48 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         return *abort_flag == 0;
     };
-    // K~ = diag(zeta) K^ without rotation: zeta_j = gamma^{n-1-j}
+    // group-local barrier (hardware barriers 1 and 2) and abort check
+    auto gsync_alive = [&]() {
+        named_sync(1 + grp, kGroup);
+        return *abort_flag == 0;
+    };
+    const bool g_leader = gtid == 0;   // waits on mbarriers for its group
+
+    // this thread's share of turning the tile at blk0 (rows r0, r0+RSG, ...);
+    // rows scaled by gamma^{n-1-r} when `zeta` is set (K~)
+    auto rotate = [&](uint32_t blk0, uint32_t blk_stride, int c, int n, bool zeta) {
+        float cc[4], sn[4], rsc[4], rss[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double th = p.theta[rc16 * 4 + e];
+            rot_cs_fast(p.pos_offset + (long long)c * kC + rr0, th, &cc[e], &sn[e]);
+            rot_cs_fast(RSG, th, &rsc[e], &rss[e]);
+        }
+        const int blk = rc16 >> 3, cw = rc16 & 7;
+        uint8_t *base = smem + blk0 + blk * blk_stride;
+#pragma unroll 4
+        for (int r = rr0; r < n; r += RSG) {
+            const float z = zeta ? decay_pow(lg, n - 1 - r) : 1.f;
+            uint4 *ptr = reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4));
+            uint4 w = *ptr;
+            uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = unpack_bf16(u[e]);
+                const float zc = z * cc[e], zs = z * sn[e];
+                u[e] = pack_bf16(x.x * zc - x.y * zs, x.x * zs + x.y * zc);
+                const float cn = cc[e] * rsc[e] - sn[e] * rss[e];
+                sn[e] = cc[e] * rss[e] + sn[e] * rsc[e];
+                cc[e] = cn;
+            }
+            *ptr = w;
+        }
+    };
+    // K~ = diag(zeta) K^ without rotation (this group's share)
     auto scale_k = [&](int n) {
         const float zeta = row < n ? decay_pow(lg, n - 1 - row) : 0.f;
 #pragma unroll 1
-        for (int kb = wg; kb < KB; kb += 4) {
+        for (int kb = gwg; kb < KB; kb += 2) {
             uint8_t *krow = smem + Ly::k_blk(kb) + row * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -267,39 +296,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
         }
     };
-    // this thread's slice of the rotation of one tile (rows r0, r0+RS, ...),
-    // rows scaled by gamma^{n-1-r} when `zeta` is set (K~)
-    auto rotate = [&](uint32_t blk0, uint32_t blk_stride, int n, bool zeta) {
-        const int blk = rc16 >> 3, cw = rc16 & 7;
-        uint8_t *base = smem + blk0 + blk * blk_stride;
-        float c[4], sn[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            c[e] = rc0[e];
-            sn[e] = rs0[e];
-        }
-#pragma unroll 2
-        for (int r = rr0; r < n; r += RS) {
-            const float z = zeta ? decay_pow(lg, n - 1 - r) : 1.f;
-            uint4 *ptr = reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4));
-            uint4 w = *ptr;
-            uint32_t *u = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 x = unpack_bf16(u[e]);
-                const float zc = z * c[e], zs = z * sn[e];
-                u[e] = pack_bf16(x.x * zc - x.y * zs, x.x * zs + x.y * zc);
-                const float cn = c[e] * rsc[e] - sn[e] * rss[e];
-                sn[e] = c[e] * rss[e] + sn[e] * rsc[e];
-                c[e] = cn;
-            }
-            *ptr = w;
-        }
+    auto prep_q = [&](int c, int n) {
+        if (p.rotate) rotate(Ly::kQ, 16384, c, n, false);
     };
-    // K~ of a chunk: turned and scaled, or scaled only
-    auto prep_k = [&](int n) {
+    auto prep_k = [&](int c, int n) {
         if (p.rotate)
-            rotate(Ly::kKR, 32768, n, true);
+            rotate(Ly::kKR, 32768, c, n, true);
         else
             scale_k(n);
     };
@@ -320,9 +322,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const bool has_in = state_in != nullptr;
     {
         const float g0 = decay_pow(lg, min(kC, L));
+        const int d_begin = wg * (DK / 4);
 #pragma unroll 1
-        for (int g = 0; g < RG; ++g) {
-            const int d0 = r_d0 + 32 * g;
+        for (int g = 0; g < DK / 128; ++g) {
+            const int d0 = d_begin + 32 * g;
             float v[32];
             uint32_t r[32];
 #pragma unroll
@@ -337,21 +340,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if (has_in) tmem_wait_st();
     }
-    // chunk 0: turn Q and K, scale K
+    // chunk 0: group A turns Q, group B prepares K~
     bool alive = true;
     {
         const int n0 = min(kC, L);
-        if (tid == 0) {
-            wait_bar(bar(BQ), 0, abort_flag, status);
-            wait_bar(bar(BK), 0, abort_flag, status);
-        }
-        alive = sync_alive();
+        if (g_leader) wait_bar(bar(grp == 0 ? BQ : BK), 0, abort_flag, status);
+        alive = gsync_alive();
         if (alive) {
-            if (p.rotate) {
-                prep_angles(0);
-                rotate(Ly::kQ, 16384, n0, false);
-            }
-            prep_k(n0);
+            if (grp == 0)
+                prep_q(0, n0);
+            else
+                prep_k(0, n0);
         }
     }
     fence_proxy_async_smem();
@@ -392,7 +391,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mma_commit(bar(BU));
         }
 
-        // ---- P = bf16(S) on j' <= j, else 0, into tensor memory
+        // ---- P = bf16(S) on j' <= j, else 0, into tensor memory (all)
         if (alive && tid == 0) {
             wait_bar(bar(BS), par, abort_flag, status);
             if (!last) load_q(c + 1);  // Q^ is no longer read
@@ -400,17 +399,18 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         alive = sync_alive();
         tc_fence_after();
         if (alive) {
+            const int c0 = wg * 32;
             uint32_t a[32], pk[16];
-            tmem_ld32(tS + lane_base + o_col0, a);
+            tmem_ld32(tS + lane_base + c0, a);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int k0 = o_col0 + 2 * i;
+                const int k0 = c0 + 2 * i;
                 pk[i] = pack_bf16(k0 <= row ? __uint_as_float(a[2 * i]) : 0.f,
                                   k0 + 1 <= row ? __uint_as_float(a[2 * i + 1]) : 0.f);
             }
             // keys [32w, 32w+32) -> columns [32w, 32w+16)
-            tmem_st16(tS + lane_base + o_col0, pk);
+            tmem_st16(tS + lane_base + c0, pk);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -426,184 +426,218 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mma_commit(bar(BPV));
         }
 
-        // ---- state: R^T -> gamma^{n'} R^T in TMEM and Rbar^T; or state_out
-        if (alive && tid == 0) {
-            wait_bar(bar(BU), par, abort_flag, status);
-            if (!last) load_k(c + 1);  // K^ is no longer read
-        }
-        alive = sync_alive();
-        tc_fence_after();
-        if (alive) {
-            const float gnext = last ? 1.f : decay_pow(lg, n_next);
+        if (grp == 0) {
+            // ================= group A: state pass, then the next Q^
+            if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier 1
+            if (alive && g_leader) {
+                wait_bar(bar(BU), par, abort_flag, status);
+                if (!last) load_k(c + 1);  // K~ is no longer read
+            }
+            alive = gsync_alive();
+            tc_fence_after();
+            if (alive) {
+                const float gnext = last ? 1.f : decay_pow(lg, n_next);
+                const int d_begin = gwg * (DK / 2);
+                // R^T columns [d0, d0+32): decay, bf16 copy, back to TMEM; or state_out
+                auto state32 = [&](uint32_t (&r)[32], int d0) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gnext;
+                    if (last) {
+                        if (state_out) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                state_out[((size_t)bh * DK + d0 + i) * dv + v0 + row] = v[i];
+                        }
+                    } else {
+                        st_rbarT_row32<DK>(smem, row, d0, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+                        tmem_st32(tR + lane_base + d0, r);
+                    }
+                };
 #pragma unroll 1
-            for (int g = 0; g < RG; ++g) {
-                const int d0 = r_d0 + 32 * g;
-                uint32_t r[32];
-                float v[32];
-                tmem_ld32(tR + lane_base + d0, r);
+                for (int g = 0; g < RGA; g += 2) {
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(tR + lane_base + d_begin + 32 * g, ra);
+                    tmem_ld32(tR + lane_base + d_begin + 32 * g + 32, rb);
+                    tmem_wait_ld();
+                    state32(ra, d_begin + 32 * g);
+                    state32(rb, d_begin + 32 * g + 32);
+                }
+                tmem_wait_st();
+            }
+            if constexpr (FUSE) {
+                cluster_wait();
+                cluster_arrive();                   // GroupNorm exchange barrier 2
+            }
+            if (alive && !last && g_leader) wait_bar(bar(BQ), par ^ 1, abort_flag, status);
+            alive = gsync_alive();
+            if (alive && !last) prep_q(c + 1, n_next);
+            if constexpr (FUSE) cluster_wait();
+        } else {
+            // ================= group B: output, then the next V and K~
+            if (alive && g_leader) wait_bar(bar(BPV), par, abort_flag, status);
+            alive = gsync_alive();
+            tc_fence_after();
+            const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite
+            const int o0 = gwg * 64;   // this thread's 64 columns of the row, 32 at a time
+            const size_t orow = ((size_t)bh * L + t0 + row) * dv + v0 + o0;
+            // 32 columns of O'' (still in tensor memory until this iteration ends)
+            auto ld_o = [&](int half, float *x) {
+                uint32_t a[32];
+                tmem_ld32(tO + lane_base + o0 + 32 * half, a);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gnext;
-                if (last) {
-                    if (state_out) {
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
+            };
+            // bf16 tiles leave through shared memory (the V tile, dead now)
+            // and a TMA store; rows past the sequence end are clipped.
+            auto stage32 = [&](int half, const float *vals) {
+                uint8_t *dst = smem + Ly::kV + gwg * 16384 + row * 128;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            state_out[((size_t)bh * DK + d0 + i) * dv + v0 + row] = v[i];
-                    }
-                } else {
-                    st_rbarT_row32<DK>(smem, row, d0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-                    tmem_st32(tR + lane_base + d0, r);
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16(vals[8 * q + 0], vals[8 * q + 1]);
+                    w.y = pack_bf16(vals[8 * q + 2], vals[8 * q + 3]);
+                    w.z = pack_bf16(vals[8 * q + 4], vals[8 * q + 5]);
+                    w.w = pack_bf16(vals[8 * q + 6], vals[8 * q + 7]);
+                    *reinterpret_cast<uint4 *>(dst + (((4 * half + q) ^ (row & 7)) << 4)) = w;
                 }
-            }
-            tmem_wait_st();
-        }
-
-        // ---- next chunk's Q^ while P V' runs
-        if (alive && !last && tid == 0) wait_bar(bar(BQ), par ^ 1, abort_flag, status);
-        alive = sync_alive();
-        if (alive && !last && p.rotate) {
-            prep_angles(c + 1);
-            rotate(Ly::kQ, 16384, n_next, false);
-        }
-
-        // ---- epilogue: o_j = alpha_j O''_j (and the fused GroupNorm + gate)
-        if (alive && tid == 0) wait_bar(bar(BPV), par, abort_flag, status);
-        alive = sync_alive();
-        tc_fence_after();
-        const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite here
-        float x[32];
-        if (alive) {
-            uint32_t a[32];
-            tmem_ld32(tO + lane_base + o_col0, a);
-            tmem_wait_ld();
+            };
+            auto store_tile = [&](const CUtensorMap *map, int x0, int y0, int z0) {
+                fence_proxy_async_smem();
+                named_sync(2, kGroup);
+                if (g_leader) {
+                    tma_store_3d(map, sbase + Ly::kV, x0, y0, z0);
+                    tma_store_3d(map, sbase + Ly::kV + 16384, x0 + 64, y0, z0);
+                    bulk_commit();
+                    bulk_wait_read();
+                }
+                named_sync(2, kGroup);
+            };
+            // O = alpha O'' into `dst` (staged tile or direct stores)
+            auto emit_o = [&]() {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float x[32];
+                    ld_o(half, x);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
-        }
-        const size_t orow = ((size_t)bh * L + t0 + row) * dv + v0 + o_col0;
-        // bf16 tiles leave through shared memory (the V tile, dead now) and a
-        // TMA store; rows past the sequence end are clipped by the store.
-        auto stage_store = [&](const float *vals, const CUtensorMap *map, int x0, int y0, int z0) {
-            uint8_t *dst = smem + Ly::kV + (wg >> 1) * 16384 + row * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 w;
-                w.x = pack_bf16(vals[8 * q + 0], vals[8 * q + 1]);
-                w.y = pack_bf16(vals[8 * q + 2], vals[8 * q + 3]);
-                w.z = pack_bf16(vals[8 * q + 4], vals[8 * q + 5]);
-                w.w = pack_bf16(vals[8 * q + 6], vals[8 * q + 7]);
-                *reinterpret_cast<uint4 *>(dst + ((((wg & 1) * 4 + q) ^ (row & 7)) << 4)) = w;
-            }
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0) {
-                tma_store_3d(map, sbase + Ly::kV, x0, y0, z0);
-                tma_store_3d(map, sbase + Ly::kV + 16384, x0 + 64, y0, z0);
-                bulk_commit();
-                bulk_wait_read();
-            }
-            __syncthreads();
-        };
-        if constexpr (!FUSE) {
-            if (alive) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] *= alpha;
-            }
-            if constexpr (kStage) {
-                if (alive) stage_store(x, &tmO, v0, t0, bh);
-            } else if (alive && row < n) {
-                st_row32<TO>(O + orow, x);
-            }
-            if (alive && tid == 0 && !last) load_v(c + 1);  // V is no longer read
-        } else {
-            const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
-            const uint32_t rank = cluster_rank();
-            const int b = bh / p.H;
-            const size_t grow =
-                ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o_col0;
-            uint4 gv[4];
-            if (alive && row < n) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) gv[q] = *reinterpret_cast<const uint4 *>(G + grow + 8 * q);
+                    for (int i = 0; i < 32; ++i) x[i] *= alpha;
+                    if constexpr (kStage)
+                        stage32(half, x);
+                    else if (row < n)
+                        st_row32<TO>(O + orow + 32 * half, x);
+                }
+                if constexpr (kStage) store_tile(&tmO, v0, t0, bh);
+            };
+            if constexpr (!FUSE) {
+                if (alive) emit_o();
             } else {
+                const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
+                const uint32_t rank = cluster_rank();
+                const int b = bh / p.H;
+                const size_t grow =
+                    ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
+                float *part = reinterpret_cast<float *>(smem + Ly::kGnPart);    // [2][128] sums
+                float *part2 = reinterpret_cast<float *>(smem + Ly::kGnPart2);  // [2][128] squares
+                const float2 *xchg = reinterpret_cast<const float2 *>(smem + Ly::kGnXchg);
+                // CTA-local mean and centred sum of squares of the row's 128
+                // columns (two warpgroups hold 64 each)
+                float s = 0.f;
+                if (alive) {
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float x[32];
+                        ld_o(half, x);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) gv[q] = make_uint4(0u, 0u, 0u, 0u);
-            }
-            float *part = reinterpret_cast<float *>(smem + Ly::kGnPart);    // [4][128] sums
-            float *part2 = reinterpret_cast<float *>(smem + Ly::kGnPart2);  // [4][128] centred squares
-            const float2 *xchg = reinterpret_cast<const float2 *>(smem + Ly::kGnXchg);
-            // CTA-local mean and centred sum of squares of the row's 128 columns
-            float s = 0.f;
+                        for (int i = 0; i < 32; ++i) s += x[i];
+                    }
+                }
+                part[gwg * 128 + row] = s;
+                named_sync(2, kGroup);
+                const float mc = (part[row] + part[128 + row]) * (1.f / kTV);
+                float q2 = 0.f;
+                if (alive) {
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float x[32];
+                        ld_o(half, x);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s += x[i];
-            part[wg * 128 + row] = s;
-            __syncthreads();
-            const float mc =
-                ((part[row] + part[128 + row]) + (part[256 + row] + part[384 + row])) * (1.f / kTV);
-            float q2 = 0.f;
+                        for (int i = 0; i < 32; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
+                    }
+                }
+                part2[gwg * 128 + row] = q2;
+                // barrier 1: every CTA of the head is past its P V product, so
+                // their V tiles are free; the partials here are visible.
+                cluster_arrive();
+                cluster_wait();
+                if (alive && gwg == 0) {
+                    const float m2c = part2[row] + part2[128 + row];
+                    const uint32_t slot = sbase + Ly::kGnXchg + (rank * 128 + row) * 8;
+                    for (int r = 0; r < nr; ++r) st_cluster_f32x2(map_to_rank(slot, r), mc, m2c);
+                }
+                cluster_arrive();                    // barrier 2: exchange written
+                cluster_wait();
+                float mean = 0.f;
+                for (int r = 0; r < nr; ++r) mean += xchg[r * 128 + row].x;
+                mean /= (float)nr;
+                float m2 = 0.f;
+                for (int r = 0; r < nr; ++r) {
+                    const float2 e = xchg[r * 128 + row];
+                    m2 += e.y + (float)kTV * (e.x - mean) * (e.x - mean);
+                }
+                const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
+                const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
+                named_sync(2, kGroup);                    // the scratch in the V tile is read
+                if (alive) {
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        uint4 gv[4];
+                        if (row < n) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
-            part2[wg * 128 + row] = q2;
-            // every CTA of the head is past its P V product: V tiles are free
-            cluster_sync();
-            if (alive && wg == 0) {
-                const float m2c = (part2[row] + part2[128 + row]) + (part2[256 + row] + part2[384 + row]);
-                const uint32_t slot = sbase + Ly::kGnXchg + (rank * 128 + row) * 8;
-                for (int r = 0; r < nr; ++r) st_cluster_f32x2(map_to_rank(slot, r), mc, m2c);
-            }
-            cluster_sync();
-            float mean = 0.f;
-            for (int r = 0; r < nr; ++r) mean += xchg[r * 128 + row].x;
-            mean /= (float)nr;
-            float m2 = 0.f;
-            for (int r = 0; r < nr; ++r) {
-                const float2 e = xchg[r * 128 + row];
-                m2 += e.y + (float)kTV * (e.x - mean) * (e.x - mean);
-            }
-            const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
-            const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
-            __syncthreads();                           // the scratch in the V tile is read
-            float y[32];
+                            for (int q = 0; q < 4; ++q)
+                                gv[q] = *reinterpret_cast<const uint4 *>(G + grow + 32 * half + 8 * q);
+                        } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t *u = reinterpret_cast<const uint32_t *>(&gv[q]);
+                            for (int q = 0; q < 4; ++q) gv[q] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        float x[32];
+                        ld_o(half, x);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 g2 = unpack_bf16(u[e]);
-                    const int i = 8 * q + 2 * e;
-                    y[i] = swish_fast(g2.x) * ((x[i] - mean) * scale);
-                    y[i + 1] = swish_fast(g2.y) * ((x[i + 1] - mean) * scale);
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t *u = reinterpret_cast<const uint32_t *>(&gv[q]);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 g2 = unpack_bf16(u[e]);
+                                const int i = 8 * q + 2 * e;
+                                x[i] = swish_fast(g2.x) * ((x[i] - mean) * scale);
+                                x[i + 1] = swish_fast(g2.y) * ((x[i + 1] - mean) * scale);
+                            }
+                        }
+                        if constexpr (kStage)
+                            stage32(half, x);
+                        else if (row < n)
+                            st_row32<TO>(Y + grow + 32 * half, x);
+                    }
+                    if constexpr (kStage) store_tile(&tmY, h * dv + v0, t0, b);
+                    if (O) emit_o();
                 }
             }
-            if constexpr (kStage) {
-                if (alive) stage_store(y, &tmY, h * dv + v0, t0, b);
-                if (alive && O) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) y[i] = x[i] * alpha;
-                    stage_store(y, &tmO, v0, t0, bh);
-                }
-            } else if (alive && row < n) {
-                st_row32<TO>(Y + grow, y);
-                if (O) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) y[i] = x[i] * alpha;
-                    st_row32<TO>(O + orow, y);
-                }
+            if (alive && g_leader && !last) {
+                load_v(c + 1);  // V is no longer read
+                wait_bar(bar(BK), par ^ 1, abort_flag, status);
             }
-            if (alive && tid == 0 && !last) load_v(c + 1);
+            alive = gsync_alive();
+            if (alive && !last) prep_k(c + 1, n_next);
         }
-
-        // ---- next chunk's K~
-        if (alive && !last && tid == 0) wait_bar(bar(BK), par ^ 1, abort_flag, status);
-        alive = sync_alive();
-        if (alive && !last) prep_k(n_next);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        alive = *abort_flag == 0;
     }
 
-    if (tid == 0) bulk_wait_all();       // output stores in flight
+    if (tid == 0 || tid == kGroup) bulk_wait_all();  // output stores in flight
     if constexpr (FUSE) cluster_sync();  // peers may still write into this CTA's smem before it
     // After an abort, copies and MMAs still in flight get a bounded time to
     // land before the shared and tensor memory are released.
