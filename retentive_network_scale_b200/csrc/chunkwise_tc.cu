@@ -61,7 +61,7 @@ constexpr int kMaxCluster = kMaxDv / kTV;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 constexpr float kMinLog2GammaTimesC = -60.f;        // gamma^C >= 2^-60
 
-enum { BQ = 0, BK, BV, BS, BU, BPV, kNumBars };
+enum { BQ = 0, BK, BV, BS, BU, BPV, BG, kNumBars };
 
 template <int DK>
 struct Layout {
@@ -78,12 +78,10 @@ struct Layout {
     static constexpr uint32_t kBar = kSmall;             // kNumBars mbarriers
     static constexpr uint32_t kTmemSlot = kSmall + 64;
     static constexpr uint32_t kAbort = kSmall + 68;
-    static constexpr uint32_t kBytes = kSmall + 128;
-    // GroupNorm scratch inside the V tile, which is dead between the P V'
-    // product and the next V load.
-    static constexpr uint32_t kGnPart = kV;              // [2 warpgroups][128] row sums
-    static constexpr uint32_t kGnPart2 = kV + 1024;      // [2 warpgroups][128] centred squares
-    static constexpr uint32_t kGnXchg = kV + 2048;       // [cluster rank][128] (mean, M2)
+    // GroupNorm: this CTA's per-row (mean, centred sum of squares) of its
+    // 128 columns, double-buffered by chunk parity; peers read it remotely.
+    static constexpr uint32_t kGnOwn = kSmall + 128;     // [2][128] float2
+    static constexpr uint32_t kBytes = kGnOwn + 2 * 128 * 8;
     static __device__ __forceinline__ uint32_t k_blk(int kb) { return kKR + kb * 32768; }
     static __device__ __forceinline__ uint32_t rbar_blk(int kb) { return kKR + kb * 32768 + 16384; }
 };
@@ -169,14 +167,14 @@ template <int DK, typename TO, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    const __grid_constant__ CUtensorMap tmY, const Params p,
+                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmG,
+                    const Params p,
                     const float *__restrict__ state_in, float *__restrict__ state_out,
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, TO *__restrict__ Y,
                     float gn_eps, int *status) {
     using Ly = Layout<DK>;
     constexpr int KB = DK / 64;         // 64-column blocks of Q^, K~, Rbar^T
     constexpr int NCH = DK / 8;         // 16-byte chunks per Q/K row
-    constexpr int RSG = kGroup / NCH;   // rows one group turns in parallel
     constexpr int RGA = DK / 64;        // 32-column groups per thread in the state pass (group A)
     constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V^T K~ (both MN-major)
     constexpr bool kStage = sizeof(TO) == 2;  // bf16 tiles leave by TMA store
@@ -211,8 +209,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tmem_alloc(sbase + Ly::kTmemSlot, 512);
         tmem_relinquish();
     }
-    // rotation (per group): column chunk and first row of this thread
-    const int rc16 = gtid % NCH, rr0 = gtid / NCH;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -246,45 +242,79 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     };
     const bool g_leader = gtid == 0;   // waits on mbarriers for its group
 
-    // this thread's share of turning the tile at blk0 (rows r0, r0+RSG, ...);
-    // rows scaled by gamma^{n-1-r} when `zeta` is set (K~)
-    auto rotate = [&](uint32_t blk0, uint32_t blk_stride, int c, int n, bool zeta) {
-        float cc[4], sn[4], rsc[4], rss[4];
+    // Turn (and for K~ scale by gamma^{n-1-r}) rows of the tile at blk0 with
+    // `nthr` threads, this one being `ti`: thread -> 16-byte column chunk
+    // (4 pairs) and the rows r0, r0+RS, r0+2RS, ... taken two at a time, the
+    // two rows in the lanes of packed fp32 pairs.  Angles start exact (fp64
+    // reduction) and advance by 2*RS*theta_j per step.
+    auto rotate = [&](uint32_t blk0, uint32_t blk_stride, int c, int n, bool zeta, int ti, int nthr) {
+        const int RS = nthr / NCH;
+        const int c16 = ti % NCH, r0 = ti / NCH;
+        const int blk = c16 >> 3, cw = c16 & 7;
+        uint8_t *base = smem + blk0 + blk * blk_stride;
+        uint64_t C[4], NS[4], c2[4], s2[4], ns2[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const double th = p.theta[rc16 * 4 + e];
-            rot_cs_fast(p.pos_offset + (long long)c * kC + rr0, th, &cc[e], &sn[e]);
-            rot_cs_fast(RSG, th, &rsc[e], &rss[e]);
+            const double th = p.theta[c16 * 4 + e];
+            float ca, sa, cb, sb, cs, ss;
+            rot_cs_fast(p.pos_offset + (long long)c * kC + r0, th, &ca, &sa);
+            rot_cs_fast(p.pos_offset + (long long)c * kC + r0 + RS, th, &cb, &sb);
+            rot_cs_fast(2 * RS, th, &cs, &ss);
+            C[e] = f2_make(ca, cb);
+            NS[e] = f2_make(-sa, -sb);
+            c2[e] = f2_make(cs, cs);
+            s2[e] = f2_make(ss, ss);
+            ns2[e] = f2_make(-ss, -ss);
         }
-        const int blk = rc16 >> 3, cw = rc16 & 7;
-        uint8_t *base = smem + blk0 + blk * blk_stride;
-#pragma unroll 4
-        for (int r = rr0; r < n; r += RSG) {
-            const float z = zeta ? decay_pow(lg, n - 1 - r) : 1.f;
-            uint4 *ptr = reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4));
-            uint4 w = *ptr;
-            uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+        // two row pairs per step: all four rows are loaded before any is written
+        auto turn_pair = [&](uint4 &wa, uint4 &wb, int ra, int rb) {
+            const float za = zeta ? (ra < n ? decay_pow(lg, n - 1 - ra) : 0.f) : 1.f;
+            const float zb = zeta ? (rb < n ? decay_pow(lg, n - 1 - rb) : 0.f) : 1.f;
+            const uint64_t Z = f2_make(za, zb);
+            uint32_t *ua = reinterpret_cast<uint32_t *>(&wa);
+            uint32_t *ub = reinterpret_cast<uint32_t *>(&wb);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 x = unpack_bf16(u[e]);
-                const float zc = z * cc[e], zs = z * sn[e];
-                u[e] = pack_bf16(x.x * zc - x.y * zs, x.x * zs + x.y * zc);
-                const float cn = cc[e] * rsc[e] - sn[e] * rss[e];
-                sn[e] = cc[e] * rss[e] + sn[e] * rsc[e];
-                cc[e] = cn;
+                // x0 = low bf16, x1 = high bf16 of each row's pair
+                const uint64_t X0 = (static_cast<uint64_t>(ub[e] << 16) << 32) | (ua[e] << 16);
+                const uint64_t X1 = (static_cast<uint64_t>(ub[e] & 0xffff0000u) << 32) | (ua[e] & 0xffff0000u);
+                const uint64_t NX0 = X0 ^ 0x8000000080000000ull;
+                const uint64_t ZC = zeta ? f2_mul(C[e], Z) : C[e];
+                const uint64_t ZNS = zeta ? f2_mul(NS[e], Z) : NS[e];
+                const uint64_t Y0 = f2_fma(X1, ZNS, f2_mul(X0, ZC));   // x0 c - x1 s
+                const uint64_t Y1 = f2_fma(X1, ZC, f2_mul(NX0, ZNS));  // x0 s + x1 c
+                ua[e] = pack_bf16(f2_lo(Y0), f2_lo(Y1));
+                ub[e] = pack_bf16(f2_hi(Y0), f2_hi(Y1));
+                const uint64_t Cn = f2_fma(C[e], c2[e], f2_mul(NS[e], s2[e]));
+                NS[e] = f2_fma(NS[e], c2[e], f2_mul(C[e], ns2[e]));
+                C[e] = Cn;
             }
-            *ptr = w;
+        };
+        auto at = [&](int r) { return reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4)); };
+        // rows r0 + RS*k, k = 0..128/RS-1 (a multiple of 4); rows at or past n
+        // are zeros from the load and are left as they are
+#pragma unroll 1
+        for (int ra = r0; ra < n; ra += 4 * RS) {
+            const int rb = ra + RS, rc = ra + 2 * RS, rd = ra + 3 * RS;
+            uint4 wa = *at(ra), wb = *at(rb), wc = *at(rc), wd = *at(rd);
+            turn_pair(wa, wb, ra, rb);
+            turn_pair(wc, wd, rc, rd);
+            *at(ra) = wa;
+            *at(rb) = wb;
+            *at(rc) = wc;
+            *at(rd) = wd;
         }
     };
-    // K~ = diag(zeta) K^ without rotation (this group's share)
-    auto scale_k = [&](int n) {
-        const float zeta = row < n ? decay_pow(lg, n - 1 - row) : 0.f;
+    // K~ = diag(zeta) K^ without rotation, `nthr` threads, this one `ti`
+    auto scale_k = [&](int n, int ti, int nthr) {
+        const int r = ti & 127;
+        const float zeta = r < n ? decay_pow(lg, n - 1 - r) : 0.f;
 #pragma unroll 1
-        for (int kb = gwg; kb < KB; kb += 2) {
-            uint8_t *krow = smem + Ly::k_blk(kb) + row * 128;
+        for (int kb = ti >> 7; kb < KB; kb += nthr >> 7) {
+            uint8_t *krow = smem + Ly::k_blk(kb) + r * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(krow + (((q + row) & 7) << 4));
+                uint4 *ptr = reinterpret_cast<uint4 *>(krow + (((q + r) & 7) << 4));
                 uint4 w = *ptr;
                 uint32_t *u = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
@@ -296,14 +326,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
         }
     };
-    auto prep_q = [&](int c, int n) {
-        if (p.rotate) rotate(Ly::kQ, 16384, c, n, false);
+    auto prep_q = [&](int c, int n, int ti, int nthr) {
+        if (p.rotate) rotate(Ly::kQ, 16384, c, n, false, ti, nthr);
     };
-    auto prep_k = [&](int c, int n) {
+    auto prep_k = [&](int c, int n, int ti, int nthr) {
         if (p.rotate)
-            rotate(Ly::kKR, 32768, c, n, true);
+            rotate(Ly::kKR, 32768, c, n, true, ti, nthr);
         else
-            scale_k(n);
+            scale_k(n, ti, nthr);
     };
     // MMA descriptors: fixed buffers, so only the start address moves
     const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);          // A of [S|O''], K-major
@@ -348,9 +378,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         alive = gsync_alive();
         if (alive) {
             if (grp == 0)
-                prep_q(0, n0);
+                prep_q(0, n0, gtid, kGroup);
             else
-                prep_k(0, n0);
+                prep_k(0, n0, gtid, kGroup);
         }
     }
     fence_proxy_async_smem();
@@ -366,7 +396,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const bool last = c + 1 == nchunks;
         const int n_next = last ? 0 : min(kC, L - t0 - kC);
 
-        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T  (thread 0)
+        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T, then R^T += V^T K~ (thread 0;
+        // S first, so that the P pass overlaps the state update)
         if (alive && tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -376,11 +407,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 mma_ss(tS, dQ + off, dKR + offkr, kIdescSX, ks > 0);
             }
             mma_commit(bar(BS));
-        }
-        // ---- R^T += V^T K~ as soon as V is in (thread 32; no data shared with
-        // the products thread 0 issues, so the two need no ordering)
-        if (alive && tid == 32) {
-            tc_fence_after();
             if (wait_bar(bar(BV), par, abort_flag, status)) {
 #pragma unroll
                 for (int ks = 0; ks < kC / 16; ++ks) {
@@ -428,7 +454,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         if (grp == 0) {
             // ================= group A: state pass, then the next Q^
-            if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier 1
+            if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier
             if (alive && g_leader) {
                 wait_bar(bar(BU), par, abort_flag, status);
                 if (!last) load_k(c + 1);  // K~ is no longer read
@@ -467,13 +493,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 tmem_wait_st();
             }
-            if constexpr (FUSE) {
-                cluster_wait();
-                cluster_arrive();                   // GroupNorm exchange barrier 2
-            }
             if (alive && !last && g_leader) wait_bar(bar(BQ), par ^ 1, abort_flag, status);
             alive = gsync_alive();
-            if (alive && !last) prep_q(c + 1, n_next);
+            if (alive && !last) prep_q(c + 1, n_next, gtid, kGroup);
             if constexpr (FUSE) cluster_wait();
         } else {
             // ================= group B: output, then the next V and K~
@@ -535,15 +557,29 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (alive) emit_o();
             } else {
                 const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
-                const uint32_t rank = cluster_rank();
                 const int b = bh / p.H;
                 const size_t grow =
                     ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
-                float *part = reinterpret_cast<float *>(smem + Ly::kGnPart);    // [2][128] sums
-                float *part2 = reinterpret_cast<float *>(smem + Ly::kGnPart2);  // [2][128] squares
-                const float2 *xchg = reinterpret_cast<const float2 *>(smem + Ly::kGnXchg);
-                // CTA-local mean and centred sum of squares of the row's 128
-                // columns (two warpgroups hold 64 each)
+                // the G tile comes by TMA into the V tile, dead since P V
+                if (alive && g_leader) {
+                    mbar_expect_tx(bar(BG), Ly::kVBytes);
+                    for (int nb = 0; nb < 2; ++nb)
+                        tma_load_3d(sbase + Ly::kV + nb * 16384, &tmG, bar(BG), h * dv + v0 + nb * 64, t0, b);
+                }
+                // row sum over the 128 columns of this CTA: the two warpgroups
+                // of the group meet in free tensor-memory columns (lane = row)
+                const uint32_t scratch = tS + lane_base;
+                auto combine2 = [&](float mine, int col) {
+                    tmem_st1(scratch + col + gwg, __float_as_uint(mine));
+                    tmem_wait_st();
+                    tc_fence_before();
+                    named_sync(2, kGroup);
+                    tc_fence_after();
+                    uint32_t u0, u1;
+                    tmem_ld2(scratch + col, u0, u1);
+                    tmem_wait_ld();
+                    return __uint_as_float(u0) + __uint_as_float(u1);
+                };
                 float s = 0.f;
                 if (alive) {
 #pragma unroll 1
@@ -554,9 +590,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         for (int i = 0; i < 32; ++i) s += x[i];
                     }
                 }
-                part[gwg * 128 + row] = s;
-                named_sync(2, kGroup);
-                const float mc = (part[row] + part[128 + row]) * (1.f / kTV);
+                const float mc = combine2(s, 0) * (1.f / kTV);
                 float q2 = 0.f;
                 if (alive) {
 #pragma unroll 1
@@ -567,46 +601,44 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         for (int i = 0; i < 32; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
                     }
                 }
-                part2[gwg * 128 + row] = q2;
-                // barrier 1: every CTA of the head is past its P V product, so
-                // their V tiles are free; the partials here are visible.
+                const float m2c = combine2(q2, 2);
+                // publish (mean, M2) of this CTA's columns; the peers read it
+                // after the cluster barrier (double buffer: a peer is never
+                // more than one chunk behind, the barrier sees to that)
+                const uint32_t own = sbase + Ly::kGnOwn + (par * 128 + row) * 8;
+                if (gwg == 0) *reinterpret_cast<float2 *>(smem + Ly::kGnOwn + (par * 128 + row) * 8) = make_float2(mc, m2c);
                 cluster_arrive();
                 cluster_wait();
-                if (alive && gwg == 0) {
-                    const float m2c = part2[row] + part2[128 + row];
-                    const uint32_t slot = sbase + Ly::kGnXchg + (rank * 128 + row) * 8;
-                    for (int r = 0; r < nr; ++r) st_cluster_f32x2(map_to_rank(slot, r), mc, m2c);
-                }
-                cluster_arrive();                    // barrier 2: exchange written
-                cluster_wait();
-                float mean = 0.f;
-                for (int r = 0; r < nr; ++r) mean += xchg[r * 128 + row].x;
-                mean /= (float)nr;
-                float m2 = 0.f;
-                for (int r = 0; r < nr; ++r) {
-                    const float2 e = xchg[r * 128 + row];
-                    m2 += e.y + (float)kTV * (e.x - mean) * (e.x - mean);
+                float mean = 0.f, m2 = 0.f;
+                {
+                    float2 e[kMaxCluster];
+#pragma unroll
+                    for (int r = 0; r < kMaxCluster; ++r)
+                        if (r < nr) e[r] = ld_cluster_f32x2(map_to_rank(own, r));
+#pragma unroll
+                    for (int r = 0; r < kMaxCluster; ++r)
+                        if (r < nr) mean += e[r].x;
+                    mean /= (float)nr;
+#pragma unroll
+                    for (int r = 0; r < kMaxCluster; ++r)
+                        if (r < nr) m2 += e[r].y + (float)kTV * (e[r].x - mean) * (e[r].x - mean);
                 }
                 const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
                 const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
-                named_sync(2, kGroup);                    // the scratch in the V tile is read
+                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
+                alive = gsync_alive();
                 if (alive) {
+                    // Y in place of G in the V tile (same thread, same bytes)
+                    uint8_t *tile = smem + Ly::kV + gwg * 16384 + row * 128;
 #pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
-                        uint4 gv[4];
-                        if (row < n) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                gv[q] = *reinterpret_cast<const uint4 *>(G + grow + 32 * half + 8 * q);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) gv[q] = make_uint4(0u, 0u, 0u, 0u);
-                        }
                         float x[32];
                         ld_o(half, x);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const uint32_t *u = reinterpret_cast<const uint32_t *>(&gv[q]);
+                            uint4 *ptr = reinterpret_cast<uint4 *>(tile + (((4 * half + q) ^ (row & 7)) << 4));
+                            uint4 gw = *ptr;
+                            uint32_t *u = reinterpret_cast<uint32_t *>(&gw);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const float2 g2 = unpack_bf16(u[e]);
@@ -614,11 +646,16 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                                 x[i] = swish_fast(g2.x) * ((x[i] - mean) * scale);
                                 x[i + 1] = swish_fast(g2.y) * ((x[i + 1] - mean) * scale);
                             }
+                            if constexpr (kStage) {
+                                u[0] = pack_bf16(x[8 * q + 0], x[8 * q + 1]);
+                                u[1] = pack_bf16(x[8 * q + 2], x[8 * q + 3]);
+                                u[2] = pack_bf16(x[8 * q + 4], x[8 * q + 5]);
+                                u[3] = pack_bf16(x[8 * q + 6], x[8 * q + 7]);
+                                *ptr = gw;
+                            }
                         }
-                        if constexpr (kStage)
-                            stage32(half, x);
-                        else if (row < n)
-                            st_row32<TO>(Y + grow + 32 * half, x);
+                        if constexpr (!kStage)
+                            if (row < n) st_row32<TO>(Y + grow + 32 * half, x);
                     }
                     if constexpr (kStage) store_tile(&tmY, h * dv + v0, t0, b);
                     if (O) emit_o();
@@ -629,7 +666,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 wait_bar(bar(BK), par ^ 1, abort_flag, status);
             }
             alive = gsync_alive();
-            if (alive && !last) prep_k(c + 1, n_next);
+            if (alive && !last) prep_k(c + 1, n_next, gtid, kGroup);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -689,13 +726,15 @@ template <int DK, typename TO, bool FUSE>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                      const void *G, void *Y, float eps, int *status, cudaStream_t st) {
-    CUtensorMap mo, my;
+    CUtensorMap mo, my, mg;
     std::memset(&mo, 0, sizeof(mo));
     std::memset(&my, 0, sizeof(my));
+    std::memset(&mg, 0, sizeof(mg));
     if (sizeof(TO) == 2) {
         if (O && !make_map(&mo, O, p.dv, p.L, p.B * p.H)) return cudaErrorInvalidValue;
         if (Y && !make_map(&my, Y, p.H * p.dv, p.L, p.B)) return cudaErrorInvalidValue;
     }
+    if (G && !make_map(&mg, G, p.H * p.dv, p.L, p.B)) return cudaErrorInvalidValue;
     auto kern = chunkwise_tc_kernel<DK, TO, FUSE>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -712,7 +751,7 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, my, p, s_in, s_out, (TO *)O,
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, my, mg, p, s_in, s_out, (TO *)O,
                            (const __nv_bfloat16 *)G, (TO *)Y, eps, status);
     if (e == cudaSuccess) note_launches(1);
     return e;
