@@ -82,10 +82,19 @@ typedef struct {
  *     Retention(X) = (Q K^T (.) D) V,  D_nm = gamma^{n-m} (n >= m), else 0,
  * with Q, K rotated as above.  Q, K, V: device, in_dtype.  O: device,
  * out_dtype, fully overwritten.  No state in or out.
- * Errors: RET_ERR_NULL, _SHAPE, _DTYPE, _ALIGN, _ARG, _UNSUPPORTED, _CUDA.
+ *   workspace  device scratch of workspace_bytes; required only when
+ *              ret_parallel_workspace_size() returns a non-zero size (it
+ *              then receives the rotated Q and K in bf16).
+ * Errors: RET_ERR_NULL, _SHAPE, _DTYPE, _ALIGN, _ARG, _WORKSPACE,
+ * _UNSUPPORTED, _CUDA.
  */
 ret_status ret_parallel(const ret_desc *desc, const void *Q, const void *K,
-                        const void *V, void *O, void *stream);
+                        const void *V, void *O, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace ret_parallel needs for this description (0 when none).
+ * Never fails (0 for descriptions ret_parallel would reject). */
+size_t ret_parallel_workspace_size(const ret_desc *desc);
 
 /*
  * ret_chunkwise -- the chunkwise recurrent representation (section 2.1,

@@ -100,19 +100,35 @@ const char *ret_status_string(ret_status s) {
     return "unknown status";
 }
 
+size_t ret_parallel_workspace_size(const ret_desc *desc) {
+    if (check_desc(desc) != RET_OK) return 0;
+    Params p;
+    make_params(desc, &p);
+    return parallel_tc_supported(p, desc->in_dtype == RET_BF16) ? parallel_tc_workspace(p) : 0;
+}
+
 ret_status ret_parallel(const ret_desc *desc, const void *Q, const void *K, const void *V,
-                        void *O, void *stream) {
+                        void *O, void *workspace, size_t workspace_bytes, void *stream) {
     ret_status s = check_desc(desc);
     if (s != RET_OK) return s;
     const bool empty = (long long)desc->B * desc->L == 0;
     if (!empty && (!Q || !K || !V || !O)) return RET_ERR_NULL;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return RET_ERR_ALIGN;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
+        return RET_ERR_ALIGN;
+    const size_t need = empty ? 0 : ret_parallel_workspace_size(desc);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return RET_ERR_WORKSPACE;
     if ((s = check_device()) != RET_OK) return s;
     if (empty) return RET_OK;
     Params p;
     make_params(desc, &p);
-    return from_cuda(launch_parallel_simt(p, desc->in_dtype == RET_BF16, desc->out_dtype == RET_BF16,
-                                          Q, K, V, O, (cudaStream_t)stream));
+    const bool in_bf16 = desc->in_dtype == RET_BF16, out_bf16 = desc->out_dtype == RET_BF16;
+    if (parallel_tc_supported(p, in_bf16)) {
+        int *status = device_status_word();
+        if (!status) return RET_ERR_CUDA;
+        return from_cuda(launch_parallel_tc(p, out_bf16, Q, K, V, O, workspace, status,
+                                            (cudaStream_t)stream));
+    }
+    return from_cuda(launch_parallel_simt(p, in_bf16, out_bf16, Q, K, V, O, (cudaStream_t)stream));
 }
 
 size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_Y) {

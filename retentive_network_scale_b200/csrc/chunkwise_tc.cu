@@ -691,37 +691,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = [] {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return static_cast<EncodeTiledFn>(nullptr);
-        return reinterpret_cast<EncodeTiledFn>(f);
-    }();
-    return fn;
-}
-
-// [bh][rows][inner] bf16, boxes of 64 x 128 x 1 with 128-byte swizzle; rows
-// past the end of a (b,h) slice read as zeros.
-bool make_map(CUtensorMap *m, const void *base, int inner, int rows, int bh) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)bh};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)rows * inner * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kC, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int DK, typename TO, bool FUSE>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
@@ -731,10 +700,10 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     std::memset(&my, 0, sizeof(my));
     std::memset(&mg, 0, sizeof(mg));
     if (sizeof(TO) == 2) {
-        if (O && !make_map(&mo, O, p.dv, p.L, p.B * p.H)) return cudaErrorInvalidValue;
-        if (Y && !make_map(&my, Y, p.H * p.dv, p.L, p.B)) return cudaErrorInvalidValue;
+        if (O && !make_tma_map_bf16(&mo, O, p.dv, p.L, p.B * p.H, kC)) return cudaErrorInvalidValue;
+        if (Y && !make_tma_map_bf16(&my, Y, p.H * p.dv, p.L, p.B, kC)) return cudaErrorInvalidValue;
     }
-    if (G && !make_map(&mg, G, p.H * p.dv, p.L, p.B)) return cudaErrorInvalidValue;
+    if (G && !make_tma_map_bf16(&mg, G, p.H * p.dv, p.L, p.B, kC)) return cudaErrorInvalidValue;
     auto kern = chunkwise_tc_kernel<DK, TO, FUSE>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -785,8 +754,8 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
                                 const void *G, void *Y, float eps, int *status, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
-    if (!make_map(&mq, Q, p.dk, p.L, bh) || !make_map(&mk, K, p.dk, p.L, bh) ||
-        !make_map(&mv, V, p.dv, p.L, bh))
+    if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC) ||
+        !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kC))
         return cudaErrorInvalidValue;
     if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);
     return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);

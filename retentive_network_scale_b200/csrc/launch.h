@@ -1,6 +1,7 @@
 // launch.h -- internal launchers behind the C ABI (not exported).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -27,6 +28,19 @@ bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16);
 cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
                                 const void *V, const float *s_in, float *s_out, void *O,
                                 const void *G, void *Y, float eps, int *status, cudaStream_t st);
+
+// Tensor map over [outer][rows][inner] bf16 with boxes of 64 x box_rows x 1
+// and 128-byte swizzle; rows past the end read as zeros and are not written.
+bool make_tma_map_bf16(CUtensorMap *m, const void *base, int inner, int rows, int outer, int box_rows);
+
+// Tensor-core parallel form: bf16 inputs, d_k 128 or 256, d_v a multiple of
+// 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
+// Q^ and K^ (bf16) into the workspace (parallel_tc_workspace bytes).
+bool parallel_tc_supported(const Params &p, bool in_bf16);
+size_t parallel_tc_workspace(const Params &p);
+cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
+                               const void *V, void *O, void *workspace, int *status,
+                               cudaStream_t st);
 
 // Address of the device status word bounded waits latch errors into.
 int *device_status_word();

@@ -1,0 +1,379 @@
+// parallel_tc.cu -- the parallel form of retention on the sm_100a tensor
+// cores ("Retentive Network" paper summary, section 2.1, form (1)):
+//     O = (Q^ K^^T (.) D) V,   D_nm = gamma^{n-m} for n >= m, else 0.
+//
+// Flash-style: one CTA owns a 128-row query tile, a slice of V columns
+// (TV = 256, or 128 when d_v is not a multiple of 256) and one (b,h).  It
+// walks the key tiles from the diagonal down:
+//     S = Q^ K^_k^T            (tcgen05, fp32 in tensor memory)
+//     P = S (.) D_tile         (CUDA cores: the decay as the rank-1 product
+//                               gamma^{Delta+j} gamma^{-j'}, Delta = q0 - k0,
+//                               and the causal mask on the diagonal tile;
+//                               bf16 back into tensor memory)
+//     O += P V_k               (tcgen05, A operand from tensor memory)
+// Key tiles whose largest weight gamma^{Delta-127} is below 2^-150 add
+// nothing representable in fp32; the walk stops there.  K and V loads for
+// the next key tile are issued as soon as the MMAs reading the current one
+// finish.  The output tile leaves through shared memory and TMA stores.
+//
+// The rotation (xPos) is applied once per row by xpos_rotate_kernel into a
+// workspace before this kernel runs: every key tile is read by many query
+// tiles, so turning it inside would repeat the work per tile pair.
+#include <cuda.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc_util.cuh"
+
+namespace ret {
+namespace {
+
+using namespace tc;
+
+constexpr int kT = 128;         // query / key tile rows
+constexpr int kThreads = 256;   // two warpgroups
+constexpr long long kTimeoutCycles = 4000000000LL;
+constexpr float kMinLog2GammaTimesT = -60.f;  // gamma^-127 stays below 2^60
+
+enum { BQ = 0, BK, BV, BS, BPV, kNumBars };
+
+template <int DK, int TV>
+struct PLayout {
+    static constexpr uint32_t kQ = 0;                     // Q^: DK/64 blocks of 16 KB
+    static constexpr uint32_t kQBytes = kT * DK * 2;
+    static constexpr uint32_t kK = kQ + kQBytes;          // K^_k
+    static constexpr uint32_t kV = kK + kQBytes;          // V_k: TV/64 blocks of 16 KB
+    static constexpr uint32_t kVBytes = kT * TV * 2;
+    static constexpr uint32_t kSmall = kV + kVBytes;
+    static constexpr uint32_t kBar = kSmall;
+    static constexpr uint32_t kTmemSlot = kSmall + 64;
+    static constexpr uint32_t kAbort = kSmall + 68;
+    static constexpr uint32_t kColScale = kSmall + 128;   // gamma^{-j'}, 128 floats
+    static constexpr uint32_t kBytes = kColScale + 512;
+};
+
+__device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                      int *status) {
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - start > kTimeoutCycles) {
+            *abort_flag = 1;
+            atomicExch(status, (int)RET_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t pk_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int DK, int TV, typename TO>
+__global__ void __launch_bounds__(kThreads, 1)
+parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Params p, TO *__restrict__ O, int *status) {
+    using Ly = PLayout<DK, TV>;
+    constexpr int KB = DK / 64, VB = TV / 64;
+    constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);  // Q^ x K^ (both K-major)
+    constexpr uint32_t kIdescPV = idesc_bf16(128, TV, 0, 1);  // P (tmem) x V (MN-major)
+    constexpr bool kStage = sizeof(TO) == 2;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+    const int nqt = (p.L + kT - 1) / kT;
+    const int qt = nqt - 1 - (int)blockIdx.x;  // long rows of tiles first
+    const int v0 = blockIdx.y * TV, bh = blockIdx.z, h = bh % p.H;
+    const int q0 = qt * kT;
+    const float lg = p.log2g[h];
+
+    if (sbase & 1023u) {
+        if (tid == 0) atomicExch(status, (int)RET_ERR_CUDA);
+        return;
+    }
+    auto bar = [&](int i) { return sbase + Ly::kBar + 8u * i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::kAbort);
+    float *colscale = reinterpret_cast<float *>(smem + Ly::kColScale);
+    if (tid == 0) {
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) {
+        tmem_alloc(sbase + Ly::kTmemSlot, 512);
+        tmem_relinquish();
+    }
+    if (tid < kT) colscale[tid] = exp2f(-(float)tid * lg);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + Ly::kTmemSlot);
+    const uint32_t tO = tmem, tS = tmem + 256;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+
+    // last key tile with a representable weight: gamma^{Delta-127} >= 2^-150
+    int kt_min = 0;
+    if (lg < 0.f) {
+        const int far = (int)floorf(-150.f / lg) + 127;  // largest Delta still kept
+        kt_min = max(0, qt - far / kT);
+    }
+    auto load_k = [&](int kt) {
+        mbar_expect_tx(bar(BK), Ly::kQBytes);
+        for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(sbase + Ly::kK + kb * 16384, &tmK, bar(BK), kb * 64, kt * kT, bh);
+    };
+    auto load_v = [&](int kt) {
+        mbar_expect_tx(bar(BV), Ly::kVBytes);
+        for (int nb = 0; nb < VB; ++nb)
+            tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, kt * kT, bh);
+    };
+    auto sync_alive = [&]() {
+        __syncthreads();
+        return *abort_flag == 0;
+    };
+    const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);
+    const uint64_t dK = sdesc_sw128(sbase + Ly::kK, 16, 1024);
+    const uint64_t dV = sdesc_sw128(sbase + Ly::kV, 16384, 1024);
+
+    if (tid == 0) {
+        mbar_expect_tx(bar(BQ), Ly::kQBytes);
+        for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQ), kb * 64, q0, bh);
+        load_k(qt);
+        load_v(qt);
+    }
+    bool alive = true;
+    int it = 0;
+#pragma unroll 1
+    for (int kt = qt; kt >= kt_min; --kt, ++it) {
+        const uint32_t par = it & 1;
+        const int delta = q0 - kt * kT;
+        // ---- S = Q^ K^_k^T
+        if (alive && tid == 0) {
+            if (it == 0) pwait(bar(BQ), 0, abort_flag, status);
+            if (pwait(bar(BK), par, abort_flag, status)) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                    mma_ss(tS, dQ + off, dK + off, kIdescS, ks > 0);
+                }
+            }
+            mma_commit(bar(BS));
+            if (pwait(bar(BS), par, abort_flag, status) && kt > kt_min) load_k(kt - 1);
+        }
+        alive = sync_alive();
+        tc_fence_after();
+        // ---- P = S (.) D into tensor memory; warpgroup w owns keys [64w, 64w+64)
+        if (alive) {
+            const int k0 = wg * 64;
+            uint32_t a[32], b[32], pk[32];
+            tmem_ld32(tS + lane_base + k0, a);
+            tmem_ld32(tS + lane_base + k0 + 32, b);
+            tmem_wait_ld();
+            const float aj = exp2f((float)(delta + row) * lg);  // gamma^{Delta + j}
+            const bool diag = delta == 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int j0 = k0 + 2 * i, j1 = k0 + 32 + 2 * i;
+                const float w00 = (diag && j0 > row) ? 0.f : aj * colscale[j0];
+                const float w01 = (diag && j0 + 1 > row) ? 0.f : aj * colscale[j0 + 1];
+                const float w10 = (diag && j1 > row) ? 0.f : aj * colscale[j1];
+                const float w11 = (diag && j1 + 1 > row) ? 0.f : aj * colscale[j1 + 1];
+                pk[i] = pk_bf16(__uint_as_float(a[2 * i]) * w00, __uint_as_float(a[2 * i + 1]) * w01);
+                pk[16 + i] = pk_bf16(__uint_as_float(b[2 * i]) * w10, __uint_as_float(b[2 * i + 1]) * w11);
+            }
+            // keys [64w, 64w+64) -> columns [64w, 64w+32) of the S region
+            tmem_st32(tS + lane_base + k0, pk);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        // ---- O += P V_k
+        if (alive && tid == 0) {
+            if (pwait(bar(BV), par, abort_flag, status)) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kT / 16; ++ks)
+                    mma_ts(tO, tS + (ks >> 2) * 64 + (ks & 3) * 8, dV + (uint64_t)((ks * 2048) >> 4),
+                           kIdescPV, (ks > 0 || it > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(BPV));
+            if (pwait(bar(BPV), par, abort_flag, status) && kt > kt_min) load_v(kt - 1);
+        }
+        alive = sync_alive();
+    }
+    tc_fence_after();
+    // ---- O tile out: bf16 through shared memory and TMA stores
+    if (alive) {
+        const int c0 = wg * (TV / 2);  // each warpgroup: TV/2 columns of the row
+#pragma unroll 1
+        for (int g = 0; g < TV / 64; ++g) {
+            uint32_t a[32];
+            float x[32];
+            tmem_ld32(tO + lane_base + c0 + 32 * g, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
+            const int col = c0 + 32 * g;
+            if constexpr (kStage) {
+                uint8_t *dst = smem + Ly::kV + (col >> 6) * 16384 + row * 128;
+                const int ch0 = (col & 63) >> 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pk_bf16(x[8 * q + 0], x[8 * q + 1]);
+                    w.y = pk_bf16(x[8 * q + 2], x[8 * q + 3]);
+                    w.z = pk_bf16(x[8 * q + 4], x[8 * q + 5]);
+                    w.w = pk_bf16(x[8 * q + 6], x[8 * q + 7]);
+                    *reinterpret_cast<uint4 *>(dst + (((ch0 + q) ^ (row & 7)) << 4)) = w;
+                }
+            } else if (q0 + row < p.L) {
+                float *dst = reinterpret_cast<float *>(O) + ((size_t)bh * p.L + q0 + row) * p.dv + v0 + col;
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+            }
+        }
+        if constexpr (kStage) {
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                for (int nb = 0; nb < VB; ++nb)
+                    tma_store_3d(&tmO, sbase + Ly::kV + nb * 16384, v0 + nb * 64, q0, bh);
+                bulk_commit();
+                bulk_wait_all();
+            }
+        }
+    }
+    if (tid == 0 && *abort_flag) {
+        const long long start = clock64();
+        while (clock64() - start < 20000000LL) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// xPos turn of [rows][dk] rows (row r at position pos_offset + r % L) into
+// bf16.  Thread -> (16-byte output chunk = 4 pairs, block of 16 consecutive
+// rows); the angles start exact and advance by theta_j per row.
+template <typename TI>
+__global__ void __launch_bounds__(256)
+xpos_rotate_kernel(Params p, long long rows, const TI *__restrict__ x, __nv_bfloat16 *__restrict__ y) {
+    constexpr int kRowsPerThread = 16;
+    const int nch = p.dk / 8;
+    const long long items = (rows + kRowsPerThread - 1) / kRowsPerThread * nch;
+    for (long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x; item < items;
+         item += (long long)gridDim.x * blockDim.x) {
+        const int c16 = (int)(item % nch);
+        const long long r0 = item / nch * kRowsPerThread;
+        float c[4], s[4], sc[4], ss[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double th = p.theta[c16 * 4 + e];
+            rot_cs(p.pos_offset + r0 % p.L, th, &c[e], &s[e]);
+            rot_cs(1, th, &sc[e], &ss[e]);
+        }
+        for (int k = 0; k < kRowsPerThread && r0 + k < rows; ++k) {
+            const long long r = r0 + k;
+            if (k > 0 && r % p.L == 0) {  // a new (b,h) slice starts: restart the angles
+#pragma unroll
+                for (int e = 0; e < 4; ++e) rot_cs(p.pos_offset, p.theta[c16 * 4 + e], &c[e], &s[e]);
+            }
+            const size_t base = (size_t)r * p.dk + c16 * 8;
+            uint4 out;
+            uint32_t *u = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float x0 = ld(x, base + 2 * e), x1 = ld(x, base + 2 * e + 1);
+                u[e] = pk_bf16(x0 * c[e] - x1 * s[e], x0 * s[e] + x1 * c[e]);
+                const float cn = c[e] * sc[e] - s[e] * ss[e];
+                s[e] = c[e] * ss[e] + s[e] * sc[e];
+                c[e] = cn;
+            }
+            *reinterpret_cast<uint4 *>(y + base) = out;
+        }
+    }
+}
+
+template <int DK, int TV, typename TO>
+cudaError_t launch_ptc(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
+                       const CUtensorMap &mv, const CUtensorMap &mo, void *O, int *status,
+                       cudaStream_t st) {
+    auto kern = parallel_tc_kernel<DK, TV, TO>;
+    const int smem = (int)PLayout<DK, TV>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.L + kT - 1) / kT, p.dv / TV, p.B * p.H);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, p, (TO *)O, status);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) note_launches(1);
+    return e;
+}
+
+template <int DK, typename TO>
+cudaError_t launch_ptc_tv(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
+                          const CUtensorMap &mv, const CUtensorMap &mo, void *O, int *status,
+                          cudaStream_t st) {
+    if (p.dv % 256 == 0) return launch_ptc<DK, 256, TO>(p, mq, mk, mv, mo, O, status, st);
+    return launch_ptc<DK, 128, TO>(p, mq, mk, mv, mo, O, status, st);
+}
+
+}  // namespace
+
+bool parallel_tc_supported(const Params &p, bool in_bf16) {
+    if (!in_bf16 || (p.dk != 128 && p.dk != 256) || p.dv % 128 != 0 || p.L < 1 ||
+        (long long)p.B * p.H > 65535 || (p.L + kT - 1) / kT > 2147483647)
+        return false;
+    for (int h = 0; h < p.H; ++h)
+        if (!(p.log2g[h] * 127.f >= kMinLog2GammaTimesT)) return false;  // also rejects gamma = 0
+    return true;
+}
+
+size_t parallel_tc_workspace(const Params &p) {
+    return p.rotate ? (size_t)2 * p.B * p.H * p.L * p.dk * sizeof(__nv_bfloat16) : 0;
+}
+
+cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
+                               const void *V, void *O, void *workspace, int *status,
+                               cudaStream_t st) {
+    const long long rows = (long long)p.B * p.H * p.L;
+    if (p.rotate) {
+        // the turned Q^ and K^ in the workspace, then the products read them
+        __nv_bfloat16 *qr = static_cast<__nv_bfloat16 *>(workspace);
+        __nv_bfloat16 *kr = qr + (size_t)rows * p.dk;
+        const long long items = (rows + 15) / 16 * (p.dk / 8);
+        const int blocks = (int)std::min<long long>((items + 255) / 256, 148LL * 32);
+        xpos_rotate_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(p, rows, (const __nv_bfloat16 *)Q, qr);
+        xpos_rotate_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(p, rows, (const __nv_bfloat16 *)K, kr);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        note_launches(2);
+        Q = qr;
+        K = kr;
+    }
+    CUtensorMap mq, mk, mv, mo;
+    std::memset(&mo, 0, sizeof(mo));
+    const int bh = p.B * p.H;
+    if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kT) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kT) ||
+        !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kT))
+        return cudaErrorInvalidValue;
+    if (out_bf16 && !make_tma_map_bf16(&mo, O, p.dv, p.L, bh, kT)) return cudaErrorInvalidValue;
+    if (p.dk == 256)
+        return out_bf16 ? launch_ptc_tv<256, __nv_bfloat16>(p, mq, mk, mv, mo, O, status, st)
+                        : launch_ptc_tv<256, float>(p, mq, mk, mv, mo, O, status, st);
+    return out_bf16 ? launch_ptc_tv<128, __nv_bfloat16>(p, mq, mk, mv, mo, O, status, st)
+                    : launch_ptc_tv<128, float>(p, mq, mk, mv, mo, O, status, st);
+}
+
+}  // namespace ret

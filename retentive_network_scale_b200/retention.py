@@ -27,7 +27,8 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
                 "RET_ERR_TIMEOUT"]
 
 # every symbol include/retention.h declares
-EXPORTS = ("ret_parallel", "ret_chunkwise", "ret_chunkwise_gate_static", "ret_workspace_size",
+EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
+           "ret_chunkwise_gate_static", "ret_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -65,7 +66,9 @@ def load_library(path: str = LIB_PATH):
             "(there is no fallback implementation)")
     lib = ctypes.CDLL(path)
     vp, st, D = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(RetDesc)
-    lib.ret_parallel.argtypes = [D, vp, vp, vp, vp, vp]
+    lib.ret_parallel.argtypes = [D, vp, vp, vp, vp, vp, st, vp]
+    lib.ret_parallel_workspace_size.argtypes = [D]
+    lib.ret_parallel_workspace_size.restype = st
     lib.ret_chunkwise.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
                                   ctypes.c_float, vp, vp, st, vp]
     lib.ret_chunkwise_gate_static.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp,
@@ -153,8 +156,10 @@ def _check(status, what):
 
 # ---------------------------------------------------------------- entry points
 def ret_parallel(Q, K, V, O, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
-                 stream=None):
-    """Parallel form: O = (Q^ K^^T (.) D) V.  Q, K [B,H,L,dk], V, O [B,H,L,dv]."""
+                 workspace=None, stream=None):
+    """Parallel form: O = (Q^ K^^T (.) D) V.  Q, K [B,H,L,dk], V, O [B,H,L,dv].
+    Allocates the workspace with torch when the call needs one and none is
+    given."""
     lib = load_library()
     B, H, L, dk = Q.shape
     dv = V.shape[-1]
@@ -162,8 +167,12 @@ def ret_parallel(Q, K, V, O, gamma, rotate=False, theta_base=10000.0, pos_offset
     _dev(O, "O", (B, H, L, dv))
     d = make_desc(B, H, L, dk, dv, _dtype_code(Q), _dtype_code(O), gamma, rotate,
                   theta_base, pos_offset)
+    need = int(lib.ret_parallel_workspace_size(ctypes.byref(d)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ret_parallel(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
-                            _stream(stream)), "ret_parallel")
+                            _ptr(workspace), ws_bytes, _stream(stream)), "ret_parallel")
     return O
 
 

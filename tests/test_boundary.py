@@ -57,8 +57,8 @@ def desc(**kw):
     return R.make_desc(**base)
 
 
-def call_parallel(lib, d, Q=FAKE, K=FAKE, V=FAKE, O=FAKE):
-    return lib.ret_parallel(ctypes.byref(d), Q, K, V, O, None)
+def call_parallel(lib, d, Q=FAKE, K=FAKE, V=FAKE, O=FAKE, ws=None, ws_bytes=0):
+    return lib.ret_parallel(ctypes.byref(d), Q, K, V, O, ws, ws_bytes, None)
 
 
 def call_chunkwise(lib, d, chunk=4, Q=FAKE, K=FAKE, V=FAKE, s_in=None, s_out=None, O=FAKE,
@@ -90,7 +90,7 @@ def test_bad_descriptions(lib, kw, status):
 
 
 def test_null_description(lib):
-    assert lib.ret_parallel(None, FAKE, FAKE, FAKE, FAKE, None) == R.STATUS_NAMES.index("RET_ERR_NULL")
+    assert lib.ret_parallel(None, FAKE, FAKE, FAKE, FAKE, None, 0, None) == R.STATUS_NAMES.index("RET_ERR_NULL")
 
 
 def test_bad_pointers(lib):
@@ -99,6 +99,12 @@ def test_bad_pointers(lib):
     assert call_parallel(lib, d, Q=None) == NULL
     assert call_parallel(lib, d, O=None) == NULL
     assert call_parallel(lib, d, V=MISALIGNED) == ALIGN
+    # the tensor-core parallel form with rotation needs workspace for the turned Q, K
+    dp = desc(d_k=128, d_v=128, gamma=[0.9, 0.99])
+    need = lib.ret_parallel_workspace_size(ctypes.byref(dp))
+    assert need == 2 * 2 * 2 * 8 * 128 * 2
+    assert call_parallel(lib, dp) == R.STATUS_NAMES.index("RET_ERR_WORKSPACE")
+    assert call_parallel(lib, desc(d_k=128, d_v=128, rotate=False)) != R.STATUS_NAMES.index("RET_ERR_WORKSPACE")
     assert call_chunkwise(lib, d, O=None) == NULL                      # nothing requested
     assert call_chunkwise(lib, d, G=FAKE, Y=None) == NULL              # G without Y
     assert call_chunkwise(lib, d, s_out=MISALIGNED) == ALIGN

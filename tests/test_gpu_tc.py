@@ -118,3 +118,24 @@ def test_small_gamma_uses_cuda_core_path():
     O = torch.empty(B, H, L, dv, device="cuda")
     R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, rotate=True)
     assert rel_l2(O, O_ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,rotate,out", [
+    (1, 3, 300, 128, 128, True, torch.float32),
+    (2, 2, 640, 256, 256, True, torch.bfloat16),
+    (1, 3, 1100, 256, 512, False, torch.bfloat16),
+    (1, 1, 1, 128, 256, True, torch.float32),
+])
+def test_tc_parallel_matches_oracle(B, H, L, dk, dv, rotate, out):
+    """Parallel form on the tensor cores (rotation pre-pass into the
+    workspace, decay as a rank-1 scaling, underflowed key tiles skipped)."""
+    Q, K, V = _inputs(B, H, L, dk, dv, 300 + L)
+    g = ([0.75, 0.96875, 1.0] * 2)[:H]
+    O_ref, _ = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=9)
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=out)
+    R.ret_parallel(Q.cuda(), K.cuda(), V.cuda(), O, g, rotate=rotate, pos_offset=9)
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
