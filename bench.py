@@ -53,6 +53,25 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def profiled_traffic(kernel_src, summary):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, scaled to the full workload; None unless the summary was taken
+    on the current source of the kernel (its sha256 prefix matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "retentive_network_scale_b200", "csrc", kernel_src)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        if line.startswith("traffic_bytes_per_full_launch:"):
+            # traffic_bytes_per_full_launch: <bytes> source_sha256: <16 hex>
+            parts = line.split()
+            if len(parts) >= 4 and parts[3] == digest:
+                return float(parts[1])
+    return None
+
+
 def chunkwise_flops_per_token_head(C, dk, dv):
     """Algorithmic flops of the chunkwise form per token and head: causal
     pairs only inside a chunk ((C+1)/2 keys on average, 2 flops per
@@ -223,8 +242,10 @@ def time_launches(fn, n, stream):
     return s.elapsed_time(e) / n
 
 
-def bench_decode(R, pk, warm=2, reps=3):
+def bench_decode(R, pk, warm=2, reps=3, batch=None):
     w = WORKLOADS["decode"]
+    if batch:
+        w = dataclasses.replace(w, B=batch)
     x = make_inputs(w, device="cuda")
     steps = make_decode_inputs(w, device="cuda")
     g = R.msr_gammas(w.H)
@@ -296,6 +317,18 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
+    if args.only in ("decode", "parallel"):
+        if args.only == "decode":
+            out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
+        else:
+            w = WORKLOADS["msr_1p3b"]
+            if args.batch:
+                w = dataclasses.replace(w, B=args.batch)
+            d = {k: v.cuda() for k, v in make_inputs(w).items()}
+            out = bench_parallel(R, w, d, pk, reps=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"only": args.only, **out}), flush=True)
+        return
     w = WORKLOADS["msr_1p3b"]
     if args.batch:
         w = dataclasses.replace(w, B=args.batch)
@@ -305,9 +338,17 @@ def run_ours(args, world, rank, local):
     g = R.msr_gammas(w.H)
     Y = torch.empty(w.B, w.L, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
     stream = torch.cuda.current_stream()
+    # workspace for the prepared Q^ / K~ (the call's streaming pass), once
+    ws = torch.empty(R.ret_chunkwise_prep_size(w.B, w.H, w.L, w.d_k, w.d_v, R.RET_BF16, R.RET_BF16,
+                                               g, w.chunk, rotate=w.rotate),
+                     dtype=torch.uint8, device="cuda")
 
     def step():
-        R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, G=d["G"], Y=Y, rotate=w.rotate)
+        R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, G=d["G"], Y=Y, rotate=w.rotate,
+                        workspace=ws)
+
+    def prep_only():
+        R.ret_chunkwise_prepare(d["Q"], d["K"], g, w.chunk, ws, rotate=w.rotate)
 
     for _ in range(args.warmup):
         step()
@@ -330,17 +371,38 @@ def run_ours(args, world, rank, local):
     tokens_step = w.B * w.L
     value = world * tokens_step / (ms * 1e-3)
 
-    # dominant kernel: the whole step is the chunkwise call
+    # The step is two launches: the streaming pass that prepares Q^ / K~
+    # and the chunk loop (the dominant kernel).  The pass is timed alone
+    # (same stream, same buffers) and the loop's time is the difference.
+    for _ in range(2):
+        prep_only()
+    ms_prep = time_launches(prep_only, max(3, args.steps), stream)
+    ms_kernel = max(ms_local - ms_prep, 1e-6)
     flops = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
+    # algorithmic bytes of the chunk loop: Q^, K~ (same sizes as Q, K), V, G in; Y out
     bytes_alg = sum(t.numel() * t.element_size() for t in d.values()) + Y.numel() * Y.element_size()
-    tf = flops / (ms_local * 1e-3) / 1e12
-    gbs = bytes_alg / (ms_local * 1e-3) / 1e9
-    roofline = {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": tf / pk["bf16_tflops"], "traffic": None,
-                "peak_source": f"{pk_src} (bf16 burst)",
-                "flops_per_launch": flops, "bytes_per_launch": bytes_alg,
-                "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": gbs / pk["hbm_gbs"]}}
+    prep_bytes = 2 * ws.numel()  # Q, K read; Q^, K~ written
+    tf = flops / (ms_kernel * 1e-3) / 1e12
+    gbs = bytes_alg / (ms_kernel * 1e-3) / 1e9
+    prep_gbs = prep_bytes / (ms_prep * 1e-3) / 1e9
+    # flops / bytes = arithmetic intensity below the ridge (peak flops / peak
+    # bandwidth): HBM is the roof that binds this kernel
+    roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"],
+                "traffic": profiled_traffic("chunkwise_tc.cu", "chunkwise_tc_msr_1p3b.md"),
+                "kernel": "chunkwise_tc_kernel<256, bf16, fused GroupNorm/gate>",
+                "peak_source": f"{pk_src} (copy bandwidth)",
+                "ms_per_launch": ms_kernel, "bytes_per_launch": bytes_alg,
+                "flops_per_launch": flops,
+                "intensity_flop_per_byte": flops / bytes_alg,
+                "ridge_flop_per_byte": pk["bf16_tflops"] * 1e3 / pk["hbm_gbs"],
+                "tensor": {"achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": tf / pk["bf16_tflops"],
+                           "peak_source": f"{pk_src} (bf16 burst)"},
+                "prep": {"kernel": "chunk_prep_kernel (rotate Q, rotate and decay-weight K)",
+                         "ms_per_launch": ms_prep, "bytes_per_launch": prep_bytes,
+                         "achieved": prep_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": prep_gbs / pk["hbm_gbs"]}}
 
     # end to end: pinned host buffers in, Y back to pinned host memory
     Y_host = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
@@ -400,6 +462,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
+    ap.add_argument("--only", choices=["main", "parallel", "decode"], default=None,
+                    help="run one measurement alone (profiler captures)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="override the decode workload's batch (small cases for profiler captures)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:

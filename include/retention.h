@@ -112,6 +112,13 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *             ret_gate_norm) is written as well, with epsilon gn_eps.
  *   workspace device scratch of workspace_bytes; required only when
  *             ret_workspace_size() returns a non-zero size for this call.
+ *             Optional on the tensor-core path (bf16 inputs, chunk 128,
+ *             d_k 128 or 256, d_v a multiple of 128 up to 512): with at
+ *             least ret_chunkwise_prep_size() bytes the rotated Q and the
+ *             decay-weighted K are prepared there in one streaming pass
+ *             before the chunk loop (faster); with less, the kernel
+ *             prepares each chunk's rows itself.  Results agree either way
+ *             up to rounding.
  * At least one of O and Y must be requested.
  * Errors: those of ret_parallel, plus RET_ERR_WORKSPACE.
  */
@@ -153,6 +160,30 @@ ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk, const void
  * for descriptions that ret_chunkwise would reject). */
 size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O,
                           int want_Y);
+
+/* Bytes of OPTIONAL workspace that let ret_chunkwise prepare its operands
+ * ahead of the chunk loop (see ret_chunkwise): 2*B*H*L*d_k bf16 values
+ * with rotation (the rotated Q, and K rotated and scaled by
+ * gamma^{n-1-j} at offset j of its chunk of n rows), B*H*L*d_k without.
+ * No counterpart in the paper: it is a layout choice of this library.
+ * 0 when the tensor-core path does not apply (ret_workspace_size then
+ * gives everything the call needs); never fails. */
+size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk);
+
+/* ret_chunkwise_prepare -- only the streaming pass that ret_chunkwise runs
+ * first when its workspace holds ret_chunkwise_prep_size() bytes: the
+ * rotated Q (bf16 [B][H][L][d_k], with rotation only) followed by
+ * K~[b,h,t] = gamma_h^{n-1-j} Theta_t K[b,h,t] (bf16, same shape) for row t
+ * at offset j of its chunk of n rows (section 2.1, chunkwise form (3): the
+ * weight of key j' in the state update).  No counterpart in the paper as a
+ * call of its own; exported so that the pass can be timed or scheduled
+ * apart.  Q, K device bf16; workspace device, caller-owned, overwritten.
+ * Errors: RET_ERR_SHAPE when the tensor-core path does not apply (nothing
+ * to prepare), _NULL, _ALIGN, _WORKSPACE (smaller than the prep size),
+ * _UNSUPPORTED, _CUDA, and the description errors of ret_parallel. */
+ret_status ret_chunkwise_prepare(const ret_desc *desc, int chunk,
+                                 const void *Q, const void *K, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /*
  * ret_recurrent_step -- one step of the recurrent representation (section

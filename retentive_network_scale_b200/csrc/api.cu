@@ -142,6 +142,33 @@ size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_
     return 0;
 }
 
+size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk) {
+    if (check_desc(desc) != RET_OK || chunk < 1) return 0;
+    Params p;
+    make_params(desc, &p);
+    return chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16) ? chunkwise_prep_bytes(p)
+                                                                        : 0;
+}
+
+ret_status ret_chunkwise_prepare(const ret_desc *desc, int chunk, const void *Q, const void *K,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    ret_status s = check_desc(desc);
+    if (s != RET_OK) return s;
+    if (chunk < 1) return RET_ERR_ARG;
+    const size_t need = ret_chunkwise_prep_size(desc, chunk);
+    if (need == 0 && (long long)desc->B * desc->L > 0) return RET_ERR_SHAPE;
+    if (need == 0) return RET_OK;  // empty problem
+    if (!Q || !K || !workspace) return RET_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace)) return RET_ERR_ALIGN;
+    if (workspace_bytes < need) return RET_ERR_WORKSPACE;
+    if ((s = check_device()) != RET_OK) return s;
+    Params p;
+    make_params(desc, &p);
+    const void *q_used = nullptr, *k_used = nullptr;
+    return from_cuda(
+        launch_chunkwise_prep(p, chunk, Q, K, workspace, &q_used, &k_used, (cudaStream_t)stream));
+}
+
 ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const void *K,
                          const void *V, const float *state_in, float *state_out, void *O,
                          const void *G, float gn_eps, void *Y, void *workspace,
@@ -185,8 +212,10 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     if (chunkwise_tc_supported(p, chunk, in_bf16)) {
         int *status = device_status_word();
         if (!status) return RET_ERR_CUDA;
+        // a workspace of ret_chunkwise_prep_size bytes holds the prepared rows
+        void *prep = workspace && workspace_bytes >= chunkwise_prep_bytes(p) ? workspace : nullptr;
         return from_cuda(launch_chunkwise_tc(p, out_bf16, Q, K, V, state_in, state_out, O, G, Y,
-                                             gn_eps, status, st));
+                                             gn_eps, prep, status, st));
     }
     cudaError_t e = launch_chunkwise_simt(p, chunk, in_bf16, o_bf16, Q, K, V, state_in, state_out,
                                           o_buf, st);

@@ -61,7 +61,10 @@ constexpr int kMaxCluster = kMaxDv / kTV;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 constexpr float kMinLog2GammaTimesC = -60.f;        // gamma^C >= 2^-60
 
-enum { BQ = 0, BK, BV, BS, BU, BPV, BG, kNumBars };
+// Q^ arrives in two parts: blocks 0,1 (BQL; between the [S|O''] product and
+// the next chunk this part is the staging area of the G, Y and O tiles) and
+// the rest (BQH; d_k 256 only).
+enum { BQL = 0, BQH, BK, BV, BS, BU, BPV, BG, kNumBars };
 
 template <int DK>
 struct Layout {
@@ -171,9 +174,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const Params p,
                     const float *__restrict__ state_in, float *__restrict__ state_out,
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, TO *__restrict__ Y,
-                    float gn_eps, int *status) {
+                    float gn_eps, int pre, int *status) {
     using Ly = Layout<DK>;
     constexpr int KB = DK / 64;         // 64-column blocks of Q^, K~, Rbar^T
+    constexpr int KHI = KB - 2;         // Q^ blocks outside the staging area
     constexpr int NCH = DK / 8;         // 16-byte chunks per Q/K row
     constexpr int RGA = DK / 64;        // 32-column groups per thread in the state pass (group A)
     constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V^T K~ (both MN-major)
@@ -186,7 +190,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int grp = tid >> 8;       // 0: state pass and Q (warpgroups 0,1); 1: output and K (2,3)
     const int gtid = tid & 255;     // thread index within the group
     const int gwg = wg & 1;         // warpgroup within the group
-    const int bh = blockIdx.y, h = bh % p.H;
+    const int bh = blockIdx.y, h = bh % p.H, b = bh / p.H;
     const int v0 = blockIdx.x * kTV;
     const float lg = p.log2g[h];
     const int L = p.L, dv = p.dv;
@@ -216,10 +220,18 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t tS = tmem, tO = tmem + 128, tR = tmem + 256;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
-    auto load_q = [&](int c) {
-        mbar_expect_tx(bar(BQ), Ly::kQBytes);
-        for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQ), kb * 64, c * kC, bh);
+    // Q^ blocks 0,1 (BQL) and the rest (BQH)
+    auto load_q_lo = [&](int c) {
+        mbar_expect_tx(bar(BQL), 2 * 16384);
+        for (int kb = 0; kb < 2; ++kb)
+            tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQL), kb * 64, c * kC, bh);
+    };
+    auto load_q_hi = [&](int c) {
+        if constexpr (KHI > 0) {
+            mbar_expect_tx(bar(BQH), KHI * 16384);
+            for (int kb = 2; kb < KB; ++kb)
+                tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQH), kb * 64, c * kC, bh);
+        }
     };
     auto load_k = [&](int c) {
         mbar_expect_tx(bar(BK), Ly::kQBytes);
@@ -230,6 +242,23 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_expect_tx(bar(BV), Ly::kVBytes);
         for (int nb = 0; nb < 2; ++nb)
             tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, c * kC, bh);
+    };
+    // the G tile of chunk c into the staging area (Q^ blocks 0,1)
+    auto load_g = [&](int c) {
+        mbar_expect_tx(bar(BG), Ly::kVBytes);
+        for (int nb = 0; nb < 2; ++nb)
+            tma_load_3d(sbase + Ly::kQ + nb * 16384, &tmG, bar(BG), h * dv + v0 + nb * 64, c * kC, b);
+    };
+    // every tile chunk c will load, into L2 ahead of time
+    auto prefetch = [&](int c) {
+        for (int kb = 0; kb < KB; ++kb) {
+            tma_prefetch_3d(&tmQ, kb * 64, c * kC, bh);
+            tma_prefetch_3d(&tmK, kb * 64, c * kC, bh);
+        }
+        for (int nb = 0; nb < 2; ++nb) {
+            tma_prefetch_3d(&tmV, v0 + nb * 64, c * kC, bh);
+            if constexpr (FUSE) tma_prefetch_3d(&tmG, h * dv + v0 + nb * 64, c * kC, b);
+        }
     };
     auto sync_alive = [&]() {
         __syncthreads();
@@ -343,9 +372,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint64_t dVb = dVa;                                           // B of P V, MN-major
 
     if (tid == 0) {
-        load_q(0);
+        load_q_lo(0);
+        load_q_hi(0);
         load_k(0);
         load_v(0);
+        if constexpr (FUSE)
+            for (int nb = 0; nb < 2; ++nb) tma_prefetch_3d(&tmG, h * dv + v0 + nb * 64, 0, b);
     }
     // Starting state: TMEM R^T = gamma^{n_0} S_in^T and Rbar^T = bf16 of the
     // same; zeros without a state (the S|X product then gives O'' = 0).
@@ -370,11 +402,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if (has_in) tmem_wait_st();
     }
-    // chunk 0: group A turns Q, group B prepares K~
+    // chunk 0 (rows not prepared ahead): group A turns Q, group B prepares K~
     bool alive = true;
-    {
+    if (!pre) {
         const int n0 = min(kC, L);
-        if (g_leader) wait_bar(bar(grp == 0 ? BQ : BK), 0, abort_flag, status);
+        if (g_leader) {
+            if (grp == 0)
+                (KHI == 0 || wait_bar(bar(BQH), 0, abort_flag, status)) &&
+                    wait_bar(bar(BQL), 0, abort_flag, status);
+            else
+                wait_bar(bar(BK), 0, abort_flag, status);
+        }
         alive = gsync_alive();
         if (alive) {
             if (grp == 0)
@@ -396,31 +434,39 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const bool last = c + 1 == nchunks;
         const int n_next = last ? 0 : min(kC, L - t0 - kC);
 
-        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T, then R^T += V^T K~ (thread 0;
-        // S first, so that the P pass overlaps the state update)
+        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T (thread 0): the Q^ blocks outside
+        // the staging area first, then blocks 0,1 (they may land later)
         if (alive && tid == 0) {
+            bool ok = true;
+            if (pre)  // prepared rows: nobody else has waited for the loads
+                ok = (KHI == 0 || wait_bar(bar(BQH), par, abort_flag, status)) &&
+                     wait_bar(bar(BK), par, abort_flag, status);
+            if (ok && !last) prefetch(c + 1);
             tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < DK / 16; ++ks) {
+            auto sx = [&](int ks, bool acc) {
                 const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
                 const uint64_t offkr = (uint64_t)(((ks >> 2) * 32768 + (ks & 3) * 32) >> 4);
-                mma_ss(tS, dQ + off, dKR + offkr, kIdescSX, ks > 0);
+                mma_ss(tS, dQ + off, dKR + offkr, kIdescSX, acc ? 1u : 0u);
+            };
+            if (ok) {
+#pragma unroll
+                for (int ks = 8; ks < DK / 16; ++ks) sx(ks, ks > 8);
+            }
+            if (ok && pre) ok = wait_bar(bar(BQL), par, abort_flag, status);
+            tc_fence_after();
+            if (ok) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) sx(ks, KHI > 0 || ks > 0);
             }
             mma_commit(bar(BS));
-            if (wait_bar(bar(BV), par, abort_flag, status)) {
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks) {
-                    const uint64_t off = (uint64_t)((ks * 2048) >> 4);
-                    mma_ss(tR, dVa + off, dKb + off, kIdescU, (ks > 0 || has_state) ? 1u : 0u);
-                }
-            }
-            mma_commit(bar(BU));
         }
 
         // ---- P = bf16(S) on j' <= j, else 0, into tensor memory (all)
         if (alive && tid == 0) {
             wait_bar(bar(BS), par, abort_flag, status);
-            if (!last) load_q(c + 1);  // Q^ is no longer read
+            // Q^ is no longer read: G into the staging area, the next Q^ around it
+            if constexpr (FUSE) load_g(c);
+            if (!last) load_q_hi(c + 1);
         }
         alive = sync_alive();
         tc_fence_after();
@@ -442,7 +488,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
 
-        // ---- O'' += P V
+        // ---- O'' += P V, then R^T += V^T K~ (the output pass starts first)
         if (alive && tid == 0 && wait_bar(bar(BV), par, abort_flag, status)) {
             tc_fence_after();
 #pragma unroll
@@ -450,6 +496,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 mma_ts(tO, tS + (ks >> 1) * 32 + (ks & 1) * 8, dVb + (uint64_t)((ks * 2048) >> 4),
                        kIdescPV, 1u);
             mma_commit(bar(BPV));
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks) {
+                const uint64_t off = (uint64_t)((ks * 2048) >> 4);
+                mma_ss(tR, dVa + off, dKb + off, kIdescU, (ks > 0 || has_state) ? 1u : 0u);
+            }
+            mma_commit(bar(BU));
         }
 
         if (grp == 0) {
@@ -457,7 +509,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier
             if (alive && g_leader) {
                 wait_bar(bar(BU), par, abort_flag, status);
-                if (!last) load_k(c + 1);  // K~ is no longer read
+                if (!last) {  // K~ and V are no longer read
+                    load_k(c + 1);
+                    load_v(c + 1);
+                }
             }
             alive = gsync_alive();
             tc_fence_after();
@@ -493,9 +548,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 tmem_wait_st();
             }
-            if (alive && !last && g_leader) wait_bar(bar(BQ), par ^ 1, abort_flag, status);
-            alive = gsync_alive();
-            if (alive && !last) prep_q(c + 1, n_next, gtid, kGroup);
+            if (!pre) {
+                // Q^ blocks 0,1 follow the output pass (group B)
+                if (alive && !last && g_leader)
+                    (KHI == 0 || wait_bar(bar(BQH), par ^ 1, abort_flag, status)) &&
+                        wait_bar(bar(BQL), par ^ 1, abort_flag, status);
+                alive = gsync_alive();
+                if (alive && !last) prep_q(c + 1, n_next, gtid, kGroup);
+            }
             if constexpr (FUSE) cluster_wait();
         } else {
             // ================= group B: output, then the next V and K~
@@ -513,10 +573,11 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
             };
-            // bf16 tiles leave through shared memory (the V tile, dead now)
-            // and a TMA store; rows past the sequence end are clipped.
+            // bf16 tiles leave through the staging area (Q^ blocks 0,1, not
+            // read again this chunk) and a TMA store; rows past the sequence
+            // end are clipped.
             auto stage32 = [&](int half, const float *vals) {
-                uint8_t *dst = smem + Ly::kV + gwg * 16384 + row * 128;
+                uint8_t *dst = smem + Ly::kQ + gwg * 16384 + row * 128;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 w;
@@ -531,8 +592,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 fence_proxy_async_smem();
                 named_sync(2, kGroup);
                 if (g_leader) {
-                    tma_store_3d(map, sbase + Ly::kV, x0, y0, z0);
-                    tma_store_3d(map, sbase + Ly::kV + 16384, x0 + 64, y0, z0);
+                    tma_store_3d(map, sbase + Ly::kQ, x0, y0, z0);
+                    tma_store_3d(map, sbase + Ly::kQ + 16384, x0 + 64, y0, z0);
                     bulk_commit();
                     bulk_wait_read();
                 }
@@ -557,15 +618,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (alive) emit_o();
             } else {
                 const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
-                const int b = bh / p.H;
                 const size_t grow =
                     ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
-                // the G tile comes by TMA into the V tile, dead since P V
-                if (alive && g_leader) {
-                    mbar_expect_tx(bar(BG), Ly::kVBytes);
-                    for (int nb = 0; nb < 2; ++nb)
-                        tma_load_3d(sbase + Ly::kV + nb * 16384, &tmG, bar(BG), h * dv + v0 + nb * 64, t0, b);
-                }
+                // (the G tile is on its way into the staging area since [S|O''])
                 // row sum over the 128 columns of this CTA: the two warpgroups
                 // of the group meet in free tensor-memory columns (lane = row)
                 const uint32_t scratch = tS + lane_base;
@@ -628,8 +683,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
                 alive = gsync_alive();
                 if (alive) {
-                    // Y in place of G in the V tile (same thread, same bytes)
-                    uint8_t *tile = smem + Ly::kV + gwg * 16384 + row * 128;
+                    // Y in place of G in the staging area (same thread, same bytes)
+                    uint8_t *tile = smem + Ly::kQ + gwg * 16384 + row * 128;
 #pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
                         float x[32];
@@ -661,12 +716,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     if (O) emit_o();
                 }
             }
-            if (alive && g_leader && !last) {
-                load_v(c + 1);  // V is no longer read
-                wait_bar(bar(BK), par ^ 1, abort_flag, status);
+            // the staging area is free again (stores have read it): the next Q^ blocks 0,1
+            if (alive && g_leader && !last) load_q_lo(c + 1);
+            if (!pre) {
+                if (alive && g_leader && !last) wait_bar(bar(BK), par ^ 1, abort_flag, status);
+                alive = gsync_alive();
+                if (alive && !last) prep_k(c + 1, n_next, gtid, kGroup);
             }
-            alive = gsync_alive();
-            if (alive && !last) prep_k(c + 1, n_next, gtid, kGroup);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -694,7 +750,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 template <int DK, typename TO, bool FUSE>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
-                     const void *G, void *Y, float eps, int *status, cudaStream_t st) {
+                     const void *G, void *Y, float eps, int pre, int *status, cudaStream_t st) {
     CUtensorMap mo, my, mg;
     std::memset(&mo, 0, sizeof(mo));
     std::memset(&my, 0, sizeof(my));
@@ -721,7 +777,7 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, my, mg, p, s_in, s_out, (TO *)O,
-                           (const __nv_bfloat16 *)G, (TO *)Y, eps, status);
+                           (const __nv_bfloat16 *)G, (TO *)Y, eps, pre, status);
     if (e == cudaSuccess) note_launches(1);
     return e;
 }
@@ -729,13 +785,13 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
 template <int DK>
 cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, const CUtensorMap &mk,
                       const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
-                      const void *G, void *Y, float eps, int *status, cudaStream_t st) {
+                      const void *G, void *Y, float eps, int pre, int *status, cudaStream_t st) {
     const bool fuse = Y != nullptr;
     if (out_bf16)
-        return fuse ? launch_t<DK, __nv_bfloat16, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st)
-                    : launch_t<DK, __nv_bfloat16, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);
-    return fuse ? launch_t<DK, float, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st)
-                : launch_t<DK, float, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);
+        return fuse ? launch_t<DK, __nv_bfloat16, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st)
+                    : launch_t<DK, __nv_bfloat16, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
+    return fuse ? launch_t<DK, float, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st)
+                : launch_t<DK, float, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
 }
 
 }  // namespace
@@ -751,14 +807,22 @@ bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
 
 cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
                                 const void *V, const float *s_in, float *s_out, void *O,
-                                const void *G, void *Y, float eps, int *status, cudaStream_t st) {
+                                const void *G, void *Y, float eps, void *prep_ws, int *status,
+                                cudaStream_t st) {
+    // With room for them, the turned Q^ and scaled K~ are written once by a
+    // streaming pass and the kernel only loads them.
+    const int pre = prep_ws != nullptr;
+    if (pre) {
+        cudaError_t e = launch_chunkwise_prep(p, kC, Q, K, prep_ws, &Q, &K, st);
+        if (e != cudaSuccess) return e;
+    }
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC) ||
         !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kC))
         return cudaErrorInvalidValue;
-    if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, status, st);
+    if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
 }
 
 }  // namespace ret

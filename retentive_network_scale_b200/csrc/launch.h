@@ -24,10 +24,21 @@ cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
 // d_v a multiple of 128 (at most 512), every gamma_h^128 >= 2^-60.  With Y
 // (and G) given it also writes Y = swish(G) (.) GroupNorm_h(O); O may then
 // be NULL.
+// With prep_ws (chunkwise_prep_bytes) the rows are first prepared by the
+// streaming pass below; with NULL the kernel turns them itself (slower).
 bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16);
 cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
                                 const void *V, const float *s_in, float *s_out, void *O,
-                                const void *G, void *Y, float eps, int *status, cudaStream_t st);
+                                const void *G, void *Y, float eps, void *prep_ws, int *status,
+                                cudaStream_t st);
+
+// Streaming pass: Q^ (rotation only) and K~ = gamma^{n-1-j} K^ per row of a
+// chunk of `chunk` rows, bf16, into the workspace ([Q^][K~], or [K~] without
+// rotation); *q_used / *k_used receive the operands to multiply.
+size_t chunkwise_prep_bytes(const Params &p);
+cudaError_t launch_chunkwise_prep(const Params &p, int chunk, const void *Q, const void *K,
+                                  void *workspace, const void **q_used, const void **k_used,
+                                  cudaStream_t st);
 
 // Tensor map over [outer][rows][inner] bf16 with boxes of 64 x box_rows x 1
 // and 128-byte swizzle; rows past the end read as zeros and are not written.

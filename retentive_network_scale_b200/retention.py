@@ -28,7 +28,8 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 
 # every symbol include/retention.h declares
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
-           "ret_chunkwise_gate_static", "ret_workspace_size",
+           "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
+           "ret_chunkwise_prepare",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -75,6 +76,9 @@ def load_library(path: str = LIB_PATH):
                                               ctypes.c_float, vp, vp]
     lib.ret_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.ret_workspace_size.restype = st
+    lib.ret_chunkwise_prep_size.argtypes = [D, ctypes.c_int]
+    lib.ret_chunkwise_prep_size.restype = st
+    lib.ret_chunkwise_prepare.argtypes = [D, ctypes.c_int, vp, vp, vp, st, vp]
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -176,6 +180,37 @@ def ret_parallel(Q, K, V, O, gamma, rotate=False, theta_base=10000.0, pos_offset
     return O
 
 
+def ret_chunkwise_prep_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk, rotate=False,
+                            theta_base=10000.0, pos_offset=0):
+    """Optional workspace bytes for the prepared operands of the
+    tensor-core chunkwise path (0 where that path does not apply)."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
+    return int(lib.ret_chunkwise_prep_size(ctypes.byref(d), int(chunk)))
+
+
+def ret_chunkwise_prepare(Q, K, gamma, chunk, workspace, rotate=False, theta_base=10000.0,
+                          pos_offset=0, stream=None):
+    """The streaming pass alone: rotated Q (with rotation) then the
+    decay-weighted rotated K, bf16, into `workspace` (a uint8 device tensor
+    of at least ret_chunkwise_prep_size bytes).  Returns (Q^ or None, K~)
+    as views of the workspace."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    _dev(Q, "Q"); _dev(K, "K", Q.shape, Q.dtype); _dev(workspace, "workspace")
+    d = make_desc(B, H, L, dk, dk, _dtype_code(Q), _dtype_code(Q), gamma, rotate, theta_base,
+                  pos_offset)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_chunkwise_prepare(ctypes.byref(d), int(chunk), _ptr(Q), _ptr(K),
+                                     _ptr(workspace), ws_bytes, _stream(stream)),
+           "ret_chunkwise_prepare")
+    n = B * H * L * dk
+    flat = workspace.view(torch.bfloat16)
+    if rotate:
+        return flat[:n].view(B, H, L, dk), flat[n:2 * n].view(B, H, L, dk)
+    return None, flat[:n].view(B, H, L, dk)
+
+
 def ret_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk,
                        want_O=True, want_Y=False, rotate=False, theta_base=10000.0,
                        pos_offset=0) -> int:
@@ -187,10 +222,13 @@ def ret_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk,
 
 def ret_chunkwise(Q, K, V, gamma, chunk, O=None, state_in=None, state_out=None, G=None,
                   Y=None, gn_eps=1e-5, rotate=False, theta_base=10000.0, pos_offset=0,
-                  workspace=None, stream=None):
+                  workspace=None, stream=None, prep=True):
     """Chunkwise recurrent form with optional state in/out and the fused
     GroupNorm + swish gate (Y).  Allocates the workspace with torch when the
-    call needs one and none is given.  Returns (O, Y, state_out)."""
+    call needs one and none is given; with `prep` it also makes room for
+    the operands the tensor-core path prepares ahead of the chunk loop
+    (ret_chunkwise_prep_size), else that path prepares them in the loop.
+    Returns (O, Y, state_out)."""
     lib = load_library()
     B, H, L, dk = Q.shape
     dv = V.shape[-1]
@@ -209,6 +247,8 @@ def ret_chunkwise(Q, K, V, gamma, chunk, O=None, state_in=None, state_out=None, 
                   theta_base, pos_offset)
     need = int(lib.ret_workspace_size(ctypes.byref(d), int(chunk), int(O is not None),
                                       int(Y is not None)))
+    if prep:
+        need = max(need, int(lib.ret_chunkwise_prep_size(ctypes.byref(d), int(chunk))))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

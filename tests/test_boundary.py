@@ -118,6 +118,26 @@ def test_bad_pointers(lib):
         R.STATUS_NAMES.index("RET_ERR_WORKSPACE")
 
 
+def test_chunkwise_prep_size(lib):
+    """Optional workspace of the tensor-core chunkwise path: the rotated Q
+    and the decay-weighted K in bf16 (only K without rotation); 0 wherever
+    that path does not apply."""
+    size = lambda d, chunk=128: lib.ret_chunkwise_prep_size(ctypes.byref(d), chunk)
+    bf = R.RET_BF16
+    base = dict(B=2, H=2, L=300, d_k=256, d_v=512, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
+    assert size(desc(**base)) == 2 * (2 * 2 * 300 * 256) * 2
+    assert size(desc(**{**base, "rotate": False})) == (2 * 2 * 300 * 256) * 2
+    assert size(desc(**{**base, "d_k": 128})) == 2 * (2 * 2 * 300 * 128) * 2
+    assert size(desc(**base), chunk=64) == 0                            # chunk other than 128
+    assert size(desc(**{**base, "in_dtype": R.RET_F32})) == 0            # fp32 inputs
+    assert size(desc(**{**base, "d_k": 64})) == 0
+    assert size(desc(**{**base, "d_v": 640})) == 0                       # more than 4 column tiles
+    assert size(desc(**{**base, "gamma": [0.5, 0.99]})) == 0             # 0.5^128 < 2^-60
+    assert size(desc(**{**base, "gamma": [1.5, 0.99]})) == 0             # rejected description
+    assert size(desc(**base), chunk=0) == 0
+    assert lib.ret_chunkwise_prep_size(None, 128) == 0
+
+
 def test_recurrent_step_arguments(lib):
     d = desc(L=2)
     assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None) == \

@@ -2,7 +2,9 @@
 or 256, d_v a multiple of 128, gamma^128 >= 2^-60) against the fp64 oracle:
 ragged tails, a single row, state in/out (aliased), rotation at large
 positions, gamma = 1 heads, fp32 and bf16 outputs, and the fused GroupNorm +
-swish gate epilogue at cluster sizes 1, 2 and 4 (one launch per call)."""
+swish gate epilogue at cluster sizes 1, 2 and 4.  Each case runs with the
+operands prepared ahead by the streaming pass (`prep`, two launches) and
+with the kernel preparing them itself (one launch)."""
 import numpy as np
 import pytest
 import torch
@@ -32,6 +34,7 @@ def _inputs(B, H, L, dk, dv, seed):
     return Q, K, V
 
 
+@pytest.mark.parametrize("prep", [True, False])
 @pytest.mark.parametrize("B,H,L,dk,dv,out", [
     (1, 2, 128, 128, 128, torch.float32),
     (1, 2, 300, 128, 128, torch.float32),
@@ -39,14 +42,14 @@ def _inputs(B, H, L, dk, dv, seed):
     (1, 3, 257, 256, 256, torch.bfloat16),
     (2, 2, 640, 256, 512, torch.bfloat16),
 ])
-def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out):
+def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out, prep):
     Q, K, V = _inputs(B, H, L, dk, dv, 100 + L)
     g = ([0.75, 0.96875, 1.0] * 2)[:H] if H > 1 else [0.96875]
     O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=5)
     O = torch.empty(B, H, L, dv, device="cuda", dtype=out)
     S = torch.empty(B, H, dk, dv, device="cuda")
     R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, state_out=S, rotate=True,
-                    pos_offset=5)
+                    pos_offset=5, prep=prep)
     torch.cuda.synchronize()
     assert R.ret_last_device_status() == 0
     for b in range(B):
@@ -55,7 +58,8 @@ def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out):
             assert rel_l2(S[b, h], S_ref[b, h]) <= TOL_BF16, (b, h)
 
 
-def test_tc_state_chaining_and_large_positions():
+@pytest.mark.parametrize("prep", [True, False])
+def test_tc_state_chaining_and_large_positions(prep):
     """Two calls joined through an aliased state equal one oracle run; the
     second starts near position 60000."""
     B, H, L1, L2, dk, dv = 1, 2, 200, 190, 128, 128
@@ -68,23 +72,26 @@ def test_tc_state_chaining_and_large_positions():
     O1 = torch.empty(B, H, L1, dv, device="cuda")
     O2 = torch.empty(B, H, L2, dv, device="cuda")
     R.ret_chunkwise(Qd[:, :, :L1].contiguous(), Kd[:, :, :L1].contiguous(), Vd[:, :, :L1].contiguous(),
-                    g, 128, O=O1, state_out=S, rotate=True, pos_offset=p0)
+                    g, 128, O=O1, state_out=S, rotate=True, pos_offset=p0, prep=prep)
     R.ret_chunkwise(Qd[:, :, L1:].contiguous(), Kd[:, :, L1:].contiguous(), Vd[:, :, L1:].contiguous(),
-                    g, 128, O=O2, state_in=S, state_out=S, rotate=True, pos_offset=p0 + L1)
+                    g, 128, O=O2, state_in=S, state_out=S, rotate=True, pos_offset=p0 + L1,
+                    prep=prep)
     got = torch.cat([O1, O2], 2)
     for h in range(H):
         assert rel_l2(got[0, h], O_ref[0, h]) <= TOL_BF16
         assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16
 
 
+@pytest.mark.parametrize("prep", [True, False])
 @pytest.mark.parametrize("dk,dv,rotate,with_O,with_state", [
     (256, 256, False, False, False),
     (256, 512, True, True, False),
     (128, 128, True, False, True),
     (128, 384, False, True, True),
 ])
-def test_tc_fused_gate_groupnorm(dk, dv, rotate, with_O, with_state):
-    """Y = swish(G) (.) GroupNorm_h(O) from the one fused launch."""
+def test_tc_fused_gate_groupnorm(dk, dv, rotate, with_O, with_state, prep):
+    """Y = swish(G) (.) GroupNorm_h(O) from the one fused launch (after the
+    preparing pass when `prep`)."""
     B, H, L = 2, 2, 300
     Q, K, V = _inputs(B, H, L, dk, dv, 21 + dv)
     G = random_tensor((B, L, H * dv), 24).bfloat16()
@@ -97,8 +104,9 @@ def test_tc_fused_gate_groupnorm(dk, dv, rotate, with_O, with_state):
     S = torch.empty(B, H, dk, dv, device="cuda")
     n0 = R.ret_kernel_launches()
     R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, 128, O=O, G=G.cuda(), Y=Y, rotate=rotate,
-                    pos_offset=17, state_in=None if S0 is None else S0.cuda(), state_out=S)
-    assert R.ret_kernel_launches() - n0 == 1
+                    pos_offset=17, state_in=None if S0 is None else S0.cuda(), state_out=S,
+                    prep=prep)
+    assert R.ret_kernel_launches() - n0 == (2 if prep else 1)
     torch.cuda.synchronize()
     assert R.ret_last_device_status() == 0
     for b in range(B):
@@ -139,3 +147,34 @@ def test_tc_parallel_matches_oracle(B, H, L, dk, dv, rotate, out):
     for b in range(B):
         for h in range(H):
             assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
+
+
+@pytest.mark.parametrize("rotate", [True, False])
+def test_prepare_pass_matches_oracle(rotate):
+    """The streaming pass alone: Q^ = Theta_t Q_t and K~ = gamma^{n-1-j}
+    Theta_t K_t (bf16) for row t at offset j of its chunk of n rows (ragged
+    last chunk), against the oracle's fp64 rotation, row by row."""
+    B, H, L, dk, p0 = 2, 3, 300, 256, 70000
+    Q, K, _ = _inputs(B, H, L, dk, 128, 41)
+    g = [0.9, 0.96875, 0.999]
+    size = R.ret_chunkwise_prep_size(B, H, L, dk, 128, R.RET_BF16, R.RET_BF16, g, 128,
+                                     rotate=rotate, pos_offset=p0)
+    assert size == (2 if rotate else 1) * B * H * L * dk * 2
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+    qh, kt = R.ret_chunkwise_prepare(Q.cuda(), K.cuda(), g, 128, ws, rotate=rotate, pos_offset=p0)
+    torch.cuda.synchronize()
+    t = np.arange(L)
+    j = t % 128
+    n = np.minimum(128, L - (t - j))
+    for b in range(B):
+        for h in range(H):
+            for name, X, got, weighted in (("Q", Q, qh, False), ("K", K, kt, True)):
+                if got is None:
+                    continue
+                x = X[b, h].double().numpy()
+                ref = np.stack([orc.xpos_rotate(x[r], p0 + r) for r in range(L)]) if rotate else x
+                if weighted:
+                    ref = ref * (g[h] ** (n - 1 - j))[:, None]
+                out = got[b, h].float().cpu().double().numpy()
+                err = np.abs(out - ref)
+                assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-6 * np.abs(ref).max()), (name, b, h)
