@@ -19,21 +19,25 @@
 //
 // One CTA owns one (b, h) and a 128-column slice of V and walks the chunks
 // in order.  Tensor memory (512 columns): S [128 x 128] (P, the bf16 mask
-// of S, overwrites half of it and feeds the P V' product as the A operand),
-// O'' [128 x 128] (the two together are one 128 x 256 accumulator), and the
-// fp32 state slice transposed, R^T [128 x d_k] (lanes are V columns).
-// Shared memory: TMA-loaded Q, K, V tiles (128-byte swizzle), with K^ and
-// Rbar^T interleaved per 64-column block so that [K~ ; Rbar^T] is the single
-// 256-row B operand of the [S | O''] product.  Loads of Q, K and V complete
-// on separate barriers and are issued as soon as the MMAs that read the
-// previous tile finish; V needs no preparation, so its load overlaps the
-// next [S | O''] product.
+// of S, overwrites half of it and feeds the P V product as the A operand),
+// O'' [128 x 128], and the fp32 state slice transposed, R^T [128 x d_k]
+// (lanes are V columns).  Shared memory: TMA-loaded Q^, K~, V tiles
+// (128-byte swizzle), with K~ and Rbar^T interleaved per 64-column block.
+// Per chunk, thread 0 issues S = Q^ K~^T, then O'' = Q^ Rbar (the P pass
+// runs on S meanwhile), then O'' += P V and R^T += V^T K~; every buffer is
+// reloaded as soon as the last product that reads it completes, and the
+// next chunk's tiles are prefetched into L2 a chunk ahead.  Q^ and K~ come
+// prepared from the streaming pass (prep.cu) when the caller provides room
+// for them; otherwise the two thread groups turn them in shared memory.
 //
 // Fused epilogue (Y = swish(G) (.) GroupNorm_h(O)): the CTAs of one head
 // form a cluster along d_v; each reduces its 128 columns of a row to a mean
 // and centred sum of squares, the partials are exchanged through
 // distributed shared memory and merged (Chan's pairwise update), and every
-// CTA normalises and gates its own columns.
+// CTA normalises and gates its own columns.  The G tile lands in the Rbar^T
+// blocks 0,1 (free between the O'' product and the state pass); the gate
+// factors are computed into registers while the peers publish, and Y leaves
+// through the V tile and a TMA store.
 //
 // Every mbarrier wait is bounded: on expiry the kernel latches
 // RET_ERR_TIMEOUT in the device status word and every thread skips the
@@ -41,6 +45,7 @@
 // cluster is left waiting), in-flight copies and MMAs get a bounded drain,
 // and TMEM is freed.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <cstring>
 
@@ -61,10 +66,10 @@ constexpr int kMaxCluster = kMaxDv / kTV;
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 constexpr float kMinLog2GammaTimesC = -60.f;        // gamma^C >= 2^-60
 
-// Q^ arrives in two parts: blocks 0,1 (BQL; between the [S|O''] product and
-// the next chunk this part is the staging area of the G, Y and O tiles) and
-// the rest (BQH; d_k 256 only).
-enum { BQL = 0, BQH, BK, BV, BS, BU, BPV, BG, kNumBars };
+// Q^ arrives in two parts, blocks 0,1 (BQL) and the rest (BQH; d_k 256
+// only), so that the S product can start on the part that lands first.
+// BSS: S done (the P pass may start); BS: S and the Q^ Rbar part done.
+enum { BQL = 0, BQH, BK, BV, BSS, BS, BU, BPV, BG, kNumBars };
 
 template <int DK>
 struct Layout {
@@ -79,8 +84,8 @@ struct Layout {
     static constexpr uint32_t kVBytes = kC * kTV * 2;
     static constexpr uint32_t kSmall = kV + kVBytes;
     static constexpr uint32_t kBar = kSmall;             // kNumBars mbarriers
-    static constexpr uint32_t kTmemSlot = kSmall + 64;
-    static constexpr uint32_t kAbort = kSmall + 68;
+    static constexpr uint32_t kTmemSlot = kSmall + 96;
+    static constexpr uint32_t kAbort = kSmall + 100;
     // GroupNorm: this CTA's per-row (mean, centred sum of squares) of its
     // 128 columns, double-buffered by chunk parity; peers read it remotely.
     static constexpr uint32_t kGnOwn = kSmall + 128;     // [2][128] float2
@@ -89,8 +94,9 @@ struct Layout {
     static __device__ __forceinline__ uint32_t rbar_blk(int kb) { return kKR + kb * 32768 + 16384; }
 };
 
-// [S | O''] = Q^ [K^ ; Rbar^T]^T : A Q^ (K-major), B 256 rows (K-major)
-constexpr uint32_t kIdescSX = idesc_bf16(128, 256, 0, 0);
+// S = Q^ K~^T and O'' = Q^ Rbar : A Q^ (K-major), B 128 rows of K~ or of
+// Rbar^T (K-major)
+constexpr uint32_t kIdescSX = idesc_bf16(128, 128, 0, 0);
 // O'' += P V' : A P from tensor memory, B V' (MN-major)
 constexpr uint32_t kIdescPV = idesc_bf16(128, kTV, 0, 1);
 
@@ -115,6 +121,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
+    return __half22float2(*reinterpret_cast<__half2 *>(&u));
 }
 
 // Row c of Rbar^T (K-major, 128-byte swizzle, inside the interleaved K^ /
@@ -163,8 +178,20 @@ __device__ __forceinline__ void st_row32<__nv_bfloat16>(__nv_bfloat16 *dst, cons
     }
 }
 
-// swish(g) = g * sigmoid(g) with the fast exponential and division.
-__device__ __forceinline__ float swish_fast(float g) { return __fdividef(g, 1.f + __expf(-g)); }
+// swish(g) = g sigmoid(g) for a pair, in fp16x2: h = g/2, sigmoid(g) =
+// (1 + tanh(h)) / 2 with the hardware's fp16x2 tanh approximation (one
+// special-function operation per pair; absolute error of sigmoid near
+// 2^-11), swish = 2h sigmoid.  fp16 holds |g| up to 65504 (beyond, swish
+// becomes infinite; for g below about -20 it is exactly 0).
+__device__ __forceinline__ uint32_t swish_pair_h2(float2 g) {
+    const __half2 h = __floats2half2_rn(0.5f * g.x, 0.5f * g.y);
+    uint32_t t;
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(*reinterpret_cast<const uint32_t *>(&h)));
+    const __half2 half2 = __float2half2_rn(0.5f);
+    const __half2 sig = __hfma2(*reinterpret_cast<const __half2 *>(&t), half2, half2);
+    const __half2 sw = __hmul2(__hadd2(h, h), sig);
+    return *reinterpret_cast<const uint32_t *>(&sw);
+}
 
 template <int DK, typename TO, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -243,15 +270,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int nb = 0; nb < 2; ++nb)
             tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, c * kC, bh);
     };
-    // the G tile of chunk c into the staging area (Q^ blocks 0,1)
+    // the G tile of chunk c into the Rbar^T blocks 0,1 (free from the O''
+    // product until the state pass writes the next Rbar)
     auto load_g = [&](int c) {
         mbar_expect_tx(bar(BG), Ly::kVBytes);
         for (int nb = 0; nb < 2; ++nb)
-            tma_load_3d(sbase + Ly::kQ + nb * 16384, &tmG, bar(BG), h * dv + v0 + nb * 64, c * kC, b);
+            tma_load_3d(sbase + Ly::rbar_blk(nb), &tmG, bar(BG), h * dv + v0 + nb * 64, c * kC, b);
     };
-    // every tile chunk c will load, into L2 ahead of time
+    // every tile chunk c will load, into L2 ahead of time (the Q^ and K~
+    // blocks, which every CTA of the head loads, shared out among them)
     auto prefetch = [&](int c) {
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = blockIdx.x; kb < KB; kb += gridDim.x) {
             tma_prefetch_3d(&tmQ, kb * 64, c * kC, bh);
             tma_prefetch_3d(&tmK, kb * 64, c * kC, bh);
         }
@@ -434,47 +463,61 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const bool last = c + 1 == nchunks;
         const int n_next = last ? 0 : min(kC, L - t0 - kC);
 
-        // ---- [S | O''] = Q^ [K~ ; Rbar^T]^T (thread 0): the Q^ blocks outside
-        // the staging area first, then blocks 0,1 (they may land later)
+        if (alive && tid == 32 && !last) prefetch(c + 1);  // off thread 0's path
+        // V of this chunk, once the previous chunk's stores have read the V
+        // tile (their last use of it; the products finished before the loop
+        // barrier)
+        if (alive && tid == kGroup && c > 0) {
+            if constexpr (kStage) bulk_wait_read();
+            load_v(c);
+        }
+
+        // ---- S = Q^ K~^T, then O'' = Q^ Rbar (thread 0; both over d_k in 16-
+        // column steps: the Q^ blocks outside the staging area first, then
+        // blocks 0,1, which may land later).  The P pass starts on S while
+        // the tensor cores compute O''.
         if (alive && tid == 0) {
             bool ok = true;
             if (pre)  // prepared rows: nobody else has waited for the loads
                 ok = (KHI == 0 || wait_bar(bar(BQH), par, abort_flag, status)) &&
                      wait_bar(bar(BK), par, abort_flag, status);
-            if (ok && !last) prefetch(c + 1);
             tc_fence_after();
-            auto sx = [&](int ks, bool acc) {
+            // part 0: S (B = K~ rows), part 1: O'' (B = Rbar^T rows, 16 KB further)
+            auto sx = [&](int part, int ks, bool acc) {
                 const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-                const uint64_t offkr = (uint64_t)(((ks >> 2) * 32768 + (ks & 3) * 32) >> 4);
-                mma_ss(tS, dQ + off, dKR + offkr, kIdescSX, acc ? 1u : 0u);
+                const uint64_t offkr =
+                    (uint64_t)(((ks >> 2) * 32768 + part * 16384 + (ks & 3) * 32) >> 4);
+                mma_ss(part ? tO : tS, dQ + off, dKR + offkr, kIdescSX, acc ? 1u : 0u);
             };
             if (ok) {
 #pragma unroll
-                for (int ks = 8; ks < DK / 16; ++ks) sx(ks, ks > 8);
+                for (int ks = 8; ks < DK / 16; ++ks) sx(0, ks, ks > 8);
             }
             if (ok && pre) ok = wait_bar(bar(BQL), par, abort_flag, status);
             tc_fence_after();
             if (ok) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) sx(ks, KHI > 0 || ks > 0);
+                for (int ks = 0; ks < 8; ++ks) sx(0, ks, KHI > 0 || ks > 0);
+            }
+            mma_commit(bar(BSS));
+            if (ok) {
+#pragma unroll
+                for (int ks = 8; ks < DK / 16; ++ks) sx(1, ks, ks > 8);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) sx(1, ks, KHI > 0 || ks > 0);
             }
             mma_commit(bar(BS));
+            wait_bar(bar(BSS), par, abort_flag, status);
         }
 
         // ---- P = bf16(S) on j' <= j, else 0, into tensor memory (all)
-        if (alive && tid == 0) {
-            wait_bar(bar(BS), par, abort_flag, status);
-            // Q^ is no longer read: G into the staging area, the next Q^ around it
-            if constexpr (FUSE) load_g(c);
-            if (!last) load_q_hi(c + 1);
-        }
         alive = sync_alive();
         tc_fence_after();
         if (alive) {
             const int c0 = wg * 32;
             uint32_t a[32], pk[16];
             tmem_ld32(tS + lane_base + c0, a);
-            tmem_wait_ld();
+            tmem_wait_ld(a);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int k0 = c0 + 2 * i;
@@ -487,6 +530,16 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         tc_fence_before();
         __syncthreads();
+
+        // Q^ and Rbar are no longer read once O'' is done: G into the Rbar
+        // blocks 0,1, the next Q^ (thread 32, while thread 0 issues products)
+        if (alive && tid == 32 && wait_bar(bar(BS), par, abort_flag, status)) {
+            if constexpr (FUSE) load_g(c);
+            if (!last) {
+                load_q_lo(c + 1);
+                load_q_hi(c + 1);
+            }
+        }
 
         // ---- O'' += P V, then R^T += V^T K~ (the output pass starts first)
         if (alive && tid == 0 && wait_bar(bar(BV), par, abort_flag, status)) {
@@ -505,15 +558,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         if (grp == 0) {
-            // ================= group A: state pass, then the next Q^
+            // ================= group A: gate factors, state pass, then the next Q^
             if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier
-            if (alive && g_leader) {
+            if (alive && tid == 0) {
                 wait_bar(bar(BU), par, abort_flag, status);
-                if (!last) {  // K~ and V are no longer read
-                    load_k(c + 1);
-                    load_v(c + 1);
-                }
+                if (!last) load_k(c + 1);  // K~ is no longer read
             }
+            // group B has taken the G tile out of the Rbar blocks
+            if constexpr (FUSE) named_sync(3, kThreads);
             alive = gsync_alive();
             tc_fence_after();
             if (alive) {
@@ -542,14 +594,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     uint32_t ra[32], rb[32];
                     tmem_ld32(tR + lane_base + d_begin + 32 * g, ra);
                     tmem_ld32(tR + lane_base + d_begin + 32 * g + 32, rb);
-                    tmem_wait_ld();
+                    tmem_wait_ld(ra);
+                    tmem_wait_ld(rb);
                     state32(ra, d_begin + 32 * g);
                     state32(rb, d_begin + 32 * g + 32);
                 }
                 tmem_wait_st();
             }
             if (!pre) {
-                // Q^ blocks 0,1 follow the output pass (group B)
                 if (alive && !last && g_leader)
                     (KHI == 0 || wait_bar(bar(BQH), par ^ 1, abort_flag, status)) &&
                         wait_bar(bar(BQL), par ^ 1, abort_flag, status);
@@ -558,26 +610,29 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             if constexpr (FUSE) cluster_wait();
         } else {
-            // ================= group B: output, then the next V and K~
+            // ================= group B: output (then, without prepared rows, the next K~)
+            const int o0 = gwg * 64;   // this thread's 64 columns of the row, 32 at a time
+            const size_t grow =
+                ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
             if (alive && g_leader) wait_bar(bar(BPV), par, abort_flag, status);
             alive = gsync_alive();
             tc_fence_after();
             const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite
-            const int o0 = gwg * 64;   // this thread's 64 columns of the row, 32 at a time
             const size_t orow = ((size_t)bh * L + t0 + row) * dv + v0 + o0;
             // 32 columns of O'' (still in tensor memory until this iteration ends)
             auto ld_o = [&](int half, float *x) {
                 uint32_t a[32];
                 tmem_ld32(tO + lane_base + o0 + 32 * half, a);
-                tmem_wait_ld();
+                tmem_wait_ld(a);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
             };
-            // bf16 tiles leave through the staging area (Q^ blocks 0,1, not
-            // read again this chunk) and a TMA store; rows past the sequence
-            // end are clipped.
+            // bf16 tiles leave through the V tile (not read again this chunk
+            // once the state update is done) and a TMA store; rows past the
+            // sequence end are clipped.  The last store of a chunk is not
+            // waited for here: the next chunk's V load waits for its read.
             auto stage32 = [&](int half, const float *vals) {
-                uint8_t *dst = smem + Ly::kQ + gwg * 16384 + row * 128;
+                uint8_t *dst = smem + Ly::kV + gwg * 16384 + row * 128;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 w;
@@ -588,18 +643,18 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     *reinterpret_cast<uint4 *>(dst + (((4 * half + q) ^ (row & 7)) << 4)) = w;
                 }
             };
-            auto store_tile = [&](const CUtensorMap *map, int x0, int y0, int z0) {
+            auto store_tile = [&](const CUtensorMap *map, int x0, int y0, int z0, bool restage) {
                 fence_proxy_async_smem();
                 named_sync(2, kGroup);
                 if (g_leader) {
-                    tma_store_3d(map, sbase + Ly::kQ, x0, y0, z0);
-                    tma_store_3d(map, sbase + Ly::kQ + 16384, x0 + 64, y0, z0);
+                    tma_store_3d(map, sbase + Ly::kV, x0, y0, z0);
+                    tma_store_3d(map, sbase + Ly::kV + 16384, x0 + 64, y0, z0);
                     bulk_commit();
-                    bulk_wait_read();
+                    if (restage) bulk_wait_read();
                 }
-                named_sync(2, kGroup);
+                if (restage) named_sync(2, kGroup);
             };
-            // O = alpha O'' into `dst` (staged tile or direct stores)
+            // O = alpha O'' (staged tile or direct stores)
             auto emit_o = [&]() {
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
@@ -612,64 +667,86 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     else if (row < n)
                         st_row32<TO>(O + orow + 32 * half, x);
                 }
-                if constexpr (kStage) store_tile(&tmO, v0, t0, bh);
+                if constexpr (kStage) store_tile(&tmO, v0, t0, bh, false);
+            };
+            // the products have read V (the state update is the last)
+            auto v_free = [&]() {
+                if (alive && g_leader) wait_bar(bar(BU), par, abort_flag, status);
+                alive = gsync_alive();
             };
             if constexpr (!FUSE) {
+                if constexpr (kStage) v_free();
                 if (alive) emit_o();
             } else {
                 const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
-                const size_t grow =
-                    ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
-                // (the G tile is on its way into the staging area since [S|O''])
-                // row sum over the 128 columns of this CTA: the two warpgroups
-                // of the group meet in free tensor-memory columns (lane = row)
-                const uint32_t scratch = tS + lane_base;
-                auto combine2 = [&](float mine, int col) {
-                    tmem_st1(scratch + col + gwg, __float_as_uint(mine));
-                    tmem_wait_st();
-                    tc_fence_before();
-                    named_sync(2, kGroup);
-                    tc_fence_after();
-                    uint32_t u0, u1;
-                    tmem_ld2(scratch + col, u0, u1);
-                    tmem_wait_ld();
-                    return __uint_as_float(u0) + __uint_as_float(u1);
-                };
-                float s = 0.f;
+                // Mean and centred sum of squares of this thread's 64 columns
+                // in one pass, shifted by its first value (no cancellation
+                // unless the mean sits many deviations from that sample).
+                float s1 = 0.f, s2 = 0.f, shift = 0.f;
                 if (alive) {
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        float x[32];
-                        ld_o(half, x);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) s += x[i];
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t a[32];
+                        tmem_ld32(tO + lane_base + o0 + 32 * half, a);
+                        tmem_wait_ld(a);
+                        if (half == 0) shift = __uint_as_float(a[0]);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float d = __uint_as_float(a[i]) - shift;
+                            s1 += d;
+                            s2 = fmaf(d, d, s2);
+                        }
                     }
                 }
-                const float mc = combine2(s, 0) * (1.f / kTV);
-                float q2 = 0.f;
-                if (alive) {
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        float x[32];
-                        ld_o(half, x);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) q2 = fmaf(x[i] - mc, x[i] - mc, q2);
-                    }
-                }
-                const float m2c = combine2(q2, 2);
-                // publish (mean, M2) of this CTA's columns; the peers read it
-                // after the cluster barrier (double buffer: a peer is never
-                // more than one chunk behind, the barrier sees to that)
+                const float m_w = shift + s1 * (1.f / 64.f);
+                const float m2_w = fmaxf(s2 - s1 * s1 * (1.f / 64.f), 0.f);
+                // The two warpgroups' halves merge (Chan's pairwise update,
+                // equal counts) in this CTA's published slot; the peers read
+                // it after the cluster barrier (double buffer by chunk parity:
+                // a peer is never more than one chunk behind, the barrier sees
+                // to that).
                 const uint32_t own = sbase + Ly::kGnOwn + (par * 128 + row) * 8;
-                if (gwg == 0) *reinterpret_cast<float2 *>(smem + Ly::kGnOwn + (par * 128 + row) * 8) = make_float2(mc, m2c);
+                float2 *slot = reinterpret_cast<float2 *>(smem + Ly::kGnOwn + (par * 128 + row) * 8);
+                if (gwg == 1) *slot = make_float2(m_w, m2_w);
+                named_sync(2, kGroup);
+                if (gwg == 0) {
+                    const float2 o = *slot;
+                    const float d = m_w - o.x;
+                    *slot = make_float2(0.5f * (m_w + o.x), m2_w + o.y + 32.f * d * d);
+                }
                 cluster_arrive();
                 cluster_wait();
-                float mean = 0.f, m2 = 0.f;
-                {
-                    float2 e[kMaxCluster];
+                // the peers' partials (distributed shared memory), in flight
+                // while the gate factors are computed
+                float2 e[kMaxCluster];
+                if (alive) {
 #pragma unroll
                     for (int r = 0; r < kMaxCluster; ++r)
                         if (r < nr) e[r] = ld_cluster_f32x2(map_to_rank(own, r));
+                }
+                // swish(G) of this thread's 64 columns (fp16 pairs in
+                // registers) from the G tile in the Rbar blocks, which then go
+                // back to the state pass
+                uint32_t sw[32];
+                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
+                alive = gsync_alive();
+                if (alive) {
+                    const uint8_t *gt = smem + Ly::rbar_blk(gwg) + row * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(gt + ((q ^ (row & 7)) << 4));
+                        sw[4 * q + 0] = swish_pair_h2(unpack_bf16(w.x));
+                        sw[4 * q + 1] = swish_pair_h2(unpack_bf16(w.y));
+                        sw[4 * q + 2] = swish_pair_h2(unpack_bf16(w.z));
+                        sw[4 * q + 3] = swish_pair_h2(unpack_bf16(w.w));
+                    }
+                }
+                named_arrive(3, kThreads);
+                v_free();
+                if (alive) {
+                    uint32_t a[32];
+                    tmem_ld32(tO + lane_base + o0, a);
+                    float mean = 0.f, m2 = 0.f;
 #pragma unroll
                     for (int r = 0; r < kMaxCluster; ++r)
                         if (r < nr) mean += e[r].x;
@@ -677,47 +754,42 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int r = 0; r < kMaxCluster; ++r)
                         if (r < nr) m2 += e[r].y + (float)kTV * (e[r].x - mean) * (e[r].x - mean);
-                }
-                const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
-                const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
-                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
-                alive = gsync_alive();
-                if (alive) {
-                    // Y in place of G in the staging area (same thread, same bytes)
-                    uint8_t *tile = smem + Ly::kQ + gwg * 16384 + row * 128;
-#pragma unroll 1
+                    const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
+                    const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
+                    // Y into the V tile
+                    uint8_t *tile = smem + Ly::kV + gwg * 16384 + row * 128;
+#pragma unroll
                     for (int half = 0; half < 2; ++half) {
+                        if (half == 1) tmem_ld32(tO + lane_base + o0 + 32, a);
+                        tmem_wait_ld(a);
                         float x[32];
-                        ld_o(half, x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            uint4 *ptr = reinterpret_cast<uint4 *>(tile + (((4 * half + q) ^ (row & 7)) << 4));
-                            uint4 gw = *ptr;
-                            uint32_t *u = reinterpret_cast<uint32_t *>(&gw);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 g2 = unpack_bf16(u[e]);
-                                const int i = 8 * q + 2 * e;
-                                x[i] = swish_fast(g2.x) * ((x[i] - mean) * scale);
-                                x[i + 1] = swish_fast(g2.y) * ((x[i + 1] - mean) * scale);
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 f = unpack_h2(sw[4 * (4 * half + q) + e2]);
+                                const int i = 8 * q + 2 * e2;
+                                x[i] = f.x * ((x[i] - mean) * scale);
+                                x[i + 1] = f.y * ((x[i + 1] - mean) * scale);
                             }
                             if constexpr (kStage) {
-                                u[0] = pack_bf16(x[8 * q + 0], x[8 * q + 1]);
-                                u[1] = pack_bf16(x[8 * q + 2], x[8 * q + 3]);
-                                u[2] = pack_bf16(x[8 * q + 4], x[8 * q + 5]);
-                                u[3] = pack_bf16(x[8 * q + 6], x[8 * q + 7]);
-                                *ptr = gw;
+                                uint4 w;
+                                w.x = pack_bf16(x[8 * q + 0], x[8 * q + 1]);
+                                w.y = pack_bf16(x[8 * q + 2], x[8 * q + 3]);
+                                w.z = pack_bf16(x[8 * q + 4], x[8 * q + 5]);
+                                w.w = pack_bf16(x[8 * q + 6], x[8 * q + 7]);
+                                *reinterpret_cast<uint4 *>(tile + (((4 * half + q) ^ (row & 7)) << 4)) = w;
                             }
                         }
                         if constexpr (!kStage)
                             if (row < n) st_row32<TO>(Y + grow + 32 * half, x);
                     }
-                    if constexpr (kStage) store_tile(&tmY, h * dv + v0, t0, b);
+                    if constexpr (kStage) store_tile(&tmY, h * dv + v0, t0, b, O != nullptr);
                     if (O) emit_o();
                 }
             }
-            // the staging area is free again (stores have read it): the next Q^ blocks 0,1
-            if (alive && g_leader && !last) load_q_lo(c + 1);
             if (!pre) {
                 if (alive && g_leader && !last) wait_bar(bar(BK), par ^ 1, abort_flag, status);
                 alive = gsync_alive();
