@@ -78,18 +78,20 @@ def _draw(gen, shape, std, dtype, device):
     return x.to(dtype)
 
 
-def make_inputs(w: Workload, device="cpu", gen_device=None, L=None, B=None):
+def make_inputs(w: Workload, device="cpu", gen_device=None, L=None, B=None, shard=0):
     """Draw Q, K, V (and G) for workload ``w``.
 
     Returns a dict with ``Q``, ``K`` ``[B,H,L,d_k]``, ``V`` ``[B,H,L,d_v]``
     and, when the workload has a gate, ``G`` ``[B,L,H*d_v]``.  ``L``/``B``
-    override the workload's sizes (same recipe, smaller draw).
+    override the workload's sizes (same recipe, smaller draw).  ``shard``
+    selects an independent draw of the same recipe (one per data-parallel
+    replica); shard 0 is the workload's own draw.
     """
     B = w.B if B is None else B
     L = w.L if L is None else L
     gen_device = device if gen_device is None else gen_device
     gen = torch.Generator(device=gen_device)
-    gen.manual_seed(w.seed)
+    gen.manual_seed(shard_seed(w.seed, shard))
     out = {
         "Q": _draw(gen, (B, w.H, L, w.d_k), w.std_qk, w.dtype, gen_device),
         "K": _draw(gen, (B, w.H, L, w.d_k), w.std_qk, w.dtype, gen_device),
@@ -98,6 +100,14 @@ def make_inputs(w: Workload, device="cpu", gen_device=None, L=None, B=None):
     if w.gate:
         out["G"] = _draw(gen, (B, L, w.H * w.d_v), w.std_g, w.dtype, gen_device)
     return {k: v.to(device) for k, v in out.items()}
+
+
+def shard_seed(seed: int, shard: int) -> int:
+    """Seed of data-parallel shard ``shard`` of a workload seeded ``seed``
+    (shard 0 keeps the workload's own seed)."""
+    if shard < 0:
+        raise ValueError("shard must be >= 0")
+    return seed + 1_000_003 * shard
 
 
 def make_decode_inputs(w: Workload, steps=None, device="cpu", gen_device=None, B=None):
