@@ -104,6 +104,9 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *     R  <- gamma^n R + sum_{j'} gamma^{n-1-j'} k^_{j'}^T v_{j'}
  * (the recurrent form unrolled over the chunk; the last chunk may be short).
  * The result equals ret_parallel's up to rounding for every chunk size.
+ * On the tensor-core path a chunk of 128*m rows is evaluated as m
+ * consecutive blocks of 128 rows (the recurrence holds exactly at every row
+ * boundary, so this is the same computation with different rounding).
  *   state_in  device fp32 [B][H][d_k][d_v] or NULL (zeros).
  *   state_out device fp32, or NULL; may alias state_in.
  *   O         device out_dtype [B][H][L][d_v], or NULL when only Y is wanted.
@@ -112,8 +115,9 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *             ret_gate_norm) is written as well, with epsilon gn_eps.
  *   workspace device scratch of workspace_bytes; required only when
  *             ret_workspace_size() returns a non-zero size for this call.
- *             Optional on the tensor-core path (bf16 inputs, chunk 128,
- *             d_k 128 or 256, d_v a multiple of 128 up to 512): with at
+ *             Optional on the tensor-core path (bf16 inputs, chunk a
+ *             multiple of 128, d_k 128 or 256, d_v a multiple of 128 up to
+ *             512, gamma_h^128 >= 2^-60 for every head): with at
  *             least ret_chunkwise_prep_size() bytes the rotated Q and the
  *             decay-weighted K are prepared there in one streaming pass
  *             before the chunk loop (faster); with less, the kernel

@@ -149,14 +149,6 @@ __device__ __forceinline__ void st_rbarT_row32(uint8_t *smem, int c, int d0, con
     }
 }
 
-// cos and sin of pos * theta: the product and its reduction to [-pi, pi]
-// in fp64, then the fast sine/cosine (absolute error near 2^-21 there).
-__device__ __forceinline__ void rot_cs_fast(long long pos, double theta, float *c, float *s) {
-    const double a = (double)pos * theta;
-    const double k = rint(a * 0.15915494309189533577);
-    __sincosf((float)fma(-k, 6.283185307179586477, a), s, c);
-}
-
 template <typename T>
 __device__ __forceinline__ void st_row32(T *dst, const float *v);
 template <>
@@ -868,8 +860,12 @@ cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, con
 
 }  // namespace
 
+// A chunk of kC * m rows is evaluated as m consecutive blocks of kC rows:
+// the chunkwise recurrence holds exactly at any row boundary (the state
+// carried between the blocks is the exact state after those rows), so this
+// is the same computation; only the rounding differs.
 bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
-    if (!in_bf16 || chunk != kC || (p.dk != 128 && p.dk != 256) || p.dv % kTV != 0 ||
+    if (!in_bf16 || chunk % kC != 0 || (p.dk != 128 && p.dk != 256) || p.dv % kTV != 0 ||
         p.dv / kTV > kMaxCluster || p.L < 1 || p.B * p.H < 1 || (long long)p.B * p.H > 65535)
         return false;
     for (int h = 0; h < p.H; ++h)

@@ -50,6 +50,15 @@ __device__ __forceinline__ void rot_cs(long long pos, double theta, float *c,
     sincosf((float)a, s, c);
 }
 
+// cos and sin of pos * theta: the product and its reduction to [-pi, pi]
+// in fp64, then the fast single-precision sine/cosine (absolute error near
+// 2^-21 on that range).
+__device__ __forceinline__ void rot_cs_fast(long long pos, double theta, float *c, float *s) {
+    const double a = (double)pos * theta;
+    const double k = rint(a * 0.15915494309189533577);
+    __sincosf((float)fma(-k, 6.283185307179586477, a), s, c);
+}
+
 // xPos turn of one pair (x0, x1) by angle with cos c, sin s:
 // (x0 + i x1) e^{i a} = (x0 c - x1 s) + i (x0 s + x1 c).
 __device__ __forceinline__ void rot_pair(float &x0, float &x1, float c, float s) {

@@ -20,7 +20,8 @@ cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
                                   const void *V, const float *s_in,
                                   float *s_out, void *O, cudaStream_t st);
 
-// Tensor-core chunkwise kernel: bf16 inputs, chunk 128, d_k 128 or 256,
+// Tensor-core chunkwise kernel: bf16 inputs, chunk a multiple of 128
+// (evaluated in blocks of 128 rows), d_k 128 or 256,
 // d_v a multiple of 128 (at most 512), every gamma_h^128 >= 2^-60.  With Y
 // (and G) given it also writes Y = swish(G) (.) GroupNorm_h(O); O may then
 // be NULL.

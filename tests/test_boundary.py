@@ -128,7 +128,9 @@ def test_chunkwise_prep_size(lib):
     assert size(desc(**base)) == 2 * (2 * 2 * 300 * 256) * 2
     assert size(desc(**{**base, "rotate": False})) == (2 * 2 * 300 * 256) * 2
     assert size(desc(**{**base, "d_k": 128})) == 2 * (2 * 2 * 300 * 128) * 2
-    assert size(desc(**base), chunk=64) == 0                            # chunk other than 128
+    assert size(desc(**base), chunk=64) == 0                            # not a multiple of 128
+    assert size(desc(**base), chunk=192) == 0
+    assert size(desc(**base), chunk=256) == size(desc(**base))          # blocks of 128 rows
     assert size(desc(**{**base, "in_dtype": R.RET_F32})) == 0            # fp32 inputs
     assert size(desc(**{**base, "d_k": 64})) == 0
     assert size(desc(**{**base, "d_v": 640})) == 0                       # more than 4 column tiles

@@ -228,6 +228,26 @@ def test_msr_1p3b_bf16_sampled():
     assert rel_l2(y_slices(Y, MSR_PAIRS, w.d_v), Y_ref) <= TOL_BF16
 
 
+def test_long_ctx_sampled():
+    """Long context at full size (B=1 H=16 L=65536 d_k=128 d_v=256, chunk
+    256, xPos): the outputs over all 65536 positions and the final state of
+    the fastest- and slowest-decaying heads against the oracle's recurrent
+    form."""
+    w = WORKLOADS["long_ctx"]
+    x = make_inputs(w)
+    d = dev(x)
+    pairs = [(0, 0), (0, w.H - 1)]
+    O_ref, S_ref = oracle_slices(x["Q"], x["K"], x["V"], pairs, orc.gammas(w.H), w.rotate)
+    O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
+    S = torch.empty(w.B, w.H, w.d_k, w.d_v, device="cuda")
+    R.ret_chunkwise(d["Q"], d["K"], d["V"], R.msr_gammas(w.H), w.chunk, O=O, state_out=S,
+                    rotate=w.rotate)
+    for i, (b, h) in enumerate(pairs):
+        assert rel_l2(O[b, h], O_ref[i]) <= TOL_BF16, (b, h)
+        assert rel_l2(O[b, h, :4096], O_ref[i, :4096]) <= TOL_BF16, (b, h)
+        assert rel_l2(S[b, h], S_ref[i]) <= TOL_BF16, (b, h)
+
+
 def test_msr_1p3b_parallel_sampled():
     w = WORKLOADS["msr_1p3b"]
     x = make_inputs(w)

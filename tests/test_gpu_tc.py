@@ -59,6 +59,32 @@ def test_tc_chunkwise_matches_oracle(B, H, L, dk, dv, out, prep):
 
 
 @pytest.mark.parametrize("prep", [True, False])
+def test_tc_chunk_multiple_of_128(prep):
+    """Chunks of 256 and 384 rows run on the tensor cores as blocks of 128
+    rows; outputs, the fused gate and the state match the oracle."""
+    B, H, L, dk, dv = 1, 2, 700, 128, 256
+    Q, K, V = _inputs(B, H, L, dk, dv, 77)
+    G = random_tensor((B, L, H * dv), 78).bfloat16()
+    g = [0.96875, 0.999]
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=3)
+    Y_ref = orc.gate_groupnorm(O_ref, G)
+    for chunk in (256, 384):
+        O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
+        Y = torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16)
+        S = torch.empty(B, H, dk, dv, device="cuda")
+        n0 = R.ret_kernel_launches()
+        R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, chunk, O=O, G=G.cuda(), Y=Y, state_out=S,
+                        rotate=True, pos_offset=3, prep=prep)
+        assert R.ret_kernel_launches() - n0 == (2 if prep else 1)   # no CUDA-core fallback
+        torch.cuda.synchronize()
+        assert R.ret_last_device_status() == 0
+        for h in range(H):
+            assert rel_l2(O[0, h], O_ref[0, h]) <= TOL_BF16, (chunk, h)
+            assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16, (chunk, h)
+        assert rel_l2(Y, Y_ref) <= TOL_BF16, chunk
+
+
+@pytest.mark.parametrize("prep", [True, False])
 def test_tc_state_chaining_and_large_positions(prep):
     """Two calls joined through an aliased state equal one oracle run; the
     second starts near position 60000."""
