@@ -499,29 +499,38 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 for (int ks = 0; ks < 8; ++ks) sx(1, ks, KHI > 0 || ks > 0);
             }
             mma_commit(bar(BS));
-            wait_bar(bar(BSS), par, abort_flag, status);
         }
 
-        // ---- P = bf16(S) on j' <= j, else 0, into tensor memory (all)
-        alive = sync_alive();
-        tc_fence_after();
-        if (alive) {
-            const int c0 = wg * 32;
-            uint32_t a[32], pk[16];
-            tmem_ld32(tS + lane_base + c0, a);
-            tmem_wait_ld(a);
+        // ---- P = bf16(S) on j' <= j, else 0, into tensor memory, by warps
+        // 1-15 as soon as S is done (warp 0 is still issuing the O'' product;
+        // warp 4 also takes warp 0's lanes and keys); warp 0 meets them at
+        // named barrier 4 before it issues P V.
+        if (warp != 0) {
+            if (alive && wait_bar(bar(BSS), par, abort_flag, status)) {
+                tc_fence_after();
+                // keys [c0, c0+32) of this warp's 32 lanes -> columns [c0, c0+16)
+                auto mask_pack = [&](int c0) {
+                    uint32_t a[32], pk[16];
+                    tmem_ld32(tS + lane_base + c0, a);
+                    tmem_wait_ld(a);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int k0 = c0 + 2 * i;
-                pk[i] = pack_bf16(k0 <= row ? __uint_as_float(a[2 * i]) : 0.f,
-                                  k0 + 1 <= row ? __uint_as_float(a[2 * i + 1]) : 0.f);
+                    for (int i = 0; i < 16; ++i) {
+                        const int k0 = c0 + 2 * i;
+                        pk[i] = pack_bf16(k0 <= row ? __uint_as_float(a[2 * i]) : 0.f,
+                                          k0 + 1 <= row ? __uint_as_float(a[2 * i + 1]) : 0.f);
+                    }
+                    tmem_st16(tS + lane_base + c0, pk);
+                };
+                mask_pack(wg * 32);
+                if (warp == 4) mask_pack(0);
+                tmem_wait_st();
             }
-            // keys [32w, 32w+32) -> columns [32w, 32w+16)
-            tmem_st16(tS + lane_base + c0, pk);
-            tmem_wait_st();
+            tc_fence_before();
+            named_arrive(4, kThreads);
+        } else {
+            named_sync(4, kThreads);
         }
-        tc_fence_before();
-        __syncthreads();
+        alive = *abort_flag == 0;
 
         // Q^ and Rbar are no longer read once O'' is done: G into the Rbar
         // blocks 0,1, the next Q^ (thread 32, while thread 0 issues products)
