@@ -190,6 +190,39 @@ ret_status ret_chunkwise_prepare(const ret_desc *desc, int chunk,
                                  size_t workspace_bytes, void *stream);
 
 /*
+ * ret_chunkwise_host -- no counterpart in the paper: ret_chunkwise from HOST
+ * buffers to HOST buffers, the end-to-end form for callers whose Q, K, V, G
+ * live in host memory.  Same description, layouts, dtypes and outputs as
+ * ret_chunkwise (O and/or Y; G with Y), starting from a zero state and with
+ * no state out.  The batch is cut into `slices` slices (1..B; more are
+ * clamped to B) of ceil(B/slices) batch elements, and the slices flow through
+ * two device slots on three streams, so that the host-to-device copies of
+ * one slice, the compute of the previous one and the copy back of the one
+ * before run at the same time.
+ *   Q, K, V, G  host, read; O, Y host, written.  Page-locked memory
+ *               (cudaHostAlloc / cudaHostRegister) lets the copies overlap;
+ *               pageable memory works but the runtime stages those copies.
+ *   dev_workspace  device, 256-byte aligned, at least
+ *               ret_chunkwise_host_workspace_size() bytes; caller-owned.
+ *   stream      the work starts after what is already queued on `stream`,
+ *               and `stream` continues only once every copy back is done.
+ *               Host buffers must stay valid until then.
+ * Errors: those of ret_chunkwise, plus RET_ERR_ARG for slices < 1.  After a
+ * failure the call waits for the copies it queued before it returns.
+ */
+ret_status ret_chunkwise_host(const ret_desc *desc, int chunk, const void *Q,
+                              const void *K, const void *V, void *O,
+                              const void *G, float gn_eps, void *Y, int slices,
+                              void *dev_workspace, size_t dev_workspace_bytes,
+                              void *stream);
+
+/* Device workspace bytes ret_chunkwise_host needs (two slots of one slice
+ * each, one slot when there is a single slice); 0 for descriptions it would
+ * reject and for empty problems.  Never fails. */
+size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
+                                         int want_O, int want_Y, int slices);
+
+/*
  * ret_recurrent_step -- one step of the recurrent representation (section
  * 2.1, form (2)): S_n = gamma S_{n-1} + k^_n^T v_n, then o_n = q^_n S_n
  * (update first, then read).  desc->L must be 1 and desc->pos_offset is the

@@ -78,6 +78,9 @@ void make_params(const ret_desc *d, Params *p) {
 ret_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RET_OK : RET_ERR_CUDA; }
 
 }  // namespace
+
+ret_status validate_desc(const ret_desc *d) { return check_desc(d); }
+
 }  // namespace ret
 
 using namespace ret;

@@ -54,6 +54,9 @@ cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, co
                                const void *V, void *O, void *workspace, int *status,
                                cudaStream_t st);
 
+// The description checks every entry point runs first (no CUDA calls).
+ret_status validate_desc(const ret_desc *d);
+
 // Address of the device status word bounded waits latch errors into.
 int *device_status_word();
 

@@ -29,7 +29,7 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 # every symbol include/retention.h declares
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
-           "ret_chunkwise_prepare",
+           "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -79,6 +79,11 @@ def load_library(path: str = LIB_PATH):
     lib.ret_chunkwise_prep_size.argtypes = [D, ctypes.c_int]
     lib.ret_chunkwise_prep_size.restype = st
     lib.ret_chunkwise_prepare.argtypes = [D, ctypes.c_int, vp, vp, vp, st, vp]
+    lib.ret_chunkwise_host.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, ctypes.c_float, vp,
+                                       ctypes.c_int, vp, st, vp]
+    lib.ret_chunkwise_host_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int]
+    lib.ret_chunkwise_host_workspace_size.restype = st
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -209,6 +214,58 @@ def ret_chunkwise_prepare(Q, K, gamma, chunk, workspace, rotate=False, theta_bas
     if rotate:
         return flat[:n].view(B, H, L, dk), flat[n:2 * n].view(B, H, L, dk)
     return None, flat[:n].view(B, H, L, dk)
+
+
+def _host(t, name, shape=None, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t
+
+
+def ret_chunkwise_host(Q, K, V, gamma, chunk, O=None, G=None, Y=None, gn_eps=1e-5, rotate=False,
+                       theta_base=10000.0, pos_offset=0, slices=None, workspace=None, stream=None):
+    """Chunkwise form from host tensors to host tensors (page-locked for
+    overlap), pipelined over batch slices on the device.  Allocates the
+    device workspace with torch when none is given.  Returns (O, Y)."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _host(Q, "Q"); _host(K, "K", Q.shape, Q.dtype); _host(V, "V", (B, H, L, dv), Q.dtype)
+    _host(O, "O", (B, H, L, dv)); _host(G, "G", (B, L, H * dv), Q.dtype); _host(Y, "Y", (B, L, H * dv))
+    out_t = O if O is not None else Y
+    if out_t is None:
+        raise ValueError("request O, Y or both")
+    if O is not None and Y is not None and O.dtype != Y.dtype:
+        raise TypeError("O and Y must share a dtype")
+    slices = min(B, 8) if slices is None else int(slices)
+    d = make_desc(B, H, L, dk, dv, _dtype_code(Q), _dtype_code(out_t), gamma, rotate,
+                  theta_base, pos_offset)
+    need = int(lib.ret_chunkwise_host_workspace_size(ctypes.byref(d), int(chunk), int(O is not None),
+                                                     int(Y is not None), max(slices, 1)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_chunkwise_host(ctypes.byref(d), int(chunk), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                  _ptr(G), float(gn_eps), _ptr(Y), slices, _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "ret_chunkwise_host")
+    return O, Y
+
+
+def ret_chunkwise_host_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk, slices,
+                                      want_O=False, want_Y=True, rotate=False, theta_base=10000.0,
+                                      pos_offset=0) -> int:
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
+    return int(lib.ret_chunkwise_host_workspace_size(ctypes.byref(d), int(chunk), int(bool(want_O)),
+                                                     int(bool(want_Y)), int(slices)))
 
 
 def ret_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk,

@@ -173,3 +173,29 @@ def test_binding_rejects_host_tensors():
     q = torch.zeros(1, 1, 4, 8)
     with pytest.raises(TypeError):
         R.ret_parallel(q, q, q, q, [0.5])
+
+
+def test_host_pipeline_arguments(lib):
+    """ret_chunkwise_host rejects bad calls before any CUDA call (so these
+    run without a GPU), and its workspace contract."""
+    d = desc(B=4, L=8)
+    call = lambda **kw: lib.ret_chunkwise_host(
+        ctypes.byref(kw.get("d", d)), kw.get("chunk", 4), kw.get("Q", FAKE), FAKE, FAKE,
+        kw.get("O", FAKE), kw.get("G", None), ctypes.c_float(1e-5), kw.get("Y", None),
+        kw.get("slices", 2), kw.get("ws", None), kw.get("ws_bytes", 0), None)
+    S = R.STATUS_NAMES.index
+    assert call(slices=0) == S("RET_ERR_ARG")
+    assert call(chunk=0) == S("RET_ERR_ARG")
+    assert call(Q=None) == S("RET_ERR_NULL")
+    assert call(O=None) == S("RET_ERR_NULL")                     # nothing requested
+    assert call(G=FAKE) == S("RET_ERR_NULL")                     # G without Y
+    assert call() == S("RET_ERR_WORKSPACE")
+    assert call(d=desc(B=0, L=8)) == S("RET_OK")                 # empty: nothing queued
+    size = lambda slices, O=1, Y=0, dd=d: lib.ret_chunkwise_host_workspace_size(
+        ctypes.byref(dd), 4, O, Y, slices)
+    assert size(1) > 0 and size(2) == size(1)                    # 1 slot of 4, or 2 slots of 2
+    assert size(4) < size(2)                                     # 2 slots of 1 batch element
+    assert size(64) == size(4)                                   # clamped to B slices
+    assert size(0) == 0 and size(2, O=0, Y=0) == 0
+    assert size(2, dd=desc(gamma=[2.0, 0.5])) == 0              # rejected description
+    assert call(ws=FAKE, ws_bytes=size(2) - 1) == S("RET_ERR_WORKSPACE")
