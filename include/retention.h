@@ -223,6 +223,19 @@ size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
                                          int want_O, int want_Y, int slices);
 
 /*
+ * ret_selftest_wait_timeout -- diagnostic, no counterpart in the paper.
+ * Queues one small kernel on `stream` that waits on an mbarrier nothing
+ * completes, through the same bounded wait every tensor-core kernel uses,
+ * giving up after `cycles` SM clock cycles (1000 to 4e9, i.e. up to about
+ * 2 s).  The expected outcome is the failure path of a stalled copy or
+ * product: RET_ERR_TIMEOUT latched in the device status word (read and
+ * cleared by ret_last_device_status), the kernel ending normally and the
+ * device staying usable.  Returns RET_OK once the kernel is queued;
+ * RET_ERR_ARG for `cycles` out of range, _UNSUPPORTED, _CUDA.
+ */
+ret_status ret_selftest_wait_timeout(long long cycles, void *stream);
+
+/*
  * ret_recurrent_step -- one step of the recurrent representation (section
  * 2.1, form (2)): S_n = gamma S_{n-1} + k^_n^T v_n, then o_n = q^_n S_n
  * (update first, then read).  desc->L must be 1 and desc->pos_offset is the

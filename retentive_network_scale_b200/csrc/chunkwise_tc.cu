@@ -102,16 +102,7 @@ constexpr uint32_t kIdescPV = idesc_bf16(128, kTV, 0, 1);
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                          int *status) {
-    const long long start = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - start > kTimeoutCycles) {
-            *abort_flag = 1;
-            atomicExch(status, (int)RET_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
+    return mbar_wait_bounded(bar, parity, abort_flag, status, kTimeoutCycles);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {

@@ -56,16 +56,7 @@ struct PLayout {
 
 __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                       int *status) {
-    const long long start = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - start > kTimeoutCycles) {
-            *abort_flag = 1;
-            atomicExch(status, (int)RET_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
+    return mbar_wait_bounded(bar, parity, abort_flag, status, kTimeoutCycles);
 }
 
 __device__ __forceinline__ uint32_t pk_bf16(float a, float b) {

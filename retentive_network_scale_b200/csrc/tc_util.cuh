@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "retention.h"
+
 namespace ret {
 namespace tc {
 
@@ -32,6 +34,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+// Waits for the phase of parity `parity` of mbarrier `bar`, for at most
+// `limit` SM clock cycles.  Returns true once the phase has completed;
+// false when another thread has raised *abort_flag, or on expiry, after
+// raising *abort_flag and latching RET_ERR_TIMEOUT in *status.  Every wait
+// of the tensor-core kernels goes through here, so none of them can spin
+// for ever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int *abort_flag, int *status,
+                                                  long long limit) {
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - start > limit) {
+            *abort_flag = 1;
+            atomicExch(status, (int)RET_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
 }
 // Makes the generic-proxy writes of this thread to shared memory visible to
 // the async proxy (TMA, tensor cores).

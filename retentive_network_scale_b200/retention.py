@@ -30,6 +30,7 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
            "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
+           "ret_selftest_wait_timeout",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -84,6 +85,7 @@ def load_library(path: str = LIB_PATH):
     lib.ret_chunkwise_host_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                       ctypes.c_int]
     lib.ret_chunkwise_host_workspace_size.restype = st
+    lib.ret_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -266,6 +268,13 @@ def ret_chunkwise_host_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, ga
     d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
     return int(lib.ret_chunkwise_host_workspace_size(ctypes.byref(d), int(chunk), int(bool(want_O)),
                                                      int(bool(want_Y)), int(slices)))
+
+
+def ret_selftest_wait_timeout(cycles, stream=None):
+    """Diagnostic: a bounded wait that runs out (see the header); afterwards
+    ret_last_device_status() reports RET_ERR_TIMEOUT."""
+    lib = load_library()
+    _check(lib.ret_selftest_wait_timeout(int(cycles), _stream(stream)), "ret_selftest_wait_timeout")
 
 
 def ret_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk,

@@ -199,3 +199,11 @@ def test_host_pipeline_arguments(lib):
     assert size(0) == 0 and size(2, O=0, Y=0) == 0
     assert size(2, dd=desc(gamma=[2.0, 0.5])) == 0              # rejected description
     assert call(ws=FAKE, ws_bytes=size(2) - 1) == S("RET_ERR_WORKSPACE")
+
+
+def test_selftest_wait_timeout_arguments(lib):
+    S = R.STATUS_NAMES.index
+    assert lib.ret_selftest_wait_timeout(999, None) == S("RET_ERR_ARG")
+    assert lib.ret_selftest_wait_timeout(4000000001, None) == S("RET_ERR_ARG")
+    if not torch.cuda.is_available():
+        assert lib.ret_selftest_wait_timeout(2000000, None) == S("RET_ERR_UNSUPPORTED")
