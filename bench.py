@@ -291,6 +291,35 @@ def bench_decode(R, pk, warm=2, reps=3, batch=None):
                   + w.B * w.H * (2 * w.d_k + w.d_v) * 2       # q, k, v (bf16)
                   + w.B * w.H * w.d_v * 2)                    # o (bf16)
     gbs = bytes_step / (ms * 1e-3) / 1e9
+    # several tokens per sequence and call (T = 8): one pass over the state
+    T = 8
+    calls = w.decode_steps // T
+    group = lambda a, i: a[i * T:(i + 1) * T].permute(1, 2, 0, 3).contiguous()  # noqa: E731
+    qs = [group(steps["q"], i) for i in range(calls)]
+    ks = [group(steps["k"], i) for i in range(calls)]
+    vs = [group(steps["v"], i) for i in range(calls)]
+    del steps
+    om = torch.empty(calls, w.B, w.H, T, w.d_v, device="cuda", dtype=torch.bfloat16)
+    state_m = S.clone()
+    graph_m = torch.cuda.CUDAGraph()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        R.ret_recurrent_step(qs[0], ks[0], vs[0], state_m, om[0], g, pos=w.L, rotate=w.rotate,
+                             stream=side)
+        side.synchronize()
+        with torch.cuda.graph(graph_m, stream=side):
+            for i in range(calls):
+                R.ret_recurrent_step(qs[i], ks[i], vs[i], state_m, om[i], g, pos=w.L + i * T,
+                                     rotate=w.rotate, stream=side)
+    stream.wait_stream(side)
+    for _ in range(warm):
+        graph_m.replay()
+    torch.cuda.synchronize()
+    ms_m = time_launches(graph_m.replay, reps, stream) / calls
+    graph_m.reset()
+    bytes_call = (2 * w.B * w.H * w.d_k * w.d_v * 4
+                  + T * w.B * w.H * (2 * w.d_k + w.d_v) * 2 + T * w.B * w.H * w.d_v * 2)
+    gbs_m = bytes_call / (ms_m * 1e-3) / 1e9
     flop_prefill = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
     return {
         "workload": f"decode: B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v}, fp32 state, bf16 q/k/v/o, "
@@ -301,6 +330,12 @@ def bench_decode(R, pk, warm=2, reps=3, batch=None):
         "prefill": {"ms": t_prefill, "tokens_per_s": w.B * w.L / (t_prefill * 1e-3),
                     "tflops": flop_prefill / (t_prefill * 1e-3) / 1e12},
         "gpu_launches_per_step": 1,
+        "multi_token": {
+            "tokens_per_call": T, "ms_per_call": ms_m,
+            "tokens_per_s": w.B * T / (ms_m * 1e-3),
+            "workload": f"{T} tokens per sequence per call, {calls} calls in one CUDA graph",
+            "roofline": {"bound": "hbm", "achieved": gbs_m, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs_m / pk["hbm_gbs"], "bytes_per_call": bytes_call}},
     }
 
 

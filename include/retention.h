@@ -48,6 +48,7 @@ extern "C" {
 #endif
 
 #define RET_MAX_HEADS 128
+#define RET_MAX_DECODE_STEPS 16  /* tokens per ret_recurrent_step call */
 
 typedef enum {
     RET_OK = 0,
@@ -68,7 +69,8 @@ typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
 
 /* Problem description.  The struct is read during the call only. */
 typedef struct {
-    int B, H, L, d_k, d_v;   /* L must be 1 for ret_recurrent_step          */
+    int B, H, L, d_k, d_v;   /* L: 1..RET_MAX_DECODE_STEPS for
+                                ret_recurrent_step                          */
     int in_dtype;            /* ret_dtype of Q, K, V (and G)                */
     int out_dtype;           /* ret_dtype of O (and Y)                      */
     const double *gamma;     /* HOST array [H]: decay of each head          */
@@ -236,14 +238,19 @@ size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
 ret_status ret_selftest_wait_timeout(long long cycles, void *stream);
 
 /*
- * ret_recurrent_step -- one step of the recurrent representation (section
- * 2.1, form (2)): S_n = gamma S_{n-1} + k^_n^T v_n, then o_n = q^_n S_n
- * (update first, then read).  desc->L must be 1 and desc->pos_offset is the
- * absolute position n of this token.
- *   q, k   device in_dtype [B][H][d_k];  v device in_dtype [B][H][d_v]
+ * ret_recurrent_step -- the recurrent representation (section 2.1, form
+ * (2)) for desc->L = T consecutive tokens of every sequence (1 <= T <=
+ * RET_MAX_DECODE_STEPS): for n = pos_offset .. pos_offset+T-1,
+ *     S_n = gamma S_{n-1} + k^_n^T v_n,  then  o_n = q^_n S_n
+ * (update first, then read).  desc->pos_offset is the absolute position of
+ * the first token.  The state is read and written once for all T tokens,
+ * so T > 1 (several accepted tokens, or a chunk of a draft) costs about the
+ * HBM traffic of one token.
+ *   q, k   device in_dtype [B][H][T][d_k];  v device in_dtype [B][H][T][d_v]
  *   state  device fp32 [B][H][d_k][d_v], updated in place
- *   o      device out_dtype [B][H][d_v]
- * Errors: those of ret_parallel.
+ *   o      device out_dtype [B][H][T][d_v]
+ * (with T = 1 these are [B][H][d]).  Errors: those of ret_parallel, and
+ * RET_ERR_SHAPE for T outside 1..RET_MAX_DECODE_STEPS.
  */
 ret_status ret_recurrent_step(const ret_desc *desc, const void *q,
                               const void *k, const void *v, float *state,

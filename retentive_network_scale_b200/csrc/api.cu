@@ -232,7 +232,7 @@ ret_status ret_recurrent_step(const ret_desc *desc, const void *q, const void *k
                               float *state, void *o, void *stream) {
     ret_status s = check_desc(desc);
     if (s != RET_OK) return s;
-    if (desc->L != 1) return RET_ERR_SHAPE;
+    if (desc->L < 1 || desc->L > RET_MAX_DECODE_STEPS) return RET_ERR_SHAPE;
     const bool empty = desc->B == 0;
     if (!empty && (!q || !k || !v || !state || !o)) return RET_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))

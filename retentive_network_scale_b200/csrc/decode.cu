@@ -117,6 +117,152 @@ recurrent_step_kernel(Params p, int ncol_tiles, const TI *q, const TI *k,
     }
 }
 
+// T > 1 consecutive tokens per sequence (positions pos_offset .. +T-1) in
+// one pass over the state: every element runs its T updates in registers,
+//   s <- gamma s + k^_t[i] v_t[c];   o_t[c] += q^_t[i] s   (t = 0 .. T-1),
+// so the state is read and written once for all T tokens.  q, k, v, o are
+// [B][H][T][d]; the rotated q^_t, k^_t of the head and the v_t of the CTA's
+// columns sit in shared memory; the column sums are reduced token by token.
+constexpr int kMultiRowsInFlight = 4;
+
+template <typename TI, typename TO, int COLS, int TMAX>
+__global__ void __launch_bounds__(kThreads)
+recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k, const TI *v,
+                       float *state, TO *o) {
+    constexpr int TPR = COLS / 4;
+    constexpr int RG = kThreads / TPR;
+    __shared__ float qs[TMAX][kMaxDk], ks[TMAX][kMaxDk];
+    __shared__ __align__(16) float vs[TMAX][COLS];
+    __shared__ float red[RG * COLS];
+
+    const int bh = blockIdx.x / ncol_tiles, ct = blockIdx.x - bh * ncol_tiles;
+    const int h = bh % p.H;
+    const int dk = p.dk, dv = p.dv;
+
+    // q^_t, k^_t (turned at position pos_offset + t) and this CTA's v_t columns
+    if (p.rotate) {
+        for (int idx = threadIdx.x; idx < T * (dk / 2); idx += kThreads) {
+            const int t = idx / (dk / 2), j = idx - t * (dk / 2);
+            const size_t base = ((size_t)bh * T + t) * dk;
+            float c, sn;
+            rot_cs(p.pos_offset + t, p.theta[j], &c, &sn);
+            float q0 = ld(q, base + 2 * j), q1 = ld(q, base + 2 * j + 1);
+            float k0 = ld(k, base + 2 * j), k1 = ld(k, base + 2 * j + 1);
+            rot_pair(q0, q1, c, sn);
+            rot_pair(k0, k1, c, sn);
+            qs[t][2 * j] = q0; qs[t][2 * j + 1] = q1;
+            ks[t][2 * j] = k0; ks[t][2 * j + 1] = k1;
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < T * dk; idx += kThreads) {
+            const int t = idx / dk, i = idx - t * dk;
+            qs[t][i] = ld(q, ((size_t)bh * T + t) * dk + i);
+            ks[t][i] = ld(k, ((size_t)bh * T + t) * dk + i);
+        }
+    }
+    for (int idx = threadIdx.x; idx < T * COLS; idx += kThreads) {
+        const int t = idx / COLS, cc = idx - t * COLS;
+        vs[t][cc] = ld(v, ((size_t)bh * T + t) * dv + ct * COLS + cc);
+    }
+    __syncthreads();
+
+    const int tpr = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+    const int c = ct * COLS + 4 * tpr;
+    const float g = exp2f(p.log2g[h]);
+    float *S = state + (size_t)bh * dk * dv + c;
+    float4 acc[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    for (int i0 = rg; i0 < dk; i0 += RG * kMultiRowsInFlight) {
+        float4 s[kMultiRowsInFlight];
+#pragma unroll
+        for (int u = 0; u < kMultiRowsInFlight; ++u) {
+            const int i = i0 + u * RG;
+            if (i < dk) s[u] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)i * dv));
+        }
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+            if (t < T) {
+                const float4 vt = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
+#pragma unroll
+                for (int u = 0; u < kMultiRowsInFlight; ++u) {
+                    const int i = i0 + u * RG;
+                    if (i < dk) {
+                        const float ki = ks[t][i], qi = qs[t][i];
+                        s[u].x = fmaf(g, s[u].x, ki * vt.x);
+                        s[u].y = fmaf(g, s[u].y, ki * vt.y);
+                        s[u].z = fmaf(g, s[u].z, ki * vt.z);
+                        s[u].w = fmaf(g, s[u].w, ki * vt.w);
+                        acc[t].x = fmaf(qi, s[u].x, acc[t].x);
+                        acc[t].y = fmaf(qi, s[u].y, acc[t].y);
+                        acc[t].z = fmaf(qi, s[u].z, acc[t].z);
+                        acc[t].w = fmaf(qi, s[u].w, acc[t].w);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kMultiRowsInFlight; ++u) {
+            const int i = i0 + u * RG;
+            if (i < dk) __stcs(reinterpret_cast<float4 *>(S + (size_t)i * dv), s[u]);
+        }
+    }
+
+    // o_t[c'] = sum over row groups, token by token; red is [RG][COLS]
+    constexpr int PARTS = kThreads / COLS;
+    constexpr int PER = RG / PARTS;
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+        if (t < T) {
+            red[rg * COLS + 4 * tpr + 0] = acc[t].x;
+            red[rg * COLS + 4 * tpr + 1] = acc[t].y;
+            red[rg * COLS + 4 * tpr + 2] = acc[t].z;
+            red[rg * COLS + 4 * tpr + 3] = acc[t].w;
+            __syncthreads();
+            const int cc = threadIdx.x % COLS, part = threadIdx.x / COLS;
+            float sum = 0.f;
+#pragma unroll
+            for (int r = 0; r < PER; ++r) sum += red[(part * PER + r) * COLS + cc];
+            __syncthreads();
+            red[part * COLS + cc] = sum;
+            __syncthreads();
+            if (threadIdx.x < COLS) {
+                float tot = 0.f;
+                for (int pt = 0; pt < PARTS; ++pt) tot += red[pt * COLS + threadIdx.x];
+                st(o, ((size_t)bh * T + t) * dv + ct * COLS + threadIdx.x, tot);
+            }
+            __syncthreads();
+        }
+    }
+}
+
+template <typename TI, typename TO, int TMAX>
+cudaError_t launch_multi(const Params &p, int T, const void *q, const void *k, const void *v,
+                         float *state, void *o, cudaStream_t st) {
+    const int cols = (p.dv % 32 == 0) ? 32 : 4;
+    const int tiles = p.dv / cols;
+    const long long blocks = (long long)p.B * p.H * tiles;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const TI *qq = (const TI *)q, *kk = (const TI *)k, *vv = (const TI *)v;
+    TO *oo = (TO *)o;
+    if (cols == 32)
+        recurrent_multi_kernel<TI, TO, 32, TMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
+    else
+        recurrent_multi_kernel<TI, TO, 4, TMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+template <typename TI, typename TO>
+cudaError_t launch_multi_t(const Params &p, int T, const void *q, const void *k, const void *v,
+                           float *state, void *o, cudaStream_t st) {
+    if (T <= 4) return launch_multi<TI, TO, 4>(p, T, q, k, v, state, o, st);
+    if (T <= 8) return launch_multi<TI, TO, 8>(p, T, q, k, v, state, o, st);
+    return launch_multi<TI, TO, 16>(p, T, q, k, v, state, o, st);
+}
+
 template <typename TI, typename TO>
 cudaError_t launch_t(const Params &p, const void *q, const void *k, const void *v,
                      float *state, void *o, cudaStream_t st) {
@@ -142,6 +288,13 @@ cudaError_t launch_t(const Params &p, const void *q, const void *k, const void *
 cudaError_t launch_recurrent_step(const Params &p, bool in_bf16, bool out_bf16,
                                   const void *q, const void *k, const void *v,
                                   float *state, void *o, cudaStream_t st) {
+    if (p.L > 1) {  // several tokens per sequence in one pass over the state
+        if (in_bf16)
+            return out_bf16 ? launch_multi_t<__nv_bfloat16, __nv_bfloat16>(p, p.L, q, k, v, state, o, st)
+                            : launch_multi_t<__nv_bfloat16, float>(p, p.L, q, k, v, state, o, st);
+        return out_bf16 ? launch_multi_t<float, __nv_bfloat16>(p, p.L, q, k, v, state, o, st)
+                        : launch_multi_t<float, float>(p, p.L, q, k, v, state, o, st);
+    }
     if (in_bf16)
         return out_bf16 ? launch_t<__nv_bfloat16, __nv_bfloat16>(p, q, k, v, state, o, st)
                         : launch_t<__nv_bfloat16, float>(p, q, k, v, state, o, st);

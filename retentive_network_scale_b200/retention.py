@@ -34,6 +34,7 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
+RET_MAX_DECODE_STEPS = 16
 
 
 class RetentionError(RuntimeError):
@@ -347,14 +348,21 @@ def ret_chunkwise_gate_static(Q, K, V, gamma, chunk, G, Y, state_in=None, state_
 
 def ret_recurrent_step(q, k, v, state, o, gamma, pos, rotate=False, theta_base=10000.0,
                        stream=None):
-    """One recurrent step at absolute position ``pos``: q, k [B,H,dk],
-    v, o [B,H,dv], state [B,H,dk,dv] fp32 updated in place."""
+    """Recurrent steps starting at absolute position ``pos``: one token with
+    q, k [B,H,dk] and v, o [B,H,dv], or T tokens (T <= RET_MAX_DECODE_STEPS)
+    with q, k [B,H,T,dk] and v, o [B,H,T,dv]; state [B,H,dk,dv] fp32 is
+    updated in place (read and written once for all T)."""
     lib = load_library()
-    B, H, dk = q.shape
+    if q.dim() == 3:
+        B, H, dk = q.shape
+        T = 1
+    else:
+        B, H, T, dk = q.shape
     dv = v.shape[-1]
-    _dev(q, "q"); _dev(k, "k", q.shape, q.dtype); _dev(v, "v", (B, H, dv), q.dtype)
-    _dev(state, "state", (B, H, dk, dv), torch.float32); _dev(o, "o", (B, H, dv))
-    d = make_desc(B, H, 1, dk, dv, _dtype_code(q), _dtype_code(o), gamma, rotate,
+    lead = tuple(q.shape[:-1])
+    _dev(q, "q"); _dev(k, "k", q.shape, q.dtype); _dev(v, "v", lead + (dv,), q.dtype)
+    _dev(state, "state", (B, H, dk, dv), torch.float32); _dev(o, "o", lead + (dv,))
+    d = make_desc(B, H, T, dk, dv, _dtype_code(q), _dtype_code(o), gamma, rotate,
                   theta_base, pos)
     _check(lib.ret_recurrent_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(state),
                                   _ptr(o), _stream(stream)), "ret_recurrent_step")

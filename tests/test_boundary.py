@@ -141,9 +141,13 @@ def test_chunkwise_prep_size(lib):
 
 
 def test_recurrent_step_arguments(lib):
-    d = desc(L=2)
-    assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
-        R.STATUS_NAMES.index("RET_ERR_SHAPE")
+    for L in (0, R.RET_MAX_DECODE_STEPS + 1):   # tokens per call: 1..RET_MAX_DECODE_STEPS
+        d = desc(L=L)
+        assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+            R.STATUS_NAMES.index("RET_ERR_SHAPE")
+    d = desc(L=R.RET_MAX_DECODE_STEPS)
+    assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_NULL")
     d = desc(L=1)
     assert lib.ret_recurrent_step(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, None) == \
         R.STATUS_NAMES.index("RET_ERR_NULL")
@@ -207,3 +211,11 @@ def test_selftest_wait_timeout_arguments(lib):
     assert lib.ret_selftest_wait_timeout(4000000001, None) == S("RET_ERR_ARG")
     if not torch.cuda.is_available():
         assert lib.ret_selftest_wait_timeout(2000000, None) == S("RET_ERR_UNSUPPORTED")
+
+
+def test_header_constants_match_binding():
+    import re
+    text = open(HEADER).read()
+    for name in ("RET_MAX_HEADS", "RET_MAX_DECODE_STEPS"):
+        m = re.search(r"#define\s+%s\s+(\d+)" % name, text)
+        assert m and int(m.group(1)) == getattr(R, name), name
