@@ -353,6 +353,36 @@ def bench_parallel(R, w, d, pk, reps=3):
                          "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"]}}
 
 
+def bench_layer(R, w, pk, reps=5):
+    """The whole multi-scale retention layer on the RetNet-1.3B head shape:
+    d_model = H*d_k, random bf16 weights (the shapes matter, not the values)."""
+    dm = w.H * w.d_k
+    n_proj = w.H * (2 * w.d_k + 2 * w.d_v)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed + 99)
+    X = torch.randn(w.B, w.L, dm, device="cuda", generator=gen).bfloat16()
+    W = (torch.randn(dm, n_proj, device="cuda", generator=gen) * dm ** -0.5).bfloat16()
+    Wo = (torch.randn(w.H * w.d_v, dm, device="cuda", generator=gen) * (w.H * w.d_v) ** -0.5).bfloat16()
+    out = torch.empty(w.B, w.L, dm, device="cuda", dtype=torch.bfloat16)
+    g = R.msr_gammas(w.H)
+    ws = torch.empty(R.lib_msr_layer_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, dm, w.chunk),
+                     dtype=torch.uint8, device="cuda")
+    fn = lambda: R.ret_msr_layer(X, W, Wo, g, w.chunk, w.d_k, w.d_v, out=out,  # noqa: E731
+                                 rotate=w.rotate, workspace=ws)
+    for _ in range(3):
+        fn()
+    ms = time_launches(fn, reps, torch.cuda.current_stream())
+    rows = w.B * w.L
+    flops = (2 * rows * dm * n_proj + 2 * rows * w.H * w.d_v * dm
+             + w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v))
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"MSR layer: B={w.B} L={w.L} d_model={dm} H={w.H} d_k={w.d_k} d_v={w.d_v}, "
+                        f"X W_qkvg (cuBLAS) + prep + fused chunkwise/GroupNorm/gate + Y W_o (cuBLAS)",
+            "ms": ms, "tokens_per_s": rows / (ms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
+
+
 def run_ours(args, world, rank, local):
     from retentive_network_scale_b200 import build as rbuild
     from retentive_network_scale_b200 import retention as R
@@ -473,6 +503,8 @@ def run_ours(args, world, rank, local):
     if not args.skip_extra:
         extra["parallel"] = bench_parallel(R, w, d, pk)
         del d
+        torch.cuda.empty_cache()
+        extra["msr_layer"] = bench_layer(R, w, pk)
         torch.cuda.empty_cache()
         extra["decode"] = bench_decode(R, pk)
 

@@ -225,6 +225,42 @@ size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
                                          int want_O, int want_Y, int slices);
 
 /*
+ * ret_msr_layer -- the multi-scale retention layer (paper summary, section
+ * 2.1: Q = (X W_Q) (.) Theta, K = (X W_K) (.) conj(Theta), V = X W_V, one
+ * decay per head; section 2.2: Y = GroupNorm_h(Concat(heads)),
+ * MSR(X) = (swish(X W_G) (.) Y) W_O):
+ *     P   = X [W_Q | W_K | W_V | W_G]
+ *     out = (swish(G) (.) GroupNorm_h(Retention(Q, K, V))) W_O
+ * with the heads, rotation, decays and GroupNorm of ret_chunkwise, from a
+ * zero state.
+ *   X       device bf16 [B][L][d_model]
+ *   W_qkvg  device bf16 [d_model][H*(2 d_k + 2 d_v)]: head h's columns of
+ *           Q at h d_k, of K at H d_k + h d_k, of V at 2 H d_k + h d_v, of G
+ *           at 2 H d_k + H d_v + h d_v
+ *   W_o     device bf16 [H d_v][d_model]
+ *   out     device bf16 [B][L][d_model]
+ *   workspace  device, 256-byte aligned, at least
+ *           ret_msr_layer_workspace_size() bytes (it holds P, the prepared
+ *           Q and K, Y and the GEMM library's scratch).
+ * desc->in_dtype and out_dtype are RET_BF16; d_model is a multiple of 8.
+ * The layer runs on the tensor-core chunkwise path only (chunk a multiple of
+ * 128, d_k 128 or 256, d_v a multiple of 128 up to 512, gamma_h^128 >=
+ * 2^-60).  The two projections are cuBLAS GEMMs with fp32 accumulation; P
+ * and Y are held in bf16.  Not safe to call from two host threads at once
+ * on one device.
+ * Errors: those of ret_chunkwise; RET_ERR_SHAPE off the tensor-core path.
+ */
+ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk,
+                         const void *X, const void *W_qkvg, const void *W_o,
+                         float gn_eps, void *out, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Device workspace bytes ret_msr_layer needs; 0 for descriptions it would
+ * reject by their arguments and for empty problems.  Never fails. */
+size_t ret_msr_layer_workspace_size(const ret_desc *desc, int d_model,
+                                    int chunk);
+
+/*
  * ret_selftest_wait_timeout -- diagnostic, no counterpart in the paper.
  * Queues one small kernel on `stream` that waits on an mbarrier nothing
  * completes, through the same bounded wait every tensor-core kernel uses,

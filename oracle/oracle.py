@@ -195,3 +195,28 @@ def gate_groupnorm(O, G, eps=1e-5, lib=None) -> np.ndarray:
     _check(lib.oracle_gate_groupnorm(B, L, H, dv, _ptr(O), _ptr(G), float(eps), _ptr(Y)),
            "gate_groupnorm")
     return Y
+
+
+def msr_layer(X, W_qkvg, W_o, gamma, d_k, d_v, rotate=False, theta_base=10000.0, pos_offset=0,
+              eps=1e-5, lib=None) -> np.ndarray:
+    """The multi-scale retention layer, fp64 ("Retentive Network" paper
+    summary, section 2.1: Q = (X W_Q) (.) Theta, K = (X W_K) (.) conj(Theta),
+    V = X W_V, one decay per head; section 2.2: Y = GroupNorm_h(Concat of
+    the heads), MSR(X) = (swish(X W_G) (.) Y) W_O).  X [B, L, d_model];
+    W_qkvg [d_model, H*(2 d_k + 2 d_v)] with the column blocks Q, K, V, G
+    (head h at h*d_k or h*d_v inside its block); W_o [H*d_v, d_model].
+    The projections are plain matrix products; the retention and the
+    GroupNorm + gate are this module's recurrent form and gate_groupnorm."""
+    X, W, Wo = _f64(X), _f64(W_qkvg), _f64(W_o)
+    B, L, _ = X.shape
+    H = len(gamma)
+    P = X @ W
+    heads = lambda a, d: a.reshape(B, L, H, d).transpose(0, 2, 1, 3)  # noqa: E731
+    Q = heads(P[..., :H * d_k], d_k)
+    K = heads(P[..., H * d_k:2 * H * d_k], d_k)
+    V = heads(P[..., 2 * H * d_k:2 * H * d_k + H * d_v], d_v)
+    G = P[..., 2 * H * d_k + H * d_v:]
+    O, _ = recurrent(np.ascontiguousarray(Q), np.ascontiguousarray(K), np.ascontiguousarray(V),
+                     gamma, rotate=rotate, theta_base=theta_base, pos_offset=pos_offset, lib=lib)
+    Y = gate_groupnorm(O, np.ascontiguousarray(G), eps=eps, lib=lib)
+    return Y @ Wo

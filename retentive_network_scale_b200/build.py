@@ -3,8 +3,8 @@
     python -m retentive_network_scale_b200.build [--verbose]
 
 Compiles every ``csrc/*.cu`` into one shared library next to this file.  The
-CUDA runtime is linked statically (nvcc's default), so the library needs no
-libcudart at run time beyond the driver.
+CUDA runtime is linked statically (nvcc's default); cuBLAS (the two plain
+GEMMs of ret_msr_layer) is linked dynamically from the CUDA toolkit.
 """
 from __future__ import annotations
 
@@ -44,7 +44,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
     cmd = [nvcc, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC,
            *(["-Xptxas", "-v"] if verbose else []),
-           *sources(), "-o", LIB + ".tmp"]
+           *sources(), "-lcublas", "-o", LIB + ".tmp"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)

@@ -80,6 +80,7 @@ ret_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RET_OK : RET_ERR
 }  // namespace
 
 ret_status validate_desc(const ret_desc *d) { return check_desc(d); }
+void params_from_desc(const ret_desc *d, Params *p) { make_params(d, p); }
 
 }  // namespace ret
 

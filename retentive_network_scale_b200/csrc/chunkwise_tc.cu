@@ -184,7 +184,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const Params p,
                     const float *__restrict__ state_in, float *__restrict__ state_out,
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, TO *__restrict__ Y,
-                    float gn_eps, int pre, int *status) {
+                    float gn_eps, int pre, int v_head_major, int *status) {
     using Ly = Layout<DK>;
     constexpr int KB = DK / 64;         // 64-column blocks of Q^, K~, Rbar^T
     constexpr int KHI = KB - 2;         // Q^ blocks outside the staging area
@@ -248,10 +248,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int kb = 0; kb < KB; ++kb)
             tma_load_3d(sbase + Ly::k_blk(kb), &tmK, bar(BK), kb * 64, c * kC, bh);
     };
+    // V as [B][H][L][d_v] (head-major) or as rows of H*d_v columns, like G
+    const int vx0 = v_head_major ? v0 : h * dv + v0, vz = v_head_major ? bh : b;
     auto load_v = [&](int c) {
         mbar_expect_tx(bar(BV), Ly::kVBytes);
         for (int nb = 0; nb < 2; ++nb)
-            tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, c * kC, bh);
+            tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), vx0 + nb * 64, c * kC, vz);
     };
     // the G tile of chunk c into the Rbar^T blocks 0,1 (free from the O''
     // product until the state pass writes the next Rbar)
@@ -268,7 +270,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tma_prefetch_3d(&tmK, kb * 64, c * kC, bh);
         }
         for (int nb = 0; nb < 2; ++nb) {
-            tma_prefetch_3d(&tmV, v0 + nb * 64, c * kC, bh);
+            tma_prefetch_3d(&tmV, vx0 + nb * 64, c * kC, vz);
             if constexpr (FUSE) tma_prefetch_3d(&tmG, h * dv + v0 + nb * 64, c * kC, b);
         }
     };
@@ -811,10 +813,19 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 }
 
 // ------------------------------------------------------------------ host side
+// G (and V when not head-major) are read as rows of H*d_v columns with the
+// row / batch strides of `g` (the C ABI's [B][L][H*d_v] has H*d_v and
+// L*H*d_v); the head stride does not apply to them.
+struct Views {
+    int v_head_major;
+    RowLayout g;
+};
+
 template <int DK, typename TO, bool FUSE>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
-                     const void *G, void *Y, float eps, int pre, int *status, cudaStream_t st) {
+                     const void *G, void *Y, float eps, int pre, const Views &vw, int *status,
+                     cudaStream_t st) {
     CUtensorMap mo, my, mg;
     std::memset(&mo, 0, sizeof(mo));
     std::memset(&my, 0, sizeof(my));
@@ -823,7 +834,8 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
         if (O && !make_tma_map_bf16(&mo, O, p.dv, p.L, p.B * p.H, kC)) return cudaErrorInvalidValue;
         if (Y && !make_tma_map_bf16(&my, Y, p.H * p.dv, p.L, p.B, kC)) return cudaErrorInvalidValue;
     }
-    if (G && !make_tma_map_bf16(&mg, G, p.H * p.dv, p.L, p.B, kC)) return cudaErrorInvalidValue;
+    if (G && !make_tma_map_bf16_strided(&mg, G, p.H * p.dv, p.L, p.B, vw.g.row, vw.g.batch, kC))
+        return cudaErrorInvalidValue;
     auto kern = chunkwise_tc_kernel<DK, TO, FUSE>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -841,7 +853,7 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, my, mg, p, s_in, s_out, (TO *)O,
-                           (const __nv_bfloat16 *)G, (TO *)Y, eps, pre, status);
+                           (const __nv_bfloat16 *)G, (TO *)Y, eps, pre, vw.v_head_major, status);
     if (e == cudaSuccess) note_launches(1);
     return e;
 }
@@ -849,13 +861,14 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
 template <int DK>
 cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, const CUtensorMap &mk,
                       const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
-                      const void *G, void *Y, float eps, int pre, int *status, cudaStream_t st) {
+                      const void *G, void *Y, float eps, int pre, const Views &vw, int *status,
+                      cudaStream_t st) {
     const bool fuse = Y != nullptr;
     if (out_bf16)
-        return fuse ? launch_t<DK, __nv_bfloat16, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st)
-                    : launch_t<DK, __nv_bfloat16, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
-    return fuse ? launch_t<DK, float, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st)
-                : launch_t<DK, float, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
+        return fuse ? launch_t<DK, __nv_bfloat16, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st)
+                    : launch_t<DK, __nv_bfloat16, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
+    return fuse ? launch_t<DK, float, true>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st)
+                : launch_t<DK, float, false>(p, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
 }
 
 }  // namespace
@@ -889,8 +902,28 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
     if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC) ||
         !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kC))
         return cudaErrorInvalidValue;
-    if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, status, st);
+    const Views vw{1, RowLayout{(long long)p.H * p.dv, 0, (long long)p.L * p.H * p.dv}};
+    if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
+}
+
+cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
+                                         const void *Kt, const void *V, RowLayout v_layout,
+                                         bool v_head_major, const void *G, RowLayout g_layout,
+                                         void *Y, float eps, int *status, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    const int bh = p.B * p.H;
+    if (!make_tma_map_bf16(&mq, Qh, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kC))
+        return cudaErrorInvalidValue;
+    const bool ok = v_head_major
+                        ? make_tma_map_bf16_strided(&mv, V, p.dv, p.L, bh, v_layout.row, v_layout.head, kC)
+                        : make_tma_map_bf16_strided(&mv, V, p.H * p.dv, p.L, p.B, v_layout.row,
+                                                    v_layout.batch, kC);
+    if (!ok) return cudaErrorInvalidValue;
+    const Views vw{v_head_major ? 1 : 0, g_layout};
+    if (p.dk == 256)
+        return launch_dk<256>(p, out_bf16, mq, mk, mv, nullptr, nullptr, nullptr, G, Y, eps, 1, vw, status, st);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, nullptr, nullptr, nullptr, G, Y, eps, 1, vw, status, st);
 }
 
 }  // namespace ret

@@ -44,6 +44,36 @@ cudaError_t launch_chunkwise_prep(const Params &p, int chunk, const void *Q, con
 // Tensor map over [outer][rows][inner] bf16 with boxes of 64 x box_rows x 1
 // and 128-byte swizzle; rows past the end read as zeros and are not written.
 bool make_tma_map_bf16(CUtensorMap *m, const void *base, int inner, int rows, int outer, int box_rows);
+// The same over a strided view: row_stride / outer_stride in elements
+// (multiples of 8, i.e. 16 bytes).
+bool make_tma_map_bf16_strided(CUtensorMap *m, const void *base, int inner, int rows, int outer,
+                               long long row_stride, long long outer_stride, int box_rows);
+
+// Element strides of a bf16 operand read as rows of (b, h, t): row t of head
+// h of batch b starts at b*batch + h*head + t*row.
+struct RowLayout {
+    long long row, head, batch;
+};
+// [B][H][L][d], the layout of the C ABI's Q, K, V
+inline RowLayout bhld_layout(const Params &p, int d) {
+    return RowLayout{d, (long long)p.L * d, (long long)p.H * p.L * d};
+}
+
+// Tensor-core chunkwise kernel on rows already prepared ([B][H][L][d_k]
+// Q^ and K~), V and G read through the given layouts (V as [B][H][L][d_v]
+// when v_head_major, else as rows of H*d_v columns like G), Y written as
+// [B][L][H*d_v].
+cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
+                                         const void *Kt, const void *V, RowLayout v_layout,
+                                         bool v_head_major, const void *G, RowLayout g_layout,
+                                         void *Y, float eps, int *status, cudaStream_t st);
+// The streaming pass reading Q and K through a layout; with always_q it
+// writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),
+// so the workspace holds 2*B*H*L*d_k values.
+cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void *Q, const void *K,
+                                          RowLayout src, bool always_q, void *workspace,
+                                          const void **q_used, const void **k_used,
+                                          cudaStream_t st);
 
 // Tensor-core parallel form: bf16 inputs, d_k 128 or 256, d_v a multiple of
 // 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
@@ -56,6 +86,8 @@ cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, co
 
 // The description checks every entry point runs first (no CUDA calls).
 ret_status validate_desc(const ret_desc *d);
+// The kernels' parameters for a checked description.
+void params_from_desc(const ret_desc *d, Params *p);
 
 // Address of the device status word bounded waits latch errors into.
 int *device_status_word();

@@ -48,10 +48,12 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
 }
 
-template <bool ROT>
+// ROT: turn Q and K (else K is only scaled); WQ: write Q^ (turned, or
+// copied as it is when the source layout differs from the kernel's).
+template <bool ROT, bool WQ>
 __global__ void __launch_bounds__(kThreads, 4)
 chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat16 *__restrict__ Q,
-                  const __nv_bfloat16 *__restrict__ K, __nv_bfloat16 *__restrict__ qh,
+                  const __nv_bfloat16 *__restrict__ K, RowLayout src, __nv_bfloat16 *__restrict__ qh,
                   __nv_bfloat16 *__restrict__ kt) {
     const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
@@ -62,14 +64,16 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
     const int t0 = (int)(rest % tiles) * kRows;
     const int bh = (int)(rest / tiles);
     const int nr = min(kRows, p.L - t0);
-    const size_t base = ((size_t)bh * p.L + t0) * p.dk + (size_t)c16 * 8;
+    const size_t base = ((size_t)bh * p.L + t0) * p.dk + (size_t)c16 * 8;  // destination
+    const size_t sbase = (size_t)(bh / p.H) * src.batch + (size_t)(bh % p.H) * src.head +
+                         (size_t)t0 * src.row + (size_t)c16 * 8;
 
     uint4 xk[kRows], xq[kRows];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
         if (r < nr) {
-            xk[r] = ld_stream(K + base + (size_t)r * p.dk);
-            if constexpr (ROT) xq[r] = ld_stream(Q + base + (size_t)r * p.dk);
+            xk[r] = ld_stream(K + sbase + (size_t)r * src.row);
+            if constexpr (WQ) xq[r] = ld_stream(Q + sbase + (size_t)r * src.row);
         }
     }
     float c[4], s[4], cs[4], ss[4];
@@ -106,7 +110,7 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
                 }
             }
             *reinterpret_cast<uint4 *>(kt + base + (size_t)r * p.dk) = xk[r];
-            if constexpr (ROT) *reinterpret_cast<uint4 *>(qh + base + (size_t)r * p.dk) = xq[r];
+            if constexpr (WQ) *reinterpret_cast<uint4 *>(qh + base + (size_t)r * p.dk) = xq[r];
         }
     }
 }
@@ -121,10 +125,19 @@ size_t chunkwise_prep_bytes(const Params &p) {
 cudaError_t launch_chunkwise_prep(const Params &p, int chunk, const void *Q, const void *K,
                                   void *workspace, const void **q_used, const void **k_used,
                                   cudaStream_t st) {
+    return launch_chunkwise_prep_strided(p, chunk, Q, K, bhld_layout(p, p.dk), false, workspace,
+                                         q_used, k_used, st);
+}
+
+cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void *Q, const void *K,
+                                          RowLayout src, bool always_q, void *workspace,
+                                          const void **q_used, const void **k_used,
+                                          cudaStream_t st) {
     const size_t rows = (size_t)p.B * p.H * p.L;
+    const bool wq = p.rotate || always_q;
     __nv_bfloat16 *ws = static_cast<__nv_bfloat16 *>(workspace);
-    __nv_bfloat16 *qh = p.rotate ? ws : nullptr;
-    __nv_bfloat16 *kt = p.rotate ? ws + rows * p.dk : ws;
+    __nv_bfloat16 *qh = wq ? ws : nullptr;
+    __nv_bfloat16 *kt = wq ? ws + rows * p.dk : ws;
     const long long items =
         (long long)p.B * p.H * ((p.L + kRows - 1) / kRows) * (p.dk / 8);
     const long long blocks = (items + kThreads - 1) / kThreads;
@@ -132,13 +145,15 @@ cudaError_t launch_chunkwise_prep(const Params &p, int chunk, const void *Q, con
     const auto *q = static_cast<const __nv_bfloat16 *>(Q);
     const auto *k = static_cast<const __nv_bfloat16 *>(K);
     if (p.rotate)
-        chunk_prep_kernel<true><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, q, k, qh, kt);
+        chunk_prep_kernel<true, true><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, q, k, src, qh, kt);
+    else if (wq)
+        chunk_prep_kernel<false, true><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, q, k, src, qh, kt);
     else
-        chunk_prep_kernel<false><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, q, k, qh, kt);
+        chunk_prep_kernel<false, false><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, q, k, src, qh, kt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     note_launches(1);
-    *q_used = p.rotate ? qh : Q;
+    *q_used = wq ? qh : Q;
     *k_used = kt;
     return cudaSuccess;
 }

@@ -27,10 +27,16 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 bool make_tma_map_bf16(CUtensorMap *m, const void *base, int inner, int rows, int outer, int box_rows) {
+    return make_tma_map_bf16_strided(m, base, inner, rows, outer, inner, (long long)rows * inner,
+                                     box_rows);
+}
+
+bool make_tma_map_bf16_strided(CUtensorMap *m, const void *base, int inner, int rows, int outer,
+                               long long row_stride, long long outer_stride, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)rows * inner * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)outer_stride * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,

@@ -30,7 +30,7 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
            "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
-           "ret_selftest_wait_timeout",
+           "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -87,6 +87,10 @@ def load_library(path: str = LIB_PATH):
                                                       ctypes.c_int]
     lib.ret_chunkwise_host_workspace_size.restype = st
     lib.ret_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    lib.ret_msr_layer.argtypes = [D, ctypes.c_int, ctypes.c_int, vp, vp, vp, ctypes.c_float, vp, vp,
+                                  st, vp]
+    lib.ret_msr_layer_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int]
+    lib.ret_msr_layer_workspace_size.restype = st
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -269,6 +273,39 @@ def ret_chunkwise_host_workspace_size(B, H, L, d_k, d_v, in_dtype, out_dtype, ga
     d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
     return int(lib.ret_chunkwise_host_workspace_size(ctypes.byref(d), int(chunk), int(bool(want_O)),
                                                      int(bool(want_Y)), int(slices)))
+
+
+def ret_msr_layer(X, W_qkvg, W_o, gamma, chunk, d_k, d_v, out=None, gn_eps=1e-5, rotate=False,
+                  theta_base=10000.0, pos_offset=0, workspace=None, stream=None):
+    """The multi-scale retention layer: X [B,L,d_model] bf16, W_qkvg
+    [d_model, H*(2 d_k + 2 d_v)], W_o [H*d_v, d_model]; returns out
+    [B,L,d_model] bf16.  Allocates the workspace with torch when none is
+    given."""
+    lib = load_library()
+    B, L, dm = X.shape
+    H = len(gamma)
+    n_proj = H * (2 * d_k + 2 * d_v)
+    _dev(X, "X", dtype=torch.bfloat16); _dev(W_qkvg, "W_qkvg", (dm, n_proj), torch.bfloat16)
+    _dev(W_o, "W_o", (H * d_v, dm), torch.bfloat16)
+    if out is None:
+        out = torch.empty(B, L, dm, device=X.device, dtype=torch.bfloat16)
+    _dev(out, "out", (B, L, dm), torch.bfloat16)
+    d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_BF16, gamma, rotate, theta_base, pos_offset)
+    need = int(lib.ret_msr_layer_workspace_size(ctypes.byref(d), int(dm), int(chunk)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_msr_layer(ctypes.byref(d), int(dm), int(chunk), _ptr(X), _ptr(W_qkvg), _ptr(W_o),
+                             float(gn_eps), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "ret_msr_layer")
+    return out
+
+
+def lib_msr_layer_workspace_size(B, H, L, d_k, d_v, gamma, d_model, chunk, rotate=False):
+    """Device workspace bytes of ret_msr_layer for these sizes."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_BF16, gamma, rotate)
+    return int(lib.ret_msr_layer_workspace_size(ctypes.byref(d), int(d_model), int(chunk)))
 
 
 def ret_selftest_wait_timeout(cycles, stream=None):

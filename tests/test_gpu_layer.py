@@ -1,0 +1,52 @@
+"""ret_msr_layer (projections, retention with the fused GroupNorm + gate,
+output projection) against the fp64 layer oracle; the layer's kernels read
+the projection in place (strided Q/K for the prep pass, strided V and G
+tensor maps), so a small case with two heads, a ragged length and both
+tensor-core d_k checks that plumbing; plus argument refusals."""
+import pytest
+import torch
+
+from oracle import oracle as orc
+from parity import rel_l2, TOL_BF16
+from retentive_network_scale_b200 import retention as R
+from retentive_network_scale_b200.synth import random_tensor
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from retentive_network_scale_b200 import build
+    build.build()
+    R.load_library()
+    yield
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+
+
+@pytest.mark.parametrize("dk,dv,rotate", [(128, 128, True), (256, 256, False), (128, 384, True)])
+def test_msr_layer_matches_oracle(dk, dv, rotate):
+    B, L, H, dm = 2, 300, 2, 256
+    g = [0.96875, 0.999]
+    n_proj = H * (2 * dk + 2 * dv)
+    X = random_tensor((B, L, dm), 700).bfloat16()
+    W = random_tensor((dm, n_proj), 701, dm ** -0.5).bfloat16()
+    Wo = random_tensor((H * dv, dm), 702, (H * dv) ** -0.5).bfloat16()
+    ref = orc.msr_layer(X, W, Wo, g, dk, dv, rotate=rotate, pos_offset=5)
+    n0 = R.ret_kernel_launches()
+    out = R.ret_msr_layer(X.cuda(), W.cuda(), Wo.cuda(), g, 128, dk, dv, rotate=rotate,
+                          pos_offset=5)
+    assert R.ret_kernel_launches() - n0 == 2          # prep pass + chunk loop (GEMMs: cuBLAS)
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    assert rel_l2(out, ref) <= TOL_BF16
+
+
+def test_msr_layer_refusals():
+    X = torch.zeros(1, 128, 64, device="cuda", dtype=torch.bfloat16)
+    W = torch.zeros(64, 2 * (2 * 128 + 2 * 128), device="cuda", dtype=torch.bfloat16)
+    Wo = torch.zeros(2 * 128, 64, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # chunk 64: CUDA-core path
+        R.ret_msr_layer(X, W, Wo, [0.9, 0.99], 64, 128, 128)
+    with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # gamma^128 below 2^-60
+        R.ret_msr_layer(X, W, Wo, [0.5, 0.99], 128, 128, 128)

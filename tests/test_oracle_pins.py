@@ -248,3 +248,35 @@ def test_empty_sequence(olib):
     S0 = np.ones((1, 2, 4, 4))
     O, S = orc.chunkwise(Q, Q, Q, [0.5, 0.6], 4, state_in=S0, lib=olib)
     assert np.array_equal(S, S0)
+
+
+def test_msr_layer_identity_projections(olib):
+    """With identity projections the layer is the retention + GroupNorm +
+    gate of the blocks of X (summary, sections 2.1-2.2): X holds, for every
+    (b, t), the heads' q, k, v and the gate side by side; W_qkvg = I selects
+    them, and W_o = [I | 0] hands Y back.  Pins the block order, the head
+    slicing and the transposes of the layer oracle."""
+    rng = np.random.default_rng(7)
+    B, L, H, dk, dv = 2, 9, 3, 4, 6
+    gam = [0.5, 0.9, 1.0]
+    Q = rng.standard_normal((B, H, L, dk)) * 0.5
+    K = rng.standard_normal((B, H, L, dk)) * 0.5
+    V = rng.standard_normal((B, H, L, dv))
+    G = rng.standard_normal((B, L, H * dv))
+    flat = lambda a: a.transpose(0, 2, 1, 3).reshape(B, L, -1)  # noqa: E731
+    X = np.concatenate([flat(Q), flat(K), flat(V), G], axis=-1)
+    n = X.shape[-1]
+    W_o = np.zeros((H * dv, n))
+    W_o[:, :H * dv] = np.eye(H * dv)
+    out = orc.msr_layer(X, np.eye(n), W_o, gam, dk, dv, rotate=True, pos_offset=3, lib=olib)
+    O, _ = orc.recurrent(Q, K, V, gam, rotate=True, pos_offset=3, lib=olib)
+    Y = orc.gate_groupnorm(O, G, lib=olib)
+    assert np.allclose(out[..., :H * dv], Y, rtol=0, atol=1e-12)
+    assert np.all(out[..., H * dv:] == 0)
+    # a projection that swaps two heads' value blocks swaps their outputs
+    P = np.eye(n)
+    v0 = 2 * H * dk
+    P[:, v0:v0 + dv], P[:, v0 + dv:v0 + 2 * dv] = np.eye(n)[:, v0 + dv:v0 + 2 * dv], np.eye(n)[:, v0:v0 + dv]
+    out2 = orc.msr_layer(X, P, W_o, [0.7, 0.7, 1.0], dk, dv, lib=olib)
+    O2, _ = orc.recurrent(Q, K, V[:, [1, 0, 2]], [0.7, 0.7, 1.0], lib=olib)
+    assert np.allclose(out2[..., :H * dv], orc.gate_groupnorm(O2, G, lib=olib), atol=1e-12)
