@@ -353,6 +353,34 @@ def bench_parallel(R, w, d, pk, reps=3):
                          "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"]}}
 
 
+def bench_backward(R, w, d, pk, reps=3):
+    """Gradients of the retention output (dQ, dK, dV, fp32) on the workload,
+    as the five tensor-core chunkwise products plus the copy passes."""
+    g = R.msr_gammas(w.H)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed + 7)
+    dO = torch.randn(w.B, w.H, w.L, w.d_v, device="cuda", generator=gen).bfloat16()
+    dQ = torch.empty(w.B, w.H, w.L, w.d_k, device="cuda")
+    dK = torch.empty_like(dQ)
+    dV = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda")
+    ws = torch.empty(R.lib_backward_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, w.chunk),
+                     dtype=torch.uint8, device="cuda")
+    fn = lambda: R.ret_backward(d["Q"], d["K"], d["V"], dO, g, w.chunk, dQ=dQ, dK=dK, dV=dV,  # noqa: E731
+                                rotate=w.rotate, workspace=ws)
+    for _ in range(2):
+        fn()
+    ms = time_launches(fn, reps, torch.cuda.current_stream())
+    C = w.chunk
+    fl = lambda dqk, dval: (C + 1) * (dqk + dval) + 4 * dqk * dval  # noqa: E731
+    per = 2 * fl(w.d_v, w.d_k) + fl(w.d_k, w.d_v)   # dQ^, dK^ (over d_v), dV
+    flops = w.B * w.H * w.L * per
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"retention backward (dQ, dK, dV fp32) on {w.name}", "ms": ms,
+            "tokens_per_s": w.B * w.L / (ms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
+
+
 def bench_layer(R, w, pk, reps=5):
     """The whole multi-scale retention layer on the RetNet-1.3B head shape:
     d_model = H*d_k, random bf16 weights (the shapes matter, not the values)."""
@@ -502,6 +530,7 @@ def run_ours(args, world, rank, local):
     extra = {}
     if not args.skip_extra:
         extra["parallel"] = bench_parallel(R, w, d, pk)
+        extra["backward"] = bench_backward(R, w, d, pk)
         del d
         torch.cuda.empty_cache()
         extra["msr_layer"] = bench_layer(R, w, pk)

@@ -261,6 +261,35 @@ size_t ret_msr_layer_workspace_size(const ret_desc *desc, int d_model,
                                     int chunk);
 
 /*
+ * ret_backward -- the gradients of the retention output O (as computed by
+ * ret_parallel / ret_chunkwise, no gate, zero state) with respect to Q, K
+ * and V, given dO (section 2.1: the parallel and chunkwise forms are the
+ * training forms).  With q^_t = Theta_t q_t, k^_m = Theta_m k_m:
+ *     dq^_t = sum_{m<=t} gamma^{t-m} (do_t . v_m) k^_m,
+ *     dk^_m = sum_{t>=m} gamma^{t-m} (v_m . do_t) q^_t,
+ *     dv_m  = sum_{t>=m} gamma^{t-m} (k^_m . q^_t) do_t,
+ *     dq_t = Theta_t^T dq^_t, dk_m = Theta_m^T dk^_m.
+ * Each is evaluated as a chunkwise retention of rearranged operands on the
+ * tensor cores (the two anti-causal ones over time-reversed copies).
+ *   Q, K    device bf16 [B][H][L][d_k];  V, dO device bf16 [B][H][L][d_v]
+ *   dQ, dK  device out_dtype [B][H][L][d_k];  dV device out_dtype
+ *           [B][H][L][d_v]; all fully overwritten
+ *   workspace  device, 256-byte aligned, at least
+ *           ret_backward_workspace_size() bytes
+ * Tensor-core shapes only: d_k 128 or 256, d_v a multiple of 128 up to 512,
+ * chunk a multiple of 128, gamma_h^128 >= 2^-60 (else RET_ERR_SHAPE).
+ * Errors: those of ret_chunkwise.
+ */
+ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q,
+                        const void *K, const void *V, const void *dO, void *dQ,
+                        void *dK, void *dV, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/* Device workspace bytes ret_backward needs; 0 for descriptions it would
+ * reject by their arguments and for empty problems.  Never fails. */
+size_t ret_backward_workspace_size(const ret_desc *desc, int chunk);
+
+/*
  * ret_selftest_wait_timeout -- diagnostic, no counterpart in the paper.
  * Queues one small kernel on `stream` that waits on an mbarrier nothing
  * completes, through the same bounded wait every tensor-core kernel uses,

@@ -220,3 +220,40 @@ def msr_layer(X, W_qkvg, W_o, gamma, d_k, d_v, rotate=False, theta_base=10000.0,
                      gamma, rotate=rotate, theta_base=theta_base, pos_offset=pos_offset, lib=lib)
     Y = gate_groupnorm(O, np.ascontiguousarray(G), eps=eps, lib=lib)
     return Y @ Wo
+
+
+def retention_backward(Q, K, V, dO, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
+                       lib=None):
+    """Gradients (dQ, dK, dV) of O = Retention(Q, K, V) from a zero state,
+    given dO, fp64 ("Retentive Network" paper summary, section 2.1: the
+    parallel form (Q^ K^T (.) D) V with q^_t = Theta_t q_t, k^_m = Theta_m
+    k_m, D_tm = gamma^{t-m} for m <= t).  Written from that definition in
+    matrix form, per (b, h):
+        A = (Q^ K^^T) (.) D,  dV = A^T dO,
+        dA = (dO V^T) (.) D,  dQ^ = dA K^,  dK^ = dA^T Q^,
+        dq_t = Theta_t^T dq^_t = Theta_{-t} dq^_t  (and the same for dk)."""
+    lib = lib or load()
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    B, H, L, dk = Q.shape
+    t = np.arange(L)
+
+    def turn(x, sign):
+        if not rotate:
+            return x.copy()
+        return np.stack([xpos_rotate(x[i], sign * (pos_offset + i), theta_base, lib=lib)
+                         for i in range(L)])
+
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for b in range(B):
+        for h in range(H):
+            g = float(gamma[h])
+            diff = t[:, None] - t[None, :]
+            D = np.where(diff >= 0, np.power(g, np.maximum(diff, 0)), 0.0)
+            D[np.arange(L), np.arange(L)] = 1.0
+            qh, kh = turn(Q[b, h], 1), turn(K[b, h], 1)
+            A = (qh @ kh.T) * D
+            dV[b, h] = A.T @ dO[b, h]
+            dA = (dO[b, h] @ V[b, h].T) * D
+            dQ[b, h] = turn(dA @ kh, -1)
+            dK[b, h] = turn(dA.T @ qh, -1)
+    return dQ, dK, dV

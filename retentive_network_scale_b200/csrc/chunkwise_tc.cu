@@ -910,7 +910,8 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
 cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
                                          const void *Kt, const void *V, RowLayout v_layout,
                                          bool v_head_major, const void *G, RowLayout g_layout,
-                                         void *Y, float eps, int *status, cudaStream_t st) {
+                                         void *Y, void *O, float eps, int *status,
+                                         cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mq, Qh, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kC))
@@ -922,8 +923,8 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
     if (!ok) return cudaErrorInvalidValue;
     const Views vw{v_head_major ? 1 : 0, g_layout};
     if (p.dk == 256)
-        return launch_dk<256>(p, out_bf16, mq, mk, mv, nullptr, nullptr, nullptr, G, Y, eps, 1, vw, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, nullptr, nullptr, nullptr, G, Y, eps, 1, vw, status, st);
+        return launch_dk<256>(p, out_bf16, mq, mk, mv, nullptr, nullptr, O, G, Y, eps, 1, vw, status, st);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, nullptr, nullptr, O, G, Y, eps, 1, vw, status, st);
 }
 
 }  // namespace ret

@@ -61,12 +61,13 @@ inline RowLayout bhld_layout(const Params &p, int d) {
 
 // Tensor-core chunkwise kernel on rows already prepared ([B][H][L][d_k]
 // Q^ and K~), V and G read through the given layouts (V as [B][H][L][d_v]
-// when v_head_major, else as rows of H*d_v columns like G), Y written as
-// [B][L][H*d_v].
+// when v_head_major, else as rows of H*d_v columns like G); writes Y
+// ([B][L][H*d_v], with G) and/or O ([B][H][L][d_v]) in the output dtype.
 cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
                                          const void *Kt, const void *V, RowLayout v_layout,
                                          bool v_head_major, const void *G, RowLayout g_layout,
-                                         void *Y, float eps, int *status, cudaStream_t st);
+                                         void *Y, void *O, float eps, int *status,
+                                         cudaStream_t st);
 // The streaming pass reading Q and K through a layout; with always_q it
 // writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),
 // so the workspace holds 2*B*H*L*d_k values.

@@ -133,7 +133,7 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
     const ret::RowLayout vg{z.n_proj, 0, (long long)desc->L * z.n_proj};
     e = ret::launch_chunkwise_tc_prepared(p, true, qh, kt, P + 2 * (size_t)H * dk, vg, false,
                                           P + 2 * (size_t)H * dk + (size_t)H * dv, vg,
-                                          ws + z.off_y, gn_eps, status, st);
+                                          ws + z.off_y, nullptr, gn_eps, status, st);
     if (e != cudaSuccess) return RET_ERR_CUDA;
     // 4. the output projection
     if (gemm_rm(h, z.rows, d_model, (long long)H * dv, ws + z.off_y, W_o, out) !=

@@ -31,6 +31,7 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
            "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
+           "ret_backward", "ret_backward_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -91,6 +92,9 @@ def load_library(path: str = LIB_PATH):
                                   st, vp]
     lib.ret_msr_layer_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int]
     lib.ret_msr_layer_workspace_size.restype = st
+    lib.ret_backward.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, st, vp]
+    lib.ret_backward_workspace_size.argtypes = [D, ctypes.c_int]
+    lib.ret_backward_workspace_size.restype = st
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -306,6 +310,38 @@ def lib_msr_layer_workspace_size(B, H, L, d_k, d_v, gamma, d_model, chunk, rotat
     lib = load_library()
     d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_BF16, gamma, rotate)
     return int(lib.ret_msr_layer_workspace_size(ctypes.byref(d), int(d_model), int(chunk)))
+
+
+def ret_backward(Q, K, V, dO, gamma, chunk, dQ=None, dK=None, dV=None, out_dtype=torch.float32,
+                 rotate=False, theta_base=10000.0, pos_offset=0, workspace=None, stream=None):
+    """Gradients of the retention output with respect to Q, K, V given dO
+    (bf16 inputs); returns (dQ, dK, dV), allocated in `out_dtype` when not
+    given.  Allocates the workspace with torch when none is given."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _dev(Q, "Q", dtype=torch.bfloat16); _dev(K, "K", Q.shape, torch.bfloat16)
+    _dev(V, "V", (B, H, L, dv), torch.bfloat16); _dev(dO, "dO", (B, H, L, dv), torch.bfloat16)
+    mk = lambda t, shape: t if t is not None else torch.empty(shape, device=Q.device, dtype=out_dtype)  # noqa: E731
+    dQ, dK, dV = mk(dQ, (B, H, L, dk)), mk(dK, (B, H, L, dk)), mk(dV, (B, H, L, dv))
+    _dev(dQ, "dQ", (B, H, L, dk)); _dev(dK, "dK", (B, H, L, dk), dQ.dtype)
+    _dev(dV, "dV", (B, H, L, dv), dQ.dtype)
+    d = make_desc(B, H, L, dk, dv, RET_BF16, _dtype_code(dQ), gamma, rotate, theta_base, pos_offset)
+    need = int(lib.ret_backward_workspace_size(ctypes.byref(d), int(chunk)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_backward(ctypes.byref(d), int(chunk), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(dQ),
+                            _ptr(dK), _ptr(dV), _ptr(workspace), ws_bytes, _stream(stream)),
+           "ret_backward")
+    return dQ, dK, dV
+
+
+def lib_backward_workspace_size(B, H, L, d_k, d_v, gamma, chunk, rotate=False):
+    """Device workspace bytes of ret_backward for these sizes."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_F32, gamma, rotate)
+    return int(lib.ret_backward_workspace_size(ctypes.byref(d), int(chunk)))
 
 
 def ret_selftest_wait_timeout(cycles, stream=None):

@@ -280,3 +280,30 @@ def test_msr_layer_identity_projections(olib):
     out2 = orc.msr_layer(X, P, W_o, [0.7, 0.7, 1.0], dk, dv, lib=olib)
     O2, _ = orc.recurrent(Q, K, V[:, [1, 0, 2]], [0.7, 0.7, 1.0], lib=olib)
     assert np.allclose(out2[..., :H * dv], orc.gate_groupnorm(O2, G, lib=olib), atol=1e-12)
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_backward_matches_finite_differences(olib, rotate):
+    """The backward oracle against central finite differences of the
+    forward oracle along random directions: d/de <dO, O(X + e dX)> at 0
+    equals <grad_X, dX> for X = Q, K, V (independent of the gradient
+    formulas: it only runs the forward recurrence)."""
+    rng = np.random.default_rng(11)
+    B, H, L, dk, dv = 1, 2, 7, 4, 6
+    gam = [0.8, 1.0]
+    Q = rng.standard_normal((B, H, L, dk)) * 0.5
+    K = rng.standard_normal((B, H, L, dk)) * 0.5
+    V = rng.standard_normal((B, H, L, dv))
+    dO = rng.standard_normal((B, H, L, dv))
+    dQ, dK, dV = orc.retention_backward(Q, K, V, dO, gam, rotate=rotate, pos_offset=5, lib=olib)
+    f = lambda q, k, v: float(np.sum(dO * orc.recurrent(q, k, v, gam, rotate=rotate,  # noqa: E731
+                                                        pos_offset=5, lib=olib)[0]))
+    eps = 1e-5
+    for grad, which in ((dQ, 0), (dK, 1), (dV, 2)):
+        for _ in range(3):
+            args = [Q, K, V]
+            d = rng.standard_normal(args[which].shape)
+            plus = list(args); plus[which] = args[which] + eps * d
+            minus = list(args); minus[which] = args[which] - eps * d
+            fd = (f(*plus) - f(*minus)) / (2 * eps)
+            assert abs(fd - float(np.sum(grad * d))) <= 1e-6 * max(1.0, abs(fd)), which
