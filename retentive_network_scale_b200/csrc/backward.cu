@@ -176,11 +176,12 @@ cudaError_t product(const Params &base, int dqk, int dval, const void *q, const 
     p.dk = dqk;
     p.dv = dval;
     p.rotate = 0;  // the operands come turned already
+    // only K~ is written: the query rows are read in place through `qk`
     const void *qh = nullptr, *kt = nullptr;
-    cudaError_t e = launch_chunkwise_prep_strided(p, 128, q, k, qk, true, prep_ws, &qh, &kt, st);
+    cudaError_t e = launch_chunkwise_prep_strided(p, 128, q, k, qk, false, prep_ws, &qh, &kt, st);
     if (e != cudaSuccess) return e;
-    return launch_chunkwise_tc_prepared(p, false, qh, kt, v, bhld_layout(p, dval), true, nullptr,
-                                        RowLayout{0, 0, 0}, nullptr, out, 0.f, status, st);
+    return launch_chunkwise_tc_prepared(p, false, qh, qk, kt, v, bhld_layout(p, dval), true,
+                                        nullptr, RowLayout{0, 0, 0}, nullptr, out, 0.f, status, st);
 }
 
 bool dims_ok(const ret_desc *d) {

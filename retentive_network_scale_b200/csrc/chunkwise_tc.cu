@@ -114,11 +114,6 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-    __half2 v = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
 __device__ __forceinline__ float2 unpack_h2(uint32_t u) {
     return __half22float2(*reinterpret_cast<__half2 *>(&u));
 }
@@ -191,7 +186,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     constexpr int NCH = DK / 8;         // 16-byte chunks per Q/K row
     constexpr int RGA = DK / 64;        // 32-column groups per thread in the state pass (group A)
     constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V^T K~ (both MN-major)
-    constexpr bool kStage = sizeof(TO) == 2;  // bf16 tiles leave by TMA store
+    constexpr bool kStage = sizeof(TO) == 2;  // bf16 Y tiles leave by TMA store (O: always)
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -453,7 +448,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // tile (their last use of it; the products finished before the loop
         // barrier)
         if (alive && tid == kGroup && c > 0) {
-            if constexpr (kStage) bulk_wait_read();
+            bulk_wait_read();
             load_v(c);
         }
 
@@ -612,7 +607,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             alive = gsync_alive();
             tc_fence_after();
             const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite
-            const size_t orow = ((size_t)bh * L + t0 + row) * dv + v0 + o0;
             // 32 columns of O'' (still in tensor memory until this iteration ends)
             auto ld_o = [&](int half, float *x) {
                 uint32_t a[32];
@@ -650,18 +644,40 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             };
             // O = alpha O'' (staged tile or direct stores)
             auto emit_o = [&]() {
+                if constexpr (sizeof(TO) == 2) {
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float x[32];
-                    ld_o(half, x);
+                    for (int half = 0; half < 2; ++half) {
+                        float x[32];
+                        ld_o(half, x);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] *= alpha;
-                    if constexpr (kStage)
+                        for (int i = 0; i < 32; ++i) x[i] *= alpha;
                         stage32(half, x);
-                    else if (row < n)
-                        st_row32<TO>(O + orow + 32 * half, x);
+                    }
+                    store_tile(&tmO, v0, t0, bh, false);
+                } else {
+                    // fp32: two rounds of 32 columns per warpgroup (128-byte
+                    // rows, one 16 KB box per warpgroup) through the V tile
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float x[32];
+                        ld_o(half, x);
+                        uint8_t *dst = smem + Ly::kV + gwg * 16384 + row * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<float4 *>(dst + ((q ^ (row & 7)) << 4)) =
+                                make_float4(x[4 * q] * alpha, x[4 * q + 1] * alpha,
+                                            x[4 * q + 2] * alpha, x[4 * q + 3] * alpha);
+                        fence_proxy_async_smem();
+                        named_sync(2, kGroup);
+                        if (g_leader) {
+                            tma_store_3d(&tmO, sbase + Ly::kV, v0 + 32 * half, t0, bh);
+                            tma_store_3d(&tmO, sbase + Ly::kV + 16384, v0 + 64 + 32 * half, t0, bh);
+                            bulk_commit();
+                            if (half == 0) bulk_wait_read();
+                        }
+                        if (half == 0) named_sync(2, kGroup);
+                    }
                 }
-                if constexpr (kStage) store_tile(&tmO, v0, t0, bh, false);
             };
             // the products have read V (the state update is the last)
             auto v_free = [&]() {
@@ -669,7 +685,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 alive = gsync_alive();
             };
             if constexpr (!FUSE) {
-                if constexpr (kStage) v_free();
+                v_free();
                 if (alive) emit_o();
             } else {
                 const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
@@ -833,6 +849,8 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     if (sizeof(TO) == 2) {
         if (O && !make_tma_map_bf16(&mo, O, p.dv, p.L, p.B * p.H, kC)) return cudaErrorInvalidValue;
         if (Y && !make_tma_map_bf16(&my, Y, p.H * p.dv, p.L, p.B, kC)) return cudaErrorInvalidValue;
+    } else if (O && !make_tma_map_f32(&mo, O, p.dv, p.L, p.B * p.H, kC)) {
+        return cudaErrorInvalidValue;
     }
     if (G && !make_tma_map_bf16_strided(&mg, G, p.H * p.dv, p.L, p.B, vw.g.row, vw.g.batch, kC))
         return cudaErrorInvalidValue;
@@ -908,13 +926,14 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
 }
 
 cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
-                                         const void *Kt, const void *V, RowLayout v_layout,
-                                         bool v_head_major, const void *G, RowLayout g_layout,
-                                         void *Y, void *O, float eps, int *status,
-                                         cudaStream_t st) {
+                                         RowLayout q_layout, const void *Kt, const void *V,
+                                         RowLayout v_layout, bool v_head_major, const void *G,
+                                         RowLayout g_layout, void *Y, void *O, float eps,
+                                         int *status, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
-    if (!make_tma_map_bf16(&mq, Qh, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kC))
+    if (!make_tma_map_bf16_strided(&mq, Qh, p.dk, p.L, bh, q_layout.row, q_layout.head, kC) ||
+        !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kC))
         return cudaErrorInvalidValue;
     const bool ok = v_head_major
                         ? make_tma_map_bf16_strided(&mv, V, p.dv, p.L, bh, v_layout.row, v_layout.head, kC)

@@ -44,6 +44,10 @@ cudaError_t launch_chunkwise_prep(const Params &p, int chunk, const void *Q, con
 // Tensor map over [outer][rows][inner] bf16 with boxes of 64 x box_rows x 1
 // and 128-byte swizzle; rows past the end read as zeros and are not written.
 bool make_tma_map_bf16(CUtensorMap *m, const void *base, int inner, int rows, int outer, int box_rows);
+// fp32 tensor map over [outer][rows][inner] with boxes of 32 x box_rows x 1
+// (128-byte rows, 128-byte swizzle).
+bool make_tma_map_f32(CUtensorMap *m, const void *base, int inner, int rows, int outer,
+                      int box_rows);
 // The same over a strided view: row_stride / outer_stride in elements
 // (multiples of 8, i.e. 16 bytes).
 bool make_tma_map_bf16_strided(CUtensorMap *m, const void *base, int inner, int rows, int outer,
@@ -59,15 +63,17 @@ inline RowLayout bhld_layout(const Params &p, int d) {
     return RowLayout{d, (long long)p.L * d, (long long)p.H * p.L * d};
 }
 
-// Tensor-core chunkwise kernel on rows already prepared ([B][H][L][d_k]
-// Q^ and K~), V and G read through the given layouts (V as [B][H][L][d_v]
-// when v_head_major, else as rows of H*d_v columns like G); writes Y
-// ([B][L][H*d_v], with G) and/or O ([B][H][L][d_v]) in the output dtype.
+// Tensor-core chunkwise kernel on rows already prepared: Q^ read through
+// `q_layout` (head-major; its batch stride must be H times its head
+// stride), K~ as [B][H][L][d_k], V and G through the given layouts (V as
+// head-major rows when v_head_major, else as rows of H*d_v columns like G);
+// writes Y ([B][L][H*d_v], with G) and/or O ([B][H][L][d_v]) in the output
+// dtype.
 cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,
-                                         const void *Kt, const void *V, RowLayout v_layout,
-                                         bool v_head_major, const void *G, RowLayout g_layout,
-                                         void *Y, void *O, float eps, int *status,
-                                         cudaStream_t st);
+                                         RowLayout q_layout, const void *Kt, const void *V,
+                                         RowLayout v_layout, bool v_head_major, const void *G,
+                                         RowLayout g_layout, void *Y, void *O, float eps,
+                                         int *status, cudaStream_t st);
 // The streaming pass reading Q and K through a layout; with always_q it
 // writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),
 // so the workspace holds 2*B*H*L*d_k values.

@@ -131,7 +131,8 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
     // 3. the chunk loop with the fused GroupNorm + gate; V and G are read as
     //    rows of H d_v columns of the projection
     const ret::RowLayout vg{z.n_proj, 0, (long long)desc->L * z.n_proj};
-    e = ret::launch_chunkwise_tc_prepared(p, true, qh, kt, P + 2 * (size_t)H * dk, vg, false,
+    e = ret::launch_chunkwise_tc_prepared(p, true, qh, ret::bhld_layout(p, dk), kt,
+                                          P + 2 * (size_t)H * dk, vg, false,
                                           P + 2 * (size_t)H * dk + (size_t)H * dv, vg,
                                           ws + z.off_y, nullptr, gn_eps, status, st);
     if (e != cudaSuccess) return RET_ERR_CUDA;

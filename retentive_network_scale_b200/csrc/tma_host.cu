@@ -31,6 +31,19 @@ bool make_tma_map_bf16(CUtensorMap *m, const void *base, int inner, int rows, in
                                      box_rows);
 }
 
+bool make_tma_map_f32(CUtensorMap *m, const void *base, int inner, int rows, int outer,
+                      int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * 4, (cuuint64_t)rows * inner * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tma_map_bf16_strided(CUtensorMap *m, const void *base, int inner, int rows, int outer,
                                long long row_stride, long long outer_stride, int box_rows) {
     EncodeTiledFn fn = encode_fn();
