@@ -34,10 +34,11 @@
 // form a cluster along d_v; each reduces its 128 columns of a row to a mean
 // and centred sum of squares, the partials are exchanged through
 // distributed shared memory and merged (Chan's pairwise update), and every
-// CTA normalises and gates its own columns.  The G tile lands in the Rbar^T
-// blocks 0,1 (free between the O'' product and the state pass); the gate
-// factors are computed into registers while the peers publish, and Y leaves
-// through the V tile and a TMA store.
+// CTA normalises and gates its own columns.  The G tile lands in the Q^
+// blocks 0,1 (free once the O'' product is done; the next chunk's blocks
+// 0,1 are loaded after the gate pass), the gate factors are computed into
+// registers between arriving at the exchange barrier and waiting on it, and
+// Y leaves through the V tile and a TMA store.
 //
 // Every mbarrier wait is bounded: on expiry the kernel latches
 // RET_ERR_TIMEOUT in the device status word and every thread skips the
@@ -45,7 +46,6 @@
 // cluster is left waiting), in-flight copies and MMAs get a bounded drain,
 // and TMEM is freed.
 #include <cuda.h>
-#include <cuda_fp16.h>
 
 #include <cstring>
 
@@ -114,8 +114,24 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
 }
 
-__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
-    return __half22float2(*reinterpret_cast<__half2 *>(&u));
+// a bf16 pair as a packed fp32 pair (lo, hi): the bf16 bits are the top
+// half of each fp32
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t u) {
+    return (static_cast<uint64_t>(u & 0xffff0000u) << 32) | (u << 16);
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_of(const uint32_t *r) {
+    return (static_cast<uint64_t>(r[1]) << 32) | r[0];
+}
+
+__device__ __forceinline__ uint32_t pack_f2_bf16(uint64_t v) {
+    return pack_bf16(f2_lo(v), f2_hi(v));
 }
 
 // Row c of Rbar^T (K-major, 128-byte swizzle, inside the interleaved K^ /
@@ -156,19 +172,17 @@ __device__ __forceinline__ void st_row32<__nv_bfloat16>(__nv_bfloat16 *dst, cons
     }
 }
 
-// swish(g) = g sigmoid(g) for a pair, in fp16x2: h = g/2, sigmoid(g) =
-// (1 + tanh(h)) / 2 with the hardware's fp16x2 tanh approximation (one
-// special-function operation per pair; absolute error of sigmoid near
-// 2^-11), swish = 2h sigmoid.  fp16 holds |g| up to 65504 (beyond, swish
-// becomes infinite; for g below about -20 it is exactly 0).
-__device__ __forceinline__ uint32_t swish_pair_h2(float2 g) {
-    const __half2 h = __floats2half2_rn(0.5f * g.x, 0.5f * g.y);
-    uint32_t t;
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(*reinterpret_cast<const uint32_t *>(&h)));
-    const __half2 half2 = __float2half2_rn(0.5f);
-    const __half2 sig = __hfma2(*reinterpret_cast<const __half2 *>(&t), half2, half2);
-    const __half2 sw = __hmul2(__hadd2(h, h), sig);
-    return *reinterpret_cast<const uint32_t *>(&sw);
+// swish(g) = g sigmoid(g) = h + h tanh(h), h = g / 2, for a bf16 pair:
+// halving is exact, the hardware's bf16x2 tanh approximation is the one
+// special-function operation, and a fused multiply-add rounds the result
+// once to bf16.  The gate factor then carries a relative error of a few
+// bf16 units, next to the one rounding of Y itself to bf16.
+__device__ __forceinline__ uint32_t swish_bf16x2(uint32_t g) {
+    uint32_t h, t, s;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(h) : "r"(g), "r"(0x3f003f00u));  // (0.5, 0.5)
+    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(s) : "r"(h), "r"(t), "r"(h));
+    return s;
 }
 
 template <int DK, typename TO, bool FUSE>
@@ -250,12 +264,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int nb = 0; nb < 2; ++nb)
             tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), vx0 + nb * 64, c * kC, vz);
     };
-    // the G tile of chunk c into the Rbar^T blocks 0,1 (free from the O''
-    // product until the state pass writes the next Rbar)
+    // the G tile of chunk c into the Q^ blocks 0,1 (free once the O''
+    // product is done; the next chunk's blocks 0,1 follow the gate pass)
     auto load_g = [&](int c) {
         mbar_expect_tx(bar(BG), Ly::kVBytes);
         for (int nb = 0; nb < 2; ++nb)
-            tma_load_3d(sbase + Ly::rbar_blk(nb), &tmG, bar(BG), h * dv + v0 + nb * 64, c * kC, b);
+            tma_load_3d(sbase + Ly::kQ + nb * 16384, &tmG, bar(BG), h * dv + v0 + nb * 64, c * kC, b);
     };
     // every tile chunk c will load, into L2 ahead of time (the Q^ and K~
     // blocks, which every CTA of the head loads, shared out among them)
@@ -520,12 +534,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         alive = *abort_flag == 0;
 
-        // Q^ and Rbar are no longer read once O'' is done: G into the Rbar
-        // blocks 0,1, the next Q^ (thread 32, while thread 0 issues products)
+        // Q^ and Rbar are no longer read once O'' is done: the next Q^ (with
+        // the gate, G takes blocks 0,1 first), by thread 32 while thread 0
+        // issues products
         if (alive && tid == 32 && wait_bar(bar(BS), par, abort_flag, status)) {
             if constexpr (FUSE) load_g(c);
             if (!last) {
-                load_q_lo(c + 1);
+                if constexpr (!FUSE) load_q_lo(c + 1);
                 load_q_hi(c + 1);
             }
         }
@@ -547,14 +562,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
 
         if (grp == 0) {
-            // ================= group A: gate factors, state pass, then the next Q^
+            // ================= group A: state pass, then (rows not prepared) the next Q^
             if constexpr (FUSE) cluster_arrive();   // GroupNorm exchange barrier
             if (alive && tid == 0) {
                 wait_bar(bar(BU), par, abort_flag, status);
                 if (!last) load_k(c + 1);  // K~ is no longer read
             }
-            // group B has taken the G tile out of the Rbar blocks
-            if constexpr (FUSE) named_sync(3, kThreads);
             alive = gsync_alive();
             tc_fence_after();
             if (alive) {
@@ -563,8 +576,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // R^T columns [d0, d0+32): decay, bf16 copy, back to TMEM; or state_out
                 auto state32 = [&](uint32_t (&r)[32], int d0) {
                     float v[32];
+                    const uint64_t G2 = f2_make(gnext, gnext);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gnext;
+                    for (int i = 0; i < 32; i += 2) {
+                        const uint64_t x = f2_mul(f2_of(r + i), G2);
+                        v[i] = f2_lo(x);
+                        v[i + 1] = f2_hi(x);
+                    }
                     if (last) {
                         if (state_out) {
 #pragma unroll
@@ -691,8 +709,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const int nr = (int)gridDim.x;        // CTAs of this head = cluster size
                 // Mean and centred sum of squares of this thread's 64 columns
                 // in one pass, shifted by its first value (no cancellation
-                // unless the mean sits many deviations from that sample).
-                float s1 = 0.f, s2 = 0.f, shift = 0.f;
+                // unless the mean sits many deviations from that sample);
+                // even and odd columns in the two lanes of packed fp32 pairs.
+                uint64_t S1 = 0, S2 = 0;
+                float shift = 0.f;
                 if (alive) {
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
@@ -700,14 +720,16 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         tmem_ld32(tO + lane_base + o0 + 32 * half, a);
                         tmem_wait_ld(a);
                         if (half == 0) shift = __uint_as_float(a[0]);
+                        const uint64_t NSH = f2_make(-shift, -shift);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float d = __uint_as_float(a[i]) - shift;
-                            s1 += d;
-                            s2 = fmaf(d, d, s2);
+                        for (int i = 0; i < 32; i += 2) {
+                            const uint64_t d = f2_add(f2_of(a + i), NSH);
+                            S1 = f2_add(S1, d);
+                            S2 = f2_fma(d, d, S2);
                         }
                     }
                 }
+                const float s1 = f2_lo(S1) + f2_hi(S1), s2 = f2_lo(S2) + f2_hi(S2);
                 const float m_w = shift + s1 * (1.f / 64.f);
                 const float m2_w = fmaxf(s2 - s1 * s1 * (1.f / 64.f), 0.f);
                 // The two warpgroups' halves merge (Chan's pairwise update,
@@ -724,34 +746,36 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const float d = m_w - o.x;
                     *slot = make_float2(0.5f * (m_w + o.x), m2_w + o.y + 32.f * d * d);
                 }
+                // swish(G) of this thread's 64 columns (bf16 pairs in
+                // registers) from the G tile in the Q^ blocks 0,1 while the
+                // peers reach the exchange barrier
                 cluster_arrive();
+                uint32_t sw[32];
+                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
+                alive = gsync_alive();
+                if (alive) {
+                    const uint8_t *gt = smem + Ly::kQ + gwg * 16384 + row * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(gt + ((q ^ (row & 7)) << 4));
+                        sw[4 * q + 0] = swish_bf16x2(w.x);
+                        sw[4 * q + 1] = swish_bf16x2(w.y);
+                        sw[4 * q + 2] = swish_bf16x2(w.z);
+                        sw[4 * q + 3] = swish_bf16x2(w.w);
+                    }
+                }
+                // the whole group has read G: the next Q^ blocks 0,1
+                alive = gsync_alive();
+                if (alive && g_leader && !last) load_q_lo(c + 1);
                 cluster_wait();
                 // the peers' partials (distributed shared memory), in flight
-                // while the gate factors are computed
+                // while the group waits for the products to release V
                 float2 e[kMaxCluster];
                 if (alive) {
 #pragma unroll
                     for (int r = 0; r < kMaxCluster; ++r)
                         if (r < nr) e[r] = ld_cluster_f32x2(map_to_rank(own, r));
                 }
-                // swish(G) of this thread's 64 columns (fp16 pairs in
-                // registers) from the G tile in the Rbar blocks, which then go
-                // back to the state pass
-                uint32_t sw[32];
-                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
-                alive = gsync_alive();
-                if (alive) {
-                    const uint8_t *gt = smem + Ly::rbar_blk(gwg) + row * 128;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(gt + ((q ^ (row & 7)) << 4));
-                        sw[4 * q + 0] = swish_pair_h2(unpack_bf16(w.x));
-                        sw[4 * q + 1] = swish_pair_h2(unpack_bf16(w.y));
-                        sw[4 * q + 2] = swish_pair_h2(unpack_bf16(w.z));
-                        sw[4 * q + 3] = swish_pair_h2(unpack_bf16(w.w));
-                    }
-                }
-                named_arrive(3, kThreads);
                 v_free();
                 if (alive) {
                     uint32_t a[32];
@@ -766,6 +790,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         if (r < nr) m2 += e[r].y + (float)kTV * (e[r].x - mean) * (e[r].x - mean);
                     const float var = m2 / (float)(nr * kTV);  // of O'' ; O = alpha O''
                     const float scale = alpha * rsqrtf(alpha * alpha * var + gn_eps);
+                    // (x - mean) scale as one fused multiply-add per pair
+                    const uint64_t SC = f2_make(scale, scale);
+                    const uint64_t NMS = f2_make(-mean * scale, -mean * scale);
                     // Y into the V tile
                     uint8_t *tile = smem + Ly::kV + gwg * 16384 + row * 128;
 #pragma unroll
@@ -774,16 +801,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         tmem_wait_ld(a);
                         float x[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
+                        for (int k = 0; k < 16; ++k) {
+                            const uint64_t y = f2_mul(f2_fma(f2_of(a + 2 * k), SC, NMS),
+                                                      bf16x2_to_f2(sw[16 * half + k]));
+                            x[2 * k] = f2_lo(y);
+                            x[2 * k + 1] = f2_hi(y);
+                        }
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 f = unpack_h2(sw[4 * (4 * half + q) + e2]);
-                                const int i = 8 * q + 2 * e2;
-                                x[i] = f.x * ((x[i] - mean) * scale);
-                                x[i + 1] = f.y * ((x[i + 1] - mean) * scale);
-                            }
                             if constexpr (kStage) {
                                 uint4 w;
                                 w.x = pack_bf16(x[8 * q + 0], x[8 * q + 1]);
