@@ -35,6 +35,11 @@ template <typename TI, bool ROT>
 __global__ void __launch_bounds__(kThreads)
 flip_turn_kernel(const Params p, int d, long long items, const TI *__restrict__ x,
                  __nv_bfloat16 *__restrict__ y, int flip) {
+    __shared__ double s_theta[kMaxDk / 2];
+    if constexpr (ROT) {
+        stage_theta(p, s_theta, d / 2);
+        __syncthreads();
+    }
     const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
     const int n8 = d / 8;
@@ -49,7 +54,7 @@ flip_turn_kernel(const Params p, int d, long long items, const TI *__restrict__ 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             float c, s;
-            rot_cs(p.pos_offset + t, p.theta[c8 * 4 + e], &c, &s);
+            rot_cs(p.pos_offset + t, s_theta[c8 * 4 + e], &c, &s);
             rot_pair(v[2 * e], v[2 * e + 1], c, s);
         }
     }
@@ -69,6 +74,11 @@ template <typename TO, bool ROT>
 __global__ void __launch_bounds__(kThreads)
 unturn_sum_kernel(const Params p, int d, long long items, const float *__restrict__ part0,
                   const float *__restrict__ part1, int flip, TO *__restrict__ out) {
+    __shared__ double s_theta[kMaxDk / 2];
+    if constexpr (ROT) {
+        stage_theta(p, s_theta, d / 2);
+        __syncthreads();
+    }
     const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
     const int n8 = d / 8;
@@ -89,7 +99,7 @@ unturn_sum_kernel(const Params p, int d, long long items, const float *__restric
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             float c, s;
-            rot_cs(p.pos_offset + t, p.theta[c8 * 4 + e], &c, &s);
+            rot_cs(p.pos_offset + t, s_theta[c8 * 4 + e], &c, &s);
             rot_pair(v[2 * e], v[2 * e + 1], c, -s);  // Theta_t^T: the opposite turn
         }
     }

@@ -130,10 +130,6 @@ __device__ __forceinline__ uint64_t f2_of(const uint32_t *r) {
     return (static_cast<uint64_t>(r[1]) << 32) | r[0];
 }
 
-__device__ __forceinline__ uint32_t pack_f2_bf16(uint64_t v) {
-    return pack_bf16(f2_lo(v), f2_hi(v));
-}
-
 // Row c of Rbar^T (K-major, 128-byte swizzle, inside the interleaved K^ /
 // Rbar^T blocks): the 32 values of d-columns [d0, d0+32).
 template <int DK>

@@ -39,6 +39,15 @@ __device__ __forceinline__ float decay_pow(float log2g, int n) {
     return n == 0 ? 1.0f : exp2f((float)n * log2g);
 }
 
+// theta_0 .. theta_{n-1} into shared memory, by all threads of the block
+// (the caller synchronises).  Kernel parameters are read through the
+// constant cache, which serves one address per request: a per-thread index
+// into Params::theta would be serialised across the warp, a shared-memory
+// table is not.
+__device__ __forceinline__ void stage_theta(const Params &p, double *s_theta, int n) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_theta[i] = p.theta[i];
+}
+
 // cos and sin of pos * theta.  The product and its reduction to
 // [-pi, pi] are done in fp64 so that positions of 10^5 and more keep full
 // fp32 accuracy; the reduced angle then goes to sincosf.

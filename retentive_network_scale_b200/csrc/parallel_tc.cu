@@ -262,6 +262,9 @@ template <typename TI>
 __global__ void __launch_bounds__(256)
 xpos_rotate_kernel(Params p, long long rows, const TI *__restrict__ x, __nv_bfloat16 *__restrict__ y) {
     constexpr int kRowsPerThread = 16;
+    __shared__ double s_theta[kMaxDk / 2];
+    stage_theta(p, s_theta, p.dk / 2);
+    __syncthreads();
     const int nch = p.dk / 8;
     const long long items = (rows + kRowsPerThread - 1) / kRowsPerThread * nch;
     for (long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x; item < items;
@@ -271,7 +274,7 @@ xpos_rotate_kernel(Params p, long long rows, const TI *__restrict__ x, __nv_bflo
         float c[4], s[4], sc[4], ss[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const double th = p.theta[c16 * 4 + e];
+            const double th = s_theta[c16 * 4 + e];
             rot_cs(p.pos_offset + r0 % p.L, th, &c[e], &s[e]);
             rot_cs(1, th, &sc[e], &ss[e]);
         }
@@ -279,7 +282,7 @@ xpos_rotate_kernel(Params p, long long rows, const TI *__restrict__ x, __nv_bflo
             const long long r = r0 + k;
             if (k > 0 && r % p.L == 0) {  // a new (b,h) slice starts: restart the angles
 #pragma unroll
-                for (int e = 0; e < 4; ++e) rot_cs(p.pos_offset, p.theta[c16 * 4 + e], &c[e], &s[e]);
+                for (int e = 0; e < 4; ++e) rot_cs(p.pos_offset, s_theta[c16 * 4 + e], &c[e], &s[e]);
             }
             const size_t base = (size_t)r * p.dk + c16 * 8;
             uint4 out;

@@ -55,6 +55,11 @@ __global__ void __launch_bounds__(kThreads, 4)
 chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat16 *__restrict__ Q,
                   const __nv_bfloat16 *__restrict__ K, RowLayout src, __nv_bfloat16 *__restrict__ qh,
                   __nv_bfloat16 *__restrict__ kt) {
+    __shared__ double s_theta[kMaxDk / 2];
+    if constexpr (ROT) {
+        stage_theta(p, s_theta, p.dk / 2);
+        __syncthreads();
+    }
     const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
     const int nch = p.dk / 8;
@@ -80,7 +85,7 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
     if constexpr (ROT) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const double th = p.theta[c16 * 4 + e];
+            const double th = s_theta[c16 * 4 + e];
             rot_cs_fast(p.pos_offset + t0, th, &c[e], &s[e]);
             __sincosf((float)th, &ss[e], &cs[e]);  // theta_j <= 1
         }
