@@ -27,37 +27,112 @@ namespace ret {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kRows = 4;  // consecutive rows per thread in the copy passes
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float4 ld_stream_f4(const float *p) {
+    const uint4 u = ld_stream(p);
+    return make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                       __uint_as_float(u.w));
+}
+
+// One copy-pass work item: the 8-column chunk c8 of rows t0 .. t0+nr-1 of
+// slice bh.  Items run chunk-fastest, so a warp reads whole rows.
+struct CopyItem {
+    int c8, t0, nr;
+    long long bh;
+};
+
+__device__ __forceinline__ bool copy_item(const Params &p, int d, long long items, CopyItem *it) {
+    const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= items) return false;
+    const int n8 = d / 8;
+    const int tiles = (p.L + kRows - 1) / kRows;
+    it->c8 = (int)(item % n8);
+    const long long rest = item / n8;
+    it->t0 = (int)(rest % tiles) * kRows;
+    it->bh = rest / tiles;
+    it->nr = min(kRows, p.L - it->t0);
+    return true;
+}
+
+// Angles of the four pairs of chunk c8 at position pos, and the per-row
+// step theta_j: the first exact (fp64 reduction), the rest by rotation.
+__device__ __forceinline__ void chunk_angles(const double *s_theta, int c8, long long pos, float *c,
+                                             float *s, float *cs, float *ss) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const double th = s_theta[c8 * 4 + e];
+        rot_cs_fast(pos, th, &c[e], &s[e]);
+        __sincosf((float)th, &ss[e], &cs[e]);  // theta_j <= 1
+    }
+}
+
+__device__ __forceinline__ void step_angles(float *c, float *s, const float *cs, const float *ss) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float cn = c[e] * cs[e] - s[e] * ss[e];
+        s[e] = c[e] * ss[e] + s[e] * cs[e];
+        c[e] = cn;
+    }
+}
 
 // y (bf16, [B][H][L][d]) = x turned by the angle of row t's own position
-// (ROT) and written at row t or, when `flip`, at row L-1-t.  One thread:
-// 8 consecutive elements (4 pairs) of one row.
-template <typename TI, bool ROT>
-__global__ void __launch_bounds__(kThreads)
-flip_turn_kernel(const Params p, int d, long long items, const TI *__restrict__ x,
+// (ROT) and written at row t or, when `flip`, at row L-1-t.
+template <bool ROT>
+__global__ void __launch_bounds__(kThreads, 4)
+flip_turn_kernel(const Params p, int d, long long items, const __nv_bfloat16 *__restrict__ x,
                  __nv_bfloat16 *__restrict__ y, int flip) {
     __shared__ double s_theta[kMaxDk / 2];
     if constexpr (ROT) {
         stage_theta(p, s_theta, d / 2);
         __syncthreads();
     }
-    const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
-    if (item >= items) return;
-    const int n8 = d / 8;
-    const long long r = item / n8;
-    const int c8 = (int)(item - r * n8);
-    const int t = (int)(r % p.L);
-    const long long rdst = flip ? r - t + (p.L - 1 - t) : r;
-    float v[8];
+    CopyItem it;
+    if (!copy_item(p, d, items, &it)) return;
+    const size_t base = (size_t)it.bh * p.L * d + (size_t)it.c8 * 8;
+    uint4 w[kRows];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = ld(x, (size_t)r * d + c8 * 8 + e);
-    if constexpr (ROT) {
+    for (int r = 0; r < kRows; ++r)
+        if (r < it.nr) w[r] = ld_stream(x + base + (size_t)(it.t0 + r) * d);
+    float c[4], s[4], cs[4], ss[4];
+    if constexpr (ROT) chunk_angles(s_theta, it.c8, p.pos_offset + it.t0, c, s, cs, ss);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float c, s;
-            rot_cs(p.pos_offset + t, s_theta[c8 * 4 + e], &c, &s);
-            rot_pair(v[2 * e], v[2 * e + 1], c, s);
+    for (int r = 0; r < kRows; ++r) {
+        if (r < it.nr) {
+            if constexpr (ROT) {
+                uint32_t *u = reinterpret_cast<uint32_t *>(&w[r]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 v = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u[e]));
+                    rot_pair(v.x, v.y, c[e], s[e]);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v.x, v.y);
+                    u[e] = *reinterpret_cast<uint32_t *>(&b2);
+                }
+                step_angles(c, s, cs, ss);
+            }
+            const int t = it.t0 + r;
+            *reinterpret_cast<uint4 *>(y + base + (size_t)(flip ? p.L - 1 - t : t) * d) = w[r];
         }
     }
+}
+
+template <typename TO>
+__device__ __forceinline__ void st8(TO *dst, const float *v);
+template <>
+__device__ __forceinline__ void st8<float>(float *dst, const float *v) {
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <>
+__device__ __forceinline__ void st8<__nv_bfloat16>(__nv_bfloat16 *dst, const float *v) {
     uint4 w;
     uint32_t *u = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
@@ -65,13 +140,13 @@ flip_turn_kernel(const Params p, int d, long long items, const TI *__restrict__ 
         __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
         u[e] = *reinterpret_cast<uint32_t *>(&b2);
     }
-    *reinterpret_cast<uint4 *>(y + (size_t)rdst * d + c8 * 8) = w;
+    *reinterpret_cast<uint4 *>(dst) = w;
 }
 
 // out row t = the sum of the fp32 partials at row t (or L-1-t when `flip`),
 // turned back by the angle of position pos_offset + t (ROT).
 template <typename TO, bool ROT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 unturn_sum_kernel(const Params p, int d, long long items, const float *__restrict__ part0,
                   const float *__restrict__ part1, int flip, TO *__restrict__ out) {
     __shared__ double s_theta[kMaxDk / 2];
@@ -79,32 +154,40 @@ unturn_sum_kernel(const Params p, int d, long long items, const float *__restric
         stage_theta(p, s_theta, d / 2);
         __syncthreads();
     }
-    const long long item = (long long)blockIdx.x * kThreads + threadIdx.x;
-    if (item >= items) return;
-    const int n8 = d / 8;
-    const long long r = item / n8;
-    const int c8 = (int)(item - r * n8);
-    const int t = (int)(r % p.L);
-    const long long rsrc = flip ? r - t + (p.L - 1 - t) : r;
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < 2; ++k) {
-        const float *part = k == 0 ? part0 : part1;
-        if (!part) continue;
-        const float4 a = *reinterpret_cast<const float4 *>(part + (size_t)rsrc * d + c8 * 8);
-        const float4 b = *reinterpret_cast<const float4 *>(part + (size_t)rsrc * d + c8 * 8 + 4);
-        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-    }
-    if constexpr (ROT) {
+    CopyItem it;
+    if (!copy_item(p, d, items, &it)) return;
+    const size_t base = (size_t)it.bh * p.L * d + (size_t)it.c8 * 8;
+    float4 a[kRows][2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float c, s;
-            rot_cs(p.pos_offset + t, s_theta[c8 * 4 + e], &c, &s);
-            rot_pair(v[2 * e], v[2 * e + 1], c, -s);  // Theta_t^T: the opposite turn
+    for (int r = 0; r < kRows; ++r) {
+        if (r < it.nr) {
+            const int t = it.t0 + r;
+            const size_t src = base + (size_t)(flip ? p.L - 1 - t : t) * d;
+            a[r][0] = ld_stream_f4(part0 + src);
+            a[r][1] = ld_stream_f4(part0 + src + 4);
+            if (part1) {
+                const float4 b0 = ld_stream_f4(part1 + src), b1 = ld_stream_f4(part1 + src + 4);
+                a[r][0].x += b0.x; a[r][0].y += b0.y; a[r][0].z += b0.z; a[r][0].w += b0.w;
+                a[r][1].x += b1.x; a[r][1].y += b1.y; a[r][1].z += b1.z; a[r][1].w += b1.w;
+            }
         }
     }
+    float c[4], s[4], cs[4], ss[4];
+    if constexpr (ROT) chunk_angles(s_theta, it.c8, p.pos_offset + it.t0, c, s, cs, ss);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) st(out, (size_t)r * d + c8 * 8 + e, v[e]);
+    for (int r = 0; r < kRows; ++r) {
+        if (r < it.nr) {
+            float v[8] = {a[r][0].x, a[r][0].y, a[r][0].z, a[r][0].w,
+                          a[r][1].x, a[r][1].y, a[r][1].z, a[r][1].w};
+            if constexpr (ROT) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    rot_pair(v[2 * e], v[2 * e + 1], c[e], -s[e]);  // Theta_t^T: the opposite turn
+                step_angles(c, s, cs, ss);
+            }
+            st8<TO>(out + base + (size_t)(it.t0 + r) * d, v);
+        }
+    }
 }
 
 constexpr size_t kAlign = 256;
@@ -143,17 +226,20 @@ BwdLayout bwd_layout(const ret_desc *d) {
     return z;
 }
 
-template <typename TI>
+long long copy_items(const Params &p, int d) {
+    return (long long)p.B * p.H * ((p.L + kRows - 1) / kRows) * (d / 8);
+}
+
 cudaError_t flip_turn(const Params &p, int d, const void *x, void *y, bool rot, bool flip,
                       cudaStream_t st) {
-    const long long items = (long long)p.B * p.H * p.L * (d / 8);
+    const long long items = copy_items(p, d);
     const long long blocks = (items + kThreads - 1) / kThreads;
+    const auto *xs = static_cast<const __nv_bfloat16 *>(x);
+    auto *yd = static_cast<__nv_bfloat16 *>(y);
     if (rot)
-        flip_turn_kernel<TI, true><<<(unsigned)blocks, kThreads, 0, st>>>(
-            p, d, items, static_cast<const TI *>(x), static_cast<__nv_bfloat16 *>(y), flip);
+        flip_turn_kernel<true><<<(unsigned)blocks, kThreads, 0, st>>>(p, d, items, xs, yd, flip);
     else
-        flip_turn_kernel<TI, false><<<(unsigned)blocks, kThreads, 0, st>>>(
-            p, d, items, static_cast<const TI *>(x), static_cast<__nv_bfloat16 *>(y), flip);
+        flip_turn_kernel<false><<<(unsigned)blocks, kThreads, 0, st>>>(p, d, items, xs, yd, flip);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) note_launches(1);
     return e;
@@ -163,7 +249,7 @@ cudaError_t flip_turn(const Params &p, int d, const void *x, void *y, bool rot, 
 template <typename TO>
 cudaError_t unturn_sum(const Params &p, int d, const float *part0, const float *part1, bool flip,
                        bool rot, void *out, cudaStream_t st) {
-    const long long items = (long long)p.B * p.H * p.L * (d / 8);
+    const long long items = copy_items(p, d);
     const long long blocks = (items + kThreads - 1) / kThreads;
     if (rot)
         unturn_sum_kernel<TO, true><<<(unsigned)blocks, kThreads, 0, st>>>(p, d, items, part0, part1, flip,
@@ -257,11 +343,11 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
     cudaError_t e = cudaSuccess;
     auto run = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
     // 1. turned and/or time-reversed bf16 copies
-    run(flip_turn<__nv_bfloat16>(p, dk, K, Kh, rot, false, st));
-    run(flip_turn<__nv_bfloat16>(p, dk, Q, Qf, rot, true, st));
-    run(flip_turn<__nv_bfloat16>(p, dk, K, Kf, rot, true, st));
-    run(flip_turn<__nv_bfloat16>(p, dv, V, Vf, false, true, st));
-    run(flip_turn<__nv_bfloat16>(p, dv, dO, Of, false, true, st));
+    run(flip_turn(p, dk, K, Kh, rot, false, st));
+    run(flip_turn(p, dk, Q, Qf, rot, true, st));
+    run(flip_turn(p, dk, K, Kf, rot, true, st));
+    run(flip_turn(p, dv, V, Vf, false, true, st));
+    run(flip_turn(p, dv, dO, Of, false, true, st));
     // 2. dQ^ (causal: dO, V, K^) and reversed dK^ (V, dO, Q^), per column block of d_v
     int w[8];
     const int n = split_dv(dv, w);
