@@ -381,6 +381,39 @@ def bench_backward(R, w, d, pk, reps=3):
                          "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
 
 
+def bench_seqshard(R, w, d, pk, reps=5, parts=8):
+    """What splitting the sequence over ranks adds per rank: the state of
+    a segment from zero (here the whole msr_1p3b sequence as one segment,
+    the most a rank does) and the scan of `parts` gathered states.  The
+    exchange itself needs several GPUs and is not timed here."""
+    g = R.msr_gammas(w.H)
+    U = torch.empty(w.B, w.H, w.d_k, w.d_v, device="cuda")
+    ws = torch.empty(R.lib_segment_state_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, w.rotate),
+                     dtype=torch.uint8, device="cuda")
+    seg = lambda: R.ret_segment_state(d["K"], d["V"], g, U=U, rotate=w.rotate, workspace=ws)  # noqa: E731
+    U_all = torch.randn(parts, w.B, w.H, w.d_k, w.d_v, device="cuda")
+    Rout = torch.empty_like(U)
+    lens = [w.L // parts] * parts
+    scan = lambda: R.ret_state_scan(U_all, lens, parts, g, R=Rout)  # noqa: E731
+    for _ in range(2):
+        seg(); scan()
+    stream = torch.cuda.current_stream()
+    ms_seg = time_launches(seg, reps, stream)
+    ms_scan = time_launches(scan, reps, stream)
+    # K read and K~ written by the streaming pass, K~ and V read and U written by the GEMM
+    rows = w.B * w.H * w.L
+    seg_bytes = rows * w.d_k * 2 * 3 + rows * w.d_v * 2 + w.B * w.H * w.d_k * w.d_v * 4
+    scan_bytes = (parts + 1) * w.B * w.H * w.d_k * w.d_v * 4
+    return {"workload": f"segment state of {w.name} (B={w.B} H={w.H}, {w.L} rows) and the scan of "
+                        f"{parts} gathered states",
+            "segment_state_ms": ms_seg, "state_scan_ms": ms_scan,
+            "roofline": {"bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"],
+                         "segment_state": seg_bytes / (ms_seg * 1e-3) / 1e9,
+                         "segment_state_frac": seg_bytes / (ms_seg * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "state_scan": scan_bytes / (ms_scan * 1e-3) / 1e9,
+                         "state_scan_frac": scan_bytes / (ms_scan * 1e-3) / 1e9 / pk["hbm_gbs"]}}
+
+
 def bench_layer(R, w, pk, reps=5):
     """The whole multi-scale retention layer on the RetNet-1.3B head shape:
     d_model = H*d_k, random bf16 weights (the shapes matter, not the values)."""
@@ -531,6 +564,7 @@ def run_ours(args, world, rank, local):
     if not args.skip_extra:
         extra["parallel"] = bench_parallel(R, w, d, pk)
         extra["backward"] = bench_backward(R, w, d, pk)
+        extra["sequence_shard"] = bench_seqshard(R, w, d, pk)
         del d
         torch.cuda.empty_cache()
         extra["msr_layer"] = bench_layer(R, w, pk)

@@ -290,6 +290,59 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q,
 size_t ret_backward_workspace_size(const ret_desc *desc, int chunk);
 
 /*
+ * ret_segment_state -- the state a segment of a sequence leaves behind when
+ * it starts from a zero state (section 2.1, form (3): the chunkwise state
+ * recurrence holds at any row boundary, so between segments as between
+ * chunks):
+ *     U = sum_{t < L} gamma^{L-1-t} k^_t^T v_t,
+ * k^_t turned at position pos_offset + t.  A segment of L rows that starts
+ * from state R leaves gamma^L R + U.  To split a long sequence over several
+ * devices, each computes the U of its own segment, the U are exchanged (an
+ * all-gather), ret_state_scan gives each segment its entering state, and
+ * ret_chunkwise with that state_in and the segment's pos_offset produces
+ * the segment's outputs.
+ *   K  device bf16 [B][H][L][d_k] (d_k a multiple of 8)
+ *   V  device bf16 [B][H][L][d_v]
+ *   U  device fp32 [B][H][d_k][d_v], fully overwritten (zeros when L = 0)
+ *   workspace  device, 256-byte aligned, at least
+ *              ret_segment_state_workspace_size() bytes
+ * A streaming pass writes the turned, decay-weighted keys into the
+ * workspace; one batched bf16 GEMM with fp32 accumulation (cuBLAS) forms U.
+ * Errors: RET_ERR_NULL, _SHAPE, _DTYPE (bf16 inputs only), _ALIGN, _ARG,
+ * _WORKSPACE, _UNSUPPORTED, _CUDA.
+ */
+ret_status ret_segment_state(const ret_desc *desc, const void *K, const void *V,
+                             float *U, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/* Device workspace bytes ret_segment_state needs; 0 for descriptions it
+ * would reject by their arguments and for empty problems.  Never fails. */
+size_t ret_segment_state_workspace_size(const ret_desc *desc);
+
+#define RET_MAX_SEGMENTS 64  /* segments of one ret_state_scan */
+
+/*
+ * ret_state_scan -- the state entering segment `rank` of a sequence cut
+ * into n_seg consecutive segments of seg_len[0..n_seg-1] rows, from the
+ * segments' own states U_s (ret_segment_state) and the state before the
+ * first segment:
+ *     R_0 = state_in (zero when NULL),  R_{s+1} = gamma^{seg_len[s]} R_s + U_s,
+ * returned for s = rank, 0 <= rank <= n_seg (rank = n_seg: the state after
+ * the whole sequence).  desc supplies B, H, d_k, d_v and gamma (it must
+ * pass the usual checks; its L and dtypes play no part).
+ *   seg_len   HOST array [n_seg], every entry >= 1
+ *   U_all     device fp32 [n_seg][B][H][d_k][d_v]; only segments below
+ *             `rank` are read (may be NULL when rank = 0)
+ *   state_in  device fp32 [B][H][d_k][d_v], or NULL
+ *   R         device fp32 [B][H][d_k][d_v], fully overwritten
+ * Errors: RET_ERR_NULL, _SHAPE (n_seg outside 1..RET_MAX_SEGMENTS, rank
+ * outside 0..n_seg, a seg_len below 1), _ALIGN, _ARG, _UNSUPPORTED, _CUDA.
+ */
+ret_status ret_state_scan(const ret_desc *desc, int n_seg, const int *seg_len,
+                          int rank, const float *U_all, const float *state_in,
+                          float *R, void *stream);
+
+/*
  * ret_selftest_wait_timeout -- diagnostic, no counterpart in the paper.
  * Queues one small kernel on `stream` that waits on an mbarrier nothing
  * completes, through the same bounded wait every tensor-core kernel uses,

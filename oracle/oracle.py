@@ -186,6 +186,36 @@ def rows(q, k, v, gamma: float, rows, rotate=False, theta_base=10000.0,
     return out
 
 
+def segment_state(K, V, gamma, rotate=False, theta_base=10000.0, pos_offset=0,
+                  nthreads=0, lib=None) -> np.ndarray:
+    """The state a segment of rows (K, V at positions pos_offset ..) leaves
+    behind from a zero state: the recurrent form's state after its last row
+    ("Retentive Network" paper summary, section 2.1, form (2)).  The query
+    rows do not enter the state, so K stands in for them."""
+    return recurrent(K, K, V, gamma, rotate=rotate, theta_base=theta_base,
+                     pos_offset=pos_offset, nthreads=nthreads, lib=lib)[1]
+
+
+def state_scan(U, seg_lens, gamma, state_in=None) -> np.ndarray:
+    """States entering each of n consecutive segments of seg_lens rows, from
+    the segments' own states U [n, B, H, dk, dv] (each the state its segment
+    leaves from a zero start) and the state before the first segment:
+    R_0 = state_in (zero if None), R_{s+1} = gamma_h^{seg_lens[s]} R_s + U_s,
+    the chunkwise form's state recurrence ("Retentive Network" paper
+    summary, section 2.1, form (3)) applied between segments.  Returns
+    R [n + 1, B, H, dk, dv]; R[n] is the state after the last segment."""
+    U = _f64(U)
+    g = np.asarray(gamma, dtype=np.float64)
+    n = U.shape[0]
+    R = np.zeros((n + 1,) + U.shape[1:])
+    if state_in is not None:
+        R[0] = _f64(state_in)
+    for s in range(n):
+        decay = g ** int(seg_lens[s])
+        R[s + 1] = decay[None, :, None, None] * R[s] + U[s]
+    return R
+
+
 def gate_groupnorm(O, G, eps=1e-5, lib=None) -> np.ndarray:
     """O [B, H, L, dv], G [B, L, H*dv] -> Y [B, L, H*dv]."""
     lib = lib or load()

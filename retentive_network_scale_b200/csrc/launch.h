@@ -1,8 +1,11 @@
 // launch.h -- internal launchers behind the C ABI (not exported).
 #pragma once
 
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "common.cuh"
 
@@ -81,6 +84,19 @@ cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void
                                           RowLayout src, bool always_q, void *workspace,
                                           const void **q_used, const void **k_used,
                                           cudaStream_t st);
+
+// K~ alone (turned when p.rotate, and weighted by gamma^{n-1-j} per row of
+// a chunk of `chunk` rows), bf16 [B][H][L][d_k], from K [B][H][L][d_k].
+cudaError_t launch_key_prep(const Params &p, int chunk, const void *K, void *kt,
+                            cudaStream_t st);
+
+// The current device's cuBLAS handle, bound to `st` and to kBlasWorkspace
+// bytes of `workspace`; the caller holds blas_mutex() for as long as it
+// uses the handle (a handle is not safe to share between host threads).
+// NULL when the handle cannot be made or bound.
+constexpr size_t kBlasWorkspace = 32ull << 20;
+std::mutex &blas_mutex();
+cublasHandle_t blas_handle(cudaStream_t st, void *workspace);
 
 // Tensor-core parallel form: bf16 inputs, d_k 128 or 256, d_v a multiple of
 // 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned

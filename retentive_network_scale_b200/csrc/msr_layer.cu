@@ -25,7 +25,6 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
-constexpr size_t kCublasWorkspace = 32ull << 20;
 
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -48,7 +47,7 @@ LayerSizes sizes_of(const ret_desc *d) {
     s.off_prep = round_up(s.proj);
     s.off_y = s.off_prep + round_up(s.prep);
     s.off_blas = s.off_y + round_up(s.y);
-    s.bytes = s.off_blas + kCublasWorkspace;
+    s.bytes = s.off_blas + ret::kBlasWorkspace;
     return s;
 }
 
@@ -63,6 +62,29 @@ cublasStatus_t gemm_rm(cublasHandle_t h, long long M, long long N, long long K, 
 }
 
 }  // namespace
+
+namespace ret {
+
+std::mutex &blas_mutex() { return g_mu; }
+
+cublasHandle_t blas_handle(cudaStream_t st, void *workspace) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (!g_handle[dev] && cublasCreate(&g_handle[dev]) != CUBLAS_STATUS_SUCCESS) {
+        g_handle[dev] = nullptr;
+        return nullptr;
+    }
+    cublasHandle_t h = g_handle[dev];
+    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS ||
+        cublasSetWorkspace(h, workspace, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
+        return nullptr;
+    return h;
+}
+
+}  // namespace ret
 
 extern "C" {
 
@@ -102,19 +124,12 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
     int *status = ret::device_status_word();
     if (!status) return RET_ERR_CUDA;
 
-    // one cuBLAS handle per device, used under the lock (handles are not
-    // safe to share between host threads)
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_handle[dev] && cublasCreate(&g_handle[dev]) != CUBLAS_STATUS_SUCCESS) {
-        g_handle[dev] = nullptr;
-        return RET_ERR_CUDA;
-    }
-    cublasHandle_t h = g_handle[dev];
+    // one cuBLAS handle per device, used under the lock
+    std::lock_guard<std::mutex> lock(ret::blas_mutex());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS ||
-        cublasSetWorkspace(h, ws + z.off_blas, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS)
-        return RET_ERR_CUDA;
+    cublasHandle_t h = ret::blas_handle(st, ws + z.off_blas);
+    if (!h) return RET_ERR_CUDA;
 
     const int H = desc->H, dk = desc->d_k, dv = desc->d_v;
     const auto *P = reinterpret_cast<const __nv_bfloat16 *>(ws);

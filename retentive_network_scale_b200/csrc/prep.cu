@@ -103,9 +103,11 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
             for (int e = 0; e < 4; ++e) {
                 const float2 k2 = unpack2(uk[e]);
                 if constexpr (ROT) {
-                    const float2 q2 = unpack2(uq[e]);
                     const float zc = z * c[e], zs = z * s[e];
-                    uq[e] = pack2(q2.x * c[e] - q2.y * s[e], q2.x * s[e] + q2.y * c[e]);
+                    if constexpr (WQ) {
+                        const float2 q2 = unpack2(uq[e]);
+                        uq[e] = pack2(q2.x * c[e] - q2.y * s[e], q2.x * s[e] + q2.y * c[e]);
+                    }
                     uk[e] = pack2(k2.x * zc - k2.y * zs, k2.x * zs + k2.y * zc);
                     const float cn = c[e] * cs[e] - s[e] * ss[e];
                     s[e] = c[e] * ss[e] + s[e] * cs[e];
@@ -161,6 +163,24 @@ cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void
     *q_used = wq ? qh : Q;
     *k_used = kt;
     return cudaSuccess;
+}
+
+cudaError_t launch_key_prep(const Params &p, int chunk, const void *K, void *kt,
+                            cudaStream_t st) {
+    const long long items =
+        (long long)p.B * p.H * ((p.L + kRows - 1) / kRows) * (p.dk / 8);
+    const long long blocks = (items + kThreads - 1) / kThreads;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const auto *k = static_cast<const __nv_bfloat16 *>(K);
+    auto *out = static_cast<__nv_bfloat16 *>(kt);
+    const RowLayout src = bhld_layout(p, p.dk);
+    if (p.rotate)
+        chunk_prep_kernel<true, false><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, k, k, src, nullptr, out);
+    else
+        chunk_prep_kernel<false, false><<<(unsigned)blocks, kThreads, 0, st>>>(p, chunk, items, k, k, src, nullptr, out);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) note_launches(1);
+    return e;
 }
 
 }  // namespace ret

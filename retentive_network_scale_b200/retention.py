@@ -32,10 +32,12 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
            "ret_backward", "ret_backward_workspace_size",
+           "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
 RET_MAX_DECODE_STEPS = 16
+RET_MAX_SEGMENTS = 64
 
 
 class RetentionError(RuntimeError):
@@ -95,6 +97,11 @@ def load_library(path: str = LIB_PATH):
     lib.ret_backward.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, st, vp]
     lib.ret_backward_workspace_size.argtypes = [D, ctypes.c_int]
     lib.ret_backward_workspace_size.restype = st
+    lib.ret_segment_state.argtypes = [D, vp, vp, vp, vp, st, vp]
+    lib.ret_segment_state_workspace_size.argtypes = [D]
+    lib.ret_segment_state_workspace_size.restype = st
+    lib.ret_state_scan.argtypes = [D, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int, vp,
+                                   vp, vp, vp]
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -342,6 +349,54 @@ def lib_backward_workspace_size(B, H, L, d_k, d_v, gamma, chunk, rotate=False):
     lib = load_library()
     d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_F32, gamma, rotate)
     return int(lib.ret_backward_workspace_size(ctypes.byref(d), int(chunk)))
+
+
+def ret_segment_state(K, V, gamma, U=None, rotate=False, theta_base=10000.0, pos_offset=0,
+                      workspace=None, stream=None):
+    """The state a segment of rows leaves behind from a zero state (bf16
+    K, V), fp32 [B][H][d_k][d_v]; allocated when not given, as is the
+    workspace."""
+    lib = load_library()
+    B, H, L, dk = K.shape
+    dv = V.shape[-1]
+    _dev(K, "K", dtype=torch.bfloat16); _dev(V, "V", (B, H, L, dv), torch.bfloat16)
+    if U is None:
+        U = torch.empty(B, H, dk, dv, device=K.device, dtype=torch.float32)
+    _dev(U, "U", (B, H, dk, dv), torch.float32)
+    d = make_desc(B, H, L, dk, dv, RET_BF16, RET_F32, gamma, rotate, theta_base, pos_offset)
+    need = int(lib.ret_segment_state_workspace_size(ctypes.byref(d)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=K.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_segment_state(ctypes.byref(d), _ptr(K), _ptr(V), _ptr(U), _ptr(workspace),
+                                 ws_bytes, _stream(stream)), "ret_segment_state")
+    return U
+
+
+def lib_segment_state_workspace_size(B, H, L, d_k, d_v, gamma, rotate=False):
+    """Device workspace bytes of ret_segment_state for these sizes."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_F32, gamma, rotate)
+    return int(lib.ret_segment_state_workspace_size(ctypes.byref(d)))
+
+
+def ret_state_scan(U_all, seg_lens, rank, gamma, state_in=None, R=None, stream=None):
+    """The state entering segment `rank` of consecutive segments of
+    seg_lens rows, from the segments' own states U_all [n_seg][B][H][d_k][d_v]
+    (fp32, device) and the state before the first segment."""
+    lib = load_library()
+    n_seg, B, H, dk, dv = U_all.shape
+    _dev(U_all, "U_all", dtype=torch.float32)
+    if state_in is not None:
+        _dev(state_in, "state_in", (B, H, dk, dv), torch.float32)
+    if R is None:
+        R = torch.empty(B, H, dk, dv, device=U_all.device, dtype=torch.float32)
+    _dev(R, "R", (B, H, dk, dv), torch.float32)
+    lens = (ctypes.c_int * len(seg_lens))(*[int(x) for x in seg_lens])
+    d = make_desc(B, H, 0, dk, dv, RET_F32, RET_F32, gamma)
+    _check(lib.ret_state_scan(ctypes.byref(d), len(seg_lens), lens, int(rank), _ptr(U_all),
+                              _ptr(state_in), _ptr(R), _stream(stream)), "ret_state_scan")
+    return R
 
 
 def ret_selftest_wait_timeout(cycles, stream=None):

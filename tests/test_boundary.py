@@ -216,6 +216,40 @@ def test_selftest_wait_timeout_arguments(lib):
 def test_header_constants_match_binding():
     import re
     text = open(HEADER).read()
-    for name in ("RET_MAX_HEADS", "RET_MAX_DECODE_STEPS"):
+    for name in ("RET_MAX_HEADS", "RET_MAX_DECODE_STEPS", "RET_MAX_SEGMENTS"):
         m = re.search(r"#define\s+%s\s+(\d+)" % name, text)
         assert m and int(m.group(1)) == getattr(R, name), name
+
+
+def test_segment_state_arguments(lib):
+    """ret_segment_state / ret_state_scan reject bad calls before any CUDA
+    call, and the workspace contract of the segment state."""
+    S = R.STATUS_NAMES.index
+    d = desc(B=2, L=300, d_k=16, d_v=8, in_dtype=R.RET_BF16)
+    seg = lambda **kw: lib.ret_segment_state(
+        ctypes.byref(kw.get("d", d)), kw.get("K", FAKE), FAKE, kw.get("U", FAKE),
+        kw.get("ws", None), kw.get("ws_bytes", 0), None)
+    assert seg(d=desc(B=2, L=300, d_k=16, d_v=8, in_dtype=R.RET_F32)) == S("RET_ERR_DTYPE")
+    assert seg(d=desc(B=2, L=300, d_k=12, d_v=8, in_dtype=R.RET_BF16)) == S("RET_ERR_SHAPE")
+    assert seg(U=None) == S("RET_ERR_NULL")
+    assert seg(U=MISALIGNED) == S("RET_ERR_ALIGN")
+    assert seg(d=desc(B=0, L=300, d_k=16, d_v=8, in_dtype=R.RET_BF16)) == S("RET_OK")
+    size = lib.ret_segment_state_workspace_size(ctypes.byref(d))
+    assert size >= 2 * 300 * 16 * 2          # the weighted keys, and cuBLAS room
+    assert lib.ret_segment_state_workspace_size(ctypes.byref(desc(B=0))) == 0
+    if not torch.cuda.is_available():
+        assert seg() == S("RET_ERR_UNSUPPORTED")
+    lens = (ctypes.c_int * 3)(4, 5, 6)
+    scan = lambda n=3, rank=1, L=lens, U=FAKE, R_=FAKE, s0=None: lib.ret_state_scan(
+        ctypes.byref(d), n, L, rank, U, s0, R_, None)
+    assert scan(n=0) == S("RET_ERR_SHAPE")
+    assert scan(n=R.RET_MAX_SEGMENTS + 1) == S("RET_ERR_SHAPE")
+    assert scan(rank=4) == S("RET_ERR_SHAPE")
+    assert scan(rank=-1) == S("RET_ERR_SHAPE")
+    assert scan(L=(ctypes.c_int * 3)(4, 0, 6)) == S("RET_ERR_SHAPE")
+    assert scan(L=None) == S("RET_ERR_NULL")
+    assert scan(U=None) == S("RET_ERR_NULL")      # segment 0 must be read for rank 1
+    assert scan(R_=None) == S("RET_ERR_NULL")
+    assert scan(s0=MISALIGNED) == S("RET_ERR_ALIGN")
+    if not torch.cuda.is_available():
+        assert scan(rank=0, U=None) == S("RET_ERR_UNSUPPORTED")

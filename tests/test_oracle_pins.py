@@ -307,3 +307,32 @@ def test_backward_matches_finite_differences(olib, rotate):
             minus = list(args); minus[which] = args[which] - eps * d
             fd = (f(*plus) - f(*minus)) / (2 * eps)
             assert abs(fd - float(np.sum(grad * d))) <= 1e-6 * max(1.0, abs(fd)), which
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_state_scan_joins_segments(olib, rotate):
+    """The segment state and the scan against the recurrent form over the
+    whole sequence: a sequence cut into unequal segments, each run from the
+    state the scan gives it (at its own absolute positions), reproduces the
+    outputs and the final state of one uncut run.  A wrong decay exponent,
+    segment order or position offset fails it."""
+    rng = np.random.default_rng(23)
+    B, H, dk, dv = 1, 3, 4, 6
+    lens = [5, 9, 3, 7]
+    L = sum(lens)
+    gam = [0.6, 0.93, 1.0]
+    Q = rng.standard_normal((B, H, L, dk)) * 0.5
+    K = rng.standard_normal((B, H, L, dk)) * 0.5
+    V = rng.standard_normal((B, H, L, dv))
+    S0 = rng.standard_normal((B, H, dk, dv))
+    O_ref, S_ref = orc.recurrent(Q, K, V, gam, rotate=rotate, pos_offset=11, state_in=S0, lib=olib)
+    starts = np.cumsum([0] + lens[:-1])
+    U = np.stack([orc.segment_state(K[:, :, a:a + n], V[:, :, a:a + n], gam, rotate=rotate,
+                                    pos_offset=11 + a, lib=olib) for a, n in zip(starts, lens)])
+    R = orc.state_scan(U, lens, gam, state_in=S0)
+    assert _normwise(R[-1], S_ref) <= 1e-12
+    for s, (a, n) in enumerate(zip(starts, lens)):
+        O_s, S_s = orc.recurrent(Q[:, :, a:a + n], K[:, :, a:a + n], V[:, :, a:a + n], gam,
+                                 rotate=rotate, pos_offset=11 + a, state_in=R[s], lib=olib)
+        assert _normwise(O_s, O_ref[:, :, a:a + n]) <= 1e-12
+        assert _normwise(S_s, R[s + 1]) <= 1e-12
