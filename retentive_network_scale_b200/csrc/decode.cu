@@ -122,7 +122,9 @@ recurrent_step_kernel(Params p, int ncol_tiles, const TI *q, const TI *k,
 //   s <- gamma s + k^_t[i] v_t[c];   o_t[c] += q^_t[i] s   (t = 0 .. T-1),
 // so the state is read and written once for all T tokens.  q, k, v, o are
 // [B][H][T][d]; the rotated q^_t, k^_t of the head and the v_t of the CTA's
-// columns sit in shared memory; the column sums are reduced token by token.
+// columns sit in shared memory.  The column sums of all T tokens are reduced
+// at the end: across the row groups of a warp by shuffles, then across the
+// warps through shared memory in one pass.
 constexpr int kMultiRowsInFlight = 4;
 
 template <typename TI, typename TO, int COLS, int TMAX>
@@ -131,9 +133,16 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
                        float *state, TO *o) {
     constexpr int TPR = COLS / 4;
     constexpr int RG = kThreads / TPR;
-    __shared__ float qs[TMAX][kMaxDk], ks[TMAX][kMaxDk];
+    constexpr int kWarps = kThreads / 32;
+    // q^_t and k^_t; after the state pass the same words hold the warps'
+    // column sums
+    __shared__ __align__(16) float qk[2 * TMAX * kMaxDk];
     __shared__ __align__(16) float vs[TMAX][COLS];
-    __shared__ float red[RG * COLS];
+    __shared__ double s_theta[kMaxDk / 2];
+    static_assert(kWarps * COLS <= 2 * kMaxDk, "column sums must fit in the q^/k^ words");
+    auto qs = reinterpret_cast<float (*)[kMaxDk]>(qk);
+    auto ks = reinterpret_cast<float (*)[kMaxDk]>(qk + TMAX * kMaxDk);
+    auto red = reinterpret_cast<float (*)[TMAX][COLS]>(qk);
 
     const int bh = blockIdx.x / ncol_tiles, ct = blockIdx.x - bh * ncol_tiles;
     const int h = bh % p.H;
@@ -141,11 +150,13 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
 
     // q^_t, k^_t (turned at position pos_offset + t) and this CTA's v_t columns
     if (p.rotate) {
+        stage_theta(p, s_theta, dk / 2);
+        __syncthreads();
         for (int idx = threadIdx.x; idx < T * (dk / 2); idx += kThreads) {
             const int t = idx / (dk / 2), j = idx - t * (dk / 2);
             const size_t base = ((size_t)bh * T + t) * dk;
             float c, sn;
-            rot_cs(p.pos_offset + t, p.theta[j], &c, &sn);
+            rot_cs_fast(p.pos_offset + t, s_theta[j], &c, &sn);
             float q0 = ld(q, base + 2 * j), q1 = ld(q, base + 2 * j + 1);
             float k0 = ld(k, base + 2 * j), k1 = ld(k, base + 2 * j + 1);
             rot_pair(q0, q1, c, sn);
@@ -209,31 +220,32 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
         }
     }
 
-    // o_t[c'] = sum over row groups, token by token; red is [RG][COLS]
-    constexpr int PARTS = kThreads / COLS;
-    constexpr int PER = RG / PARTS;
+    // o_t[c'] = the sum over row groups: the lanes of a warp that share this
+    // thread's columns (lane bits TPR and up) by shuffles, then the warps
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int t = 0; t < TMAX; ++t) {
         if (t < T) {
-            red[rg * COLS + 4 * tpr + 0] = acc[t].x;
-            red[rg * COLS + 4 * tpr + 1] = acc[t].y;
-            red[rg * COLS + 4 * tpr + 2] = acc[t].z;
-            red[rg * COLS + 4 * tpr + 3] = acc[t].w;
-            __syncthreads();
-            const int cc = threadIdx.x % COLS, part = threadIdx.x / COLS;
-            float sum = 0.f;
 #pragma unroll
-            for (int r = 0; r < PER; ++r) sum += red[(part * PER + r) * COLS + cc];
-            __syncthreads();
-            red[part * COLS + cc] = sum;
-            __syncthreads();
-            if (threadIdx.x < COLS) {
-                float tot = 0.f;
-                for (int pt = 0; pt < PARTS; ++pt) tot += red[pt * COLS + threadIdx.x];
-                st(o, ((size_t)bh * T + t) * dv + ct * COLS + threadIdx.x, tot);
+            for (int off = TPR; off < 32; off <<= 1) {
+                acc[t].x += __shfl_xor_sync(0xffffffffu, acc[t].x, off);
+                acc[t].y += __shfl_xor_sync(0xffffffffu, acc[t].y, off);
+                acc[t].z += __shfl_xor_sync(0xffffffffu, acc[t].z, off);
+                acc[t].w += __shfl_xor_sync(0xffffffffu, acc[t].w, off);
             }
-            __syncthreads();
         }
+    }
+    __syncthreads();  // every thread is done with q^ and k^
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t)
+        if (t < T && lane < TPR) *reinterpret_cast<float4 *>(&red[warp][t][4 * tpr]) = acc[t];
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < T * COLS; idx += kThreads) {
+        const int t = idx / COLS, cc = idx - t * COLS;
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) tot += red[w][t][cc];
+        st(o, ((size_t)bh * T + t) * dv + ct * COLS + cc, tot);
     }
 }
 

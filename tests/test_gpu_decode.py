@@ -1,7 +1,8 @@
 """Several tokens per ret_recurrent_step call (1 < T <= RET_MAX_DECODE_STEPS):
 outputs and the in-place state against the oracle's recurrent form run on
-from the same state, for both column-tile widths of the kernel (d_v a
-multiple of 32, and not), fp32 and bf16, with rotation at a large offset;
+from the same state, for the three column layouts of the kernels (d_v a
+multiple of 128, of 32, neither), fp32 and bf16, with rotation at a large
+offset;
 T-token calls chained, and agreement with T single-token calls."""
 import numpy as np
 import pytest
@@ -34,7 +35,8 @@ def _case(B, H, T, dk, dv, dtype, seed):
 
 
 @pytest.mark.parametrize("T", [2, 5, 8, 16])
-@pytest.mark.parametrize("dtype,dv", [(torch.float32, 96), (torch.bfloat16, 36)])
+@pytest.mark.parametrize("dtype,dv", [(torch.float32, 96), (torch.bfloat16, 36),
+                                      (torch.float32, 256), (torch.bfloat16, 128)])
 def test_multi_token_step_matches_oracle(T, dtype, dv):
     B, H, dk, p0 = 2, 3, 64, 1000
     q, k, v, s0 = _case(B, H, T, dk, dv, dtype, 40 + T)
