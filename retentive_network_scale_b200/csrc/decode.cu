@@ -12,6 +12,7 @@
 // the state is larger than L2 and is not read again within the step.
 #include "common.cuh"
 #include "launch.h"
+#include "tc_util.cuh"
 
 namespace ret {
 namespace {
@@ -126,8 +127,9 @@ recurrent_step_kernel(Params p, int ncol_tiles, const TI *q, const TI *k,
 // at the end: across the row groups of a warp by shuffles, then across the
 // warps through shared memory in one pass.
 constexpr int kMultiRowsInFlight = 4;
+constexpr bool kMultiPacked = true;  // packed fp32 pairs on the rescaled path
 
-template <typename TI, typename TO, int COLS, int TMAX>
+template <typename TI, typename TO, int COLS, int TMAX, bool PACKED>
 __global__ void __launch_bounds__(kThreads)
 recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k, const TI *v,
                        float *state, TO *o) {
@@ -147,6 +149,19 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
     const int bh = blockIdx.x / ncol_tiles, ct = blockIdx.x - bh * ncol_tiles;
     const int h = bh % p.H;
     const int dk = p.dk, dv = p.dv;
+    // With gamma^T >= 2^-60 the T updates run on a rescaled state: with
+    // s_t = gamma s_{t-1} + k_t v_t from s_{-1} = S,
+    //   s_t = gamma^{t+1} a_t,  a_t = S + sum_{tau<=t} gamma^{-(tau+1)} k_tau v_tau,
+    //   o_t = q_t . s_t = (gamma^{t+1} q_t) . a_t,
+    // so with k~_t = gamma^{-(t+1)} k_t and q~_t = gamma^{t+1} q_t each token
+    // costs a += k~ v and o += q~ a, and the state leaves as gamma^T a.  The
+    // final scaling brings every term back to its own magnitude, so the
+    // relative rounding is that of the direct form.  Other decays (gamma = 0
+    // among them) take the direct form.
+    const float lg = p.log2g[h];
+    const bool scaled = (float)T * lg >= -60.f;
+    auto fq = [&](int t) { return scaled ? exp2f((float)(t + 1) * lg) : 1.f; };
+    auto fk = [&](int t) { return scaled ? exp2f(-(float)(t + 1) * lg) : 1.f; };
 
     // q^_t, k^_t (turned at position pos_offset + t) and this CTA's v_t columns
     if (p.rotate) {
@@ -161,14 +176,15 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
             float k0 = ld(k, base + 2 * j), k1 = ld(k, base + 2 * j + 1);
             rot_pair(q0, q1, c, sn);
             rot_pair(k0, k1, c, sn);
-            qs[t][2 * j] = q0; qs[t][2 * j + 1] = q1;
-            ks[t][2 * j] = k0; ks[t][2 * j + 1] = k1;
+            const float a = fq(t), b = fk(t);
+            qs[t][2 * j] = a * q0; qs[t][2 * j + 1] = a * q1;
+            ks[t][2 * j] = b * k0; ks[t][2 * j + 1] = b * k1;
         }
     } else {
         for (int idx = threadIdx.x; idx < T * dk; idx += kThreads) {
             const int t = idx / dk, i = idx - t * dk;
-            qs[t][i] = ld(q, ((size_t)bh * T + t) * dk + i);
-            ks[t][i] = ld(k, ((size_t)bh * T + t) * dk + i);
+            qs[t][i] = fq(t) * ld(q, ((size_t)bh * T + t) * dk + i);
+            ks[t][i] = fk(t) * ld(k, ((size_t)bh * T + t) * dk + i);
         }
     }
     for (int idx = threadIdx.x; idx < T * COLS; idx += kThreads) {
@@ -179,36 +195,84 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
 
     const int tpr = threadIdx.x % TPR, rg = threadIdx.x / TPR;
     const int c = ct * COLS + 4 * tpr;
-    const float g = exp2f(p.log2g[h]);
+    const float g = exp2f(lg);
+    const float gT = scaled ? exp2f((float)T * lg) : 1.f;
     float *S = state + (size_t)bh * dk * dv + c;
     float4 acc[TMAX];
 #pragma unroll
     for (int t = 0; t < TMAX; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 
+    // packed fp32 pairs (x, y) and (z, w) of a float4
+    union P4 {
+        float4 f;
+        uint64_t u[2];
+    };
     for (int i0 = rg; i0 < dk; i0 += RG * kMultiRowsInFlight) {
-        float4 s[kMultiRowsInFlight];
+        P4 s[kMultiRowsInFlight];
 #pragma unroll
         for (int u = 0; u < kMultiRowsInFlight; ++u) {
             const int i = i0 + u * RG;
-            if (i < dk) s[u] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)i * dv));
+            if (i < dk) s[u].f = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)i * dv));
         }
+        if (scaled) {
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
-            if (t < T) {
-                const float4 vt = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    P4 vt, at;
+                    vt.f = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
+                    at.f = acc[t];
 #pragma unroll
-                for (int u = 0; u < kMultiRowsInFlight; ++u) {
-                    const int i = i0 + u * RG;
-                    if (i < dk) {
-                        const float ki = ks[t][i], qi = qs[t][i];
-                        s[u].x = fmaf(g, s[u].x, ki * vt.x);
-                        s[u].y = fmaf(g, s[u].y, ki * vt.y);
-                        s[u].z = fmaf(g, s[u].z, ki * vt.z);
-                        s[u].w = fmaf(g, s[u].w, ki * vt.w);
-                        acc[t].x = fmaf(qi, s[u].x, acc[t].x);
-                        acc[t].y = fmaf(qi, s[u].y, acc[t].y);
-                        acc[t].z = fmaf(qi, s[u].z, acc[t].z);
-                        acc[t].w = fmaf(qi, s[u].w, acc[t].w);
+                    for (int u = 0; u < kMultiRowsInFlight; ++u) {
+                        const int i = i0 + u * RG;
+                        if (i < dk) {
+                            const float ki = ks[t][i], qi = qs[t][i];
+                            if constexpr (PACKED) {
+                                const uint64_t K2 = tc::f2_make(ki, ki), Q2 = tc::f2_make(qi, qi);
+                                s[u].u[0] = tc::f2_fma(K2, vt.u[0], s[u].u[0]);
+                                s[u].u[1] = tc::f2_fma(K2, vt.u[1], s[u].u[1]);
+                                at.u[0] = tc::f2_fma(Q2, s[u].u[0], at.u[0]);
+                                at.u[1] = tc::f2_fma(Q2, s[u].u[1], at.u[1]);
+                            } else {
+                                s[u].f.x = fmaf(ki, vt.f.x, s[u].f.x);
+                                s[u].f.y = fmaf(ki, vt.f.y, s[u].f.y);
+                                s[u].f.z = fmaf(ki, vt.f.z, s[u].f.z);
+                                s[u].f.w = fmaf(ki, vt.f.w, s[u].f.w);
+                                at.f.x = fmaf(qi, s[u].f.x, at.f.x);
+                                at.f.y = fmaf(qi, s[u].f.y, at.f.y);
+                                at.f.z = fmaf(qi, s[u].f.z, at.f.z);
+                                at.f.w = fmaf(qi, s[u].f.w, at.f.w);
+                            }
+                        }
+                    }
+                    acc[t] = at.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMultiRowsInFlight; ++u) {
+                s[u].f.x *= gT;
+                s[u].f.y *= gT;
+                s[u].f.z *= gT;
+                s[u].f.w *= gT;
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    const float4 vt = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
+#pragma unroll
+                    for (int u = 0; u < kMultiRowsInFlight; ++u) {
+                        const int i = i0 + u * RG;
+                        if (i < dk) {
+                            const float ki = ks[t][i], qi = qs[t][i];
+                            s[u].f.x = fmaf(g, s[u].f.x, ki * vt.x);
+                            s[u].f.y = fmaf(g, s[u].f.y, ki * vt.y);
+                            s[u].f.z = fmaf(g, s[u].f.z, ki * vt.z);
+                            s[u].f.w = fmaf(g, s[u].f.w, ki * vt.w);
+                            acc[t].x = fmaf(qi, s[u].f.x, acc[t].x);
+                            acc[t].y = fmaf(qi, s[u].f.y, acc[t].y);
+                            acc[t].z = fmaf(qi, s[u].f.z, acc[t].z);
+                            acc[t].w = fmaf(qi, s[u].f.w, acc[t].w);
+                        }
                     }
                 }
             }
@@ -216,7 +280,7 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
 #pragma unroll
         for (int u = 0; u < kMultiRowsInFlight; ++u) {
             const int i = i0 + u * RG;
-            if (i < dk) __stcs(reinterpret_cast<float4 *>(S + (size_t)i * dv), s[u]);
+            if (i < dk) __stcs(reinterpret_cast<float4 *>(S + (size_t)i * dv), s[u].f);
         }
     }
 
@@ -259,9 +323,9 @@ cudaError_t launch_multi(const Params &p, int T, const void *q, const void *k, c
     const TI *qq = (const TI *)q, *kk = (const TI *)k, *vv = (const TI *)v;
     TO *oo = (TO *)o;
     if (cols == 32)
-        recurrent_multi_kernel<TI, TO, 32, TMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
+        recurrent_multi_kernel<TI, TO, 32, TMAX, kMultiPacked><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
     else
-        recurrent_multi_kernel<TI, TO, 4, TMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
+        recurrent_multi_kernel<TI, TO, 4, TMAX, kMultiPacked><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
     cudaError_t err = cudaGetLastError();
     if (err == cudaSuccess) note_launches(1);
     return err;
