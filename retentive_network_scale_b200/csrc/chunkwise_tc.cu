@@ -617,8 +617,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int o0 = gwg * 64;   // this thread's 64 columns of the row, 32 at a time
             const size_t grow =
                 ((size_t)b * L + t0 + row) * ((size_t)p.H * dv) + (size_t)h * dv + v0 + o0;
-            if (alive && g_leader) wait_bar(bar(BPV), par, abort_flag, status);
-            alive = gsync_alive();
+            // every thread observes the barriers it depends on itself: a
+            // completed phase orders its own reads, no group barrier needed
+            if (alive) alive = wait_bar(bar(BPV), par, abort_flag, status);
             tc_fence_after();
             const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}; lg finite
             // 32 columns of O'' (still in tensor memory until this iteration ends)
@@ -695,8 +696,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             };
             // the products have read V (the state update is the last)
             auto v_free = [&]() {
-                if (alive && g_leader) wait_bar(bar(BU), par, abort_flag, status);
-                alive = gsync_alive();
+                if (alive) alive = wait_bar(bar(BU), par, abort_flag, status);
             };
             if constexpr (!FUSE) {
                 v_free();
@@ -747,8 +747,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // peers reach the exchange barrier
                 cluster_arrive();
                 uint32_t sw[32];
-                if (alive && g_leader) wait_bar(bar(BG), par, abort_flag, status);
-                alive = gsync_alive();
+                if (alive) alive = wait_bar(bar(BG), par, abort_flag, status);
                 if (alive) {
                     const uint8_t *gt = smem + Ly::kQ + gwg * 16384 + row * 128;
 #pragma unroll
