@@ -483,7 +483,7 @@ def run_ours(args, world, rank, local):
                         workspace=ws)
 
     def prep_only():
-        R.ret_chunkwise_prepare(d["Q"], d["K"], g, w.chunk, ws, rotate=w.rotate)
+        return R.ret_chunkwise_prepare(d["Q"], d["K"], g, w.chunk, ws, rotate=w.rotate)
 
     for _ in range(args.warmup):
         step()
@@ -506,13 +506,20 @@ def run_ours(args, world, rank, local):
     tokens_step = w.B * w.L
     value = whole_job_value(world, tokens_step, ms)
 
-    # The step is two launches: the streaming pass that prepares Q^ / K~
-    # and the chunk loop (the dominant kernel).  The pass is timed alone
-    # (same stream, same buffers) and the loop's time is the difference.
+    # The step is the streaming pass that prepares Q^ / K~ and the chunk loop
+    # (the dominant kernel); with the loop taking more than one wave of CTAs
+    # the call cuts the batch into slices and the pass of the next slice runs
+    # under the loop of the current one.  Each is timed alone here (same
+    # stream, same buffers): the pass, then the loop over the whole batch in
+    # one launch on the rows the pass prepared.
     for _ in range(2):
-        prep_only()
+        qh, kt = prep_only()
     ms_prep = time_launches(prep_only, max(3, args.steps), stream)
-    ms_kernel = max(ms_local - ms_prep, 1e-6)
+    loop_only = lambda: R.ret_chunkwise_prepared(  # noqa: E731
+        qh if w.rotate else d["Q"], kt, d["V"], g, w.chunk, G=d["G"], Y=Y, rotate=w.rotate)
+    for _ in range(2):
+        loop_only()
+    ms_kernel = time_launches(loop_only, max(3, args.steps), stream)
     flops = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
     # algorithmic bytes of the chunk loop: Q^, K~ (same sizes as Q, K), V, G in; Y out
     bytes_alg = sum(t.numel() * t.element_size() for t in d.values()) + Y.numel() * Y.element_size()

@@ -180,8 +180,10 @@ size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk);
  * first when its workspace holds ret_chunkwise_prep_size() bytes: the
  * rotated Q (bf16 [B][H][L][d_k], with rotation only) followed by
  * K~[b,h,t] = gamma_h^{n-1-j} Theta_t K[b,h,t] (bf16, same shape) for row t
- * at offset j of its chunk of n rows (section 2.1, chunkwise form (3): the
- * weight of key j' in the state update).  No counterpart in the paper as a
+ * at offset j of its block of n rows (section 2.1, chunkwise form (3): the
+ * weight of key j' in the state update).  The tensor-core loop evaluates a
+ * chunk of any multiple of 128 rows as blocks of 128 (the recurrence holds
+ * at every row boundary), so the blocks are 128 rows whatever `chunk` is.  No counterpart in the paper as a
  * call of its own; exported so that the pass can be timed or scheduled
  * apart.  Q, K device bf16; workspace device, caller-owned, overwritten.
  * Errors: RET_ERR_SHAPE when the tensor-core path does not apply (nothing
@@ -190,6 +192,23 @@ size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk);
 ret_status ret_chunkwise_prepare(const ret_desc *desc, int chunk,
                                  const void *Q, const void *K, void *workspace,
                                  size_t workspace_bytes, void *stream);
+
+/* ret_chunkwise_prepared -- the chunk loop of ret_chunkwise alone, on rows
+ * that ret_chunkwise_prepare wrote: the tensor-core loop, one launch over
+ * the whole batch.  No counterpart in the paper as a call of its own;
+ * exported for callers that schedule the streaming pass themselves, and so
+ * that the loop can be timed apart.
+ *   Qh  device bf16 [B][H][L][d_k]: the rotated Q from the workspace, or Q
+ *       itself when desc->rotate is 0
+ *   Kt  device bf16 [B][H][L][d_k]: the weighted K~ from the workspace
+ *   V, state_in, state_out, O, G, gn_eps, Y  as ret_chunkwise
+ * desc and chunk must be those the rows were prepared with.  Errors:
+ * RET_ERR_SHAPE when the tensor-core path does not apply or the problem is
+ * empty, and those of ret_chunkwise. */
+ret_status ret_chunkwise_prepared(const ret_desc *desc, int chunk,
+                                  const void *Qh, const void *Kt, const void *V,
+                                  const float *state_in, float *state_out, void *O,
+                                  const void *G, float gn_eps, void *Y, void *stream);
 
 /*
  * ret_chunkwise_host -- no counterpart in the paper: ret_chunkwise from HOST

@@ -169,8 +169,32 @@ ret_status ret_chunkwise_prepare(const ret_desc *desc, int chunk, const void *Q,
     Params p;
     make_params(desc, &p);
     const void *q_used = nullptr, *k_used = nullptr;
-    return from_cuda(
-        launch_chunkwise_prep(p, chunk, Q, K, workspace, &q_used, &k_used, (cudaStream_t)stream));
+    // the weights follow the 128-row blocks the tensor-core loop works in
+    return from_cuda(launch_chunkwise_prep(p, kChunkBlock, Q, K, workspace, &q_used, &k_used,
+                                           (cudaStream_t)stream));
+}
+
+ret_status ret_chunkwise_prepared(const ret_desc *desc, int chunk, const void *Qh, const void *Kt,
+                                  const void *V, const float *state_in, float *state_out,
+                                  void *O, const void *G, float gn_eps, void *Y, void *stream) {
+    ret_status s = check_desc(desc);
+    if (s != RET_OK) return s;
+    if (chunk < 1) return RET_ERR_ARG;
+    if ((long long)desc->B * desc->L == 0) return RET_ERR_SHAPE;  // nothing was prepared
+    Params p;
+    make_params(desc, &p);
+    if (!chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16)) return RET_ERR_SHAPE;
+    if ((G == nullptr) != (Y == nullptr) || (!O && !Y) || !Qh || !Kt || !V) return RET_ERR_NULL;
+    if (Y && !(gn_eps >= 0.0f && std::isfinite(gn_eps))) return RET_ERR_ARG;
+    if (!aligned16(Qh) || !aligned16(Kt) || !aligned16(V) || !aligned16(O) || !aligned16(G) ||
+        !aligned16(Y) || !aligned16(state_in) || !aligned16(state_out))
+        return RET_ERR_ALIGN;
+    if ((s = check_device()) != RET_OK) return s;
+    int *status = device_status_word();
+    if (!status) return RET_ERR_CUDA;
+    return from_cuda(launch_chunkwise_tc_rows(p, desc->out_dtype == RET_BF16, Qh, Kt, V, state_in,
+                                              state_out, O, G, Y, gn_eps, status,
+                                              (cudaStream_t)stream));
 }
 
 ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const void *K,

@@ -47,7 +47,9 @@
 // and TMEM is freed.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -924,17 +926,12 @@ bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
     return true;
 }
 
-cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
-                                const void *V, const float *s_in, float *s_out, void *O,
-                                const void *G, void *Y, float eps, void *prep_ws, int *status,
-                                cudaStream_t st) {
-    // With room for them, the turned Q^ and scaled K~ are written once by a
-    // streaming pass and the kernel only loads them.
-    const int pre = prep_ws != nullptr;
-    if (pre) {
-        cudaError_t e = launch_chunkwise_prep(p, kC, Q, K, prep_ws, &Q, &K, st);
-        if (e != cudaSuccess) return e;
-    }
+namespace {
+
+// The chunk loop on rows that are ready (prepared when `pre`).
+cudaError_t launch_tc_rows(const Params &p, bool out_bf16, const void *Q, const void *K,
+                           const void *V, const float *s_in, float *s_out, void *O, const void *G,
+                           void *Y, float eps, int pre, int *status, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC) ||
@@ -943,6 +940,122 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
     const Views vw{1, RowLayout{(long long)p.H * p.dv, 0, (long long)p.L * p.H * p.dv}};
     if (p.dk == 256) return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
     return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, Y, eps, pre, vw, status, st);
+}
+
+// A second stream per device on which the streaming pass of the next batch
+// slice runs while the chunk loop of the current one holds the SMs, and the
+// two events that join it to the caller's stream.  Made once; the lock
+// keeps the enqueue sequences of concurrent callers apart.
+struct SideStream {
+    std::mutex mu;
+    bool made = false, ok = false;
+    cudaStream_t s = nullptr;
+    cudaEvent_t start = nullptr, ready = nullptr;
+    int sms = 0;
+};
+constexpr int kMaxDevices = 64;
+SideStream g_side[kMaxDevices];
+
+SideStream *side_stream() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    SideStream &ss = g_side[dev];
+    std::lock_guard<std::mutex> lock(ss.mu);
+    if (!ss.made) {
+        ss.made = true;
+        // the lowest priority: the loop's CTAs take the SMs first, the pass
+        // fills those left over
+        int least = 0, greatest = 0;
+        ss.ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
+                cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, least) == cudaSuccess &&
+                cudaEventCreateWithFlags(&ss.start, cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&ss.ready, cudaEventDisableTiming) == cudaSuccess &&
+                cudaDeviceGetAttribute(&ss.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                ss.sms > 0;
+        if (!ss.ok) cudaGetLastError();
+    }
+    return ss.ok ? &ss : nullptr;
+}
+
+}  // namespace
+
+// With room for them, the turned Q^ and scaled K~ are written once by a
+// streaming pass and the kernel only loads them.  When the chunk loop needs
+// more than one wave of CTAs (one per SM: its shared memory and registers
+// fill an SM), the batch is cut into as many slices as waves, each at most
+// a wave: the loop of slice i then leaves SMs free on which the streaming
+// pass of slice i+1 runs from the side stream, so only the first slice's
+// pass is exposed.  The slices compute exactly what one launch would (every
+// (b, h) and every row of the pass is independent).
+cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
+                                const void *V, const float *s_in, float *s_out, void *O,
+                                const void *G, void *Y, float eps, void *prep_ws, int *status,
+                                cudaStream_t st) {
+    if (!prep_ws) return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 0, status, st);
+    SideStream *ss = side_stream();
+    const long long ctas_per_b = (long long)p.H * (p.dv / kTV);
+    constexpr int kMaxSlices = 16;  // beyond, a slice takes several waves
+    const int slices =
+        ss ? (int)std::min<long long>(std::min(p.B, kMaxSlices), (ctas_per_b * p.B + ss->sms - 1) / ss->sms)
+           : 1;
+    if (slices <= 1) {
+        cudaError_t e = launch_chunkwise_prep(p, kC, Q, K, prep_ws, &Q, &K, st);
+        if (e != cudaSuccess) return e;
+        return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 1, status, st);
+    }
+    // slice i: batch elements [b0(i), b0(i+1)); byte offsets per batch element
+    auto b0 = [&](int i) { return (int)((long long)p.B * i / slices); };
+    const size_t ob = out_bf16 ? 2 : 4;
+    const size_t qk_b = (size_t)p.H * p.L * p.dk * 2, v_b = (size_t)p.H * p.L * p.dv * 2;
+    const size_t o_b = (size_t)p.H * p.L * p.dv * ob, st_b = (size_t)p.H * p.dk * p.dv;
+    const size_t ws_b = chunkwise_prep_bytes(p) / p.B;
+    auto at = [](const void *base, size_t off) {
+        return base ? static_cast<const void *>(static_cast<const uint8_t *>(base) + off) : nullptr;
+    };
+    auto at_w = [](void *base, size_t off) {
+        return base ? static_cast<void *>(static_cast<uint8_t *>(base) + off) : nullptr;
+    };
+    auto sub = [&](int i) {
+        Params q = p;
+        q.B = b0(i + 1) - b0(i);
+        return q;
+    };
+    const void *qh[kMaxSlices], *kt[kMaxSlices];  // prepared operands per slice
+    auto prep = [&](int i, cudaStream_t on) {
+        const size_t b = b0(i);
+        return launch_chunkwise_prep(sub(i), kC, at(Q, b * qk_b), at(K, b * qk_b),
+                                     at_w(prep_ws, b * ws_b), &qh[i], &kt[i], on);
+    };
+    // pass 0 on the caller's stream; the side stream starts after it (and so
+    // after whatever the caller queued before), when the loop of slice 0
+    // starts: the passes of the later slices run beside the loops
+    std::lock_guard<std::mutex> lock(ss->mu);
+    cudaError_t e = prep(0, st);
+    if (e == cudaSuccess) e = cudaEventRecord(ss->start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->start, 0);
+    for (int i = 0; i < slices && e == cudaSuccess; ++i) {
+        const size_t b = b0(i);
+        e = launch_tc_rows(sub(i), out_bf16, qh[i], kt[i], at(V, b * v_b),
+                           s_in ? s_in + b * st_b : nullptr, s_out ? s_out + b * st_b : nullptr,
+                           at_w(O, b * o_b), at(G, b * v_b), at_w(Y, b * o_b), eps, 1, status, st);
+        if (e == cudaSuccess && i + 1 < slices) {
+            e = prep(i + 1, ss->s);
+            if (e == cudaSuccess) e = cudaEventRecord(ss->ready, ss->s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ss->ready, 0);
+        }
+    }
+    return e;
+}
+
+cudaError_t launch_chunkwise_tc_rows(const Params &p, bool out_bf16, const void *Qh, const void *Kt,
+                                     const void *V, const float *s_in, float *s_out, void *O,
+                                     const void *G, void *Y, float eps, int *status,
+                                     cudaStream_t st) {
+    static_assert(kChunkBlock == kC, "the streaming pass and the loop share the row blocks");
+    return launch_tc_rows(p, out_bf16, Qh, Kt, V, s_in, s_out, O, G, Y, eps, 1, status, st);
 }
 
 cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const void *Qh,

@@ -36,6 +36,14 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
                                 const void *G, void *Y, float eps, void *prep_ws, int *status,
                                 cudaStream_t st);
 
+// The chunk loop alone on rows prepared by the streaming pass (blocks of
+// kChunkBlock rows), one launch over the whole batch.
+constexpr int kChunkBlock = 128;
+cudaError_t launch_chunkwise_tc_rows(const Params &p, bool out_bf16, const void *Qh, const void *Kt,
+                                     const void *V, const float *s_in, float *s_out, void *O,
+                                     const void *G, void *Y, float eps, int *status,
+                                     cudaStream_t st);
+
 // Streaming pass: Q^ (rotation only) and K~ = gamma^{n-1-j} K^ per row of a
 // chunk of `chunk` rows, bf16, into the workspace ([Q^][K~], or [K~] without
 // rotation); *q_used / *k_used receive the operands to multiply.

@@ -29,7 +29,7 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 # every symbol include/retention.h declares
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
-           "ret_chunkwise_prepare", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
+           "ret_chunkwise_prepare", "ret_chunkwise_prepared", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
            "ret_backward", "ret_backward_workspace_size",
            "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.ret_chunkwise_prep_size.argtypes = [D, ctypes.c_int]
     lib.ret_chunkwise_prep_size.restype = st
     lib.ret_chunkwise_prepare.argtypes = [D, ctypes.c_int, vp, vp, vp, st, vp]
+    lib.ret_chunkwise_prepared.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                           ctypes.c_float, vp, vp]
     lib.ret_chunkwise_host.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, ctypes.c_float, vp,
                                        ctypes.c_int, vp, st, vp]
     lib.ret_chunkwise_host_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -232,6 +234,31 @@ def ret_chunkwise_prepare(Q, K, gamma, chunk, workspace, rotate=False, theta_bas
     if rotate:
         return flat[:n].view(B, H, L, dk), flat[n:2 * n].view(B, H, L, dk)
     return None, flat[:n].view(B, H, L, dk)
+
+
+def ret_chunkwise_prepared(Qh, Kt, V, gamma, chunk, O=None, state_in=None, state_out=None,
+                           G=None, Y=None, gn_eps=1e-5, rotate=False, theta_base=10000.0,
+                           pos_offset=0, stream=None):
+    """The chunk loop alone on rows ret_chunkwise_prepare wrote (its views;
+    Q itself for Qh without rotation).  Returns (O, Y, state_out)."""
+    lib = load_library()
+    B, H, L, dk = Qh.shape
+    dv = V.shape[-1]
+    _dev(Qh, "Qh", dtype=torch.bfloat16); _dev(Kt, "Kt", Qh.shape, torch.bfloat16)
+    _dev(V, "V", (B, H, L, dv), torch.bfloat16)
+    _dev(O, "O", (B, H, L, dv)); _dev(G, "G", (B, L, H * dv)); _dev(Y, "Y", (B, L, H * dv))
+    _dev(state_in, "state_in", (B, H, dk, dv), torch.float32)
+    _dev(state_out, "state_out", (B, H, dk, dv), torch.float32)
+    out = O if O is not None else Y
+    if out is None:
+        raise ValueError("ret_chunkwise_prepared needs O or Y")
+    d = make_desc(B, H, L, dk, dv, RET_BF16, _dtype_code(out), gamma, rotate, theta_base,
+                  pos_offset)
+    _check(lib.ret_chunkwise_prepared(ctypes.byref(d), int(chunk), _ptr(Qh), _ptr(Kt), _ptr(V),
+                                      _ptr(state_in), _ptr(state_out), _ptr(O), _ptr(G),
+                                      ctypes.c_float(gn_eps), _ptr(Y), _stream(stream)),
+           "ret_chunkwise_prepared")
+    return O, Y, state_out
 
 
 def _host(t, name, shape=None, dtype=None):

@@ -253,3 +253,22 @@ def test_segment_state_arguments(lib):
     assert scan(s0=MISALIGNED) == S("RET_ERR_ALIGN")
     if not torch.cuda.is_available():
         assert scan(rank=0, U=None) == S("RET_ERR_UNSUPPORTED")
+
+
+def test_chunkwise_prepared_arguments(lib):
+    """ret_chunkwise_prepared rejects bad calls before any CUDA call."""
+    S = R.STATUS_NAMES.index
+    d = desc(B=2, L=300, d_k=128, d_v=128, gamma=[0.9, 0.99])
+    call = lambda dd=d, chunk=128, Qh=FAKE, Kt=FAKE, V=FAKE, O=FAKE, G=None, Y=None: \
+        lib.ret_chunkwise_prepared(ctypes.byref(dd), chunk, Qh, Kt, V, None, None, O, G,
+                                   ctypes.c_float(1e-5), Y, None)
+    assert call(chunk=0) == S("RET_ERR_ARG")
+    assert call(dd=desc(B=0, L=300, d_k=128, d_v=128)) == S("RET_ERR_SHAPE")   # nothing prepared
+    assert call(dd=desc(B=2, L=300, d_k=64, d_v=128)) == S("RET_ERR_SHAPE")    # not a tensor-core shape
+    assert call(chunk=64) == S("RET_ERR_SHAPE")
+    assert call(Kt=None) == S("RET_ERR_NULL")
+    assert call(O=None) == S("RET_ERR_NULL")                                   # nothing requested
+    assert call(G=FAKE) == S("RET_ERR_NULL")                                   # G without Y
+    assert call(V=MISALIGNED) == S("RET_ERR_ALIGN")
+    if not torch.cuda.is_available():
+        assert call() == S("RET_ERR_UNSUPPORTED")

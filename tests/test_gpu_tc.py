@@ -204,3 +204,48 @@ def test_prepare_pass_matches_oracle(rotate):
                 out = got[b, h].float().cpu().double().numpy()
                 err = np.abs(out - ref)
                 assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-6 * np.abs(ref).max()), (name, b, h)
+
+
+def test_batch_slices_and_prepared_loop_are_exact():
+    """More CTAs than one wave (B=4 x H=20 x d_v/128=4 = 320 > 148 SMs): the
+    call cuts the batch into slices and overlaps the streaming pass of one
+    with the loop of the other.  Every (b, h) is independent, so the result
+    is bitwise that of one call per batch element (80 CTAs, no slices) and of
+    the loop alone on rows prepared by ret_chunkwise_prepare; and it matches
+    the oracle on sampled slices."""
+    B, H, L, dk, dv = 4, 20, 300, 128, 512
+    Q, K, V = _inputs(B, H, L, dk, dv, 61)
+    G = random_tensor((B, L, H * dv), 62).bfloat16()
+    S0 = random_tensor((B, H, dk, dv), 63, 0.1)
+    g = [1 - 2.0 ** (-5 - (h % 8)) for h in range(H)]
+    Qd, Kd, Vd, Gd, S0d = Q.cuda(), K.cuda(), V.cuda(), G.cuda(), S0.cuda()
+    mk = lambda: (torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16),  # noqa: E731
+                  torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16),
+                  torch.empty(B, H, dk, dv, device="cuda"))
+    O1, Y1, S1 = mk()
+    n0 = R.ret_kernel_launches()
+    R.ret_chunkwise(Qd, Kd, Vd, g, 128, O=O1, G=Gd, Y=Y1, state_in=S0d, state_out=S1, rotate=True,
+                    pos_offset=9)
+    assert R.ret_kernel_launches() - n0 == 6          # three slices: pass + loop each
+    O2, Y2, S2 = mk()
+    for b in range(B):
+        R.ret_chunkwise(Qd[b:b + 1], Kd[b:b + 1], Vd[b:b + 1], g, 128, O=O2[b:b + 1], G=Gd[b:b + 1],
+                        Y=Y2[b:b + 1], state_in=S0d[b:b + 1], state_out=S2[b:b + 1], rotate=True,
+                        pos_offset=9)
+    size = R.ret_chunkwise_prep_size(B, H, L, dk, dv, R.RET_BF16, R.RET_BF16, g, 128, rotate=True,
+                                     pos_offset=9)
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+    qh, kt = R.ret_chunkwise_prepare(Qd, Kd, g, 128, ws, rotate=True, pos_offset=9)
+    O3, Y3, S3 = mk()
+    R.ret_chunkwise_prepared(qh, kt, Vd, g, 128, O=O3, G=Gd, Y=Y3, state_in=S0d, state_out=S3,
+                             rotate=True, pos_offset=9)
+    torch.cuda.synchronize()
+    for a, b in ((O1, O2), (Y1, Y2), (S1, S2), (O1, O3), (Y1, Y3), (S1, S3)):
+        assert torch.equal(a, b)
+    pairs = [(0, 0), (1, 7), (3, 19)]
+    pick = lambda X: np.stack([X[b, h].double().numpy() for b, h in pairs])[None]  # noqa: E731
+    O_ref, S_ref = orc.recurrent(pick(Q), pick(K), pick(V), [g[h] for _, h in pairs], rotate=True,
+                                 pos_offset=9, state_in=pick(S0))
+    for i, (b, h) in enumerate(pairs):
+        assert rel_l2(O1[b, h], O_ref[0, i]) <= TOL_BF16, (b, h)
+        assert rel_l2(S1[b, h], S_ref[0, i]) <= TOL_BF16, (b, h)
