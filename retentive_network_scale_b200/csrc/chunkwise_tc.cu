@@ -996,11 +996,17 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
                                 cudaStream_t st) {
     if (!prep_ws) return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 0, status, st);
     SideStream *ss = side_stream();
+    // as many slices as waves, when every slice then fits in one wave (so
+    // slicing never adds a wave); otherwise one launch
+    constexpr int kMaxSlices = 16;
     const long long ctas_per_b = (long long)p.H * (p.dv / kTV);
-    constexpr int kMaxSlices = 16;  // beyond, a slice takes several waves
-    const int slices =
-        ss ? (int)std::min<long long>(std::min(p.B, kMaxSlices), (ctas_per_b * p.B + ss->sms - 1) / ss->sms)
-           : 1;
+    int slices = 1;
+    if (ss) {
+        const long long waves = (ctas_per_b * p.B + ss->sms - 1) / ss->sms;
+        const long long per_slice = (p.B + waves - 1) / waves;  // batch elements, at most
+        if (waves > 1 && waves <= std::min(p.B, kMaxSlices) && per_slice * ctas_per_b <= ss->sms)
+            slices = (int)waves;
+    }
     if (slices <= 1) {
         cudaError_t e = launch_chunkwise_prep(p, kC, Q, K, prep_ws, &Q, &K, st);
         if (e != cudaSuccess) return e;
