@@ -19,9 +19,17 @@
  *    device (or managed memory); every one must be 16-byte aligned.  Pointers
  *    named as host pointers are read during the call only.
  *  - The caller owns every buffer and the stream.  The library allocates no
- *    device memory, keeps no per-call state, and never synchronises unless a
- *    function says so.  `stream` is a cudaStream_t passed as void*; NULL is
- *    the legacy default stream.
+ *    device memory (cuBLAS allocates its own when the library first makes a
+ *    handle on a device, for ret_msr_layer and ret_segment_state), keeps no
+ *    per-call state, and never synchronises unless a function says so.
+ *    `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.
+ *  - Process-level objects, made once per device under a lock: the device
+ *    status word of the bounded waits (a __device__ variable), the cuBLAS
+ *    handle, and the side stream with two events on which ret_chunkwise runs
+ *    the streaming pass of its next batch slice.  Calls from several host
+ *    threads are safe; on one device they take those locks in turn while
+ *    they enqueue work.
  *  - Arguments are checked before any launch.  A call that returns an error
  *    launched nothing and wrote nothing.  A call that returns RET_OK has only
  *    queued work: kernel faults surface on the stream, and a bounded device
