@@ -217,7 +217,11 @@ def run_reference(args, world, rank):
     val = statistics.median(values)
     line = {"impl": "reference", "metric": "retention fwd tokens/s (RetNet-1.3B MSR chunkwise + GN/gate)",
             "value": val, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "warmup": args.warmup,
+            # each step is a bounded sample of the workload: the time a whole
+            # step (B*L tokens) would take at the sampled rate
+            "ms_per_step": w.B * w.L / val * 1e3, "ms_per_step_extrapolated": True,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w),
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -414,6 +418,42 @@ def bench_seqshard(R, w, d, pk, reps=5, parts=8):
                          "state_scan_frac": scan_bytes / (ms_scan * 1e-3) / 1e9 / pk["hbm_gbs"]}}
 
 
+def bench_long_ctx(R, pk, reps=3, segments=8):
+    """Long context (B=1 H=16 L=65536 d_k=128 d_v=256, chunk 256, xPos, O and
+    the final state): the plain chunk loop (32 CTAs on 148 SMs) against the
+    same sequences cut into `segments` segments that run at once."""
+    w = WORKLOADS["long_ctx"]
+    d = make_inputs(w, device="cuda")
+    g = R.msr_gammas(w.H)
+    O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
+    S = torch.empty(w.B, w.H, w.d_k, w.d_v, device="cuda")
+    ws_plain = torch.empty(R.ret_chunkwise_prep_size(w.B, w.H, w.L, w.d_k, w.d_v, R.RET_BF16,
+                                                     R.RET_BF16, g, w.chunk, rotate=w.rotate),
+                           dtype=torch.uint8, device="cuda")
+    ws_seg = torch.empty(R.lib_segmented_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, w.chunk,
+                                                        segments, w.rotate),
+                         dtype=torch.uint8, device="cuda")
+    plain = lambda: R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, O=O, state_out=S,  # noqa: E731
+                                    rotate=w.rotate, workspace=ws_plain)
+    seg = lambda: R.ret_chunkwise_segmented(d["Q"], d["K"], d["V"], g, w.chunk, segments, O=O,  # noqa: E731
+                                            state_out=S, rotate=w.rotate, workspace=ws_seg)
+    for _ in range(2):
+        plain(); seg()
+    stream = torch.cuda.current_stream()
+    ms_plain = time_launches(plain, reps, stream)
+    ms_seg = time_launches(seg, reps, stream)
+    tokens = w.B * w.L
+    # algorithmic bytes of the loop: Q, K (prepared copies), V read, O written
+    loop_bytes = sum(t.numel() * t.element_size() for k, t in d.items() if k in ("Q", "K", "V")) + \
+        O.numel() * O.element_size()
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d_k={w.d_k} d_v={w.d_v} chunk={w.chunk}, "
+                        f"O and the final state",
+            "plain_ms": ms_plain, "segmented_ms": ms_seg, "segments": segments,
+            "tokens_per_s_plain": tokens / (ms_plain * 1e-3),
+            "tokens_per_s_segmented": tokens / (ms_seg * 1e-3),
+            "segmented_gbs": loop_bytes / (ms_seg * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"]}
+
+
 def bench_layer(R, w, pk, reps=5):
     """The whole multi-scale retention layer on the RetNet-1.3B head shape:
     d_model = H*d_k, random bf16 weights (the shapes matter, not the values)."""
@@ -573,6 +613,8 @@ def run_ours(args, world, rank, local):
         extra["backward"] = bench_backward(R, w, d, pk)
         extra["sequence_shard"] = bench_seqshard(R, w, d, pk)
         del d
+        torch.cuda.empty_cache()
+        extra["long_ctx"] = bench_long_ctx(R, pk)
         torch.cuda.empty_cache()
         extra["msr_layer"] = bench_layer(R, w, pk)
         torch.cuda.empty_cache()

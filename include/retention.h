@@ -370,6 +370,37 @@ ret_status ret_state_scan(const ret_desc *desc, int n_seg, const int *seg_len,
                           float *R, void *stream);
 
 /*
+ * ret_chunkwise_segmented -- ret_chunkwise for few long sequences, on one
+ * device: every sequence is cut into `segments` equal segments of L /
+ * segments rows, which run at once (the chunkwise recurrence of section
+ * 2.1, form (3), holds between segments as between chunks).  Each segment's
+ * own state comes from a streaming pass and one batched GEMM (as in
+ * ret_segment_state), a scan gives every segment its entering state, and
+ * one launch of the tensor-core chunk loop computes all segments, each from
+ * its state: S times the CTAs of the plain loop, for B*H*d_v/128 well below
+ * the number of SMs.  Same result as ret_chunkwise up to rounding.
+ *   Q, K  device bf16 [B][H][L][d_k];  V device bf16 [B][H][L][d_v]
+ *   state_in   device fp32 [B][H][d_k][d_v] or NULL (zero state)
+ *   state_out  device fp32 [B][H][d_k][d_v] or NULL: after the last row
+ *   O          device out_dtype [B][H][L][d_v], fully overwritten
+ *   workspace  device, 256-byte aligned, at least
+ *              ret_chunkwise_segmented_workspace_size() bytes
+ * Tensor-core shapes only; L a multiple of `segments`, H * segments <=
+ * RET_MAX_HEADS, B * H * segments <= 65535 (else RET_ERR_SHAPE).  No gate
+ * (use ret_gate_norm on O).  Errors: those of ret_chunkwise.
+ */
+ret_status ret_chunkwise_segmented(const ret_desc *desc, int chunk, int segments,
+                                   const void *Q, const void *K, const void *V,
+                                   const float *state_in, float *state_out,
+                                   void *O, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/* Device workspace bytes ret_chunkwise_segmented needs; 0 for calls it
+ * would reject by their arguments.  Never fails. */
+size_t ret_chunkwise_segmented_workspace_size(const ret_desc *desc, int chunk,
+                                              int segments);
+
+/*
  * ret_selftest_wait_timeout -- diagnostic, no counterpart in the paper.
  * Queues one small kernel on `stream` that waits on an mbarrier nothing
  * completes, through the same bounded wait every tensor-core kernel uses,

@@ -22,6 +22,12 @@ struct Params {
     long long pos_offset;
     float log2g[RET_MAX_HEADS];
     double theta[kMaxDk / 2];  // theta_j = base^(-2j/dk), fp64 from the host
+    // Rows of head h sit at positions pos_offset + (h mod seg_heads) * seg_len
+    // + t: a sequence read as seg_heads segments of seg_len rows, each segment
+    // a head of its own ([B][H][L][d] is [B][H*S][L/S][d]).  1 and 0 for
+    // plain heads; only the streaming pass reads them.
+    int seg_heads;
+    long long seg_len;
 };
 
 // ------------------------------------------------------------------ dtypes

@@ -83,10 +83,12 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
     }
     float c[4], s[4], cs[4], ss[4];
     if constexpr (ROT) {
+        const long long pos0 =
+            p.pos_offset + (long long)((bh % p.H) % p.seg_heads) * p.seg_len + t0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const double th = s_theta[c16 * 4 + e];
-            rot_cs_fast(p.pos_offset + t0, th, &c[e], &s[e]);
+            rot_cs_fast(pos0, th, &c[e], &s[e]);
             __sincosf((float)th, &ss[e], &cs[e]);  // theta_j <= 1
         }
     }

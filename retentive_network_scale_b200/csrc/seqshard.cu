@@ -1,5 +1,6 @@
-// seqshard.cu -- ret_segment_state and ret_state_scan: a long sequence cut
-// into consecutive segments (one per device), joined through their states.
+// seqshard.cu -- a long sequence cut into consecutive segments, joined
+// through their states: across devices (ret_segment_state, ret_state_scan)
+// and on one device (ret_chunkwise_segmented, for few long sequences).
 //
 // "Retentive Network" paper summary, section 2.1, chunkwise form (3):
 // parallel inside a block of rows, a decayed state carried between blocks.
@@ -10,7 +11,11 @@
 // its own segment at once (a streaming pass that turns and decay-weights the
 // keys, then one batched GEMM), the U are exchanged (an all-gather), and a
 // scan gives each segment its entering state; the segment's outputs then
-// come from ret_chunkwise started from that state.
+// come from ret_chunkwise started from that state.  On one device the same
+// steps run for all segments at once: a [B][H][L][d] tensor read as
+// [B][H*S][L/S][d] is S segment heads per head with uniform strides, so one
+// streaming pass, one batched product, one scan and one chunk-loop launch
+// cover them, with S times the CTAs of the plain loop.
 #include <mutex>
 
 #include "launch.h"
@@ -74,6 +79,78 @@ bool sm100() {
 
 bool a16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
+// U_bh [d_k][d_v] = K~_bh^T V_bh for every (b, h) of p, i.e. in column-major
+// terms the (d_v x d_k) product V_cm (d_v x L) * K~_cm^T (L x d_k); the
+// caller holds blas_mutex().
+ret_status segment_gemm(const Params &p, const void *V, const void *kt, float *U,
+                        void *blas_ws, cudaStream_t st) {
+    cublasHandle_t h = blas_handle(st, blas_ws);
+    if (!h) return RET_ERR_CUDA;
+    const float one = 1.f, zero = 0.f;
+    const long long L = p.L, dk = p.dk, dv = p.dv;
+    const cublasStatus_t r = cublasGemmStridedBatchedEx(
+        h, CUBLAS_OP_N, CUBLAS_OP_T, (int)dv, (int)dk, (int)L, &one, V, CUDA_R_16BF, (int)dv,
+        L * dv, kt, CUDA_R_16BF, (int)dk, L * dk, &zero, U, CUDA_R_32F, (int)dv, dk * dv,
+        p.B * p.H, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+    return r == CUBLAS_STATUS_SUCCESS ? RET_OK : RET_ERR_CUDA;
+}
+
+// The entering state of every segment of every sequence at once, segments
+// of n rows each (R_0 = state_in or 0, R_{s+1} = gamma^n R_s + U_s): one
+// thread per four elements of a (b, h) state walks its S segments in order.
+// U and R are [B][H*S][d_k][d_v] (segment s of head h at h*S + s); state_in
+// is [B][H][d_k][d_v].
+__global__ void __launch_bounds__(256)
+segment_scan_kernel(const Params p, int S, long long n, long long quads,
+                    const float *__restrict__ U, const float *__restrict__ state_in,
+                    float *__restrict__ R) {
+    const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= quads) return;
+    const size_t per = (size_t)p.dk * p.dv;
+    const size_t e = (size_t)q * 4;                  // element of the [B][H] states
+    const size_t bh = e / per, off = e - bh * per;
+    const int h = (int)(bh % p.H);
+    const float g = decay_pow_ll(p.log2g[h], n);
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in) r = *reinterpret_cast<const float4 *>(state_in + e);
+    const size_t first = (bh * S) * per + off;       // segment 0 of this (b, h)
+    for (int s = 0; s < S; ++s) {
+        *reinterpret_cast<float4 *>(R + first + (size_t)s * per) = r;
+        const float4 u = *reinterpret_cast<const float4 *>(U + first + (size_t)s * per);
+        r = make_float4(fmaf(g, r.x, u.x), fmaf(g, r.y, u.y), fmaf(g, r.z, u.z), fmaf(g, r.w, u.w));
+    }
+}
+
+// [B][H][L] heads as [B][H*S][L/S] segment heads: decays repeated per
+// segment, rows at their absolute positions.
+Params segment_params(const Params &p, int S) {
+    Params q = p;
+    q.H = p.H * S;
+    q.L = p.L / S;
+    for (int h = p.H - 1; h >= 0; --h)
+        for (int s = S - 1; s >= 0; --s) q.log2g[h * S + s] = p.log2g[h];
+    q.seg_heads = S;
+    q.seg_len = q.L;
+    return q;
+}
+
+struct SegLayout {
+    size_t prep, states, off_u, off_r, off_s, off_blas, bytes;
+};
+
+SegLayout seg_layout(const Params &p, int S) {
+    const Params q = segment_params(p, S);
+    SegLayout z{};
+    z.prep = round_up(chunkwise_prep_bytes(q));
+    z.states = round_up((size_t)q.B * q.H * q.dk * q.dv * sizeof(float));
+    z.off_u = z.prep;
+    z.off_r = z.off_u + z.states;
+    z.off_s = z.off_r + z.states;
+    z.off_blas = z.off_s + z.states;
+    z.bytes = z.off_blas + kBlasWorkspace;
+    return z;
+}
+
 }  // namespace
 }  // namespace ret
 
@@ -115,18 +192,8 @@ ret_status ret_segment_state(const ret_desc *desc, const void *K, const void *V,
     void *kt = ws;
     // K~ = gamma^{L-1-t} k^_t: the whole segment as one block of rows
     if (launch_key_prep(p, desc->L, K, kt, st) != cudaSuccess) return RET_ERR_CUDA;
-    // U_bh [d_k][d_v] = K~_bh^T V_bh, i.e. in column-major terms the
-    // (d_v x d_k) product V_cm (d_v x L) * K~_cm^T (L x d_k)
     std::lock_guard<std::mutex> lock(blas_mutex());
-    cublasHandle_t h = blas_handle(st, ws + round_up((size_t)bh * desc->L * desc->d_k * 2));
-    if (!h) return RET_ERR_CUDA;
-    const float one = 1.f, zero = 0.f;
-    const long long L = desc->L, dk = desc->d_k, dv = desc->d_v;
-    const cublasStatus_t r = cublasGemmStridedBatchedEx(
-        h, CUBLAS_OP_N, CUBLAS_OP_T, (int)dv, (int)dk, (int)L, &one, V, CUDA_R_16BF, (int)dv,
-        L * dv, kt, CUDA_R_16BF, (int)dk, L * dk, &zero, U, CUDA_R_32F, (int)dv, dk * dv, (int)bh,
-        CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-    return r == CUBLAS_STATUS_SUCCESS ? RET_OK : RET_ERR_CUDA;
+    return segment_gemm(p, V, kt, U, ws + round_up((size_t)bh * desc->L * desc->d_k * 2), st);
 }
 
 ret_status ret_state_scan(const ret_desc *desc, int n_seg, const int *seg_len, int rank,
@@ -159,6 +226,89 @@ ret_status ret_state_scan(const ret_desc *desc, int n_seg, const int *seg_len, i
     state_scan_kernel<<<(unsigned)blocks, 256, 0, st>>>(p, a, quads, seg_elems, U_all, state_in, R);
     if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
     note_launches(1);
+    return RET_OK;
+}
+
+namespace {
+
+// The checks ret_chunkwise_segmented and its size share; fills p.
+ret_status check_segmented(const ret_desc *desc, int chunk, int segments, ret::Params *p) {
+    using namespace ret;
+    ret_status s = validate_desc(desc);
+    if (s != RET_OK) return s;
+    if (desc->in_dtype != RET_BF16) return RET_ERR_DTYPE;
+    if (chunk < 1 || segments < 1) return RET_ERR_ARG;
+    if ((long long)desc->B * desc->L == 0 || desc->L % segments != 0 ||
+        (long long)desc->H * segments > RET_MAX_HEADS ||
+        (long long)desc->B * desc->H * segments > 65535)  // one CTA row per segment head
+        return RET_ERR_SHAPE;
+    params_from_desc(desc, p);
+    if (!chunkwise_tc_supported(*p, chunk, true)) return RET_ERR_SHAPE;
+    return RET_OK;
+}
+
+}  // namespace
+
+size_t ret_chunkwise_segmented_workspace_size(const ret_desc *desc, int chunk, int segments) {
+    ret::Params p;
+    if (check_segmented(desc, chunk, segments, &p) != RET_OK) return 0;
+    return ret::seg_layout(p, segments).bytes;
+}
+
+ret_status ret_chunkwise_segmented(const ret_desc *desc, int chunk, int segments, const void *Q,
+                                   const void *K, const void *V, const float *state_in,
+                                   float *state_out, void *O, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    using namespace ret;
+    Params p;
+    ret_status s = check_segmented(desc, chunk, segments, &p);
+    if (s != RET_OK) return s;
+    if (!Q || !K || !V || !O) return RET_ERR_NULL;
+    if (!a16(Q) || !a16(K) || !a16(V) || !a16(O) || (state_in && !a16(state_in)) ||
+        (state_out && !a16(state_out)))
+        return RET_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return RET_ERR_ALIGN;
+    const SegLayout z = seg_layout(p, segments);
+    if (!workspace || workspace_bytes < z.bytes) return RET_ERR_WORKSPACE;
+    if (!sm100()) return RET_ERR_UNSUPPORTED;
+    int *status = device_status_word();
+    if (!status) return RET_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *U = reinterpret_cast<float *>(ws + z.off_u);
+    float *R = reinterpret_cast<float *>(ws + z.off_r);
+    float *Sout = reinterpret_cast<float *>(ws + z.off_s);
+    const Params q = segment_params(p, segments);
+    // 1. every segment's own state: its keys weighted over the whole segment
+    //    (one block of L/S rows), then the batched product
+    if (launch_key_prep(q, q.L, K, ws, st) != cudaSuccess) return RET_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(blas_mutex());
+        if ((s = segment_gemm(q, V, ws, U, ws + z.off_blas, st)) != RET_OK) return s;
+    }
+    // 2. the state entering each segment
+    const long long quads = (long long)p.B * p.H * p.dk * p.dv / 4;
+    segment_scan_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(p, segments, q.L, quads, U,
+                                                                          state_in, R);
+    if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
+    note_launches(1);
+    // 3. the chunk loop over all segments at once, each from its state (the
+    //    workspace's first part now holds the rows prepared for the loop)
+    const void *qh = nullptr, *kt = nullptr;
+    if (launch_chunkwise_prep(q, kChunkBlock, Q, K, ws, &qh, &kt, st) != cudaSuccess)
+        return RET_ERR_CUDA;
+    if (launch_chunkwise_tc_rows(q, desc->out_dtype == RET_BF16, qh, kt, V, R,
+                                 state_out ? Sout : nullptr, O, nullptr, nullptr, 0.f, status,
+                                 st) != cudaSuccess)
+        return RET_ERR_CUDA;
+    // 4. the state after the last segment of each sequence
+    if (state_out) {
+        const size_t per = (size_t)p.dk * p.dv * sizeof(float);
+        if (cudaMemcpy2DAsync(state_out, per, Sout + (size_t)(segments - 1) * p.dk * p.dv,
+                              per * segments, per, (size_t)p.B * p.H, cudaMemcpyDeviceToDevice,
+                              st) != cudaSuccess)
+            return RET_ERR_CUDA;
+    }
     return RET_OK;
 }
 

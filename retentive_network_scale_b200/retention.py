@@ -33,6 +33,7 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
            "ret_backward", "ret_backward_workspace_size",
            "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
+           "ret_chunkwise_segmented", "ret_chunkwise_segmented_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
            "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
@@ -104,6 +105,10 @@ def load_library(path: str = LIB_PATH):
     lib.ret_segment_state_workspace_size.restype = st
     lib.ret_state_scan.argtypes = [D, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int, vp,
                                    vp, vp, vp]
+    lib.ret_chunkwise_segmented.argtypes = [D, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp,
+                                            vp, st, vp]
+    lib.ret_chunkwise_segmented_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int]
+    lib.ret_chunkwise_segmented_workspace_size.restype = st
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
@@ -424,6 +429,42 @@ def ret_state_scan(U_all, seg_lens, rank, gamma, state_in=None, R=None, stream=N
     _check(lib.ret_state_scan(ctypes.byref(d), len(seg_lens), lens, int(rank), _ptr(U_all),
                               _ptr(state_in), _ptr(R), _stream(stream)), "ret_state_scan")
     return R
+
+
+def ret_chunkwise_segmented(Q, K, V, gamma, chunk, segments, O=None, state_in=None,
+                            state_out=None, rotate=False, theta_base=10000.0, pos_offset=0,
+                            workspace=None, out_dtype=torch.bfloat16, stream=None):
+    """ret_chunkwise for few long sequences: each cut into `segments` equal
+    segments that run at once, joined through their states.  Returns
+    (O, state_out); O is allocated in `out_dtype` when not given, as is the
+    workspace."""
+    lib = load_library()
+    B, H, L, dk = Q.shape
+    dv = V.shape[-1]
+    _dev(Q, "Q", dtype=torch.bfloat16); _dev(K, "K", Q.shape, torch.bfloat16)
+    _dev(V, "V", (B, H, L, dv), torch.bfloat16)
+    if O is None:
+        O = torch.empty(B, H, L, dv, device=Q.device, dtype=out_dtype)
+    _dev(O, "O", (B, H, L, dv))
+    _dev(state_in, "state_in", (B, H, dk, dv), torch.float32)
+    _dev(state_out, "state_out", (B, H, dk, dv), torch.float32)
+    d = make_desc(B, H, L, dk, dv, RET_BF16, _dtype_code(O), gamma, rotate, theta_base, pos_offset)
+    need = int(lib.ret_chunkwise_segmented_workspace_size(ctypes.byref(d), int(chunk), int(segments)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ret_chunkwise_segmented(ctypes.byref(d), int(chunk), int(segments), _ptr(Q), _ptr(K),
+                                       _ptr(V), _ptr(state_in), _ptr(state_out), _ptr(O),
+                                       _ptr(workspace), ws_bytes, _stream(stream)),
+           "ret_chunkwise_segmented")
+    return O, state_out
+
+
+def lib_segmented_workspace_size(B, H, L, d_k, d_v, gamma, chunk, segments, rotate=False):
+    """Device workspace bytes of ret_chunkwise_segmented for these sizes."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, RET_BF16, RET_BF16, gamma, rotate)
+    return int(lib.ret_chunkwise_segmented_workspace_size(ctypes.byref(d), int(chunk), int(segments)))
 
 
 def ret_selftest_wait_timeout(cycles, stream=None):

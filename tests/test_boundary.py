@@ -272,3 +272,27 @@ def test_chunkwise_prepared_arguments(lib):
     assert call(V=MISALIGNED) == S("RET_ERR_ALIGN")
     if not torch.cuda.is_available():
         assert call() == S("RET_ERR_UNSUPPORTED")
+
+
+def test_chunkwise_segmented_arguments(lib):
+    """ret_chunkwise_segmented rejects bad calls before any CUDA call, and
+    its workspace size is 0 for the calls it would reject."""
+    S = R.STATUS_NAMES.index
+    d = desc(B=1, H=4, L=1024, d_k=128, d_v=256, gamma=[0.9, 0.95, 0.99, 0.999])
+    call = lambda dd=d, chunk=128, seg=4, Q=FAKE, O=FAKE, ws=None, nb=0: \
+        lib.ret_chunkwise_segmented(ctypes.byref(dd), chunk, seg, Q, FAKE, FAKE, None, None, O,
+                                    ws, nb, None)
+    size = lambda dd=d, chunk=128, seg=4: lib.ret_chunkwise_segmented_workspace_size(
+        ctypes.byref(dd), chunk, seg)
+    assert call(seg=0) == S("RET_ERR_ARG") and size(seg=0) == 0
+    assert call(seg=3) == S("RET_ERR_SHAPE") and size(seg=3) == 0          # L % segments
+    assert call(seg=64) == S("RET_ERR_SHAPE")                                # H * segments > 128
+    assert call(chunk=64) == S("RET_ERR_SHAPE")                              # not a tensor-core chunk
+    assert call(dd=desc(B=1, H=4, L=1024, d_k=128, d_v=256, in_dtype=R.RET_F32,
+                        gamma=[0.9] * 4)) == S("RET_ERR_DTYPE")
+    assert call(O=None) == S("RET_ERR_NULL")
+    assert call(Q=MISALIGNED) == S("RET_ERR_ALIGN")
+    assert size() > 0
+    assert call() == S("RET_ERR_WORKSPACE")
+    if not torch.cuda.is_available():
+        assert call(ws=FAKE, nb=size()) == S("RET_ERR_UNSUPPORTED")

@@ -246,6 +246,15 @@ def test_long_ctx_sampled():
         assert rel_l2(O[b, h], O_ref[i]) <= TOL_BF16, (b, h)
         assert rel_l2(O[b, h, :4096], O_ref[i, :4096]) <= TOL_BF16, (b, h)
         assert rel_l2(S[b, h], S_ref[i]) <= TOL_BF16, (b, h)
+    # the same with the sequence cut into 8 segments that run at once
+    O8 = torch.empty_like(O)
+    S8 = torch.empty_like(S)
+    R.ret_chunkwise_segmented(d["Q"], d["K"], d["V"], R.msr_gammas(w.H), w.chunk, 8, O=O8,
+                              state_out=S8, rotate=w.rotate)
+    for i, (b, h) in enumerate(pairs):
+        assert rel_l2(O8[b, h], O_ref[i]) <= TOL_BF16, (b, h)
+        assert rel_l2(O8[b, h, :4096], O_ref[i, :4096]) <= TOL_BF16, (b, h)
+        assert rel_l2(S8[b, h], S_ref[i]) <= TOL_BF16, (b, h)
 
 
 def test_msr_1p3b_parallel_sampled():

@@ -3,7 +3,8 @@ ret_state_scan against the fp64 oracle (itself pinned to one uncut
 recurrent run), and whole sequences cut into segments that run one after
 another on this GPU -- each through the same function a rank runs, with the
 all-gather replaced by the stacked segment states -- against the oracle's
-uncut run: outputs, the fused GroupNorm + gate, and the final state.
+uncut run: outputs, the fused GroupNorm + gate, and the final state; and
+ret_chunkwise_segmented, which runs all segments of a sequence at once.
 
 "Retentive Network" paper summary, section 2.1, chunkwise form (3)."""
 import numpy as np
@@ -109,3 +110,30 @@ def test_segments_reproduce_the_uncut_sequence(L, parts, dk, dv, gate):
                               Y_ref[0, a:a + n, h * dv:(h + 1) * dv]) <= TOL_BF16, (r, h)
     for h in range(H):
         assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16, h
+
+
+@pytest.mark.parametrize("L,S,dk,dv,with_in", [
+    (2048, 4, 128, 256, True),     # segments of 512 rows
+    (1200, 3, 256, 128, False),    # segments of 400 rows: ragged last block in each
+    (384, 1, 128, 128, True),      # one segment: the plain loop
+])
+def test_segmented_matches_oracle(L, S, dk, dv, with_in):
+    """ret_chunkwise_segmented: all segments of every sequence at once, each
+    from the state the scan gives it, against the oracle's uncut run
+    (outputs of every head and the final state)."""
+    B, H = 1, 3
+    g = [0.96875, 0.99, 0.999]
+    Q, K, V = _qkv(B, H, L, dk, dv, 130)
+    S0 = random_tensor((B, H, dk, dv), 135, 0.1) if with_in else None
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=77, state_in=S0)
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
+    St = torch.empty(B, H, dk, dv, device="cuda")
+    n0 = R.ret_kernel_launches()
+    R.ret_chunkwise_segmented(Q.cuda(), K.cuda(), V.cuda(), g, 128, S, O=O,
+                              state_in=None if S0 is None else S0.cuda(), state_out=St,
+                              rotate=True, pos_offset=77)
+    assert R.ret_kernel_launches() - n0 == 4        # key pass, scan, prep pass, chunk loop
+    torch.cuda.synchronize()
+    for h in range(H):
+        assert rel_l2(O[0, h], O_ref[0, h]) <= TOL_BF16, h
+        assert rel_l2(St[0, h], S_ref[0, h]) <= TOL_BF16, h
