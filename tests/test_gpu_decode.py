@@ -84,3 +84,24 @@ def test_multi_token_chained_and_single_steps():
     assert normwise(st, S_ref) <= TOL_F32
     assert normwise(got, o_single.cpu().double().numpy()) <= TOL_F32
     assert normwise(st, st1.cpu().double().numpy()) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_multi_token_fast_decays_take_the_direct_form(dtype):
+    """Heads with gamma^T below 2^-60 (gamma 0 and 0.01 at T = 16) run the
+    direct update in the same call as a slow head on the rescaled one; all
+    three match the oracle."""
+    B, H, T, dk, dv, p0 = 2, 3, 16, 64, 128, 500
+    q, k, v, s0 = _case(B, H, T, dk, dv, dtype, 77)
+    g = [0.0, 0.01, 0.9]
+    O_ref, S_ref = orc.recurrent(q, k, v, g, rotate=True, pos_offset=p0, state_in=s0)
+    state = s0.cuda()
+    o = torch.empty(B, H, T, dv, device="cuda", dtype=dtype)
+    R.ret_recurrent_step(q.cuda(), k.cuda(), v.cuda(), state, o, g, pos=p0, rotate=True)
+    torch.cuda.synchronize()
+    if dtype == torch.float32:
+        assert normwise(o, O_ref) <= TOL_F32
+        assert normwise(state, S_ref) <= TOL_F32
+    else:
+        assert rel_l2(o, O_ref) <= TOL_BF16
+        assert rel_l2(state, S_ref) <= TOL_BF16
