@@ -155,13 +155,16 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q,
  * it until the process exits.  Nothing is allocated by this call.
  *   - Problems whose scratch would exceed the array return
  *     RET_ERR_WORKSPACE before anything runs.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first
- *     call before any stream capture.
+ *   - The first call on each device that needs the array looks up its
+ *     device address (cudaGetSymbolAddress) with that device current; make
+ *     that first call before any stream capture.  A failed lookup returns
+ *     RET_ERR_CUDA, leaves no CUDA error pending and is tried again by the
+ *     next call.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents; calls that overlap on the GPU (other streams or threads)
  *     race on it.
- * Arguments, layouts and other errors are those of ret_chunkwise.
+ * Arguments, layouts and other errors are those of ret_chunkwise; the
+ * description, chunk and NULL checks come before the size check.
  */
 #define RET_STATIC_SCRATCH_FLOATS (4u << 20)
 ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk, const void *Q,

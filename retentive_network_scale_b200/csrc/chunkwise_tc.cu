@@ -928,10 +928,20 @@ bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
 
 namespace {
 
-// The chunk loop on rows that are ready (prepared when `pre`).
+// The chunk loop on rows that are ready: prepared by the streaming pass
+// (`pre`, the key rows carry their weight) or, without rotation, Q and K as
+// they are (the loop weights the value rows).  Both run on the pipelined
+// kernel of chunkwise_ws.cu; rotated rows that nobody prepared go to the
+// kernel below, which turns them itself.
 cudaError_t launch_tc_rows(const Params &p, bool out_bf16, const void *Q, const void *K,
                            const void *V, const float *s_in, float *s_out, void *O, const void *G,
                            void *Y, float eps, int pre, int *status, cudaStream_t st) {
+    if (pre || !p.rotate) {
+        const RowLayout hm = bhld_layout(p, p.dk), vl = bhld_layout(p, p.dv);
+        const RowLayout gl{(long long)p.H * p.dv, 0, (long long)p.L * p.H * p.dv};
+        return launch_chunkwise_ws(p, out_bf16, Q, hm, K, V, vl, true, s_in, s_out, O, G, gl, Y,
+                                   eps, !pre, status, st);
+    }
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kC) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC) ||
@@ -994,7 +1004,8 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
                                 const void *V, const float *s_in, float *s_out, void *O,
                                 const void *G, void *Y, float eps, void *prep_ws, int *status,
                                 cudaStream_t st) {
-    if (!prep_ws) return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 0, status, st);
+    if (!prep_ws || !p.rotate)
+        return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 0, status, st);
     SideStream *ss = side_stream();
     // as many slices as waves, when every slice then fits in one wave (so
     // slicing never adds a wave); otherwise one launch
@@ -1069,20 +1080,8 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
                                          RowLayout v_layout, bool v_head_major, const void *G,
                                          RowLayout g_layout, void *Y, void *O, float eps,
                                          int *status, cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
-    const int bh = p.B * p.H;
-    if (!make_tma_map_bf16_strided(&mq, Qh, p.dk, p.L, bh, q_layout.row, q_layout.head, kC) ||
-        !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kC))
-        return cudaErrorInvalidValue;
-    const bool ok = v_head_major
-                        ? make_tma_map_bf16_strided(&mv, V, p.dv, p.L, bh, v_layout.row, v_layout.head, kC)
-                        : make_tma_map_bf16_strided(&mv, V, p.H * p.dv, p.L, p.B, v_layout.row,
-                                                    v_layout.batch, kC);
-    if (!ok) return cudaErrorInvalidValue;
-    const Views vw{v_head_major ? 1 : 0, g_layout};
-    if (p.dk == 256)
-        return launch_dk<256>(p, out_bf16, mq, mk, mv, nullptr, nullptr, O, G, Y, eps, 1, vw, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, nullptr, nullptr, O, G, Y, eps, 1, vw, status, st);
+    return launch_chunkwise_ws(p, out_bf16, Qh, q_layout, Kt, V, v_layout, v_head_major, nullptr,
+                               nullptr, O, G, g_layout, Y, eps, false, status, st);
 }
 
 }  // namespace ret

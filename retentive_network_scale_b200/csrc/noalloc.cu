@@ -24,23 +24,29 @@ constexpr int kMaxDevices = 64;
 // device address comes from cudaGetSymbolAddress, once per device.
 __device__ __align__(256) float g_chunkwise_scratch[kScratchFloats];
 
-std::once_flag g_setup_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_setup_err[kMaxDevices];
+std::mutex g_setup_mu[kMaxDevices];
+void *g_scratch_ptr[kMaxDevices];  // NULL until a lookup on that device succeeded
 
-// Device address of the scratch on the current device (set up on first use).
+// Device address of the scratch on the current device, looked up on first
+// use with that device current.  Only a successful lookup is kept; after a
+// failure (for instance a first call made inside a stream capture) the
+// CUDA error is cleared, so that it is not reported by a later, unrelated
+// launch, and the next call tries again.
 ret_status scratch_on_current_device(void **ptr) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
         return RET_ERR_UNSUPPORTED;
     }
-    std::call_once(g_setup_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_setup_mu[dev]);
+    if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
-        g_setup_err[dev] = cudaGetSymbolAddress(&p, g_chunkwise_scratch);
+        if (cudaGetSymbolAddress(&p, g_chunkwise_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return RET_ERR_CUDA;
+        }
         g_scratch_ptr[dev] = p;
-    });
-    if (g_setup_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return RET_ERR_CUDA;
+    }
     *ptr = g_scratch_ptr[dev];
     return RET_OK;
 }
@@ -52,7 +58,13 @@ extern "C" ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk,
                                                 const float *state_in, float *state_out,
                                                 const void *G, float gn_eps, void *Y,
                                                 void *stream) {
-    // Same argument checks as ret_chunkwise; then the scratch it would need.
+    // The description, the chunk and the G / Y pair are checked first, so
+    // that these errors are the ones ret_chunkwise would report; then the
+    // scratch this call needs against the array.
+    ret_status s = ret::validate_desc(desc);
+    if (s != RET_OK) return s;
+    if (chunk < 1) return RET_ERR_ARG;
+    if ((long long)desc->B * desc->L > 0 && (!G || !Y)) return RET_ERR_NULL;
     const size_t need = ret_workspace_size(desc, chunk, 0, 1);
     if (need > kScratchFloats * sizeof(float)) return RET_ERR_WORKSPACE;
     if (need == 0) {
@@ -62,7 +74,7 @@ extern "C" ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk,
                              nullptr, 0, stream);
     }
     void *scratch = nullptr;
-    ret_status s = scratch_on_current_device(&scratch);
+    s = scratch_on_current_device(&scratch);
     if (s != RET_OK) return s;
     return ret_chunkwise(desc, chunk, Q, K, V, state_in, state_out, nullptr, G, gn_eps, Y, scratch,
                          kScratchFloats * sizeof(float), stream);

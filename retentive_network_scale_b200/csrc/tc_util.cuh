@@ -55,6 +55,47 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
     return true;
 }
+// One arrival on a barrier of this CTA (release at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// One arrival on a barrier of another CTA of the cluster (`addr` from
+// map_to_rank), releasing at CTA scope.  (A cluster-scope release here was
+// measured to wait several microseconds for the memory traffic of the
+// whole SM; callers order what the peers read themselves.)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// mbar_wait_bounded for a barrier that other CTAs of the cluster arrive on:
+// the completed phase also acquires their released writes.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity,
+                                                          volatile int *abort_flag, int *status,
+                                                          long long limit) {
+    const long long start = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - start > limit) {
+            *abort_flag = 1;
+            atomicExch(status, (int)RET_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
 // Makes the generic-proxy writes of this thread to shared memory visible to
 // the async proxy (TMA, tensor cores).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -235,6 +276,20 @@ __device__ __forceinline__ void named_arrive(int id, int n) {
 // Barrier over `count` threads of this CTA on hardware barrier `id` (1..15).
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Barrier over `count` threads of this CTA on hardware barrier `id` that
+// also returns, to every one of them, whether `pred` held for all.
+__device__ __forceinline__ bool named_sync_and(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {

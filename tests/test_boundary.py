@@ -296,3 +296,20 @@ def test_chunkwise_segmented_arguments(lib):
     assert call() == S("RET_ERR_WORKSPACE")
     if not torch.cuda.is_available():
         assert call(ws=FAKE, nb=size()) == S("RET_ERR_UNSUPPORTED")
+
+
+def test_static_entry_checks_arguments_before_its_scratch_limit(lib):
+    """ret_chunkwise_gate_static reports the errors ret_chunkwise would
+    before it compares the problem with its fixed scratch: a missing Y on a
+    shape far beyond the array is a NULL error, not a workspace one."""
+    S = lambda n: R.STATUS_NAMES.index(n)  # noqa: E731
+    big_L = R.RET_STATIC_SCRATCH_FLOATS  # B*H*L*d_v floats far beyond the array
+    d = desc(B=1, H=1, L=big_L, d_k=16, d_v=64, in_dtype=R.RET_F32, out_dtype=R.RET_F32,
+             gamma=[0.9])
+    call = lambda dd, chunk=16, G=FAKE, Y=FAKE: lib.ret_chunkwise_gate_static(  # noqa: E731
+        ctypes.byref(dd), chunk, FAKE, FAKE, FAKE, None, None, G, ctypes.c_float(1e-5), Y, None)
+    assert call(d, Y=None) == S("RET_ERR_NULL")
+    assert call(d, G=None) == S("RET_ERR_NULL")
+    assert call(d, chunk=0) == S("RET_ERR_ARG")
+    assert call(desc(gamma=[1.5, 0.9])) == S("RET_ERR_ARG")
+    assert call(d) == S("RET_ERR_WORKSPACE")

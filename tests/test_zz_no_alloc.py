@@ -1,16 +1,20 @@
 """ret_chunkwise_gate_static: the chunkwise forward with the fused
 GroupNorm + swish gate for callers that may not allocate device memory
 (memory reserved up front by a host framework, or a fixed budget once
-serving starts).  Its scratch is the library's fixed device array, so the
-test checks, through the C ABI, that two calls in a row match the
-allocating entry point ret_chunkwise on the same inputs, and that a problem
-too large for the array is refused.  It sits in a file of its own, collected
-last, and must pass alone in a fresh process as well."""
+serving starts).  Its scratch is the library's fixed device array.  The
+tests call it through the C ABI, twice in a row (the calls share the
+array), and check Y and the final state against the fp64 oracle and against
+the allocating entry point ret_chunkwise on the same inputs: on the CUDA-core
+path, which uses the array, and on the tensor-core path, which needs none.
+A problem too large for the array is refused.  The file sits on its own,
+collected last, and must pass alone in a fresh process as well."""
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+from oracle import oracle as orc
 from parity import normwise, rel_l2, TOL_BF16, TOL_F32
 from retentive_network_scale_b200 import build
 from retentive_network_scale_b200 import retention as R
@@ -29,41 +33,56 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _call_static(lib, Q, K, V, G, Y, g, chunk, rotate):
+def _call_static(lib, Q, K, V, G, Y, g, chunk, rotate, S_in=None, S_out=None):
     B, H, L, dk = Q.shape
     dv = V.shape[-1]
     code = R.RET_F32 if Q.dtype == torch.float32 else R.RET_BF16
     d = R.make_desc(B, H, L, dk, dv, code, code, g, rotate)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    return lib.ret_chunkwise_gate_static(ctypes.byref(d), chunk, _ptr(Q), _ptr(K), _ptr(V), None,
-                                         None, _ptr(G), ctypes.c_float(1e-5), _ptr(Y), stream)
+    return lib.ret_chunkwise_gate_static(ctypes.byref(d), chunk, _ptr(Q), _ptr(K), _ptr(V),
+                                         _ptr(S_in), _ptr(S_out), _ptr(G), ctypes.c_float(1e-5),
+                                         _ptr(Y), stream)
 
 
-@pytest.mark.parametrize("dtype,dk,dv,rotate", [
-    (torch.float32, 32, 48, True),
-    (torch.bfloat16, 64, 64, False),
+@pytest.mark.parametrize("dtype,dk,dv,chunk,rotate,with_state,scratch", [
+    (torch.float32, 32, 48, 32, True, False, True),     # CUDA-core path: uses the array
+    (torch.bfloat16, 64, 64, 32, False, True, True),    # CUDA-core path: uses the array
+    (torch.bfloat16, 128, 128, 128, True, True, False),  # tensor-core path: no scratch
 ])
-def test_static_scratch_matches_allocating_entry(lib, dtype, dk, dv, rotate):
-    B, H, L, chunk = 2, 3, 150, 32
-    Q = random_tensor((B, H, L, dk), 61, dk ** -0.5).to(dtype).cuda()
-    K = random_tensor((B, H, L, dk), 62, dk ** -0.5).to(dtype).cuda()
-    V = random_tensor((B, H, L, dv), 63).to(dtype).cuda()
-    G = random_tensor((B, L, H * dv), 64).to(dtype).cuda()
+def test_static_scratch_matches_oracle_and_allocating_entry(lib, dtype, dk, dv, chunk, rotate,
+                                                            with_state, scratch):
+    B, H, L = 2, 3, 150
+    Q = random_tensor((B, H, L, dk), 61, dk ** -0.5).to(dtype)
+    K = random_tensor((B, H, L, dk), 62, dk ** -0.5).to(dtype)
+    V = random_tensor((B, H, L, dv), 63).to(dtype)
+    G = random_tensor((B, L, H * dv), 64).to(dtype)
+    S0 = random_tensor((B, H, dk, dv), 65, 0.2) if with_state else None
     g = [0.9, 0.96875, 0.999]
-    # this shape needs scratch in ret_chunkwise (the CUDA-core path)
-    assert R.ret_workspace_size(B, H, L, dk, dv, R._dtype_code(Q), R._dtype_code(Q), g, chunk,
-                                want_O=False, want_Y=True, rotate=rotate) > 0
-    Y_ref = torch.empty(B, L, H * dv, device="cuda", dtype=dtype)
-    R.ret_chunkwise(Q, K, V, g, chunk, G=G, Y=Y_ref, rotate=rotate)
-    for _ in range(2):  # two calls in a row share the scratch
+    need = R.ret_workspace_size(B, H, L, dk, dv, R._dtype_code(Q), R._dtype_code(Q), g, chunk,
+                                want_O=False, want_Y=True, rotate=rotate)
+    assert (need > 0) == scratch
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=rotate, state_in=S0)
+    Y_ref = orc.gate_groupnorm(O_ref, G)
+    Qd, Kd, Vd, Gd = Q.cuda(), K.cuda(), V.cuda(), G.cuda()
+    S0d = None if S0 is None else S0.cuda()
+    # the allocating entry point, with its workspace (or the prep workspace
+    # of the tensor-core path)
+    Y_alloc = torch.empty(B, L, H * dv, device="cuda", dtype=dtype)
+    S_alloc = torch.empty(B, H, dk, dv, device="cuda")
+    R.ret_chunkwise(Qd, Kd, Vd, g, chunk, G=Gd, Y=Y_alloc, rotate=rotate, state_in=S0d,
+                    state_out=S_alloc, prep=not scratch)
+    metric, tol = (normwise, TOL_F32) if dtype == torch.float32 else (rel_l2, TOL_BF16)
+    for _ in range(2):  # two calls in a row share the array
         Y = torch.full((B, L, H * dv), float("nan"), device="cuda", dtype=dtype)
-        assert _call_static(lib, Q, K, V, G, Y, g, chunk, rotate) == 0
+        S = torch.full((B, H, dk, dv), float("nan"), device="cuda")
+        assert _call_static(lib, Qd, Kd, Vd, Gd, Y, g, chunk, rotate, S0d, S) == 0
         torch.cuda.synchronize()
         assert R.ret_last_device_status() == 0
-        if dtype == torch.float32:
-            assert normwise(Y, Y_ref) <= TOL_F32
-        else:
-            assert rel_l2(Y, Y_ref) <= TOL_BF16
+        assert metric(Y, Y_ref) <= tol
+        assert metric(S, S_ref) <= tol
+        assert metric(Y, Y_alloc) <= tol
+        assert metric(S, S_alloc) <= tol
+        assert np.isfinite(Y.float().cpu().numpy()).all()
 
 
 def test_static_scratch_refuses_oversized_problem(lib):
