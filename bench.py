@@ -443,15 +443,25 @@ def bench_long_ctx(R, pk, reps=3, segments=8):
     ms_plain = time_launches(plain, reps, stream)
     ms_seg = time_launches(seg, reps, stream)
     tokens = w.B * w.L
-    # algorithmic bytes of the loop: Q, K (prepared copies), V read, O written
-    loop_bytes = sum(t.numel() * t.element_size() for k, t in d.items() if k in ("Q", "K", "V")) + \
+    # algorithmic bytes: Q, K, V read once, O written (bf16); algorithmic
+    # flops of the chunkwise form at the workload's chunk
+    alg_bytes = sum(t.numel() * t.element_size() for k, t in d.items() if k in ("Q", "K", "V")) + \
         O.numel() * O.element_size()
+    flops = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
+    gbs = alg_bytes / (ms_seg * 1e-3) / 1e9
+    tf = flops / (ms_seg * 1e-3) / 1e12
     return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d_k={w.d_k} d_v={w.d_v} chunk={w.chunk}, "
                         f"O and the final state",
             "plain_ms": ms_plain, "segmented_ms": ms_seg, "segments": segments,
             "tokens_per_s_plain": tokens / (ms_plain * 1e-3),
             "tokens_per_s_segmented": tokens / (ms_seg * 1e-3),
-            "segmented_gbs": loop_bytes / (ms_seg * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"]}
+            # the whole segmented call (key pass, segment states on the
+            # tensor cores, scan, prep pass, chunk loop) against the
+            # algorithmic work of the workload
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": alg_bytes,
+                         "tensor": {"achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                    "frac": tf / pk["bf16_tflops"], "flops": flops}}}
 
 
 def bench_layer(R, w, pk, reps=5):
@@ -492,9 +502,11 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
-    if args.only in ("decode", "parallel"):
+    if args.only in ("decode", "parallel", "long_ctx"):
         if args.only == "decode":
             out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
+        elif args.only == "long_ctx":
+            out = bench_long_ctx(R, pk)
         else:
             w = WORKLOADS["msr_1p3b"]
             if args.batch:
@@ -647,15 +659,15 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-extra", action="store_true", help="only the main step")
     ap.add_argument("--skip-cpu", action="store_true", help="no CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
-    ap.add_argument("--only", choices=["main", "parallel", "decode"], default=None,
+    ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx"], default=None,
                     help="run one measurement alone (profiler captures)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="override the decode workload's batch (small cases for profiler captures)")

@@ -929,10 +929,11 @@ bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
 namespace {
 
 // The chunk loop on rows that are ready: prepared by the streaming pass
-// (`pre`, the key rows carry their weight) or, without rotation, Q and K as
-// they are (the loop weights the value rows).  Both run on the pipelined
-// kernel of chunkwise_ws.cu; rotated rows that nobody prepared go to the
-// kernel below, which turns them itself.
+// (`pre`, the key rows carry their weight) or, without rotation and
+// without a workspace for that pass, Q and K as they are (the loop then
+// weights the value rows in shared memory, which measured slower than the
+// pass).  Both run on the pipelined kernel of chunkwise_ws.cu; rotated rows
+// that nobody prepared go to the kernel below, which turns them itself.
 cudaError_t launch_tc_rows(const Params &p, bool out_bf16, const void *Q, const void *K,
                            const void *V, const float *s_in, float *s_out, void *O, const void *G,
                            void *Y, float eps, int pre, int *status, cudaStream_t st) {
@@ -1004,7 +1005,7 @@ cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, c
                                 const void *V, const float *s_in, float *s_out, void *O,
                                 const void *G, void *Y, float eps, void *prep_ws, int *status,
                                 cudaStream_t st) {
-    if (!prep_ws || !p.rotate)
+    if (!prep_ws)
         return launch_tc_rows(p, out_bf16, Q, K, V, s_in, s_out, O, G, Y, eps, 0, status, st);
     SideStream *ss = side_stream();
     // as many slices as waves, when every slice then fits in one wave (so

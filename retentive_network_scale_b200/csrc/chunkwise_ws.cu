@@ -187,34 +187,30 @@ __device__ __forceinline__ void st_rbarT_row32(uint8_t *smem, int c, int d0, con
     }
 }
 
-// One row segment of 64 values (this thread's row) leaves as TO, in pieces
-// of 16 bytes that a 4 x 4 transpose among groups of 4 lanes gathers, so
-// that one store instruction covers 64 contiguous bytes of 8 rows: bf16 in
-// two rounds of 32 columns, fp32 in four of 16.  `pair(k)` gives columns
-// 2k, 2k+1 as a packed fp32 pair; `dst(i)` is the address of column 0 of
-// row 4j+i of this lane's group (j = lane >> 2) and `ok(i)` whether that
-// row exists.
+// 32 values of one row (this thread's, columns [col0, col0 + 32)) leave as
+// TO, in pieces of 16 bytes that a 4 x 4 transpose among groups of 4 lanes
+// gathers, so that one store instruction covers 64 contiguous bytes of 8
+// rows: bf16 in one round, fp32 in two of 16 columns.  `pair(k)` gives
+// columns col0 + 2k, col0 + 2k + 1 as a packed fp32 pair; `dst(i)` is the
+// address of column 0 of row 4j+i of this lane's group (j = lane >> 2) and
+// `ok(i)` whether that row exists.
 template <typename TO, typename Pair, typename Dst, typename Ok>
-__device__ __forceinline__ void store_row64(Pair pair, int m, Dst dst, Ok ok) {
+__device__ __forceinline__ void store_row32(Pair pair, int m, int col0, Dst dst, Ok ok) {
     if constexpr (sizeof(TO) == 2) {
+        uint4 a[4];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            uint4 a[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int p0 = 16 * hf + 4 * k;
-                const uint64_t v0 = pair(p0), v1 = pair(p0 + 1), v2 = pair(p0 + 2), v3 = pair(p0 + 3);
-                a[k] = make_uint4(pack_bf16(f2_lo(v0), f2_hi(v0)), pack_bf16(f2_lo(v1), f2_hi(v1)),
-                                  pack_bf16(f2_lo(v2), f2_hi(v2)), pack_bf16(f2_lo(v3), f2_hi(v3)));
-            }
-            xpose4(a, m);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (ok(i)) st_na(reinterpret_cast<__nv_bfloat16 *>(dst(i)) + 32 * hf + 8 * m, a[i]);
+        for (int k = 0; k < 4; ++k) {
+            const uint64_t v0 = pair(4 * k), v1 = pair(4 * k + 1), v2 = pair(4 * k + 2), v3 = pair(4 * k + 3);
+            a[k] = make_uint4(pack_bf16(f2_lo(v0), f2_hi(v0)), pack_bf16(f2_lo(v1), f2_hi(v1)),
+                              pack_bf16(f2_lo(v2), f2_hi(v2)), pack_bf16(f2_lo(v3), f2_hi(v3)));
         }
+        xpose4(a, m);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (ok(i)) st_na(reinterpret_cast<__nv_bfloat16 *>(dst(i)) + col0 + 8 * m, a[i]);
     } else {
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < 2; ++qq) {
             uint4 a[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -225,7 +221,7 @@ __device__ __forceinline__ void store_row64(Pair pair, int m, Dst dst, Ok ok) {
             xpose4(a, m);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok(i)) st_na(reinterpret_cast<float *>(dst(i)) + 16 * qq + 4 * m, a[i]);
+                if (ok(i)) st_na(reinterpret_cast<float *>(dst(i)) + col0 + 16 * qq + 4 * m, a[i]);
         }
     }
 }
@@ -417,7 +413,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         uint8_t *rowp = smem + Ly::kV + nb * 16384 + r * 128;
 #pragma unroll
                         for (int ch = 0; ch < 8; ++ch) {
-                            uint4 *ptr = reinterpret_cast<uint4 *>(rowp + (ch << 4));
+                            // rows of a phase start at different 16-byte pieces: no bank conflicts
+                            uint4 *ptr = reinterpret_cast<uint4 *>(rowp + (((ch + r) & 7) << 4));
                             uint4 w = *ptr;
                             uint32_t *u = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
@@ -625,11 +622,15 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const float off = (shift_p - mean) * scale;
             const uint64_t OFF = f2_make(off, off);
             // Y = swish(G) ((O'' - shift) scale + (shift - mean) scale)
-            store_row64<TO>(
-                [&](int k) { return f2_mul(f2_fma(bf16x2_to_f2(rp[k]), SC, OFF), bf16x2_to_f2(sw[k])); },
-                m4,
-                [&](int i) { return Y + ((size_t)b * L + t0_p + grow(i)) * ((size_t)p.H * dv) + ycol; },
-                [&](int i) { return grow(i) < n_p; });
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                store_row32<TO>(
+                    [&](int k) {
+                        return f2_mul(f2_fma(bf16x2_to_f2(rp[16 * hf + k]), SC, OFF), bf16x2_to_f2(sw[16 * hf + k]));
+                    },
+                    m4, 32 * hf,
+                    [&](int i) { return Y + ((size_t)b * L + t0_p + grow(i)) * ((size_t)p.H * dv) + ycol; },
+                    [&](int i) { return grow(i) < n_p; });
         };
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
@@ -647,33 +648,39 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (!ok) break;
             }
             tc_fence_after();
-            uint32_t x[64];
-            tmem_ld32(tO + lane_base + o0, *reinterpret_cast<uint32_t(*)[32]>(x));
-            tmem_ld32(tO + lane_base + o0 + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-            tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(x));
-            tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(x + 32));
-            tc_fence_before();
-            warp_arrive(OF);  // the next chunk's O'' may overwrite tensor memory
             const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}
-            if (O) {
-                const uint64_t A2 = f2_make(alpha, alpha);
-                store_row64<TO>([&](int k) { return f2_mul(f2_of(x + 2 * k), A2); }, m4,
-                                [&](int i) { return O + ((size_t)bh * L + t0 + grow(i)) * dv + v0 + o0; },
-                                row_ok);
+            const uint64_t A2 = f2_make(alpha, alpha);
+            // O'' in two halves of 32 columns: O (when asked for), the
+            // running statistics (shifted by the row's first value, even
+            // and odd columns in packed fp32 lanes) and the residuals
+            float shift = 0.f;
+            uint64_t S1 = 0, S2 = 0;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t x[32];
+                tmem_ld32(tO + lane_base + o0 + 32 * hf, x);
+                tmem_wait_ld(x);
+                if (hf == 1) {
+                    tc_fence_before();
+                    warp_arrive(OF);  // the next chunk's O'' may overwrite tensor memory
+                }
+                if (O)
+                    store_row32<TO>([&](int k) { return f2_mul(f2_of(x + 2 * k), A2); }, m4, 32 * hf,
+                                    [&](int i) { return O + ((size_t)bh * L + t0 + grow(i)) * dv + v0 + o0; },
+                                    row_ok);
+                if constexpr (FUSE) {
+                    if (hf == 0) shift = __uint_as_float(x[0]);
+                    const uint64_t NSH = f2_make(-shift, -shift);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const uint64_t d = f2_add(f2_of(x + i), NSH);
+                        S1 = f2_add(S1, d);
+                        S2 = f2_fma(d, d, S2);
+                        rp[16 * hf + i / 2] = pack_bf16(f2_lo(d), f2_hi(d));
+                    }
+                }
             }
             if constexpr (FUSE) {
-                // mean and centred sum of squares of the 64 columns, shifted
-                // by the first value; even/odd columns in packed fp32 lanes
-                const float shift = __uint_as_float(x[0]);
-                const uint64_t NSH = f2_make(-shift, -shift);
-                uint64_t S1 = 0, S2 = 0;
-#pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    const uint64_t d = f2_add(f2_of(x + i), NSH);
-                    S1 = f2_add(S1, d);
-                    S2 = f2_fma(d, d, S2);
-                    rp[i / 2] = pack_bf16(f2_lo(d), f2_hi(d));
-                }
                 const float s1 = f2_lo(S1) + f2_hi(S1), s2 = f2_lo(S2) + f2_hi(S2);
                 const float m_w = shift + s1 * (1.f / 64.f);
                 const float m2_w = fmaxf(s2 - s1 * s1 * (1.f / 64.f), 0.f);
@@ -691,8 +698,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // the slots are written (the barrier above ordered them before
                 // this arrival); warp 3 announces them to the cluster
                 if (gtid == 0) mbar_arrive(bar(SL));
-                // G of this chunk (coalesced: one instruction reads four whole
-                // 128-byte row segments), used one chunk later
+                // G of this chunk (coalesced: one instruction reads 64
+                // contiguous bytes of each of 8 rows), used one chunk later
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
 #pragma unroll

@@ -120,6 +120,17 @@ constexpr size_t kBlasWorkspace = 32ull << 20;
 std::mutex &blas_mutex();
 cublasHandle_t blas_handle(cudaStream_t st, void *workspace);
 
+// U = sum_t gamma^{L-1-t} k^_t^T v_t per (b, h) ([d_k][d_v] fp32) on the
+// tensor cores (segstate.cu): K~ [B][H][L][d_k], V [B][H][L][d_v], d_k 128
+// or 256, d_v a multiple of 128.  zeta_v 0: the weight is on K~ already
+// (the streaming pass with the segment as one block); 1: K~ = K^ and the
+// kernel weights the value rows; 2: K~ carries the weights of 128-row
+// blocks (the chunk loop's streaming pass) and the kernel scales each
+// block's value rows by the rest.
+bool segment_state_tc_supported(const Params &p);
+cudaError_t launch_segment_state_tc(const Params &p, const void *V, const void *Kt, int zeta_v,
+                                    float *U, int *status, cudaStream_t st);
+
 // Tensor-core parallel form: bf16 inputs, d_k 128 or 256, d_v a multiple of
 // 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
 // Q^ and K^ (bf16) into the workspace (parallel_tc_workspace bytes).

@@ -9,13 +9,15 @@
 //     R' = gamma^n R + U,   U = sum_{t<n} gamma^{n-1-t} k^_t^T v_t,
 // where U depends on the segment alone.  So every device computes the U of
 // its own segment at once (a streaming pass that turns and decay-weights the
-// keys, then one batched GEMM), the U are exchanged (an all-gather), and a
+// keys, then one product K~^T V on the tensor cores), the U are exchanged
+// (an all-gather), and a
 // scan gives each segment its entering state; the segment's outputs then
 // come from ret_chunkwise started from that state.  On one device the same
 // steps run for all segments at once: a [B][H][L][d] tensor read as
-// [B][H*S][L/S][d] is S segment heads per head with uniform strides, so one
-// streaming pass, one batched product, one scan and one chunk-loop launch
-// cover them, with S times the CTAs of the plain loop.
+// [B][H*S][L/S][d] is S segment heads per head with uniform strides, so the
+// chunk loop's streaming pass (whose weighted keys also serve the segment
+// states), one launch for the segment states, one scan and one chunk-loop
+// launch cover them, with S times the CTAs of the plain loop.
 #include <mutex>
 
 #include "launch.h"
@@ -79,11 +81,20 @@ bool sm100() {
 
 bool a16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
-// U_bh [d_k][d_v] = K~_bh^T V_bh for every (b, h) of p, i.e. in column-major
-// terms the (d_v x d_k) product V_cm (d_v x L) * K~_cm^T (L x d_k); the
-// caller holds blas_mutex().
+// U_bh [d_k][d_v] = K~_bh^T V_bh for every (b, h) of p: on the tensor-core
+// kernel of segstate.cu where it applies (d_k 128 or 256, d_v a multiple of
+// 128); otherwise as one cuBLAS batched GEMM, in column-major terms the
+// (d_v x d_k) product V_cm (d_v x L) * K~_cm^T (L x d_k).
 ret_status segment_gemm(const Params &p, const void *V, const void *kt, float *U,
                         void *blas_ws, cudaStream_t st) {
+    if (segment_state_tc_supported(p)) {
+        int *status = device_status_word();
+        if (!status) return RET_ERR_CUDA;
+        return launch_segment_state_tc(p, V, kt, 0, U, status, st) == cudaSuccess
+                   ? RET_OK
+                   : RET_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(blas_mutex());
     cublasHandle_t h = blas_handle(st, blas_ws);
     if (!h) return RET_ERR_CUDA;
     const float one = 1.f, zero = 0.f;
@@ -192,7 +203,6 @@ ret_status ret_segment_state(const ret_desc *desc, const void *K, const void *V,
     void *kt = ws;
     // K~ = gamma^{L-1-t} k^_t: the whole segment as one block of rows
     if (launch_key_prep(p, desc->L, K, kt, st) != cudaSuccess) return RET_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(blas_mutex());
     return segment_gemm(p, V, kt, U, ws + round_up((size_t)bh * desc->L * desc->d_k * 2), st);
 }
 
@@ -279,29 +289,27 @@ ret_status ret_chunkwise_segmented(const ret_desc *desc, int chunk, int segments
     float *R = reinterpret_cast<float *>(ws + z.off_r);
     float *Sout = reinterpret_cast<float *>(ws + z.off_s);
     const Params q = segment_params(p, segments);
-    // 1. every segment's own state: its keys weighted over the whole segment
-    //    (one block of L/S rows), then the batched product
-    if (launch_key_prep(q, q.L, K, ws, st) != cudaSuccess) return RET_ERR_CUDA;
-    {
-        std::lock_guard<std::mutex> lock(blas_mutex());
-        if ((s = segment_gemm(q, V, ws, U, ws + z.off_blas, st)) != RET_OK) return s;
-    }
-    // 2. the state entering each segment
+    // 1. the chunk loop's streaming pass: Q^ (with rotation) and K~, the keys
+    //    turned and weighted by gamma^{m-1-j} within each block of m <= 128
+    //    rows of each segment
+    const void *qh = nullptr, *kt = nullptr;
+    if (launch_chunkwise_prep(q, kChunkBlock, Q, K, ws, &qh, &kt, st) != cudaSuccess)
+        return RET_ERR_CUDA;
+    // 2. every segment's own state from the same K~, each block's value rows
+    //    scaled by the rest of the segment's weight
+    if (launch_segment_state_tc(q, V, kt, 2, U, status, st) != cudaSuccess) return RET_ERR_CUDA;
+    // 3. the state entering each segment
     const long long quads = (long long)p.B * p.H * p.dk * p.dv / 4;
     segment_scan_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(p, segments, q.L, quads, U,
                                                                           state_in, R);
     if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
     note_launches(1);
-    // 3. the chunk loop over all segments at once, each from its state (the
-    //    workspace's first part now holds the rows prepared for the loop)
-    const void *qh = nullptr, *kt = nullptr;
-    if (launch_chunkwise_prep(q, kChunkBlock, Q, K, ws, &qh, &kt, st) != cudaSuccess)
-        return RET_ERR_CUDA;
+    // 4. the chunk loop over all segments at once, each from its state
     if (launch_chunkwise_tc_rows(q, desc->out_dtype == RET_BF16, qh, kt, V, R,
                                  state_out ? Sout : nullptr, O, nullptr, nullptr, 0.f, status,
                                  st) != cudaSuccess)
         return RET_ERR_CUDA;
-    // 4. the state after the last segment of each sequence
+    // 5. the state after the last segment of each sequence
     if (state_out) {
         const size_t per = (size_t)p.dk * p.dv * sizeof(float);
         if (cudaMemcpy2DAsync(state_out, per, Sout + (size_t)(segments - 1) * p.dk * p.dv,

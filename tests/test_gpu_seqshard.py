@@ -112,12 +112,13 @@ def test_segments_reproduce_the_uncut_sequence(L, parts, dk, dv, gate):
         assert rel_l2(S[0, h], S_ref[0, h]) <= TOL_BF16, h
 
 
-@pytest.mark.parametrize("L,S,dk,dv,with_in", [
-    (2048, 4, 128, 256, True),     # segments of 512 rows
-    (1200, 3, 256, 128, False),    # segments of 400 rows: ragged last block in each
-    (384, 1, 128, 128, True),      # one segment: the plain loop
+@pytest.mark.parametrize("L,S,dk,dv,with_in,rotate", [
+    (2048, 4, 128, 256, True, True),     # segments of 512 rows
+    (1200, 3, 256, 128, False, True),    # segments of 400 rows: ragged last block in each
+    (384, 1, 128, 128, True, True),      # one segment: the plain loop
+    (1200, 3, 128, 256, True, False),    # without rotation: no streaming pass
 ])
-def test_segmented_matches_oracle(L, S, dk, dv, with_in):
+def test_segmented_matches_oracle(L, S, dk, dv, with_in, rotate):
     """ret_chunkwise_segmented: all segments of every sequence at once, each
     from the state the scan gives it, against the oracle's uncut run
     (outputs of every head and the final state)."""
@@ -125,14 +126,15 @@ def test_segmented_matches_oracle(L, S, dk, dv, with_in):
     g = [0.96875, 0.99, 0.999]
     Q, K, V = _qkv(B, H, L, dk, dv, 130)
     S0 = random_tensor((B, H, dk, dv), 135, 0.1) if with_in else None
-    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=True, pos_offset=77, state_in=S0)
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=77, state_in=S0)
     O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
     St = torch.empty(B, H, dk, dv, device="cuda")
     n0 = R.ret_kernel_launches()
     R.ret_chunkwise_segmented(Q.cuda(), K.cuda(), V.cuda(), g, 128, S, O=O,
                               state_in=None if S0 is None else S0.cuda(), state_out=St,
-                              rotate=True, pos_offset=77)
-    assert R.ret_kernel_launches() - n0 == 4        # key pass, scan, prep pass, chunk loop
+                              rotate=rotate, pos_offset=77)
+    # the streaming pass, the segment states, the scan, the chunk loop
+    assert R.ret_kernel_launches() - n0 == 4
     torch.cuda.synchronize()
     for h in range(H):
         assert rel_l2(O[0, h], O_ref[0, h]) <= TOL_BF16, h
