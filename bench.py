@@ -464,6 +464,62 @@ def bench_long_ctx(R, pk, reps=3, segments=8):
                                     "frac": tf / pk["bf16_tflops"], "flops": flops}}}
 
 
+def time_flushed(fn, n, stream, flush):
+    """Median device time (ms) of n calls, each after writing a buffer larger
+    than L2 (so no call finds its inputs in L2), CUDA events per call."""
+    times = []
+    for _ in range(n):
+        flush.zero_()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    return statistics.median(times)
+
+
+def bench_msr_small(R, pk, reps=50):
+    """The small MSR layer's retention (B=4 H=8 L=2048 d_k=d_v=64, chunk 64,
+    no rotation, GroupNorm + swish gate, bf16): the chunkwise call for Y, and
+    the parallel form for O.  Its inputs (42 MB) fit in L2, so L2 is flushed
+    before every timed call."""
+    w = WORKLOADS["msr_small"]
+    d = make_inputs(w, device="cuda")
+    g = R.msr_gammas(w.H)
+    Y = torch.empty(w.B, w.L, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
+    O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(max(1, R.ret_chunkwise_prep_size(w.B, w.H, w.L, w.d_k, w.d_v, R.RET_BF16,
+                                                      R.RET_BF16, g, w.chunk, rotate=w.rotate)),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    chunk = lambda: R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, G=d["G"], Y=Y,  # noqa: E731
+                                    rotate=w.rotate, workspace=ws)
+    par = lambda: R.ret_parallel(d["Q"], d["K"], d["V"], O, g, rotate=w.rotate)  # noqa: E731
+    for _ in range(3):
+        chunk(); par()
+    stream = torch.cuda.current_stream()
+    ms_c = time_flushed(chunk, reps, stream, flush)
+    ms_p = time_flushed(par, reps, stream, flush)
+    alg_bytes = sum(d[k].numel() * d[k].element_size() for k in ("Q", "K", "V", "G")) + \
+        Y.numel() * Y.element_size()
+    fl_c = w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v)
+    fl_p = w.B * w.H * w.L * parallel_flops_per_token_head(w.L, w.d_k, w.d_v)
+    gbs = alg_bytes / (ms_c * 1e-3) / 1e9
+    tf_p = fl_p / (ms_p * 1e-3) / 1e12
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d_k={w.d_k} d_v={w.d_v} chunk={w.chunk}, "
+                        f"no rotation, Y = swish(G) GroupNorm(O), bf16; L2 flushed before each call",
+            "chunkwise_ms": ms_c, "tokens_per_s": w.B * w.L / (ms_c * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": alg_bytes,
+                         "tensor_frac": fl_c / (ms_c * 1e-3) / 1e12 / pk["bf16_tflops"]},
+            "parallel": {"ms": ms_p, "tokens_per_s": w.B * w.L / (ms_p * 1e-3),
+                         "roofline": {"bound": "tensor", "achieved": tf_p, "peak": pk["bf16_tflops"],
+                                      "unit": "TFLOP/s", "frac": tf_p / pk["bf16_tflops"],
+                                      "flops": fl_p}}}
+
+
 def bench_layer(R, w, pk, reps=5):
     """The whole multi-scale retention layer on the RetNet-1.3B head shape:
     d_model = H*d_k, random bf16 weights (the shapes matter, not the values)."""
@@ -502,11 +558,13 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
-    if args.only in ("decode", "parallel", "long_ctx"):
+    if args.only in ("decode", "parallel", "long_ctx", "msr_small"):
         if args.only == "decode":
             out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
         elif args.only == "long_ctx":
             out = bench_long_ctx(R, pk)
+        elif args.only == "msr_small":
+            out = bench_msr_small(R, pk)
         else:
             w = WORKLOADS["msr_1p3b"]
             if args.batch:
@@ -628,6 +686,8 @@ def run_ours(args, world, rank, local):
         torch.cuda.empty_cache()
         extra["long_ctx"] = bench_long_ctx(R, pk)
         torch.cuda.empty_cache()
+        extra["msr_small"] = bench_msr_small(R, pk)
+        torch.cuda.empty_cache()
         extra["msr_layer"] = bench_layer(R, w, pk)
         torch.cuda.empty_cache()
         extra["decode"] = bench_decode(R, pk)
@@ -667,7 +727,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
-    ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx"], default=None,
+    ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx", "msr_small"],
+                    default=None,
                     help="run one measurement alone (profiler captures)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="override the decode workload's batch (small cases for profiler captures)")

@@ -114,9 +114,10 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *     R  <- gamma^n R + sum_{j'} gamma^{n-1-j'} k^_{j'}^T v_{j'}
  * (the recurrent form unrolled over the chunk; the last chunk may be short).
  * The result equals ret_parallel's up to rounding for every chunk size.
- * On the tensor-core path a chunk of 128*m rows is evaluated as m
- * consecutive blocks of 128 rows (the recurrence holds exactly at every row
- * boundary, so this is the same computation with different rounding).
+ * The tensor-core path works in blocks of 128 rows: a chunk of 128*m rows
+ * is m consecutive blocks, a chunk of 64 rows two chunks per block (the
+ * recurrence holds exactly at every row boundary, so this is the same
+ * computation with different rounding).
  *   state_in  device fp32 [B][H][d_k][d_v] or NULL (zeros).
  *   state_out device fp32, or NULL; may alias state_in.
  *   O         device out_dtype [B][H][L][d_v], or NULL when only Y is wanted.
@@ -125,14 +126,17 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *             ret_gate_norm) is written as well, with epsilon gn_eps.
  *   workspace device scratch of workspace_bytes; required only when
  *             ret_workspace_size() returns a non-zero size for this call.
- *             Optional on the tensor-core path (bf16 inputs, chunk a
- *             multiple of 128, d_k 128 or 256, d_v a multiple of 128 up to
- *             512, gamma_h^128 >= 2^-60 for every head): with at
- *             least ret_chunkwise_prep_size() bytes the rotated Q and the
+ *             On the tensor-core path (bf16 inputs, chunk a multiple of
+ *             64, d_k 64, 128 or 256, d_v 64 or a multiple of 128 up to
+ *             512, gamma_h^128 >= 2^-60 for every head): with at least
+ *             ret_chunkwise_prep_size() bytes the rotated Q and the
  *             decay-weighted K are prepared there in one streaming pass
- *             before the chunk loop (faster); with less, the kernel
- *             prepares each chunk's rows itself.  Results agree either way
- *             up to rounding.
+ *             before the chunk loop (faster); with less, the loop turns
+ *             the rows itself (d_k and d_v from 128 and chunks of 128*m
+ *             only: for the other shapes of the path ret_workspace_size
+ *             asks for the prep size when rotating) or, without rotation,
+ *             weights the value rows itself.  Results agree either way up
+ *             to rounding.
  * At least one of O and Y must be requested.
  * Errors: those of ret_parallel, plus RET_ERR_WORKSPACE.
  */

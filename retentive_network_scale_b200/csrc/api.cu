@@ -139,12 +139,14 @@ ret_status ret_parallel(const ret_desc *desc, const void *Q, const void *K, cons
 
 size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_Y) {
     if (check_desc(desc) != RET_OK || chunk < 1) return 0;
-    // The tensor-core kernel normalises in its epilogue.  The CUDA-core
+    // The tensor-core kernel normalises in its epilogue; some of its shapes
+    // need the streaming pass's workspace when rotated.  The CUDA-core
     // chunkwise path needs an fp32 O to normalise when only Y is requested.
     Params p;
     make_params(desc, &p);
-    if (want_Y && !want_O && !chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16))
-        return sizeof(float) * (size_t)desc->B * desc->H * desc->L * desc->d_v;
+    if (chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16))
+        return chunkwise_tc_needs_prep(p, chunk) ? chunkwise_prep_bytes(p) : 0;
+    if (want_Y && !want_O) return sizeof(float) * (size_t)desc->B * desc->H * desc->L * desc->d_v;
     return 0;
 }
 

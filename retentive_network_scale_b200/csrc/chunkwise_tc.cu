@@ -913,17 +913,27 @@ cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, con
 
 }  // namespace
 
-// A chunk of kC * m rows is evaluated as m consecutive blocks of kC rows:
-// the chunkwise recurrence holds exactly at any row boundary (the state
-// carried between the blocks is the exact state after those rows), so this
-// is the same computation; only the rounding differs.
+// The loop works in blocks of kC rows whatever the chunk: a chunk of
+// kC * m rows is m consecutive blocks, and a chunk of 64 rows pairs up two
+// chunks per block.  The chunkwise recurrence holds exactly at any row
+// boundary (the state carried between blocks is the exact state after
+// those rows), so either is the same computation; only the rounding
+// differs.  d_k 64, d_v 64 and chunks of 64 rows are served by the
+// pipelined kernel of chunkwise_ws.cu only: with rotation they need the
+// streaming pass's workspace (chunkwise_tc_needs_prep).
 bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16) {
-    if (!in_bf16 || chunk % kC != 0 || (p.dk != 128 && p.dk != 256) || p.dv % kTV != 0 ||
-        p.dv / kTV > kMaxCluster || p.L < 1 || p.B * p.H < 1 || (long long)p.B * p.H > 65535)
+    const bool dk_ok = p.dk == 64 || p.dk == 128 || p.dk == 256;
+    const bool dv_ok = p.dv == 64 || (p.dv % kTV == 0 && p.dv / kTV <= kMaxCluster);
+    if (!in_bf16 || chunk % 64 != 0 || !dk_ok || !dv_ok || p.L < 1 || p.B * p.H < 1 ||
+        (long long)p.B * p.H > 65535)
         return false;
     for (int h = 0; h < p.H; ++h)
         if (!(p.log2g[h] * kC >= kMinLog2GammaTimesC)) return false;  // also rejects gamma = 0
     return true;
+}
+
+bool chunkwise_tc_needs_prep(const Params &p, int chunk) {
+    return p.rotate && (p.dk == 64 || p.dv == 64 || chunk % kC != 0);
 }
 
 namespace {

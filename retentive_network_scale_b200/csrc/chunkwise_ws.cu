@@ -15,8 +15,9 @@
 // this needs no pass over Q and K at all when there is no rotation).  Both
 // give gamma^{j+1-n} gamma^{n-1-j'} = gamma^{j-j'} term by term.
 //
-// One CTA owns one (b, h) and 128 value columns; the d_v/128 CTAs of a head
-// form a cluster.  Unlike chunkwise_tc.cu, no role waits for a whole chunk
+// One CTA owns one (b, h) and 128 value columns (d_v = 64: one CTA with 64,
+// the rest of its V tile zero); the CTAs of a head form a cluster.  d_k is
+// 64, 128 or 256.  Unlike chunkwise_tc.cu, no role waits for a whole chunk
 // to finish: every hand-over is an mbarrier, so the epilogue of chunk c runs
 // while the tensor cores work on chunk c+1.  Roles (16 warps):
 //   warp 0      issues the MMAs (one thread), chunk by chunk:
@@ -242,6 +243,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.y, h = bh % p.H, b = bh / p.H;
     const int v0 = blockIdx.x * kTV;
+    const int dvr = min(kTV, p.dv - v0);  // value columns of this CTA: 128, or 64 when d_v = 64
     const float lg = p.log2g[h];
     const int L = p.L, dv = p.dv;
     const int nchunks = (L + kC - 1) / kC;
@@ -274,6 +276,12 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     if (warp == 0) {
         tmem_alloc(sbase + Ly::kTmemSlot, 512);
         tmem_relinquish();
+    }
+    if (dvr < kTV) {
+        // d_v = 64: the V tile's second block is never loaded and stays zero
+        for (int i = tid; i < 16384 / 16; i += kThreads)
+            reinterpret_cast<uint4 *>(smem + Ly::kV + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -376,8 +384,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tma_load_3d(sbase + Ly::k_blk(kb), &tmK, bar(KF), kb * 64, c * kC, bh);
         };
         auto load_v = [&](int c) {
-            mbar_expect_tx(bar(VF), Ly::kVBytes);
-            for (int nb = 0; nb < 2; ++nb)
+            mbar_expect_tx(bar(VF), dvr * kC * 2);
+            for (int nb = 0; nb < dvr / 64; ++nb)
                 tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(VF), vx0 + nb * 64, c * kC, vz);
         };
         if (lane == 0) {
@@ -450,6 +458,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================ P pass and state pass (warps 4-7, one TMEM lane each)
         const int row = tid & 127;  // chunk row for S, value column for R^T
         const int quad = warp & 3;
+        const bool vcol = row < dvr;  // this lane's value column exists
         {
             // starting state: R^T = gamma^{n_0} S_in^T in TMEM and Rbar^T =
             // bf16 of the same; zeros without a state
@@ -461,7 +470,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 uint32_t r[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    v[i] = has_in ? state_in[((size_t)bh * DK + d0 + i) * dv + v0 + row] * g0 : 0.f;
+                    v[i] = has_in && vcol ? state_in[((size_t)bh * DK + d0 + i) * dv + v0 + row] * g0 : 0.f;
                 st_rbarT_row32<DK>(smem, row, d0, v);
                 if (has_in) {
 #pragma unroll
@@ -537,7 +546,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         v[i + 1] = f2_hi(x);
                     }
                     if (last) {
-                        if (state_out) {
+                        if (state_out && vcol) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
                                 state_out[((size_t)bh * DK + dd + i) * dv + v0 + row] = v[i];
@@ -551,7 +560,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 };
                 pass32(ra, d0);
                 pass32(rb, d0 + 32);
-                if (d0 + 64 == DK / 2) {
+                if (DK >= 128 && d0 + 64 == DK / 2) {
                     // the first half of Rbar^T is ready for the next O'' product
                     tmem_wait_st();
                     fence_proxy_async_smem();
@@ -562,6 +571,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
+            if constexpr (DK < 128) warp_arrive(RBL);  // no first half to publish early
             warp_arrive(RB);
         }
     } else {
@@ -572,6 +582,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int row = 32 * quad + lane;   // this thread's row (TMEM lane)
         const int j4 = lane >> 2, m4 = lane & 3;  // groups of 4 lanes
         const int o0 = gwg * 64;
+        const bool ocols = o0 < dvr;  // this thread's 64 columns exist (d_v = 64: group 0 only)
         const size_t ycol = (size_t)h * dv + v0 + o0;  // column of Y / G of this thread's segment
         // rows of this lane group's 16-byte row pieces: 32 quad + 4 j4 + i
         auto grow = [&](int i) { return 32 * quad + 4 * j4 + i; };
@@ -615,8 +626,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mean /= (float)nr;
 #pragma unroll
             for (int r = 0; r < kMaxCluster; ++r)
-                if (r < nr) m2 += e[r].y + (float)kTV * (e[r].x - mean) * (e[r].x - mean);
-            const float var = m2 / (float)(nr * kTV);  // of O''; O = alpha O''
+                if (r < nr) m2 += e[r].y + (float)dvr * (e[r].x - mean) * (e[r].x - mean);
+            const float var = m2 / (float)(nr * dvr);  // of O''; O = alpha O''
             const float scale = alpha_p * rsqrtf(alpha_p * alpha_p * var + gn_eps);
             const uint64_t SC = f2_make(scale, scale);
             const float off = (shift_p - mean) * scale;
@@ -630,14 +641,14 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     },
                     m4, 32 * hf,
                     [&](int i) { return Y + ((size_t)b * L + t0_p + grow(i)) * ((size_t)p.H * dv) + ycol; },
-                    [&](int i) { return grow(i) < n_p; });
+                    [&](int i) { return ocols && grow(i) < n_p; });
         };
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const int t0 = c * kC;
             const int n = min(kC, L - t0);
-            auto row_ok = [&](int i) { return grow(i) < n; };
+            auto row_ok = [&](int i) { return ocols && grow(i) < n; };
             if constexpr (FUSE)
                 if (c > 0) finish(c - 1);
             {
@@ -687,12 +698,16 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // the two halves of the row merge (Chan's update, equal
                 // counts) in this CTA's published slot
                 float2 *slot = reinterpret_cast<float2 *>(smem + Ly::kSlot + (par * 128 + row) * 8);
-                if (gwg == 1) *slot = make_float2(m_w, m2_w);
+                if (gwg == 1 && dvr == kTV) *slot = make_float2(m_w, m2_w);
                 named_sync(1, 256);
                 if (gwg == 0) {
-                    const float2 o = *slot;
-                    const float d = m_w - o.x;
-                    *slot = make_float2(0.5f * (m_w + o.x), m2_w + o.y + 32.f * d * d);
+                    if (dvr == kTV) {
+                        const float2 o = *slot;
+                        const float d = m_w - o.x;
+                        *slot = make_float2(0.5f * (m_w + o.x), m2_w + o.y + 32.f * d * d);
+                    } else {
+                        *slot = make_float2(m_w, m2_w);  // the row's only 64 columns
+                    }
                 }
                 named_sync(1, 256);
                 // the slots are written (the barrier above ordered them before
@@ -705,8 +720,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int r = grow(i);
-                        gp[4 * hf + i] = r < n ? ld_nc(Gb + (size_t)(t0 + r) * g_row + 32 * hf + 8 * m4)
-                                               : make_uint4(0u, 0u, 0u, 0u);
+                        gp[4 * hf + i] = ocols && r < n ? ld_nc(Gb + (size_t)(t0 + r) * g_row + 32 * hf + 8 * m4)
+                                                        : make_uint4(0u, 0u, 0u, 0u);
                     }
                 shift_p = shift;
                 alpha_p = alpha;
@@ -744,13 +759,13 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.dv / kTV, p.B * p.H);
+    cfg.gridDim = dim3((p.dv + kTV - 1) / kTV, p.B * p.H);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = FUSE ? p.dv / kTV : 1;
+    attr[0].val.clusterDim.x = FUSE ? (p.dv + kTV - 1) / kTV : 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -795,6 +810,8 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
     const int zv = zeta_on_v ? 1 : 0, vhm = v_head_major ? 1 : 0;
     if (p.dk == 256)
         return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
+    if (p.dk == 64)
+        return launch_dk<64>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
     return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
 }
 

@@ -23,14 +23,17 @@ cudaError_t launch_chunkwise_simt(const Params &p, int chunk, bool in_bf16,
                                   const void *V, const float *s_in,
                                   float *s_out, void *O, cudaStream_t st);
 
-// Tensor-core chunkwise kernel: bf16 inputs, chunk a multiple of 128
-// (evaluated in blocks of 128 rows), d_k 128 or 256,
-// d_v a multiple of 128 (at most 512), every gamma_h^128 >= 2^-60.  With Y
+// Tensor-core chunkwise kernel: bf16 inputs, chunk a multiple of 64
+// (evaluated in blocks of 128 rows), d_k 64, 128 or 256, d_v 64 or a
+// multiple of 128 (at most 512), every gamma_h^128 >= 2^-60.  With Y
 // (and G) given it also writes Y = swish(G) (.) GroupNorm_h(O); O may then
 // be NULL.
 // With prep_ws (chunkwise_prep_bytes) the rows are first prepared by the
 // streaming pass below; with NULL the kernel turns them itself (slower).
 bool chunkwise_tc_supported(const Params &p, int chunk, bool in_bf16);
+// Shapes of the tensor-core path whose rotated rows must come from the
+// streaming pass (the workspace ret_chunkwise_prep_size gives).
+bool chunkwise_tc_needs_prep(const Params &p, int chunk);
 cudaError_t launch_chunkwise_tc(const Params &p, bool out_bf16, const void *Q, const void *K,
                                 const void *V, const float *s_in, float *s_out, void *O,
                                 const void *G, void *Y, float eps, void *prep_ws, int *status,

@@ -253,7 +253,8 @@ ret_status check_segmented(const ret_desc *desc, int chunk, int segments, ret::P
         (long long)desc->B * desc->H * segments > 65535)  // one CTA row per segment head
         return RET_ERR_SHAPE;
     params_from_desc(desc, p);
-    if (!chunkwise_tc_supported(*p, chunk, true)) return RET_ERR_SHAPE;
+    if (!chunkwise_tc_supported(*p, chunk, true) || !segment_state_tc_supported(*p))
+        return RET_ERR_SHAPE;
     return RET_OK;
 }
 

@@ -128,11 +128,15 @@ def test_chunkwise_prep_size(lib):
     assert size(desc(**base)) == 2 * (2 * 2 * 300 * 256) * 2
     assert size(desc(**{**base, "rotate": False})) == (2 * 2 * 300 * 256) * 2
     assert size(desc(**{**base, "d_k": 128})) == 2 * (2 * 2 * 300 * 128) * 2
-    assert size(desc(**base), chunk=64) == 0                            # not a multiple of 128
-    assert size(desc(**base), chunk=192) == 0
-    assert size(desc(**base), chunk=256) == size(desc(**base))          # blocks of 128 rows
+    assert size(desc(**base), chunk=64) == size(desc(**base))           # blocks of 128 rows
+    assert size(desc(**base), chunk=192) == size(desc(**base))
+    assert size(desc(**base), chunk=256) == size(desc(**base))
+    assert size(desc(**base), chunk=96) == 0                            # not a multiple of 64
     assert size(desc(**{**base, "in_dtype": R.RET_F32})) == 0            # fp32 inputs
-    assert size(desc(**{**base, "d_k": 64})) == 0
+    assert size(desc(**{**base, "d_k": 64})) == 2 * (2 * 2 * 300 * 64) * 2
+    assert size(desc(**{**base, "d_v": 64})) == size(desc(**base))
+    assert size(desc(**{**base, "d_k": 32})) == 0
+    assert size(desc(**{**base, "d_v": 192})) == 0                       # neither 64 nor 128 m
     assert size(desc(**{**base, "d_v": 640})) == 0                       # more than 4 column tiles
     assert size(desc(**{**base, "gamma": [0.5, 0.99]})) == 0             # 0.5^128 < 2^-60
     assert size(desc(**{**base, "gamma": [1.5, 0.99]})) == 0             # rejected description
@@ -264,8 +268,8 @@ def test_chunkwise_prepared_arguments(lib):
                                    ctypes.c_float(1e-5), Y, None)
     assert call(chunk=0) == S("RET_ERR_ARG")
     assert call(dd=desc(B=0, L=300, d_k=128, d_v=128)) == S("RET_ERR_SHAPE")   # nothing prepared
-    assert call(dd=desc(B=2, L=300, d_k=64, d_v=128)) == S("RET_ERR_SHAPE")    # not a tensor-core shape
-    assert call(chunk=64) == S("RET_ERR_SHAPE")
+    assert call(dd=desc(B=2, L=300, d_k=32, d_v=128)) == S("RET_ERR_SHAPE")    # not a tensor-core shape
+    assert call(chunk=96) == S("RET_ERR_SHAPE")
     assert call(Kt=None) == S("RET_ERR_NULL")
     assert call(O=None) == S("RET_ERR_NULL")                                   # nothing requested
     assert call(G=FAKE) == S("RET_ERR_NULL")                                   # G without Y
@@ -287,7 +291,9 @@ def test_chunkwise_segmented_arguments(lib):
     assert call(seg=0) == S("RET_ERR_ARG") and size(seg=0) == 0
     assert call(seg=3) == S("RET_ERR_SHAPE") and size(seg=3) == 0          # L % segments
     assert call(seg=64) == S("RET_ERR_SHAPE")                                # H * segments > 128
-    assert call(chunk=64) == S("RET_ERR_SHAPE")                              # not a tensor-core chunk
+    assert call(chunk=96) == S("RET_ERR_SHAPE")                              # not a tensor-core chunk
+    assert call(dd=desc(B=1, H=4, L=1024, d_k=64, d_v=256,
+                        gamma=[0.9] * 4)) == S("RET_ERR_SHAPE")              # no segment states at d_k 64
     assert call(dd=desc(B=1, H=4, L=1024, d_k=128, d_v=256, in_dtype=R.RET_F32,
                         gamma=[0.9] * 4)) == S("RET_ERR_DTYPE")
     assert call(O=None) == S("RET_ERR_NULL")
@@ -313,3 +319,23 @@ def test_static_entry_checks_arguments_before_its_scratch_limit(lib):
     assert call(d, chunk=0) == S("RET_ERR_ARG")
     assert call(desc(gamma=[1.5, 0.9])) == S("RET_ERR_ARG")
     assert call(d) == S("RET_ERR_WORKSPACE")
+
+
+def test_workspace_size_of_tensor_core_shapes(lib):
+    """The tensor-core path needs no workspace, except for rotated shapes
+    that only the prepared-rows loop serves (d_k 64, d_v 64, chunks of 64
+    rows): there ret_workspace_size asks for the streaming pass's room."""
+    bf = R.RET_BF16
+    ws = lambda d, chunk=128, o=0, y=1: lib.ret_workspace_size(ctypes.byref(d), chunk, o, y)  # noqa: E731
+    prep = lambda d, chunk=128: lib.ret_chunkwise_prep_size(ctypes.byref(d), chunk)  # noqa: E731
+    big = dict(B=1, H=2, L=300, d_k=256, d_v=512, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
+    assert ws(desc(**big)) == 0 and ws(desc(**big), chunk=256) == 0
+    assert ws(desc(**big), chunk=64) == prep(desc(**big), chunk=64) > 0
+    small = {**big, "d_k": 64, "d_v": 64}
+    assert ws(desc(**small), chunk=64) == prep(desc(**small), chunk=64) > 0
+    assert ws(desc(**small), chunk=64, o=1, y=0) == prep(desc(**small), chunk=64)
+    assert ws(desc(**{**small, "rotate": False}), chunk=64) == 0
+    # fp32 inputs take the CUDA-core path: an fp32 O to normalise for Y alone
+    f32 = {**small, "in_dtype": R.RET_F32, "out_dtype": R.RET_F32}
+    assert ws(desc(**f32), chunk=64) == 1 * 2 * 300 * 64 * 4
+    assert ws(desc(**f32), chunk=64, o=1, y=1) == 0

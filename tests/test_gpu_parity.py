@@ -186,14 +186,23 @@ def test_msr_small_bf16():
     O = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda", dtype=torch.bfloat16)
     Y = torch.empty(w.B, w.L, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
     S = torch.empty(w.B, w.H, w.d_k, w.d_v, device="cuda")
+    # the tensor-core path: no workspace for Y alone, and one launch of the
+    # loop when called without a workspace (the CUDA-core path would need an
+    # fp32 O to normalise and a second launch for the gate)
+    assert R.ret_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, R.RET_BF16, R.RET_BF16, g, w.chunk,
+                                want_O=False, want_Y=True, rotate=w.rotate) == 0
+    n0 = R.ret_kernel_launches()
     R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, O=O, state_out=S, G=d["G"], Y=Y,
-                    rotate=w.rotate)
+                    rotate=w.rotate, prep=False)
+    assert R.ret_kernel_launches() - n0 == 1
     assert rel_l2(O.reshape(-1, w.L, w.d_v), O_ref) <= TOL_BF16
     assert rel_l2(S.reshape(-1, w.d_k, w.d_v), S_ref) <= TOL_BF16
     assert rel_l2(y_slices(Y, pairs, w.d_v), Y_ref) <= TOL_BF16
-    # Y alone (the benchmarked call)
+    # Y alone (the benchmarked call: streaming pass of the keys, then the loop)
     Y2 = torch.empty_like(Y)
+    n0 = R.ret_kernel_launches()
     R.ret_chunkwise(d["Q"], d["K"], d["V"], g, w.chunk, G=d["G"], Y=Y2, rotate=w.rotate)
+    assert R.ret_kernel_launches() - n0 == 2
     assert rel_l2(y_slices(Y2, pairs, w.d_v), Y_ref) <= TOL_BF16
     # parallel form
     Op = torch.empty_like(O)

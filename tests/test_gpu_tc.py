@@ -250,3 +250,36 @@ def test_batch_slices_and_prepared_loop_are_exact():
     for i, (b, h) in enumerate(pairs):
         assert rel_l2(O1[b, h], O_ref[0, i]) <= TOL_BF16, (b, h)
         assert rel_l2(S1[b, h], S_ref[0, i]) <= TOL_BF16, (b, h)
+
+
+@pytest.mark.parametrize("dk,dv,chunk,rotate,prep", [
+    (64, 64, 64, True, True),      # the small MSR head (rotated: prepared rows)
+    (64, 64, 64, False, False),    # value rows weighted inside the loop
+    (64, 256, 128, True, True),    # d_k 64 with two CTAs of columns per head
+    (128, 64, 64, False, True),    # d_v 64 under a wider d_k
+])
+def test_tc_small_heads(dk, dv, chunk, rotate, prep):
+    """d_k 64 and d_v 64 on the tensor cores (a CTA with 64 value columns,
+    the rest of its tile zero), chunks of 64 rows (two per block of 128):
+    O, Y and the state against the oracle, ragged tail, with a state in."""
+    B, H, L = 2, 3, 333
+    Q, K, V = _inputs(B, H, L, dk, dv, 500 + dk + dv)
+    G = random_tensor((B, L, H * dv), 520).bfloat16()
+    S0 = random_tensor((B, H, dk, dv), 521, 0.2)
+    g = [0.96875, 0.99, 0.999]
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=11, state_in=S0)
+    Y_ref = orc.gate_groupnorm(O_ref, G)
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
+    Y = torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16)
+    S = torch.empty(B, H, dk, dv, device="cuda")
+    n0 = R.ret_kernel_launches()
+    R.ret_chunkwise(Q.cuda(), K.cuda(), V.cuda(), g, chunk, O=O, G=G.cuda(), Y=Y, rotate=rotate,
+                    pos_offset=11, state_in=S0.cuda(), state_out=S, prep=prep)
+    assert R.ret_kernel_launches() - n0 == (2 if prep else 1)   # no CUDA-core fallback
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
+            assert rel_l2(S[b, h], S_ref[b, h]) <= TOL_BF16, (b, h)
+            assert rel_l2(Y[b, :, h * dv:(h + 1) * dv], Y_ref[b, :, h * dv:(h + 1) * dv]) <= TOL_BF16
