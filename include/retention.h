@@ -196,9 +196,9 @@ size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk);
  * rotated Q (bf16 [B][H][L][d_k], with rotation only) followed by
  * K~[b,h,t] = gamma_h^{n-1-j} Theta_t K[b,h,t] (bf16, same shape) for row t
  * at offset j of its block of n rows (section 2.1, chunkwise form (3): the
- * weight of key j' in the state update).  The tensor-core loop evaluates a
- * chunk of any multiple of 128 rows as blocks of 128 (the recurrence holds
- * at every row boundary), so the blocks are 128 rows whatever `chunk` is.  No counterpart in the paper as a
+ * weight of key j' in the state update).  The tensor-core loop works in
+ * blocks of 128 rows whatever `chunk` is (a multiple of 64; the recurrence
+ * holds at every row boundary), so the weights follow those blocks.  No counterpart in the paper as a
  * call of its own; exported so that the pass can be timed or scheduled
  * apart.  Q, K device bf16; workspace device, caller-owned, overwritten.
  * Errors: RET_ERR_SHAPE when the tensor-core path does not apply (nothing
@@ -278,7 +278,7 @@ size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
  *           Q and K, Y and the GEMM library's scratch).
  * desc->in_dtype and out_dtype are RET_BF16; d_model is a multiple of 8.
  * The layer runs on the tensor-core chunkwise path only (chunk a multiple of
- * 128, d_k 128 or 256, d_v a multiple of 128 up to 512, gamma_h^128 >=
+ * 64, d_k 128 or 256, d_v a multiple of 128 up to 512, gamma_h^128 >=
  * 2^-60).  The two projections are cuBLAS GEMMs with fp32 accumulation; P
  * and Y are held in bf16.  Not safe to call from two host threads at once
  * on one device.
@@ -311,7 +311,7 @@ size_t ret_msr_layer_workspace_size(const ret_desc *desc, int d_model,
  *   workspace  device, 256-byte aligned, at least
  *           ret_backward_workspace_size() bytes
  * Tensor-core shapes only: d_k 128 or 256, d_v a multiple of 128 up to 512,
- * chunk a multiple of 128, gamma_h^128 >= 2^-60 (else RET_ERR_SHAPE).
+ * chunk a multiple of 64, gamma_h^128 >= 2^-60 (else RET_ERR_SHAPE).
  * Errors: those of ret_chunkwise.
  */
 ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q,

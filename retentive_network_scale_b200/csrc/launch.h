@@ -134,8 +134,8 @@ bool segment_state_tc_supported(const Params &p);
 cudaError_t launch_segment_state_tc(const Params &p, const void *V, const void *Kt, int zeta_v,
                                     float *U, int *status, cudaStream_t st);
 
-// Tensor-core parallel form: bf16 inputs, d_k 128 or 256, d_v a multiple of
-// 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
+// Tensor-core parallel form: bf16 inputs, d_k 64, 128 or 256, d_v 64 or a
+// multiple of 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
 // Q^ and K^ (bf16) into the workspace (parallel_tc_workspace bytes).
 bool parallel_tc_supported(const Params &p, bool in_bf16);
 size_t parallel_tc_workspace(const Params &p);

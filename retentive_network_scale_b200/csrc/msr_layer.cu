@@ -104,8 +104,12 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
     if (chunk < 1 || !(gn_eps >= 0.0f && gn_eps < 3.0e38f)) return RET_ERR_ARG;
     ret::Params p;
     ret::params_from_desc(desc, &p);
-    if ((long long)desc->B * desc->L > 0 && !ret::chunkwise_tc_supported(p, chunk, true))
-        return RET_ERR_SHAPE;  // the layer runs on the tensor-core chunkwise path only
+    // the layer runs on the tensor-core chunkwise path only, at the head
+    // shapes its tests cover (d_k 128 or 256, d_v a multiple of 128)
+    if ((long long)desc->B * desc->L > 0 &&
+        (!ret::chunkwise_tc_supported(p, chunk, true) || (p.dk != 128 && p.dk != 256) ||
+         p.dv % 128 != 0))
+        return RET_ERR_SHAPE;
     if ((long long)desc->B * desc->L == 0) return RET_OK;
     if (!X || !W_qkvg || !W_o || !out) return RET_ERR_NULL;
     auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };

@@ -3,7 +3,8 @@
 //     O = (Q^ K^^T (.) D) V,   D_nm = gamma^{n-m} for n >= m, else 0.
 //
 // Flash-style: one CTA owns a 128-row query tile, a slice of V columns
-// (TV = 256, or 128 when d_v is not a multiple of 256) and one (b,h).  It
+// (TV = 256, or 128 when d_v is not a multiple of 256, or 64 when d_v is
+// 64) and one (b,h); d_k is 64, 128 or 256.  It
 // walks the key tiles from the diagonal down:
 //     S = Q^ K^_k^T            (tcgen05, fp32 in tensor memory)
 //     P = S (.) D_tile         (CUDA cores: the decay as the rank-1 product
@@ -320,13 +321,15 @@ cudaError_t launch_ptc_tv(const Params &p, const CUtensorMap &mq, const CUtensor
                           const CUtensorMap &mv, const CUtensorMap &mo, void *O, int *status,
                           cudaStream_t st) {
     if (p.dv % 256 == 0) return launch_ptc<DK, 256, TO>(p, mq, mk, mv, mo, O, status, st);
-    return launch_ptc<DK, 128, TO>(p, mq, mk, mv, mo, O, status, st);
+    if (p.dv % 128 == 0) return launch_ptc<DK, 128, TO>(p, mq, mk, mv, mo, O, status, st);
+    return launch_ptc<DK, 64, TO>(p, mq, mk, mv, mo, O, status, st);
 }
 
 }  // namespace
 
 bool parallel_tc_supported(const Params &p, bool in_bf16) {
-    if (!in_bf16 || (p.dk != 128 && p.dk != 256) || p.dv % 128 != 0 || p.L < 1 ||
+    if (!in_bf16 || (p.dk != 64 && p.dk != 128 && p.dk != 256) || (p.dv % 128 != 0 && p.dv != 64) ||
+        p.L < 1 ||
         (long long)p.B * p.H > 65535 || (p.L + kT - 1) / kT > 2147483647)
         return false;
     for (int h = 0; h < p.H; ++h)
@@ -366,6 +369,9 @@ cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, co
     if (p.dk == 256)
         return out_bf16 ? launch_ptc_tv<256, __nv_bfloat16>(p, mq, mk, mv, mo, O, status, st)
                         : launch_ptc_tv<256, float>(p, mq, mk, mv, mo, O, status, st);
+    if (p.dk == 64)
+        return out_bf16 ? launch_ptc_tv<64, __nv_bfloat16>(p, mq, mk, mv, mo, O, status, st)
+                        : launch_ptc_tv<64, float>(p, mq, mk, mv, mo, O, status, st);
     return out_bf16 ? launch_ptc_tv<128, __nv_bfloat16>(p, mq, mk, mv, mo, O, status, st)
                     : launch_ptc_tv<128, float>(p, mq, mk, mv, mo, O, status, st);
 }

@@ -46,7 +46,7 @@ def test_msr_layer_refusals():
     X = torch.zeros(1, 128, 64, device="cuda", dtype=torch.bfloat16)
     W = torch.zeros(64, 2 * (2 * 128 + 2 * 128), device="cuda", dtype=torch.bfloat16)
     Wo = torch.zeros(2 * 128, 64, device="cuda", dtype=torch.bfloat16)
-    with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # chunk 64: CUDA-core path
-        R.ret_msr_layer(X, W, Wo, [0.9, 0.99], 64, 128, 128)
+    with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # chunk 96: CUDA-core path
+        R.ret_msr_layer(X, W, Wo, [0.9, 0.99], 96, 128, 128)
     with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # gamma^128 below 2^-60
         R.ret_msr_layer(X, W, Wo, [0.5, 0.99], 128, 128, 128)

@@ -283,3 +283,28 @@ def test_tc_small_heads(dk, dv, chunk, rotate, prep):
             assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
             assert rel_l2(S[b, h], S_ref[b, h]) <= TOL_BF16, (b, h)
             assert rel_l2(Y[b, :, h * dv:(h + 1) * dv], Y_ref[b, :, h * dv:(h + 1) * dv]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,rotate,out", [
+    (2, 3, 333, 64, 64, True, torch.bfloat16),
+    (1, 2, 500, 64, 256, False, torch.float32),
+    (1, 2, 300, 128, 64, True, torch.bfloat16),
+])
+def test_tc_parallel_small_heads(B, H, L, dk, dv, rotate, out):
+    """The parallel form on the tensor cores at d_k 64 and d_v 64 (value
+    slices of 64 columns): against the oracle, and on the tensor-core path
+    (with rotation it needs the workspace for the turned rows and launches
+    the two turning passes and the product)."""
+    Q, K, V = _inputs(B, H, L, dk, dv, 700 + L)
+    g = ([0.75, 0.96875, 1.0] * 2)[:H]
+    O_ref, _ = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=3)
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=out)
+    n0 = R.ret_kernel_launches()
+    R.ret_parallel(Q.cuda(), K.cuda(), V.cuda(), O, g, rotate=rotate, pos_offset=3)
+    if rotate:
+        assert R.ret_kernel_launches() - n0 == 3
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(O[b, h], O_ref[b, h]) <= TOL_BF16, (b, h)
