@@ -13,9 +13,14 @@
 //                               bf16 back into tensor memory)
 //     O += P V_k               (tcgen05, A operand from tensor memory)
 // Key tiles whose largest weight gamma^{Delta-127} is below 2^-150 add
-// nothing representable in fp32; the walk stops there.  K and V loads for
-// the next key tile are issued as soon as the MMAs reading the current one
-// finish.  The output tile leaves through shared memory and TMA stores.
+// nothing representable in fp32; the walk stops there.  Roles (12 warps):
+// one thread issues the MMAs -- S of tile t into one of two tensor-memory
+// buffers, then P V of tile t-1 -- so that the P pass of one tile runs while
+// the tensor cores multiply its neighbour; one thread issues the TMA loads
+// (the next K tile once S has read the current one, the next V tile once
+// P V has); warps 4-11 run the P pass and finally move the output tile out
+// through shared memory and TMA stores.  Every hand-over is an mbarrier with
+// a bounded wait.
 //
 // The rotation (xPos) is applied once per row by xpos_rotate_kernel into a
 // workspace before this kernel runs: every key tile is read by many query
@@ -34,11 +39,15 @@ namespace {
 using namespace tc;
 
 constexpr int kT = 128;         // query / key tile rows
-constexpr int kThreads = 256;   // two warpgroups
+constexpr int kThreads = 384;   // three warpgroups
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr float kMinLog2GammaTimesT = -60.f;  // gamma^-127 stays below 2^60
 
-enum { BQ = 0, BK, BV, BS, BPV, kNumBars };
+// BQ/BK/BV: tile landed; SD0/SD1: S of the tile in S buffer b done; PR0/PR1:
+// P of buffer b written; PV0/PV1: P V of buffer b's tile done (the buffer,
+// and the V tile, free again).  The buffer barriers complete once every two
+// key tiles, so no waiter can fall two phases behind.
+enum { BQ = 0, BK, BV, SD0, SD1, PR0, PR1, PV0, PV1, kNumBars };
 
 template <int DK, int TV>
 struct PLayout {
@@ -49,8 +58,8 @@ struct PLayout {
     static constexpr uint32_t kVBytes = kT * TV * 2;
     static constexpr uint32_t kSmall = kV + kVBytes;
     static constexpr uint32_t kBar = kSmall;
-    static constexpr uint32_t kTmemSlot = kSmall + 64;
-    static constexpr uint32_t kAbort = kSmall + 68;
+    static constexpr uint32_t kTmemSlot = kSmall + 8 * kNumBars;
+    static constexpr uint32_t kAbort = kTmemSlot + 4;
     static constexpr uint32_t kColScale = kSmall + 128;   // gamma^{-j'}, 128 floats
     static constexpr uint32_t kBytes = kColScale + 512;
 };
@@ -77,7 +86,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     constexpr bool kStage = sizeof(TO) == 2;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
-    const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, row = tid & 127;
     const int nqt = (p.L + kT - 1) / kT;
     const int qt = nqt - 1 - (int)blockIdx.x;  // long rows of tiles first
     const int v0 = blockIdx.y * TV, bh = blockIdx.z, h = bh % p.H;
@@ -92,7 +101,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::kAbort);
     float *colscale = reinterpret_cast<float *>(smem + Ly::kColScale);
     if (tid == 0) {
-        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == PR0 || i == PR1) ? 8 : 1);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -106,7 +115,8 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + Ly::kTmemSlot);
-    const uint32_t tO = tmem, tS = tmem + 256;
+    const uint32_t tO = tmem;
+    auto tS = [&](int b) { return tmem + 256 + 128 * b; };
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
     // last key tile with a representable weight: gamma^{Delta-127} >= 2^-150
@@ -115,60 +125,100 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int far = (int)floorf(-150.f / lg) + 127;  // largest Delta still kept
         kt_min = max(0, qt - far / kT);
     }
-    auto load_k = [&](int kt) {
-        mbar_expect_tx(bar(BK), Ly::kQBytes);
-        for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(sbase + Ly::kK + kb * 16384, &tmK, bar(BK), kb * 64, kt * kT, bh);
+    const int nit = qt - kt_min + 1;  // key tiles qt, qt-1, ..., kt_min
+    auto wait_all = [&](int i, uint32_t parity) {
+        return __all_sync(0xffffffffu, pwait(bar(i), parity, abort_flag, status));
     };
-    auto load_v = [&](int kt) {
-        mbar_expect_tx(bar(BV), Ly::kVBytes);
-        for (int nb = 0; nb < VB; ++nb)
-            tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, kt * kT, bh);
-    };
-    auto sync_alive = [&]() {
-        __syncthreads();
-        return *abort_flag == 0;
-    };
-    const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);
-    const uint64_t dK = sdesc_sw128(sbase + Ly::kK, 16, 1024);
-    const uint64_t dV = sdesc_sw128(sbase + Ly::kV, 16384, 1024);
 
-    if (tid == 0) {
-        mbar_expect_tx(bar(BQ), Ly::kQBytes);
-        for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQ), kb * 64, q0, bh);
-        load_k(qt);
-        load_v(qt);
-    }
-    bool alive = true;
-    int it = 0;
+    if (warp == 0) {
+        // ====== MMA issue (one thread): S of tile it into buffer it & 1,
+        // then P V of tile it-1 while the P pass works on tile it
+        const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);
+        const uint64_t dK = sdesc_sw128(sbase + Ly::kK, 16, 1024);
+        const uint64_t dV = sdesc_sw128(sbase + Ly::kV, 16384, 1024);
+        auto pv = [&](int j) {  // P V of tile j (buffer j & 1)
+            const int b = j & 1;
+            if (!(wait_all(PR0 + b, (j >> 1) & 1) && wait_all(BV, j & 1))) return false;
+            tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+                for (int ks = 0; ks < kT / 16; ++ks)
+                    mma_ts(tO, tS(b) + (ks >> 2) * 64 + (ks & 3) * 8, dV + (uint64_t)((ks * 2048) >> 4),
+                           kIdescPV, (ks > 0 || j > 0) ? 1u : 0u);
+                mma_commit(bar(PV0 + b));
+            }
+            __syncwarp();
+            return true;
+        };
+        bool ok = wait_all(BQ, 0);
 #pragma unroll 1
-    for (int kt = qt; kt >= kt_min; --kt, ++it) {
-        const uint32_t par = it & 1;
-        const int delta = q0 - kt * kT;
-        // ---- S = Q^ K^_k^T
-        if (alive && tid == 0) {
-            if (it == 0) pwait(bar(BQ), 0, abort_flag, status);
-            if (pwait(bar(BK), par, abort_flag, status)) {
-                tc_fence_after();
+        for (int it = 0; it < nit && ok; ++it) {
+            const int b = it & 1;
+            // the K tile, and buffer b free (P V of tile it-2 done)
+            ok = wait_all(BK, it & 1) && (it < 2 || wait_all(PV0 + b, ((it - 2) >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-                    mma_ss(tS, dQ + off, dK + off, kIdescS, ks > 0);
+                    mma_ss(tS(b), dQ + off, dK + off, kIdescS, ks > 0);
                 }
+                mma_commit(bar(SD0 + b));
             }
-            mma_commit(bar(BS));
-            if (pwait(bar(BS), par, abort_flag, status) && kt > kt_min) load_k(kt - 1);
+            __syncwarp();
+            if (it > 0) ok = pv(it - 1);
         }
-        alive = sync_alive();
-        tc_fence_after();
-        // ---- P = S (.) D into tensor memory; warpgroup w owns keys [64w, 64w+64)
-        if (alive) {
-            const int k0 = wg * 64;
-            uint32_t a[32], b[32], pk[32];
-            tmem_ld32(tS + lane_base + k0, a);
-            tmem_ld32(tS + lane_base + k0 + 32, b);
-            tmem_wait_ld();
+        if (ok) pv(nit - 1);
+    } else if (warp == 1) {
+        // ====== TMA loads: K of the next tile once S has read the current,
+        // V of the next tile once P V has read the current
+        auto load_k = [&](int kt) {
+            mbar_expect_tx(bar(BK), Ly::kQBytes);
+            for (int kb = 0; kb < KB; ++kb)
+                tma_load_3d(sbase + Ly::kK + kb * 16384, &tmK, bar(BK), kb * 64, kt * kT, bh);
+        };
+        auto load_v = [&](int kt) {
+            mbar_expect_tx(bar(BV), Ly::kVBytes);
+            for (int nb = 0; nb < VB; ++nb)
+                tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, kt * kT, bh);
+        };
+        if (lane == 0) {
+            mbar_expect_tx(bar(BQ), Ly::kQBytes);
+            for (int kb = 0; kb < KB; ++kb)
+                tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQ), kb * 64, q0, bh);
+            load_k(qt);
+            load_v(qt);
+        }
+#pragma unroll 1
+        for (int it = 0; it + 1 < nit; ++it) {
+            const int b = it & 1;
+            if (!wait_all(SD0 + b, (it >> 1) & 1)) break;
+            if (lane == 0) load_k(qt - it - 1);
+            if (!wait_all(PV0 + b, (it >> 1) & 1)) break;
+            if (lane == 0) load_v(qt - it - 1);
+            __syncwarp();
+        }
+    } else if (warp >= 4) {
+        // ====== P = S (.) D into tensor memory (warpgroup pw owns keys
+        // [64 pw, 64 pw + 64)), then the output tile
+        const int pw = (warp - 4) >> 2, gtid = tid - 128;
+        const int k0 = pw * 64;
+        bool ok = true;
+#pragma unroll 1
+        for (int it = 0; it < nit; ++it) {
+            const int b = it & 1;
+            const int delta = q0 - (qt - it) * kT;
+            if (!wait_all(SD0 + b, (it >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t a[32], c[32], pk[32];
+            tmem_ld32(tS(b) + lane_base + k0, a);
+            tmem_ld32(tS(b) + lane_base + k0 + 32, c);
+            tmem_wait_ld(a);
+            tmem_wait_ld(c);
             const float aj = exp2f((float)(delta + row) * lg);  // gamma^{Delta + j}
             const bool diag = delta == 0;
 #pragma unroll
@@ -179,71 +229,65 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const float w10 = (diag && j1 > row) ? 0.f : aj * colscale[j1];
                 const float w11 = (diag && j1 + 1 > row) ? 0.f : aj * colscale[j1 + 1];
                 pk[i] = pk_bf16(__uint_as_float(a[2 * i]) * w00, __uint_as_float(a[2 * i + 1]) * w01);
-                pk[16 + i] = pk_bf16(__uint_as_float(b[2 * i]) * w10, __uint_as_float(b[2 * i + 1]) * w11);
+                pk[16 + i] = pk_bf16(__uint_as_float(c[2 * i]) * w10, __uint_as_float(c[2 * i + 1]) * w11);
             }
-            // keys [64w, 64w+64) -> columns [64w, 64w+32) of the S region
-            tmem_st32(tS + lane_base + k0, pk);
+            // keys [64w, 64w+64) -> columns [64w, 64w+32) of the buffer
+            tmem_st32(tS(b) + lane_base + k0, pk);
             tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(PR0 + b));
         }
-        tc_fence_before();
-        __syncthreads();
-        // ---- O += P V_k
-        if (alive && tid == 0) {
-            if (pwait(bar(BV), par, abort_flag, status)) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kT / 16; ++ks)
-                    mma_ts(tO, tS + (ks >> 2) * 64 + (ks & 3) * 8, dV + (uint64_t)((ks * 2048) >> 4),
-                           kIdescPV, (ks > 0 || it > 0) ? 1u : 0u);
-            }
-            mma_commit(bar(BPV));
-            if (pwait(bar(BPV), par, abort_flag, status) && kt > kt_min) load_v(kt - 1);
-        }
-        alive = sync_alive();
-    }
-    tc_fence_after();
-    // ---- O tile out: bf16 through shared memory and TMA stores
-    if (alive) {
-        const int c0 = wg * (TV / 2);  // each warpgroup: TV/2 columns of the row
+        // the output tile once the last P V has landed (the group decides
+        // together: it meets at a barrier before the store)
+        const int last = nit - 1;
+        ok = ok && wait_all(PV0 + (last & 1), (last >> 1) & 1);
+        ok = named_sync_and(1, 256, ok);
+        if (ok) {
+            tc_fence_after();
+            const int c0 = pw * (TV / 2);  // each warpgroup: TV/2 columns of the row
 #pragma unroll 1
-        for (int g = 0; g < TV / 64; ++g) {
-            uint32_t a[32];
-            float x[32];
-            tmem_ld32(tO + lane_base + c0 + 32 * g, a);
-            tmem_wait_ld();
+            for (int g = 0; g < TV / 64; ++g) {
+                uint32_t a[32];
+                tmem_ld32(tO + lane_base + c0 + 32 * g, a);
+                tmem_wait_ld(a);
+                const int col = c0 + 32 * g;
+                if constexpr (kStage) {
+                    // bf16 through the V tile (free: the last P V has read it)
+                    uint8_t *dst = smem + Ly::kV + (col >> 6) * 16384 + row * 128;
+                    const int ch0 = (col & 63) >> 3;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
-            const int col = c0 + 32 * g;
-            if constexpr (kStage) {
-                uint8_t *dst = smem + Ly::kV + (col >> 6) * 16384 + row * 128;
-                const int ch0 = (col & 63) >> 3;
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pk_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1]));
+                        w.y = pk_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3]));
+                        w.z = pk_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5]));
+                        w.w = pk_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7]));
+                        *reinterpret_cast<uint4 *>(dst + (((ch0 + q) ^ (row & 7)) << 4)) = w;
+                    }
+                } else if (q0 + row < p.L) {
+                    float *dst = reinterpret_cast<float *>(O) + ((size_t)bh * p.L + q0 + row) * p.dv + v0 + col;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 w;
-                    w.x = pk_bf16(x[8 * q + 0], x[8 * q + 1]);
-                    w.y = pk_bf16(x[8 * q + 2], x[8 * q + 3]);
-                    w.z = pk_bf16(x[8 * q + 4], x[8 * q + 5]);
-                    w.w = pk_bf16(x[8 * q + 6], x[8 * q + 7]);
-                    *reinterpret_cast<uint4 *>(dst + (((ch0 + q) ^ (row & 7)) << 4)) = w;
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(dst + i) =
+                            make_float4(__uint_as_float(a[i]), __uint_as_float(a[i + 1]),
+                                        __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
                 }
-            } else if (q0 + row < p.L) {
-                float *dst = reinterpret_cast<float *>(O) + ((size_t)bh * p.L + q0 + row) * p.dv + v0 + col;
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
             }
-        }
-        if constexpr (kStage) {
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0) {
-                for (int nb = 0; nb < VB; ++nb)
-                    tma_store_3d(&tmO, sbase + Ly::kV + nb * 16384, v0 + nb * 64, q0, bh);
-                bulk_commit();
-                bulk_wait_all();
+            if constexpr (kStage) {
+                fence_proxy_async_smem();
+                named_sync(1, 256);
+                if (gtid == 0) {
+                    for (int nb = 0; nb < VB; ++nb)
+                        tma_store_3d(&tmO, sbase + Ly::kV + nb * 16384, v0 + nb * 64, q0, bh);
+                    bulk_commit();
+                    bulk_wait_all();
+                }
             }
         }
     }
+    __syncthreads();
+    // after an abort, copies and MMAs in flight get a bounded time to land
     if (tid == 0 && *abort_flag) {
         const long long start = clock64();
         while (clock64() - start < 20000000LL) __nanosleep(1000);
