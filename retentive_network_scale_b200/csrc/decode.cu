@@ -10,6 +10,9 @@
 // eight rows of loads in flight.  The column sums of q^ S are reduced
 // through shared memory.  State traffic uses streaming (evict-first) hints:
 // the state is larger than L2 and is not read again within the step.
+#include <algorithm>
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc_util.cuh"
@@ -122,33 +125,88 @@ recurrent_step_kernel(Params p, int ncol_tiles, const TI *q, const TI *k,
 // one pass over the state: every element runs its T updates in registers,
 //   s <- gamma s + k^_t[i] v_t[c];   o_t[c] += q^_t[i] s   (t = 0 .. T-1),
 // so the state is read and written once for all T tokens.  q, k, v, o are
-// [B][H][T][d]; the rotated q^_t, k^_t of the head and the v_t of the CTA's
-// columns sit in shared memory.  The column sums of all T tokens are reduced
-// at the end: across the row groups of a warp by shuffles, then across the
-// warps through shared memory in one pass.
-constexpr int kMultiRowsInFlight = 4;
-constexpr bool kMultiPacked = true;  // packed fp32 pairs on the rescaled path
+// [B][H][T][d].  A thread owns CPT adjacent columns of one head's state and
+// streams through all d_k rows of them, so o_t of its columns is complete
+// in its registers at the end: no reduction across threads.  A warp reads
+// 32 CPT adjacent floats of a row per load (whole 128-byte lines); every
+// thread keeps AHEAD rows of loads in flight in a ring of registers
+// that is updated in place, the first of them issued before the operands
+// are set up.  The operands of row i, the rotated (and rescaled, below)
+// k~_t[i] and q~_t[i] for every t, sit in shared memory as packed fp32
+// pairs (k, k, q, q), one 16-byte broadcast load per row and token; every
+// update is a packed fused multiply-add on two columns, two rows at a time
+// for independent chains, and v_t of the thread's columns stays in
+// registers.
+constexpr int kMultiThreads = 128;  // threads (columns / CPT) per CTA, at most
 
-template <typename TI, typename TO, int COLS, int TMAX, bool PACKED>
-__global__ void __launch_bounds__(kThreads)
+// Per token count: columns per thread (v_t and o_t live in registers), rows
+// of loads in flight per thread (even) and the CTAs per SM the registers are
+// budgeted for; measured on B200 at B=64, H=16, d_k=256, d_v=512.
+template <int TMAX>
+struct MultiCfg {
+    static constexpr int CPT = TMAX > 8 ? 2 : 4;
+    static constexpr int NPR = CPT / 2;  // fp32 pairs per row piece
+    static constexpr int AHEAD = TMAX > 4 ? 10 : 8;
+    static constexpr int MIN_CTAS = TMAX > 4 ? 3 : 4;
+    static __host__ __device__ size_t rec_bytes(int dk) { return (size_t)dk * TMAX * 16; }
+    static __host__ __device__ size_t smem_bytes(int dk) { return rec_bytes(dk) + (size_t)(kMaxDk / 2) * 8; }
+};
+
+template <int NPR>
+struct Piece {
+    uint64_t u[NPR];
+};
+__device__ __forceinline__ void ld_piece(Piece<2> &r, const float *p) {
+    const ulonglong2 x = __ldcs(reinterpret_cast<const ulonglong2 *>(p));
+    r.u[0] = x.x;
+    r.u[1] = x.y;
+}
+__device__ __forceinline__ void ld_piece(Piece<1> &r, const float *p) {
+    r.u[0] = __ldcs(reinterpret_cast<const unsigned long long *>(p));
+}
+__device__ __forceinline__ void st_piece(float *p, const Piece<2> &r) {
+    __stcs(reinterpret_cast<ulonglong2 *>(p), make_ulonglong2(r.u[0], r.u[1]));
+}
+__device__ __forceinline__ void st_piece(float *p, const Piece<1> &r) {
+    __stcs(reinterpret_cast<unsigned long long *>(p), (unsigned long long)r.u[0]);
+}
+
+template <typename TI, typename TO, int TMAX>
+__global__ void __launch_bounds__(kMultiThreads, MultiCfg<TMAX>::MIN_CTAS)
 recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k, const TI *v,
                        float *state, TO *o) {
-    constexpr int TPR = COLS / 4;
-    constexpr int RG = kThreads / TPR;
-    constexpr int kWarps = kThreads / 32;
-    // q^_t and k^_t; after the state pass the same words hold the warps'
-    // column sums
-    __shared__ __align__(16) float qk[2 * TMAX * kMaxDk];
-    __shared__ __align__(16) float vs[TMAX][COLS];
-    __shared__ double s_theta[kMaxDk / 2];
-    static_assert(kWarps * COLS <= 2 * kMaxDk, "column sums must fit in the q^/k^ words");
-    auto qs = reinterpret_cast<float (*)[kMaxDk]>(qk);
-    auto ks = reinterpret_cast<float (*)[kMaxDk]>(qk + TMAX * kMaxDk);
-    auto red = reinterpret_cast<float (*)[TMAX][COLS]>(qk);
+    using Cfg = MultiCfg<TMAX>;
+    constexpr int CPT = Cfg::CPT, NPR = Cfg::NPR;
+    constexpr int R = Cfg::AHEAD;
+    static_assert(R % 2 == 0, "rows go in pairs");
+    extern __shared__ __align__(16) uint8_t dsm[];
+    const int dk = p.dk, dv = p.dv;
+    float4 *rec = reinterpret_cast<float4 *>(dsm);  // [dk][TMAX]: (k~, k~, q~, q~)
+    double *s_theta = reinterpret_cast<double *>(dsm + Cfg::rec_bytes(dk));
 
     const int bh = blockIdx.x / ncol_tiles, ct = blockIdx.x - bh * ncol_tiles;
     const int h = bh % p.H;
-    const int dk = p.dk, dv = p.dv;
+    const int c = (ct * blockDim.x + threadIdx.x) * CPT;
+    const bool active = c < dv;
+    float *S = state + (size_t)bh * dk * dv + c;
+
+    // rows 0 .. R-1 of the thread's columns, in flight during the set-up
+    Piece<NPR> ring[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (active && r < dk) ld_piece(ring[r], S + (size_t)r * dv);
+        else
+#pragma unroll
+            for (int j = 0; j < NPR; ++j) ring[r].u[j] = 0ull;
+    }
+    Piece<NPR> vt[TMAX];  // zero past T
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t)
+#pragma unroll
+        for (int j = 0; j < NPR; ++j) {
+            const size_t base = ((size_t)bh * T + t) * dv + c + 2 * j;
+            vt[t].u[j] = active && t < T ? tc::f2_make(ld(v, base), ld(v, base + 1)) : 0ull;
+        }
     // With gamma^T >= 2^-60 the T updates run on a rescaled state: with
     // s_t = gamma s_{t-1} + k_t v_t from s_{-1} = S,
     //   s_t = gamma^{t+1} a_t,  a_t = S + sum_{tau<=t} gamma^{-(tau+1)} k_tau v_tau,
@@ -157,178 +215,152 @@ recurrent_multi_kernel(Params p, int T, int ncol_tiles, const TI *q, const TI *k
     // costs a += k~ v and o += q~ a, and the state leaves as gamma^T a.  The
     // final scaling brings every term back to its own magnitude, so the
     // relative rounding is that of the direct form.  Other decays (gamma = 0
-    // among them) take the direct form.
+    // among them) take the direct form with k~ = k^, q~ = q^.
     const float lg = p.log2g[h];
     const bool scaled = (float)T * lg >= -60.f;
     auto fq = [&](int t) { return scaled ? exp2f((float)(t + 1) * lg) : 1.f; };
     auto fk = [&](int t) { return scaled ? exp2f(-(float)(t + 1) * lg) : 1.f; };
 
-    // q^_t, k^_t (turned at position pos_offset + t) and this CTA's v_t columns
+    // operands (q~_t, k~_t turned at position pos_offset + t)
     if (p.rotate) {
         stage_theta(p, s_theta, dk / 2);
         __syncthreads();
-        for (int idx = threadIdx.x; idx < T * (dk / 2); idx += kThreads) {
+        for (int idx = threadIdx.x; idx < T * (dk / 2); idx += blockDim.x) {
             const int t = idx / (dk / 2), j = idx - t * (dk / 2);
             const size_t base = ((size_t)bh * T + t) * dk;
-            float c, sn;
-            rot_cs_fast(p.pos_offset + t, s_theta[j], &c, &sn);
+            float cs, sn;
+            rot_cs_fast(p.pos_offset + t, s_theta[j], &cs, &sn);
             float q0 = ld(q, base + 2 * j), q1 = ld(q, base + 2 * j + 1);
             float k0 = ld(k, base + 2 * j), k1 = ld(k, base + 2 * j + 1);
-            rot_pair(q0, q1, c, sn);
-            rot_pair(k0, k1, c, sn);
+            rot_pair(q0, q1, cs, sn);
+            rot_pair(k0, k1, cs, sn);
             const float a = fq(t), b = fk(t);
-            qs[t][2 * j] = a * q0; qs[t][2 * j + 1] = a * q1;
-            ks[t][2 * j] = b * k0; ks[t][2 * j + 1] = b * k1;
+            rec[(2 * j) * TMAX + t] = make_float4(b * k0, b * k0, a * q0, a * q0);
+            rec[(2 * j + 1) * TMAX + t] = make_float4(b * k1, b * k1, a * q1, a * q1);
         }
     } else {
-        for (int idx = threadIdx.x; idx < T * dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < T * dk; idx += blockDim.x) {
             const int t = idx / dk, i = idx - t * dk;
-            qs[t][i] = fq(t) * ld(q, ((size_t)bh * T + t) * dk + i);
-            ks[t][i] = fk(t) * ld(k, ((size_t)bh * T + t) * dk + i);
+            const float kk = fk(t) * ld(k, ((size_t)bh * T + t) * dk + i);
+            const float qq = fq(t) * ld(q, ((size_t)bh * T + t) * dk + i);
+            rec[i * TMAX + t] = make_float4(kk, kk, qq, qq);
         }
     }
-    for (int idx = threadIdx.x; idx < T * COLS; idx += kThreads) {
-        const int t = idx / COLS, cc = idx - t * COLS;
-        vs[t][cc] = ld(v, ((size_t)bh * T + t) * dv + ct * COLS + cc);
+    // tokens T .. TMAX-1 carry zero operands: on the rescaled path they add
+    // nothing (a += 0 v), so its loops need no test on t
+    for (int idx = threadIdx.x; idx < (TMAX - T) * dk; idx += blockDim.x) {
+        const int t = T + idx / dk, i = idx % dk;
+        rec[i * TMAX + t] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
+    if (!active) return;
 
-    const int tpr = threadIdx.x % TPR, rg = threadIdx.x / TPR;
-    const int c = ct * COLS + 4 * tpr;
     const float g = exp2f(lg);
-    const float gT = scaled ? exp2f((float)T * lg) : 1.f;
-    float *S = state + (size_t)bh * dk * dv + c;
-    float4 acc[TMAX];
-#pragma unroll
-    for (int t = 0; t < TMAX; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-
-    // packed fp32 pairs (x, y) and (z, w) of a float4
-    union P4 {
-        float4 f;
-        uint64_t u[2];
-    };
-    for (int i0 = rg; i0 < dk; i0 += RG * kMultiRowsInFlight) {
-        P4 s[kMultiRowsInFlight];
-#pragma unroll
-        for (int u = 0; u < kMultiRowsInFlight; ++u) {
-            const int i = i0 + u * RG;
-            if (i < dk) s[u].f = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)i * dv));
-        }
-        if (scaled) {
-#pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
-                if (t < T) {
-                    P4 vt, at;
-                    vt.f = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
-                    at.f = acc[t];
-#pragma unroll
-                    for (int u = 0; u < kMultiRowsInFlight; ++u) {
-                        const int i = i0 + u * RG;
-                        if (i < dk) {
-                            const float ki = ks[t][i], qi = qs[t][i];
-                            if constexpr (PACKED) {
-                                const uint64_t K2 = tc::f2_make(ki, ki), Q2 = tc::f2_make(qi, qi);
-                                s[u].u[0] = tc::f2_fma(K2, vt.u[0], s[u].u[0]);
-                                s[u].u[1] = tc::f2_fma(K2, vt.u[1], s[u].u[1]);
-                                at.u[0] = tc::f2_fma(Q2, s[u].u[0], at.u[0]);
-                                at.u[1] = tc::f2_fma(Q2, s[u].u[1], at.u[1]);
-                            } else {
-                                s[u].f.x = fmaf(ki, vt.f.x, s[u].f.x);
-                                s[u].f.y = fmaf(ki, vt.f.y, s[u].f.y);
-                                s[u].f.z = fmaf(ki, vt.f.z, s[u].f.z);
-                                s[u].f.w = fmaf(ki, vt.f.w, s[u].f.w);
-                                at.f.x = fmaf(qi, s[u].f.x, at.f.x);
-                                at.f.y = fmaf(qi, s[u].f.y, at.f.y);
-                                at.f.z = fmaf(qi, s[u].f.z, at.f.z);
-                                at.f.w = fmaf(qi, s[u].f.w, at.f.w);
-                            }
-                        }
-                    }
-                    acc[t] = at.f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kMultiRowsInFlight; ++u) {
-                s[u].f.x *= gT;
-                s[u].f.y *= gT;
-                s[u].f.z *= gT;
-                s[u].f.w *= gT;
-            }
-        } else {
-#pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
-                if (t < T) {
-                    const float4 vt = *reinterpret_cast<const float4 *>(&vs[t][4 * tpr]);
-#pragma unroll
-                    for (int u = 0; u < kMultiRowsInFlight; ++u) {
-                        const int i = i0 + u * RG;
-                        if (i < dk) {
-                            const float ki = ks[t][i], qi = qs[t][i];
-                            s[u].f.x = fmaf(g, s[u].f.x, ki * vt.x);
-                            s[u].f.y = fmaf(g, s[u].f.y, ki * vt.y);
-                            s[u].f.z = fmaf(g, s[u].f.z, ki * vt.z);
-                            s[u].f.w = fmaf(g, s[u].f.w, ki * vt.w);
-                            acc[t].x = fmaf(qi, s[u].f.x, acc[t].x);
-                            acc[t].y = fmaf(qi, s[u].f.y, acc[t].y);
-                            acc[t].z = fmaf(qi, s[u].f.z, acc[t].z);
-                            acc[t].w = fmaf(qi, s[u].f.w, acc[t].w);
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kMultiRowsInFlight; ++u) {
-            const int i = i0 + u * RG;
-            if (i < dk) __stcs(reinterpret_cast<float4 *>(S + (size_t)i * dv), s[u].f);
-        }
-    }
-
-    // o_t[c'] = the sum over row groups: the lanes of a warp that share this
-    // thread's columns (lane bits TPR and up) by shuffles, then the warps
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int t = 0; t < TMAX; ++t) {
-        if (t < T) {
-#pragma unroll
-            for (int off = TPR; off < 32; off <<= 1) {
-                acc[t].x += __shfl_xor_sync(0xffffffffu, acc[t].x, off);
-                acc[t].y += __shfl_xor_sync(0xffffffffu, acc[t].y, off);
-                acc[t].z += __shfl_xor_sync(0xffffffffu, acc[t].z, off);
-                acc[t].w += __shfl_xor_sync(0xffffffffu, acc[t].w, off);
-            }
-        }
-    }
-    __syncthreads();  // every thread is done with q^ and k^
+    const uint64_t G2 = tc::f2_make(g, g);
+    const float gT = exp2f((float)T * lg);
+    const uint64_t GT2 = tc::f2_make(gT, gT);
+    Piece<NPR> acc[TMAX];
 #pragma unroll
     for (int t = 0; t < TMAX; ++t)
-        if (t < T && lane < TPR) *reinterpret_cast<float4 *>(&red[warp][t][4 * tpr]) = acc[t];
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < T * COLS; idx += kThreads) {
-        const int t = idx / COLS, cc = idx - t * COLS;
-        float tot = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) tot += red[w][t][cc];
-        st(o, ((size_t)bh * T + t) * dv + ct * COLS + cc, tot);
-    }
+        for (int j = 0; j < NPR; ++j) acc[t].u[j] = 0ull;
+
+    // rows i and (with TWO) i+1, updated in place in their ring slots and
+    // stored
+    auto rows = [&](auto sc, auto two, int i, Piece<NPR> &s0, Piece<NPR> &s1) {
+        constexpr bool SC = decltype(sc)::value, TWO = decltype(two)::value;
+        const float4 *rc = rec + i * TMAX;
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+            if (SC || t < T) {
+                const ulonglong2 a = *reinterpret_cast<const ulonglong2 *>(rc + t);
+                ulonglong2 b;
+                if (TWO) b = *reinterpret_cast<const ulonglong2 *>(rc + TMAX + t);
+#pragma unroll
+                for (int j = 0; j < NPR; ++j) {
+                    if (SC) {
+                        s0.u[j] = tc::f2_fma(a.x, vt[t].u[j], s0.u[j]);
+                        if (TWO) s1.u[j] = tc::f2_fma(b.x, vt[t].u[j], s1.u[j]);
+                    } else {
+                        s0.u[j] = tc::f2_fma(G2, s0.u[j], tc::f2_mul(a.x, vt[t].u[j]));
+                        if (TWO) s1.u[j] = tc::f2_fma(G2, s1.u[j], tc::f2_mul(b.x, vt[t].u[j]));
+                    }
+                    acc[t].u[j] = tc::f2_fma(a.y, s0.u[j], acc[t].u[j]);
+                    if (TWO) acc[t].u[j] = tc::f2_fma(b.y, s1.u[j], acc[t].u[j]);
+                }
+            }
+        }
+        if (SC) {
+#pragma unroll
+            for (int j = 0; j < NPR; ++j) {
+                s0.u[j] = tc::f2_mul(GT2, s0.u[j]);
+                if (TWO) s1.u[j] = tc::f2_mul(GT2, s1.u[j]);
+            }
+        }
+        st_piece(S + (size_t)i * dv, s0);
+        if (TWO) st_piece(S + (size_t)(i + 1) * dv, s1);
+    };
+    auto pass = [&](auto sc) {
+        const std::true_type two;
+        const std::false_type one;
+        // whole groups of R rows: no tests on the row index; after a pair is
+        // stored its slots take the rows R further on
+        const int full = dk - dk % R;
+#pragma unroll 1
+        for (int i0 = 0; i0 < full; i0 += R) {
+            const bool more = i0 + R < dk;
+#pragma unroll
+            for (int r = 0; r < R; r += 2) {
+                rows(sc, two, i0 + r, ring[r], ring[r + 1]);
+                if (more) {
+                    if (i0 + R + r < dk) ld_piece(ring[r], S + (size_t)(i0 + R + r) * dv);
+                    if (i0 + R + r + 1 < dk) ld_piece(ring[r + 1], S + (size_t)(i0 + R + r + 1) * dv);
+                }
+            }
+        }
+        // the last dk % R rows, already in slots 0 ..
+#pragma unroll
+        for (int r = 0; r < R; r += 2) {
+            if (full + r + 1 < dk)
+                rows(sc, two, full + r, ring[r], ring[r + 1]);
+            else if (full + r < dk)
+                rows(sc, one, full + r, ring[r], ring[r + 1]);
+        }
+    };
+    if (scaled)
+        pass(std::true_type{});
+    else
+        pass(std::false_type{});
+
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t)
+        if (t < T)
+#pragma unroll
+            for (int j = 0; j < NPR; ++j) {
+                const size_t base = ((size_t)bh * T + t) * dv + c + 2 * j;
+                st(o, base, tc::f2_lo(acc[t].u[j]));
+                st(o, base + 1, tc::f2_hi(acc[t].u[j]));
+            }
 }
 
 template <typename TI, typename TO, int TMAX>
 cudaError_t launch_multi(const Params &p, int T, const void *q, const void *k, const void *v,
                          float *state, void *o, cudaStream_t st) {
-    const int cols = (p.dv % 32 == 0) ? 32 : 4;
-    const int tiles = p.dv / cols;
+    constexpr int CPT = MultiCfg<TMAX>::CPT;
+    const int nthr = p.dv / CPT;  // d_v is a multiple of 4
+    const int threads = std::min(kMultiThreads, (nthr + 31) / 32 * 32);
+    const int tiles = (nthr + threads - 1) / threads;
     const long long blocks = (long long)p.B * p.H * tiles;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const TI *qq = (const TI *)q, *kk = (const TI *)k, *vv = (const TI *)v;
-    TO *oo = (TO *)o;
-    if (cols == 32)
-        recurrent_multi_kernel<TI, TO, 32, TMAX, kMultiPacked><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
-    else
-        recurrent_multi_kernel<TI, TO, 4, TMAX, kMultiPacked><<<(unsigned)blocks, kThreads, 0, st>>>(p, T, tiles, qq, kk, vv, state, oo);
-    cudaError_t err = cudaGetLastError();
-    if (err == cudaSuccess) note_launches(1);
-    return err;
+    auto kern = recurrent_multi_kernel<TI, TO, TMAX>;
+    const size_t smem = MultiCfg<TMAX>::smem_bytes(p.dk);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, threads, smem, st>>>(p, T, tiles, (const TI *)q, (const TI *)k,
+                                                  (const TI *)v, state, (TO *)o);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) note_launches(1);
+    return e;
 }
 
 template <typename TI, typename TO>
