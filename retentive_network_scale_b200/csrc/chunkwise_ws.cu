@@ -57,6 +57,7 @@
 #include <cuda.h>
 
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -166,25 +167,113 @@ __device__ __forceinline__ uint4 ld_nc(const void *p) {
                  : "l"(p));
     return v;
 }
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void st_na(void *p, uint4 v) {
     asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
                  "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 
-// Row c of Rbar^T (K-major, 128-byte swizzle): 32 values of d-columns [d0, d0+32).
-template <int DK>
-__device__ __forceinline__ void st_rbarT_row32(uint8_t *smem, int c, int d0, const float *v) {
+// Row c of Rbar^T (K-major, 128-byte swizzle): N (16 or 32) values of
+// d-columns [d0, d0+N).
+template <int DK, int N = 32>
+__device__ __forceinline__ void st_rbarT_row(uint8_t *smem, int c, int d0, const float *v) {
     uint8_t *blk = smem + Layout<DK>::rbar_blk(d0 >> 6) + c * 128;
     const int ch0 = (d0 & 63) >> 3;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < N / 8; ++q) {
         uint4 w;
         w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
         w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
         w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
         w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
         *reinterpret_cast<uint4 *>(blk + (((ch0 + q) ^ (c & 7)) << 4)) = w;
+    }
+}
+
+// R^T columns [D0, D1) of this thread's TMEM lane (value column `row`)
+// after a chunk's state update: scaled by g2 (the next chunk's gamma^n,
+// packed) back into TMEM and, as bf16, into Rbar^T for the next O''
+// product; after the last chunk into state_out instead (`so` points at the
+// lane's value column of d-row 0, or is null).  Units of W (16 or 32)
+// columns; with PIPE the load of the next unit is in flight while the
+// current one is processed (W more registers).
+template <int DK, int D0, int D1, int W, bool PIPE>
+__device__ __forceinline__ void state_cols(uint8_t *smem, uint32_t t_lane, int row, uint64_t g2,
+                                           bool last, float *so, int dv) {
+    static_assert((W == 16 || W == 32) && D0 % W == 0 && D1 % W == 0 && D1 > D0, "whole units");
+    constexpr int NU = (D1 - D0) / W;
+    constexpr int NB = PIPE ? 2 : 1;
+    auto ld = [&](int col, uint32_t(&x)[W]) {
+        if constexpr (W == 32) tmem_ld32(t_lane + col, x);
+        else tmem_ld16(t_lane + col, x);
+    };
+    if (last) {
+        // the final state, unit by unit
+#pragma unroll 1
+        for (int dd = D0; dd < D1; dd += W) {
+            uint32_t x[W];
+            ld(dd, x);
+            tmem_wait_ld(x);
+            if (so) {
+#pragma unroll
+                for (int i = 0; i < W; i += 2) {
+                    const uint64_t y = f2_mul((static_cast<uint64_t>(x[i + 1]) << 32) | x[i], g2);
+                    so[(size_t)(dd + i) * dv] = f2_lo(y);
+                    so[(size_t)(dd + i + 1) * dv] = f2_hi(y);
+                }
+            }
+        }
+        return;
+    }
+    uint32_t r[NB][W];
+    ld(D0, r[0]);
+    tmem_wait_ld(r[0]);
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+        uint32_t(&cur)[W] = r[u % NB];
+        if (PIPE && u + 1 < NU) ld(D0 + W * (u + 1), r[(u + 1) % NB]);
+        const int dd = D0 + W * u;
+        float v[W];
+#pragma unroll
+        for (int i = 0; i < W; i += 2) {
+            const uint64_t x = f2_mul((static_cast<uint64_t>(cur[i + 1]) << 32) | cur[i], g2);
+            v[i] = f2_lo(x);
+            v[i + 1] = f2_hi(x);
+        }
+        st_rbarT_row<DK, W>(smem, row, dd, v);
+#pragma unroll
+        for (int i = 0; i < W; ++i) cur[i] = __float_as_uint(v[i]);
+        if constexpr (W == 32) tmem_st32(t_lane + dd, cur);
+        else tmem_st16(t_lane + dd, cur);
+        if (u + 1 < NU) {
+            if (!PIPE) ld(D0 + W * (u + 1), r[(u + 1) % NB]);
+            tmem_wait_ld(r[(u + 1) % NB]);
+        }
+    }
+}
+
+// The starting state of R^T columns [D0, D1): gamma^{n_0} S_in^T into TMEM
+// and its bf16 copy into Rbar^T (`si` points at the lane's value column of
+// d-row 0, or is null for a lane past d_v: zeros); without a state
+// (has_in false) zeros into Rbar^T only.
+template <int DK, int D0, int D1>
+__device__ __forceinline__ void state_init_cols(uint8_t *smem, uint32_t t_lane, int row, bool has_in,
+                                                const float *si, float g0, int dv) {
+#pragma unroll 1
+    for (int d0 = D0; d0 < D1; d0 += 32) {
+        float v[32];
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = si ? si[(size_t)(d0 + i) * dv] * g0 : 0.f;
+        st_rbarT_row<DK>(smem, row, d0, v);
+        if (has_in) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+            tmem_st32(t_lane + d0, r);
+        }
     }
 }
 
@@ -459,25 +548,13 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int row = tid & 127;  // chunk row for S, value column for R^T
         const int quad = warp & 3;
         const bool vcol = row < dvr;  // this lane's value column exists
+        float *so = state_out && vcol ? state_out + (size_t)bh * DK * dv + v0 + row : nullptr;
         {
             // starting state: R^T = gamma^{n_0} S_in^T in TMEM and Rbar^T =
             // bf16 of the same; zeros without a state
-            const bool has_in = state_in != nullptr;
-            const float g0 = decay_pow(lg, min(kC, L));
-#pragma unroll 1
-            for (int d0 = 0; d0 < DK; d0 += 32) {
-                float v[32];
-                uint32_t r[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    v[i] = has_in && vcol ? state_in[((size_t)bh * DK + d0 + i) * dv + v0 + row] * g0 : 0.f;
-                st_rbarT_row32<DK>(smem, row, d0, v);
-                if (has_in) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-                    tmem_st32(tR + lane_base + d0, r);
-                }
-            }
+            const float *si = state_in && vcol ? state_in + (size_t)bh * DK * dv + v0 + row : nullptr;
+            state_init_cols<DK, 0, DK>(smem, tR + lane_base, row, state_in != nullptr, si,
+                                       decay_pow(lg, min(kC, L)), dv);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -527,51 +604,24 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // product no longer reads Rbar^T
             if (!(wait_all(UD, par) && wait_all(SOD, par))) break;
             tc_fence_after();
+            // (the first half of Rbar^T is published as soon as it is written)
             const float gnext = last ? 1.f : decay_pow(lg, n_next);
-            const uint64_t G2 = f2_make(gnext, gnext);
-#pragma unroll 1
-            for (int d0 = 0; d0 < DK; d0 += 64) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tR + lane_base + d0, ra);
-                tmem_ld32(tR + lane_base + d0 + 32, rb);
-                tmem_wait_ld(ra);
-                tmem_wait_ld(rb);
-                // R^T columns [dd, dd+32): decay, bf16 copy, back to TMEM; or state_out
-                auto pass32 = [&](uint32_t (&r)[32], int dd) {
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const uint64_t x = f2_mul(f2_of(r + i), G2);
-                        v[i] = f2_lo(x);
-                        v[i + 1] = f2_hi(x);
-                    }
-                    if (last) {
-                        if (state_out && vcol) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                state_out[((size_t)bh * DK + dd + i) * dv + v0 + row] = v[i];
-                        }
-                    } else {
-                        st_rbarT_row32<DK>(smem, row, dd, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-                        tmem_st32(tR + lane_base + dd, r);
-                    }
-                };
-                pass32(ra, d0);
-                pass32(rb, d0 + 32);
-                if (DK >= 128 && d0 + 64 == DK / 2) {
-                    // the first half of Rbar^T is ready for the next O'' product
-                    tmem_wait_st();
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    warp_arrive(RBL);
-                }
+            const uint64_t g2 = f2_make(gnext, gnext);
+            const uint32_t tl = tR + lane_base;
+            if constexpr (DK >= 128) {
+                state_cols<DK, 0, DK / 2, 32, true>(smem, tl, row, g2, last, so, dv);
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                warp_arrive(RBL);
+                state_cols<DK, DK / 2, DK, 32, true>(smem, tl, row, g2, last, so, dv);
+            } else {
+                state_cols<DK, 0, DK, 32, true>(smem, tl, row, g2, last, so, dv);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
-            if constexpr (DK < 128) warp_arrive(RBL);  // no first half to publish early
+            if constexpr (DK < 128) warp_arrive(RBL);
             warp_arrive(RB);
         }
     } else {
@@ -587,20 +637,21 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // rows of this lane group's 16-byte row pieces: 32 quad + 4 j4 + i
         auto grow = [&](int i) { return 32 * quad + 4 * j4 + i; };
         const __nv_bfloat16 *Gb = G + (size_t)b * g_batch + ycol;
-        // With the gate, chunk c's outputs are finished one chunk later: at
-        // chunk c the epilogue copies O''(c) out of tensor memory, publishes
-        // its row statistics and starts loading G(c), then completes Y(c-1),
-        // whose statistics exchange and G loads have had a whole chunk to
-        // land.  What is carried over is, per row segment of 64 columns,
-        // O'' - shift as bf16 (the shift is the segment's first value, so the
+        // With the gate, each chunk goes: G(c) loads issued; O''(c) copied
+        // out of tensor memory (which is then released at once to the next
+        // chunk's product); its row statistics published to the cluster;
+        // then Y(c), once every CTA of the head has published.  The G loads
+        // land while O'' is read out and the statistics are exchanged.  What
+        // Y(c) needs of O'' is kept, per row segment of 64 columns, as
+        // O'' - shift in bf16 (the shift is the segment's first value, so the
         // residuals are of the size of the row's spread and keep fp32's
-        // range), the shift and the raw G tile.
-        uint32_t rp[32];  // residuals of the carried chunk, bf16 pairs
+        // range) with the shift.
+        uint32_t rp[32];  // residuals of the chunk, bf16 pairs
         uint4 gp[8];      // its G, two halves of 32 columns (16-byte pieces as loaded, rows 4 j4 + i)
         float shift_p = 0.f, alpha_p = 1.f;
         int t0_p = 0, n_p = 0;
-        // Y of the carried chunk (parity par_p), once every CTA of the head
-        // has published its statistics.  A wait that runs out leaves the
+        // Y of chunk c_p (parity par_p), once every CTA of the head has
+        // published its statistics.  A wait that runs out leaves the
         // chunk's Y unwritten; the group stops at the next barrier.
         auto finish = [&](int c_p) {
             const uint32_t par_p = c_p & 1;
@@ -649,8 +700,26 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int t0 = c * kC;
             const int n = min(kC, L - t0);
             auto row_ok = [&](int i) { return ocols && grow(i) < n; };
-            if constexpr (FUSE)
-                if (c > 0) finish(c - 1);
+            if constexpr (FUSE) {
+                // G of this chunk (coalesced: one instruction reads 64
+                // contiguous bytes of each of 8 rows)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = grow(i);
+                        gp[4 * hf + i] = ocols && r < n ? ld_nc(Gb + (size_t)(t0 + r) * g_row + 32 * hf + 8 * m4)
+                                                        : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                // and the next chunk's G into L2 (a row segment of 64 columns
+                // is one 128-byte line), so that its loads do not wait on HBM
+                if (m4 == 0 && ocols && c + 1 < nchunks) {
+                    const int n1 = min(kC, L - t0 - kC);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (grow(i) < n1) prefetch_l2(Gb + (size_t)(t0 + kC + grow(i)) * g_row);
+                }
+            }
             {
                 // with the gate the group meets at named barriers below, so it
                 // decides together whether to go on
@@ -713,23 +782,12 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // the slots are written (the barrier above ordered them before
                 // this arrival); warp 3 announces them to the cluster
                 if (gtid == 0) mbar_arrive(bar(SL));
-                // G of this chunk (coalesced: one instruction reads 64
-                // contiguous bytes of each of 8 rows), used one chunk later
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = grow(i);
-                        gp[4 * hf + i] = ocols && r < n ? ld_nc(Gb + (size_t)(t0 + r) * g_row + 32 * hf + 8 * m4)
-                                                        : make_uint4(0u, 0u, 0u, 0u);
-                    }
                 shift_p = shift;
                 alpha_p = alpha;
                 t0_p = t0;
                 n_p = n;
             }
-            if constexpr (FUSE)
-                if (c + 1 == nchunks) finish(c);
+            if constexpr (FUSE) finish(c);
         }
     }
 
