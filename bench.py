@@ -641,8 +641,8 @@ def run_ours(args, world, rank, local):
     # bandwidth): HBM is the roof that binds this kernel
     roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / pk["hbm_gbs"],
-                "traffic": profiled_traffic("chunkwise_tc.cu", "chunkwise_tc_msr_1p3b.md"),
-                "kernel": "chunkwise_tc_kernel<256, bf16, fused GroupNorm/gate>",
+                "traffic": profiled_traffic("chunkwise_ws.cu", "chunkwise_ws_msr_1p3b.md"),
+                "kernel": "chunkwise_ws_kernel<256, bf16, fused GroupNorm/gate>",
                 "peak_source": f"{pk_src} (copy bandwidth)",
                 "ms_per_launch": ms_kernel, "bytes_per_launch": bytes_alg,
                 "flops_per_launch": flops,
