@@ -69,6 +69,7 @@ void make_params(const ret_desc *d, Params *p) {
     p->rotate = d->rotate;
     p->pos_offset = d->pos_offset;
     p->seg_heads = 1;
+    p->reverse = 0;
     p->seg_len = 0;
     for (int h = 0; h < d->H; ++h)
         p->log2g[h] = d->gamma[h] > 0.0 ? (float)std::log2(d->gamma[h]) : -INFINITY;

@@ -11,12 +11,14 @@
 //   dv_m  = sum_{t>=m} gamma^{t-m} (k^_m . q^_t) do_t    anti-causal
 //   dq_t = Theta_t^T dq^_t,  dk_m = Theta_m^T dk^_m.
 // Each is a retention of rearranged operands: (query, key, value) =
-// (dO, V, K^) causally, and (V, dO, Q^), (K^, Q^, dO) over the time-reversed
-// sequences.  Retention is linear in its scores, so a contraction over d_v
-// (the dO . V scores) splits into column blocks of 128 or 256 whose outputs
-// add: every product then fits the tensor-core chunkwise kernel.  The
-// operands are first copied (bf16) turned and/or time-reversed; the fp32
-// partial outputs are summed, turned back and un-reversed at the end.
+// (dO, V, K^) causally, and (V, dO, Q^), (K^, Q^, dO) anti-causally, which
+// the tensor-core chunk loop runs in its reverse mode (blocks from last to
+// first, mirrored mask and weights) on the operands as they are.
+// Retention is linear in its scores, so a contraction over d_v (the dO . V
+// scores) splits into column blocks of 128 or 256 whose outputs add: every
+// product then fits the tensor-core chunkwise kernel.  With rotation, Q and
+// K are first copied turned (bf16); the fp32 partial outputs are summed and
+// turned back at the end.
 #include <algorithm>
 
 #include "common.cuh"
@@ -202,7 +204,7 @@ int split_dv(int dv, int *w) {  // at most two blocks for d_v <= 512
 }
 
 struct BwdLayout {
-    size_t kh, qf, kf, vf, of, prep, part_dk, part_dv;  // offsets
+    size_t kh, qh, prep, part_dk, part_dv;  // offsets
     size_t bytes;
     int nsplit;
 };
@@ -214,11 +216,9 @@ BwdLayout bwd_layout(const ret_desc *d) {
     const size_t rows = (size_t)d->B * d->H * d->L;
     const size_t bk = rows * d->d_k * 2, bv = rows * d->d_v * 2;
     size_t o = 0;
-    z.kh = o; o += round_up(bk);
-    z.qf = o; o += round_up(bk);
-    z.kf = o; o += round_up(bk);
-    z.vf = o; o += round_up(bv);
-    z.of = o; o += round_up(bv);
+    (void)bv;
+    z.kh = o; o += d->rotate ? round_up(bk) : 0;  // turned K and Q
+    z.qh = o; o += d->rotate ? round_up(bk) : 0;
     z.prep = o; o += round_up(2 * rows * 256 * 2);            // prepared Q^, K~ of one call
     z.part_dk = o; o += round_up(rows * d->d_k * 4) * 2 * z.nsplit;  // dQ^, dK^ partials
     z.part_dv = o; o += round_up(rows * d->d_v * 4);
@@ -266,12 +266,13 @@ cudaError_t unturn_sum(const Params &p, int d, const float *part0, const float *
 // `qk` (column offset already in the pointers), value rows [B][H][L][dv']
 // contiguous, fp32 output [B][H][L][dv'].
 cudaError_t product(const Params &base, int dqk, int dval, const void *q, const void *k,
-                    RowLayout qk, const void *v, void *prep_ws, float *out, int *status,
+                    RowLayout qk, const void *v, bool anti, void *prep_ws, float *out, int *status,
                     cudaStream_t st) {
     Params p = base;
     p.dk = dqk;
     p.dv = dval;
     p.rotate = 0;  // the operands come turned already
+    p.reverse = anti ? 1 : 0;
     // only K~ is written: the query rows are read in place through `qk`
     const void *qh = nullptr, *kt = nullptr;
     cudaError_t e = launch_chunkwise_prep_strided(p, 128, q, k, qk, false, prep_ws, &qh, &kt, st);
@@ -333,7 +334,8 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
     const int dk = desc->d_k, dv = desc->d_v;
     const bool rot = desc->rotate != 0;
     const size_t rows = (size_t)desc->B * desc->H * desc->L;
-    void *Kh = ws + z.kh, *Qf = ws + z.qf, *Kf = ws + z.kf, *Vf = ws + z.vf, *Of = ws + z.of;
+    const void *Kh = rot ? static_cast<const void *>(ws + z.kh) : K;
+    const void *Qh = rot ? static_cast<const void *>(ws + z.qh) : Q;
     void *prep = ws + z.prep;
     float *partA = reinterpret_cast<float *>(ws + z.part_dk);
     const size_t part_stride = round_up(rows * dk * 4) / 4;      // floats between partials
@@ -342,37 +344,37 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
 
     cudaError_t e = cudaSuccess;
     auto run = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
-    // 1. turned and/or time-reversed bf16 copies
-    run(flip_turn(p, dk, K, Kh, rot, false, st));
-    run(flip_turn(p, dk, Q, Qf, rot, true, st));
-    run(flip_turn(p, dk, K, Kf, rot, true, st));
-    run(flip_turn(p, dv, V, Vf, false, true, st));
-    run(flip_turn(p, dv, dO, Of, false, true, st));
-    // 2. dQ^ (causal: dO, V, K^) and reversed dK^ (V, dO, Q^), per column block of d_v
+    // 1. turned bf16 copies of K and Q
+    if (rot) {
+        run(flip_turn(p, dk, K, ws + z.kh, true, false, st));
+        run(flip_turn(p, dk, Q, ws + z.qh, true, false, st));
+    }
+    // 2. dQ^ (causal: dO, V, K^) and dK^ (anti-causal: V, dO, Q^), per
+    //    column block of d_v
     int w[8];
     const int n = split_dv(dv, w);
     const RowLayout full_v = bhld_layout(p, dv);
     const auto *dO8 = static_cast<const uint8_t *>(dO), *V8 = static_cast<const uint8_t *>(V);
     for (int i = 0, c0 = 0; i < n && e == cudaSuccess; c0 += w[i], ++i) {
         const size_t off = (size_t)c0 * 2;
-        run(product(p, w[i], dk, dO8 + off, V8 + off, full_v, Kh, prep, partA + i * part_stride,
-                    status, st));
-        run(product(p, w[i], dk, static_cast<uint8_t *>(Vf) + off, static_cast<uint8_t *>(Of) + off,
-                    full_v, Qf, prep, partB + i * part_stride, status, st));
+        run(product(p, w[i], dk, dO8 + off, V8 + off, full_v, Kh, false, prep,
+                    partA + i * part_stride, status, st));
+        run(product(p, w[i], dk, V8 + off, dO8 + off, full_v, Qh, true, prep,
+                    partB + i * part_stride, status, st));
     }
-    // 3. reversed dV (K^, Q^, dO)
-    run(product(p, dk, dv, Kf, Qf, bhld_layout(p, dk), Of, prep, partC, status, st));
-    // 4. sums, the opposite turn, and back to forward time
+    // 3. dV (anti-causal: K^, Q^, dO)
+    run(product(p, dk, dv, Kh, Qh, bhld_layout(p, dk), dO, true, prep, partC, status, st));
+    // 4. sums and the opposite turn
     const float *a1 = n > 1 ? partA + part_stride : nullptr;
     const float *b1 = n > 1 ? partB + part_stride : nullptr;
     if (desc->out_dtype == RET_BF16) {
         run(unturn_sum<__nv_bfloat16>(p, dk, partA, a1, false, rot, dQ, st));
-        run(unturn_sum<__nv_bfloat16>(p, dk, partB, b1, true, rot, dK, st));
-        run(unturn_sum<__nv_bfloat16>(p, dv, partC, nullptr, true, false, dV, st));
+        run(unturn_sum<__nv_bfloat16>(p, dk, partB, b1, false, rot, dK, st));
+        run(unturn_sum<__nv_bfloat16>(p, dv, partC, nullptr, false, false, dV, st));
     } else {
         run(unturn_sum<float>(p, dk, partA, a1, false, rot, dQ, st));
-        run(unturn_sum<float>(p, dk, partB, b1, true, rot, dK, st));
-        run(unturn_sum<float>(p, dv, partC, nullptr, true, false, dV, st));
+        run(unturn_sum<float>(p, dk, partB, b1, false, rot, dK, st));
+        run(unturn_sum<float>(p, dv, partC, nullptr, false, false, dV, st));
     }
     return e == cudaSuccess ? RET_OK : RET_ERR_CUDA;
 }

@@ -337,6 +337,10 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int L = p.L, dv = p.dv;
     const int nchunks = (L + kC - 1) / kC;
     const int nr = (int)gridDim.x;  // CTAs of this head (the cluster when FUSE)
+    // the block of rows handled at step c: in order, or last to first for
+    // the anti-causal form (the mask and the weights mirror within a block)
+    const bool rev = p.reverse != 0;
+    auto blk = [&](int c) { return rev ? nchunks - 1 - c : c; };
 
     if (sbase & 1023u) {  // swizzle atoms need 1024-byte alignment (same for every CTA)
         if (tid == 0) atomicExch(status, (int)RET_ERR_CUDA);
@@ -465,17 +469,17 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         auto load_q = [&](int c) {
             mbar_expect_tx(bar(QF), Ly::kQBytes);
             for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(QF), kb * 64, c * kC, bh);
+                tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(QF), kb * 64, blk(c) * kC, bh);
         };
         auto load_k = [&](int c) {
             mbar_expect_tx(bar(KF), Ly::kQBytes);
             for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(sbase + Ly::k_blk(kb), &tmK, bar(KF), kb * 64, c * kC, bh);
+                tma_load_3d(sbase + Ly::k_blk(kb), &tmK, bar(KF), kb * 64, blk(c) * kC, bh);
         };
         auto load_v = [&](int c) {
             mbar_expect_tx(bar(VF), dvr * kC * 2);
             for (int nb = 0; nb < dvr / 64; ++nb)
-                tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(VF), vx0 + nb * 64, c * kC, vz);
+                tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(VF), vx0 + nb * 64, blk(c) * kC, vz);
         };
         if (lane == 0) {
             load_q(0);
@@ -498,12 +502,12 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (zeta_v) {
 #pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
-                const int n = min(kC, L - c * kC);
+                const int n = min(kC, L - blk(c) * kC);
                 if (!wait_all(VF, c & 1)) break;
 #pragma unroll 1
                 for (int rr = 0; rr < 4; ++rr) {
                     const int r = lane + 32 * rr;  // rows of both 64-column blocks
-                    const float z = r < n ? decay_pow(lg, n - 1 - r) : 0.f;
+                    const float z = r < n ? decay_pow(lg, rev ? r : n - 1 - r) : 0.f;
                     const uint64_t Z = f2_make(z, z);
 #pragma unroll
                     for (int nb = 0; nb < 2; ++nb) {
@@ -554,7 +558,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // bf16 of the same; zeros without a state
             const float *si = state_in && vcol ? state_in + (size_t)bh * DK * dv + v0 + row : nullptr;
             state_init_cols<DK, 0, DK>(smem, tR + lane_base, row, state_in != nullptr, si,
-                                       decay_pow(lg, min(kC, L)), dv);
+                                       decay_pow(lg, min(kC, L - blk(0) * kC)), dv);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -565,24 +569,24 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const bool last = c + 1 == nchunks;
-            const int t0 = c * kC;
-            const int n_next = last ? 0 : min(kC, L - t0 - kC);
+            const int n_next = last ? 0 : min(kC, L - blk(c + 1) * kC);
             if (!wait_all(SSD, par)) break;
             tc_fence_after();
-            // P = bf16(S) on keys j' <= j, else 0: keys [32 cb, 32 cb + 32)
-            // into columns [32 cb, 32 cb + 16); groups right of the diagonal
-            // block are zero for every row of this warp
+            // P = bf16(S) on keys j' <= j (j' >= j anti-causal), else 0: keys
+            // [32 cb, 32 cb + 32) into columns [32 cb, 32 cb + 16); groups on
+            // the far side of the diagonal block are zero for every row of
+            // this warp
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t pk[16];
-                if (cb > quad) {
+                if (rev ? cb < quad : cb > quad) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 } else {
                     uint32_t a[32];
                     tmem_ld32(tS + lane_base + 32 * cb, a);
                     tmem_wait_ld(a);
-                    if (cb < quad) {
+                    if (cb != quad) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
@@ -590,8 +594,10 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int k0 = 32 * cb + 2 * i;
-                            pk[i] = pack_bf16(k0 <= row ? __uint_as_float(a[2 * i]) : 0.f,
-                                              k0 + 1 <= row ? __uint_as_float(a[2 * i + 1]) : 0.f);
+                            const bool in0 = rev ? k0 >= row : k0 <= row;
+                            const bool in1 = rev ? k0 + 1 >= row : k0 + 1 <= row;
+                            pk[i] = pack_bf16(in0 ? __uint_as_float(a[2 * i]) : 0.f,
+                                              in1 ? __uint_as_float(a[2 * i + 1]) : 0.f);
                         }
                     }
                 }
@@ -697,7 +703,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
-            const int t0 = c * kC;
+            const int t0 = blk(c) * kC;
             const int n = min(kC, L - t0);
             auto row_ok = [&](int i) { return ocols && grow(i) < n; };
             if constexpr (FUSE) {
@@ -714,10 +720,10 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // and the next chunk's G into L2 (a row segment of 64 columns
                 // is one 128-byte line), so that its loads do not wait on HBM
                 if (m4 == 0 && ocols && c + 1 < nchunks) {
-                    const int n1 = min(kC, L - t0 - kC);
+                    const int t1 = blk(c + 1) * kC, n1 = min(kC, L - t1);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        if (grow(i) < n1) prefetch_l2(Gb + (size_t)(t0 + kC + grow(i)) * g_row);
+                        if (grow(i) < n1) prefetch_l2(Gb + (size_t)(t1 + grow(i)) * g_row);
                 }
             }
             {
@@ -728,7 +734,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (!ok) break;
             }
             tc_fence_after();
-            const float alpha = exp2f((float)(row + 1 - n) * lg);  // gamma^{row+1-n}
+            // gamma^{row+1-n} (gamma^{-row} anti-causal)
+            const float alpha = exp2f((float)(rev ? -row : row + 1 - n) * lg);
             const uint64_t A2 = f2_make(alpha, alpha);
             // O'' in two halves of 32 columns: O (when asked for), the
             // running statistics (shifted by the row's first value, even

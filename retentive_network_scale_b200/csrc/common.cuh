@@ -28,6 +28,12 @@ struct Params {
     // plain heads; only the streaming pass reads them.
     int seg_heads;
     long long seg_len;
+    // Anti-causal retention, o_t = sum over m >= t of gamma^{m-t} (q^_t . k^_m)
+    // v_m (the time-reversed products of the backward pass): the streaming
+    // pass weights key row j of a block by gamma^j and the tensor-core chunk
+    // loop walks the blocks from last to first with the mirrored mask.  0
+    // for the forward forms; no other kernel reads it.
+    int reverse;
 };
 
 // ------------------------------------------------------------------ dtypes

@@ -7,7 +7,8 @@
 // gamma^{n-1-j} in the state update.  The tensor-core kernel multiplies
 //   Q^_t = Theta_t Q_t                        (Q itself without rotation)
 //   K~_t = zeta_t Theta_t K_t,  zeta_t = gamma_h^{n-1-j}
-// (t = chunk start + j).  Computing them here, once per row, takes the
+// (t = chunk start + j; zeta_t = gamma_h^j for the anti-causal products of
+// the backward pass, whose chunk loop runs from the last block to the first).  Computing them here, once per row, takes the
 // turn off the kernel's critical path; inside the kernel the CUDA cores
 // would turn each tile while the tensor cores wait, and every CTA of a head
 // would turn the same rows.  The kernel then loads the prepared rows from
@@ -98,7 +99,7 @@ chunk_prep_kernel(const Params p, int chunk, long long items, const __nv_bfloat1
         if (r < nr) {
             const int t = t0 + r, j = t % chunk;
             const int n = min(chunk, p.L - (t - j));
-            const float z = decay_pow(lg, n - 1 - j);
+            const float z = decay_pow(lg, p.reverse ? j : n - 1 - j);
             uint32_t *uk = reinterpret_cast<uint32_t *>(&xk[r]);
             uint32_t *uq = reinterpret_cast<uint32_t *>(&xq[r]);
 #pragma unroll
