@@ -9,7 +9,7 @@
 // segment's rows.  The weight comes
 //   - on the keys, K~_t = gamma^{n-1-t} k^_t (the streaming pass of prep.cu
 //     with the segment as one block), or
-//   - on the value rows (value mode 1), which warps 1-3 scale in shared
+//   - on the value rows (value mode 1), which warps 1-7 scale in shared
 //     memory as each block of 128 rows lands, or
 //   - split (value mode 2): keys weighted per block of 128 rows by the
 //     streaming pass of the chunk loop, K~_t = gamma^{m-1-j} k^_t for row j
@@ -18,7 +18,7 @@
 // owns one (b, h) and 128 value columns and accumulates U^T = V^T K~ in
 // tensor memory over blocks of 128 rows, which TMA brings through a ring
 // of stages; its one MMA thread also reissues each stage's loads once the
-// product that read it has completed.  The four warps then move U^T out
+// product that read it has completed.  The eight warps then move U^T out
 // of tensor memory into U [d_k][d_v] (fp32), one value column per lane.
 //
 // Every wait is bounded (about 2 s): on expiry RET_ERR_TIMEOUT is latched in
@@ -37,6 +37,8 @@ using namespace tc;
 
 constexpr int kRows = 128;  // rows per block (the MMA's K extent, 8 steps of 16)
 constexpr int kTV = 128;    // value columns per CTA (MMA M)
+constexpr int kThreads = 256;                // warp 0 issues, warps 1-7 scale value rows
+constexpr int kScalers = kThreads - 32;
 constexpr long long kTimeoutCycles = 4000000000LL;
 
 template <int DK>
@@ -52,7 +54,7 @@ struct SLayout {
 };
 
 template <int DK>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK,
                      const Params p, int zeta_v, float *__restrict__ U, int *status) {
     using Ly = SLayout<DK>;
@@ -77,7 +79,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::kAbort);
     if (tid == 0) {
         for (int i = 0; i < 3 * NS + 1; ++i)
-            mbar_init(sbase + Ly::kBar + 8u * i, (i >= 2 * NS && i < 3 * NS) ? 3 : 1);
+            mbar_init(sbase + Ly::kBar + 8u * i, (i >= 2 * NS && i < 3 * NS) ? kScalers / 32 : 1);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -128,7 +130,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
     } else if (zeta_v && warp > 0) {
         // V' = diag(zeta) V as each block lands, zeta_t = gamma^{L-1-t}
         // (mode 1) or gamma^{L - 128 blk - m} for the block's m rows (mode
-        // 2): warps 1-3, one row per thread and pass (rows past L are zeros)
+        // 2): warps 1-7, one row per thread and pass (rows past L are zeros)
         const int t = tid - 32;
         const int lane = tid & 31;
 #pragma unroll 1
@@ -140,7 +142,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
                 break;
             uint8_t *vt = smem + s * Ly::kStage;
 #pragma unroll 1
-            for (int r = t; r < kRows; r += 96) {
+            for (int r = t; r < kRows; r += kScalers) {
                 const int row = blk * kRows + r;
                 const int m = min(kRows, L - blk * kRows);
                 const float z = row >= L ? 0.f
@@ -170,15 +172,17 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
         }
     }
     __syncthreads();
-    // U[d][v0 + lane] of every d-column of U^T (lanes are value columns)
+    // U[d][v0 + lane] of every d-column of U^T (lanes are value columns;
+    // warps 0-3 take the first half of the d-columns, warps 4-7 the rest)
     const int row = tid & 127;
+    const int dbeg = warp < 4 ? 0 : DK / 2;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = *abort_flag == 0 && mbar_wait_bounded(done, 0, abort_flag, status, kTimeoutCycles);
     ok = __all_sync(0xffffffffu, ok);
     if (ok && *abort_flag == 0) {
         tc_fence_after();
 #pragma unroll 1
-        for (int d0 = 0; d0 < DK; d0 += 32) {
+        for (int d0 = dbeg; d0 < dbeg + DK / 2; d0 += 32) {
             uint32_t r[32];
             tmem_ld32(tmem + lane_base + d0, r);
             tmem_wait_ld(r);
@@ -206,7 +210,7 @@ cudaError_t launch_dk(const Params &p, const CUtensorMap &mv, const CUtensorMap 
     const int smem = (int)SLayout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(p.dv / kTV, p.B * p.H), 128, smem, st>>>(mv, mk, p, zeta_v, U, status);
+    kern<<<dim3(p.dv / kTV, p.B * p.H), kThreads, smem, st>>>(mv, mk, p, zeta_v, U, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) note_launches(1);
     return e;
