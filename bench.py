@@ -367,7 +367,8 @@ def bench_backward(R, w, d, pk, reps=3):
     dQ = torch.empty(w.B, w.H, w.L, w.d_k, device="cuda")
     dK = torch.empty_like(dQ)
     dV = torch.empty(w.B, w.H, w.L, w.d_v, device="cuda")
-    ws = torch.empty(R.lib_backward_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, w.chunk),
+    ws = torch.empty(R.lib_backward_workspace_size(w.B, w.H, w.L, w.d_k, w.d_v, g, w.chunk,
+                                                   rotate=w.rotate),
                      dtype=torch.uint8, device="cuda")
     fn = lambda: R.ret_backward(d["Q"], d["K"], d["V"], dO, g, w.chunk, dQ=dQ, dK=dK, dV=dV,  # noqa: E731
                                 rotate=w.rotate, workspace=ws)

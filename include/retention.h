@@ -304,7 +304,8 @@ size_t ret_msr_layer_workspace_size(const ret_desc *desc, int d_model,
  *     dv_m  = sum_{t>=m} gamma^{t-m} (k^_m . q^_t) do_t,
  *     dq_t = Theta_t^T dq^_t, dk_m = Theta_m^T dk^_m.
  * Each is evaluated as a chunkwise retention of rearranged operands on the
- * tensor cores (the two anti-causal ones over time-reversed copies).
+ * tensor cores (the two anti-causal ones by the chunk loop's reverse mode,
+ * on the operands in place; with rotation Q and K are first copied turned).
  *   Q, K    device bf16 [B][H][L][d_k];  V, dO device bf16 [B][H][L][d_v]
  *   dQ, dK  device out_dtype [B][H][L][d_k];  dV device out_dtype
  *           [B][H][L][d_v]; all fully overwritten
@@ -319,8 +320,9 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q,
                         void *dK, void *dV, void *workspace,
                         size_t workspace_bytes, void *stream);
 
-/* Device workspace bytes ret_backward needs; 0 for descriptions it would
- * reject by their arguments and for empty problems.  Never fails. */
+/* Device workspace bytes ret_backward needs (it depends on desc->rotate:
+ * the turned copies of Q and K); 0 for descriptions it would reject by their
+ * arguments and for empty problems.  Never fails. */
 size_t ret_backward_workspace_size(const ret_desc *desc, int chunk);
 
 /*

@@ -316,7 +316,7 @@ __device__ __forceinline__ void store_row32(Pair pair, int m, int col0, Dst dst,
     }
 }
 
-template <int DK, typename TO, bool FUSE>
+template <int DK, typename TO, bool FUSE, bool REV>
 __global__ void __launch_bounds__(kThreads, 1)
 chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p,
@@ -339,7 +339,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int nr = (int)gridDim.x;  // CTAs of this head (the cluster when FUSE)
     // the block of rows handled at step c: in order, or last to first for
     // the anti-causal form (the mask and the weights mirror within a block)
-    const bool rev = p.reverse != 0;
+    constexpr bool rev = REV;
     auto blk = [&](int c) { return rev ? nchunks - 1 - c : c; };
 
     if (sbase & 1023u) {  // swizzle atoms need 1024-byte alignment (same for every CTA)
@@ -569,7 +569,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const bool last = c + 1 == nchunks;
-            const int n_next = last ? 0 : min(kC, L - blk(c + 1) * kC);
+            const int n_next = last ? 0 : min(kC, L - (rev ? blk(c + 1) : c + 1) * kC);
             if (!wait_all(SSD, par)) break;
             tc_fence_after();
             // P = bf16(S) on keys j' <= j (j' >= j anti-causal), else 0: keys
@@ -586,7 +586,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     uint32_t a[32];
                     tmem_ld32(tS + lane_base + 32 * cb, a);
                     tmem_wait_ld(a);
-                    if (cb != quad) {
+                    if (rev ? cb > quad : cb < quad) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
@@ -720,7 +720,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // and the next chunk's G into L2 (a row segment of 64 columns
                 // is one 128-byte line), so that its loads do not wait on HBM
                 if (m4 == 0 && ocols && c + 1 < nchunks) {
-                    const int t1 = blk(c + 1) * kC, n1 = min(kC, L - t1);
+                    const int t1 = rev ? blk(c + 1) * kC : t0 + kC, n1 = min(kC, L - t1);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         if (grow(i) < n1) prefetch_l2(Gb + (size_t)(t1 + grow(i)) * g_row);
@@ -814,12 +814,12 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 }
 
-template <int DK, typename TO, bool FUSE>
+template <int DK, typename TO, bool FUSE, bool REV = false>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                      const void *G, RowLayout g, void *Y, float eps, int zeta_v,
                      int v_head_major, int *status, cudaStream_t st) {
-    auto kern = chunkwise_ws_kernel<DK, TO, FUSE>;
+    auto kern = chunkwise_ws_kernel<DK, TO, FUSE, REV>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -848,6 +848,14 @@ cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, con
                       const void *G, RowLayout g, void *Y, float eps, int zeta_v, int vhm,
                       int *status, cudaStream_t st) {
     const bool fuse = Y != nullptr;
+    if (p.reverse) {
+        // the anti-causal products of the backward pass: fp32 O, no gate
+        if constexpr (DK >= 128) {
+            if (!out_bf16 && !fuse)
+                return launch_t<DK, float, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
+        }
+        return cudaErrorInvalidValue;
+    }
     if (out_bf16)
         return fuse ? launch_t<DK, __nv_bfloat16, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st)
                     : launch_t<DK, __nv_bfloat16, false>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
