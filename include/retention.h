@@ -383,8 +383,8 @@ ret_status ret_state_scan(const ret_desc *desc, int n_seg, const int *seg_len,
  * device: every sequence is cut into `segments` equal segments of L /
  * segments rows, which run at once (the chunkwise recurrence of section
  * 2.1, form (3), holds between segments as between chunks).  Each segment's
- * own state comes from a streaming pass and one batched GEMM (as in
- * ret_segment_state), a scan gives every segment its entering state, and
+ * own state comes from the streaming pass's keys and a tensor-core
+ * reduction over its rows, a scan gives every segment its entering state, and
  * one launch of the tensor-core chunk loop computes all segments, each from
  * its state: S times the CTAs of the plain loop, for B*H*d_v/128 well below
  * the number of SMs.  Same result as ret_chunkwise up to rounding.
