@@ -135,8 +135,10 @@ size_t ret_parallel_workspace_size(const ret_desc *desc);
  *             the rows itself (d_k and d_v from 128 and chunks of 128*m
  *             only: for the other shapes of the path ret_workspace_size
  *             asks for the prep size when rotating) or, without rotation,
- *             weights the value rows itself.  Results agree either way up
- *             to rounding.
+ *             weights the value rows itself.  With at least
+ *             ret_chunkwise_fast_size() bytes a call on few heads cuts
+ *             every sequence into segments that run at once (see there).
+ *             Results agree either way up to rounding.
  * At least one of O and Y must be requested.
  * Errors: those of ret_parallel, plus RET_ERR_WORKSPACE.
  */
@@ -181,6 +183,17 @@ ret_status ret_chunkwise_gate_static(const ret_desc *desc, int chunk, const void
  * for descriptions that ret_chunkwise would reject). */
 size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O,
                           int want_Y);
+
+/* Bytes of OPTIONAL workspace with which ret_chunkwise takes its fastest
+ * path for this description and chunk: on the tensor-core path the room of
+ * ret_chunkwise_prep_size, or, when B*H*ceil(d_v/128) is below 64 (most
+ * SMs would idle) and L splits into 2 to 16 equal segments of at least 512
+ * rows, the room of ret_chunkwise_segmented_workspace_size for the number
+ * of segments that keeps one CTA per SM: ret_chunkwise then cuts every
+ * sequence into segments that run at once, with the gate when G and Y are
+ * given (same result up to rounding).  0 when the tensor-core path does not
+ * apply; never fails.  No counterpart in the paper. */
+size_t ret_chunkwise_fast_size(const ret_desc *desc, int chunk);
 
 /* Bytes of OPTIONAL workspace that let ret_chunkwise prepare its operands
  * ahead of the chunk loop (see ret_chunkwise): 2*B*H*L*d_k bf16 values

@@ -151,6 +151,15 @@ size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_
     return 0;
 }
 
+size_t ret_chunkwise_fast_size(const ret_desc *desc, int chunk) {
+    if (check_desc(desc) != RET_OK || chunk < 1 || (long long)desc->B * desc->L == 0) return 0;
+    Params p;
+    make_params(desc, &p);
+    if (!chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16)) return 0;
+    const int S = auto_segments(p, chunk);
+    return S > 1 ? segmented_bytes(p, S) : chunkwise_prep_bytes(p);
+}
+
 size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk) {
     if (check_desc(desc) != RET_OK || chunk < 1) return 0;
     Params p;
@@ -245,6 +254,12 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     if (chunkwise_tc_supported(p, chunk, in_bf16)) {
         int *status = device_status_word();
         if (!status) return RET_ERR_CUDA;
+        // few (b, h) heads and room for the segment states: every sequence
+        // cut into segments that run at once
+        const int S = auto_segments(p, chunk);
+        if (S > 1 && workspace && workspace_bytes >= segmented_bytes(p, S))
+            return from_cuda(launch_segmented(p, S, out_bf16, Q, K, V, state_in, state_out, O, G,
+                                              Y, gn_eps, workspace, status, st));
         // a workspace of ret_chunkwise_prep_size bytes holds the prepared rows
         void *prep = workspace && workspace_bytes >= chunkwise_prep_bytes(p) ? workspace : nullptr;
         return from_cuda(launch_chunkwise_tc(p, out_bf16, Q, K, V, state_in, state_out, O, G, Y,

@@ -949,7 +949,9 @@ cudaError_t launch_tc_rows(const Params &p, bool out_bf16, const void *Q, const 
                            void *Y, float eps, int pre, int *status, cudaStream_t st) {
     if (pre || !p.rotate) {
         const RowLayout hm = bhld_layout(p, p.dk), vl = bhld_layout(p, p.dv);
-        const RowLayout gl{(long long)p.H * p.dv, 0, (long long)p.L * p.H * p.dv};
+        // G [B][L][H d_v] of the real heads (segment heads: H = real heads x
+        // seg_heads, L = rows of one segment; the batch stride is the same)
+        const RowLayout gl{(long long)(p.H / p.seg_heads) * p.dv, 0, (long long)p.L * p.H * p.dv};
         return launch_chunkwise_ws(p, out_bf16, Q, hm, K, V, vl, true, s_in, s_out, O, G, gl, Y,
                                    eps, !pre, status, st);
     }

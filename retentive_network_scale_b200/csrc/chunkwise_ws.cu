@@ -639,10 +639,15 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int j4 = lane >> 2, m4 = lane & 3;  // groups of 4 lanes
         const int o0 = gwg * 64;
         const bool ocols = o0 < dvr;  // this thread's 64 columns exist (d_v = 64: group 0 only)
-        const size_t ycol = (size_t)h * dv + v0 + o0;  // column of Y / G of this thread's segment
+        // A segment head (p.seg_heads = S > 1: head h is segment h mod S of
+        // head h / S, rows at (h mod S) * L of that head's sequence of S * L
+        // rows) reads G and writes Y of its own rows of the real head.
+        const int S = p.seg_heads, hr = h / S, sg = h - hr * S;
+        const size_t ycol = (size_t)hr * dv + v0 + o0;  // column of Y / G of this thread's segment
+        const size_t ypitch = (size_t)(p.H / S) * dv, yrow0 = (size_t)b * S * L + (size_t)sg * L;
         // rows of this lane group's 16-byte row pieces: 32 quad + 4 j4 + i
         auto grow = [&](int i) { return 32 * quad + 4 * j4 + i; };
-        const __nv_bfloat16 *Gb = G + (size_t)b * g_batch + ycol;
+        const __nv_bfloat16 *Gb = G + (size_t)b * g_batch + (size_t)sg * L * g_row + ycol;
         // With the gate, each chunk goes: G(c) loads issued; O''(c) copied
         // out of tensor memory (which is then released at once to the next
         // chunk's product); its row statistics published to the cluster;
@@ -697,7 +702,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         return f2_mul(f2_fma(bf16x2_to_f2(rp[16 * hf + k]), SC, OFF), bf16x2_to_f2(sw[16 * hf + k]));
                     },
                     m4, 32 * hf,
-                    [&](int i) { return Y + ((size_t)b * L + t0_p + grow(i)) * ((size_t)p.H * dv) + ycol; },
+                    [&](int i) { return Y + (yrow0 + t0_p + grow(i)) * ypitch + ycol; },
                     [&](int i) { return ocols && grow(i) < n_p; });
         };
 #pragma unroll 1

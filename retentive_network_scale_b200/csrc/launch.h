@@ -124,8 +124,8 @@ std::mutex &blas_mutex();
 cublasHandle_t blas_handle(cudaStream_t st, void *workspace);
 
 // U = sum_t gamma^{L-1-t} k^_t^T v_t per (b, h) ([d_k][d_v] fp32) on the
-// tensor cores (segstate.cu): K~ [B][H][L][d_k], V [B][H][L][d_v], d_k 128
-// or 256, d_v a multiple of 128.  zeta_v 0: the weight is on K~ already
+// tensor cores (segstate.cu): K~ [B][H][L][d_k], V [B][H][L][d_v], d_k 64,
+// 128 or 256, d_v 64 or a multiple of 128.  zeta_v 0: the weight is on K~ already
 // (the streaming pass with the segment as one block); 1: K~ = K^ and the
 // kernel weights the value rows; 2: K~ carries the weights of 128-row
 // blocks (the chunk loop's streaming pass) and the kernel scales each
@@ -133,6 +133,21 @@ cublasHandle_t blas_handle(cudaStream_t st, void *workspace);
 bool segment_state_tc_supported(const Params &p);
 cudaError_t launch_segment_state_tc(const Params &p, const void *V, const void *Kt, int zeta_v,
                                     float *U, int *status, cudaStream_t st);
+
+// The chunkwise form with every sequence cut into S equal segments that run
+// at once (seqshard.cu): streaming pass, segment states, scan of the
+// entering states, one chunk-loop launch over the B*H*S segment heads (with
+// the gate when G and Y are given), the final state copied out.  The
+// workspace holds segmented_bytes(p, S), the streaming pass's rows first.
+// auto_segments gives the S that ret_chunkwise uses when the plain loop
+// would leave most SMs idle (1: none).
+bool segmented_supported(const Params &p, int chunk, int S);
+size_t segmented_bytes(const Params &p, int S);
+int auto_segments(const Params &p, int chunk);
+cudaError_t launch_segmented(const Params &p, int S, bool out_bf16, const void *Q, const void *K,
+                             const void *V, const float *state_in, float *state_out, void *O,
+                             const void *G, void *Y, float eps, void *workspace, int *status,
+                             cudaStream_t st);
 
 // Tensor-core parallel form: bf16 inputs, d_k 64, 128 or 256, d_v 64 or a
 // multiple of 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned

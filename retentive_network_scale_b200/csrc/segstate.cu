@@ -15,7 +15,8 @@
 //     streaming pass of the chunk loop, K~_t = gamma^{m-1-j} k^_t for row j
 //     of a block of m rows, and the value rows of block b scaled by
 //     gamma^{n - 128 b - m}, which makes up the rest of gamma^{n-1-t}.  One CTA
-// owns one (b, h) and 128 value columns and accumulates U^T = V^T K~ in
+// owns one (b, h) and 128 value columns (d_v = 64: the 64, the rest of its
+// V tile held at zero; d_k 64, 128 or 256) and accumulates U^T = V^T K~ in
 // tensor memory over blocks of 128 rows, which TMA brings through a ring
 // of stages; its one MMA thread also reissues each stage's loads once the
 // product that read it has completed.  The eight warps then move U^T out
@@ -43,7 +44,7 @@ constexpr long long kTimeoutCycles = 4000000000LL;
 
 template <int DK>
 struct SLayout {
-    static constexpr int kStages = DK == 256 ? 2 : 3;
+    static constexpr int kStages = DK == 256 ? 2 : DK == 128 ? 3 : 4;
     static constexpr uint32_t kVBytes = kRows * kTV * 2;  // 2 blocks of 64 columns
     static constexpr uint32_t kKBytes = kRows * DK * 2;   // DK/64 blocks of 64 columns
     static constexpr uint32_t kStage = kVBytes + kKBytes;
@@ -66,6 +67,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
     const int tid = threadIdx.x, warp = tid >> 5;
     const int bh = blockIdx.y, v0 = blockIdx.x * kTV;
     const int L = p.L, dv = p.dv;
+    const int dvr = min(kTV, dv - v0);  // value columns of this CTA: 128, or 64 when d_v = 64
     const float lg = p.log2g[bh % p.H];
     const int nblk = (L + kRows - 1) / kRows;
     if (sbase & 1023u) {
@@ -88,6 +90,14 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
         tmem_alloc(sbase + Ly::kTmemSlot, DK);
         tmem_relinquish();
     }
+    if (dvr < kTV) {
+        // d_v = 64: the second 64-column block of every stage's V tile is
+        // never loaded and stays zero
+        for (int s = 0; s < NS; ++s)
+            for (int i = tid; i < 16384 / 16; i += kThreads)
+                reinterpret_cast<uint4 *>(smem + s * Ly::kStage + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -96,8 +106,8 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
     if (tid == 0) {
         auto load = [&](int s, int blk) {
             const uint32_t st = sbase + s * Ly::kStage;
-            mbar_expect_tx(full(s), Ly::kStage);
-            for (int nb = 0; nb < 2; ++nb)
+            mbar_expect_tx(full(s), dvr * kRows * 2 + Ly::kKBytes);
+            for (int nb = 0; nb < dvr / 64; ++nb)
                 tma_load_3d(st + nb * 16384, &tmV, full(s), v0 + nb * 64, blk * kRows, bh);
             for (int kb = 0; kb < KB; ++kb)
                 tma_load_3d(st + Ly::kVBytes + kb * 16384, &tmK, full(s), kb * 64, blk * kRows, bh);
@@ -150,6 +160,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
                 const uint64_t Z = f2_make(z, z);
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb)
+                    if (nb * 64 < dvr)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
                         // rows of a phase start at different 16-byte pieces: no bank conflicts
@@ -188,7 +199,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
             tmem_wait_ld(r);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                U[((size_t)bh * DK + d0 + i) * dv + v0 + row] = __uint_as_float(r[i]);
+                if (row < dvr) U[((size_t)bh * DK + d0 + i) * dv + v0 + row] = __uint_as_float(r[i]);
         }
     }
     if (tid == 0 && *abort_flag) {
@@ -210,7 +221,7 @@ cudaError_t launch_dk(const Params &p, const CUtensorMap &mv, const CUtensorMap 
     const int smem = (int)SLayout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(p.dv / kTV, p.B * p.H), kThreads, smem, st>>>(mv, mk, p, zeta_v, U, status);
+    kern<<<dim3((p.dv + kTV - 1) / kTV, p.B * p.H), kThreads, smem, st>>>(mv, mk, p, zeta_v, U, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) note_launches(1);
     return e;
@@ -219,7 +230,8 @@ cudaError_t launch_dk(const Params &p, const CUtensorMap &mv, const CUtensorMap 
 }  // namespace
 
 bool segment_state_tc_supported(const Params &p) {
-    return (p.dk == 128 || p.dk == 256) && p.dv % kTV == 0 && p.dv <= kMaxDv && p.L >= 1 &&
+    return (p.dk == 64 || p.dk == 128 || p.dk == 256) && (p.dv == 64 || p.dv % kTV == 0) &&
+           p.dv <= kMaxDv && p.L >= 1 &&
            (long long)p.B * p.H >= 1 && (long long)p.B * p.H <= 65535;
 }
 
@@ -229,8 +241,9 @@ cudaError_t launch_segment_state_tc(const Params &p, const void *V, const void *
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kRows) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kRows))
         return cudaErrorInvalidValue;
-    return p.dk == 256 ? launch_dk<256>(p, mv, mk, zeta_v, U, status, st)
-                       : launch_dk<128>(p, mv, mk, zeta_v, U, status, st);
+    if (p.dk == 256) return launch_dk<256>(p, mv, mk, zeta_v, U, status, st);
+    if (p.dk == 64) return launch_dk<64>(p, mv, mk, zeta_v, U, status, st);
+    return launch_dk<128>(p, mv, mk, zeta_v, U, status, st);
 }
 
 }  // namespace ret

@@ -82,8 +82,8 @@ bool sm100() {
 bool a16(const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
 // U_bh [d_k][d_v] = K~_bh^T V_bh for every (b, h) of p: on the tensor-core
-// kernel of segstate.cu where it applies (d_k 128 or 256, d_v a multiple of
-// 128); otherwise as one cuBLAS batched GEMM, in column-major terms the
+// kernel of segstate.cu where it applies (d_k 64, 128 or 256, d_v 64 or a
+// multiple of 128); otherwise as one cuBLAS batched GEMM, in column-major terms the
 // (d_v x d_k) product V_cm (d_v x L) * K~_cm^T (L x d_k).
 ret_status segment_gemm(const Params &p, const void *V, const void *kt, float *U,
                         void *blas_ws, cudaStream_t st) {
@@ -163,6 +163,69 @@ SegLayout seg_layout(const Params &p, int S) {
 }
 
 }  // namespace
+
+bool segmented_supported(const Params &p, int chunk, int S) {
+    if (S < 1 || p.L % S != 0 || (long long)p.H * S > RET_MAX_HEADS ||
+        (long long)p.B * p.H * S > 65535)  // one CTA row per segment head
+        return false;
+    return chunkwise_tc_supported(p, chunk, true) && segment_state_tc_supported(p);
+}
+
+size_t segmented_bytes(const Params &p, int S) { return seg_layout(p, S).bytes; }
+
+int auto_segments(const Params &p, int chunk) {
+    // the plain loop's CTAs; segments only when they leave most SMs idle,
+    // as many as keep one wave (148 SMs) and at least four blocks of 128
+    // rows per segment (below that the three extra launches cost more than
+    // the shorter chain saves)
+    const long long ctas = (long long)p.B * p.H * ((p.dv + 127) / 128);
+    if (ctas >= 64) return 1;
+    int S = 1;
+    while (ctas * S * 2 <= 148 && p.L % (S * 2) == 0 && p.L / (S * 2) >= 4 * kChunkBlock &&
+           segmented_supported(p, chunk, S * 2))
+        S *= 2;
+    return S;
+}
+
+cudaError_t launch_segmented(const Params &p, int S, bool out_bf16, const void *Q, const void *K,
+                             const void *V, const float *state_in, float *state_out, void *O,
+                             const void *G, void *Y, float eps, void *workspace, int *status,
+                             cudaStream_t st) {
+    const SegLayout z = seg_layout(p, S);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *U = reinterpret_cast<float *>(ws + z.off_u);
+    float *R = reinterpret_cast<float *>(ws + z.off_r);
+    float *Sout = reinterpret_cast<float *>(ws + z.off_s);
+    const Params q = segment_params(p, S);
+    // 1. the chunk loop's streaming pass: Q^ (with rotation) and K~, the keys
+    //    turned and weighted by gamma^{m-1-j} within each block of m <= 128
+    //    rows of each segment
+    const void *qh = nullptr, *kt = nullptr;
+    cudaError_t e = launch_chunkwise_prep(q, kChunkBlock, Q, K, ws, &qh, &kt, st);
+    if (e != cudaSuccess) return e;
+    // 2. every segment's own state from the same K~, each block's value rows
+    //    scaled by the rest of the segment's weight
+    if ((e = launch_segment_state_tc(q, V, kt, 2, U, status, st)) != cudaSuccess) return e;
+    // 3. the state entering each segment
+    const long long quads = (long long)p.B * p.H * p.dk * p.dv / 4;
+    segment_scan_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(p, S, q.L, quads, U,
+                                                                          state_in, R);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    note_launches(1);
+    // 4. the chunk loop over all segments at once, each from its state (with
+    //    the gate: G and Y of each segment's own rows)
+    if ((e = launch_chunkwise_tc_rows(q, out_bf16, qh, kt, V, R, state_out ? Sout : nullptr, O, G,
+                                      Y, eps, status, st)) != cudaSuccess)
+        return e;
+    // 5. the state after the last segment of each sequence
+    if (state_out) {
+        const size_t per = (size_t)p.dk * p.dv * sizeof(float);
+        e = cudaMemcpy2DAsync(state_out, per, Sout + (size_t)(S - 1) * p.dk * p.dv, per * S, per,
+                              (size_t)p.B * p.H, cudaMemcpyDeviceToDevice, st);
+    }
+    return e;
+}
+
 }  // namespace ret
 
 extern "C" {
@@ -248,13 +311,9 @@ ret_status check_segmented(const ret_desc *desc, int chunk, int segments, ret::P
     if (s != RET_OK) return s;
     if (desc->in_dtype != RET_BF16) return RET_ERR_DTYPE;
     if (chunk < 1 || segments < 1) return RET_ERR_ARG;
-    if ((long long)desc->B * desc->L == 0 || desc->L % segments != 0 ||
-        (long long)desc->H * segments > RET_MAX_HEADS ||
-        (long long)desc->B * desc->H * segments > 65535)  // one CTA row per segment head
-        return RET_ERR_SHAPE;
+    if ((long long)desc->B * desc->L == 0) return RET_ERR_SHAPE;
     params_from_desc(desc, p);
-    if (!chunkwise_tc_supported(*p, chunk, true) || !segment_state_tc_supported(*p))
-        return RET_ERR_SHAPE;
+    if (!segmented_supported(*p, chunk, segments)) return RET_ERR_SHAPE;
     return RET_OK;
 }
 
@@ -284,41 +343,11 @@ ret_status ret_chunkwise_segmented(const ret_desc *desc, int chunk, int segments
     if (!sm100()) return RET_ERR_UNSUPPORTED;
     int *status = device_status_word();
     if (!status) return RET_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    float *U = reinterpret_cast<float *>(ws + z.off_u);
-    float *R = reinterpret_cast<float *>(ws + z.off_r);
-    float *Sout = reinterpret_cast<float *>(ws + z.off_s);
-    const Params q = segment_params(p, segments);
-    // 1. the chunk loop's streaming pass: Q^ (with rotation) and K~, the keys
-    //    turned and weighted by gamma^{m-1-j} within each block of m <= 128
-    //    rows of each segment
-    const void *qh = nullptr, *kt = nullptr;
-    if (launch_chunkwise_prep(q, kChunkBlock, Q, K, ws, &qh, &kt, st) != cudaSuccess)
-        return RET_ERR_CUDA;
-    // 2. every segment's own state from the same K~, each block's value rows
-    //    scaled by the rest of the segment's weight
-    if (launch_segment_state_tc(q, V, kt, 2, U, status, st) != cudaSuccess) return RET_ERR_CUDA;
-    // 3. the state entering each segment
-    const long long quads = (long long)p.B * p.H * p.dk * p.dv / 4;
-    segment_scan_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, st>>>(p, segments, q.L, quads, U,
-                                                                          state_in, R);
-    if (cudaGetLastError() != cudaSuccess) return RET_ERR_CUDA;
-    note_launches(1);
-    // 4. the chunk loop over all segments at once, each from its state
-    if (launch_chunkwise_tc_rows(q, desc->out_dtype == RET_BF16, qh, kt, V, R,
-                                 state_out ? Sout : nullptr, O, nullptr, nullptr, 0.f, status,
-                                 st) != cudaSuccess)
-        return RET_ERR_CUDA;
-    // 5. the state after the last segment of each sequence
-    if (state_out) {
-        const size_t per = (size_t)p.dk * p.dv * sizeof(float);
-        if (cudaMemcpy2DAsync(state_out, per, Sout + (size_t)(segments - 1) * p.dk * p.dv,
-                              per * segments, per, (size_t)p.B * p.H, cudaMemcpyDeviceToDevice,
-                              st) != cudaSuccess)
-            return RET_ERR_CUDA;
-    }
-    return RET_OK;
+    return launch_segmented(p, segments, desc->out_dtype == RET_BF16, Q, K, V, state_in, state_out,
+                            O, nullptr, nullptr, 0.f, workspace, status,
+                            static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? RET_OK
+               : RET_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -29,6 +29,7 @@ STATUS_NAMES = ["RET_OK", "RET_ERR_NULL", "RET_ERR_SHAPE", "RET_ERR_DTYPE", "RET
 # every symbol include/retention.h declares
 EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_gate_static", "ret_workspace_size", "ret_chunkwise_prep_size",
+           "ret_chunkwise_fast_size",
            "ret_chunkwise_prepare", "ret_chunkwise_prepared", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
            "ret_backward", "ret_backward_workspace_size",
@@ -82,6 +83,8 @@ def load_library(path: str = LIB_PATH):
                                               ctypes.c_float, vp, vp]
     lib.ret_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.ret_workspace_size.restype = st
+    lib.ret_chunkwise_fast_size.argtypes = [D, ctypes.c_int]
+    lib.ret_chunkwise_fast_size.restype = st
     lib.ret_chunkwise_prep_size.argtypes = [D, ctypes.c_int]
     lib.ret_chunkwise_prep_size.restype = st
     lib.ret_chunkwise_prepare.argtypes = [D, ctypes.c_int, vp, vp, vp, st, vp]
@@ -217,6 +220,15 @@ def ret_chunkwise_prep_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk
     lib = load_library()
     d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
     return int(lib.ret_chunkwise_prep_size(ctypes.byref(d), int(chunk)))
+
+
+def ret_chunkwise_fast_size(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, chunk, rotate=False,
+                            theta_base=10000.0, pos_offset=0):
+    """Optional workspace bytes with which ret_chunkwise takes its fastest
+    path (the prepared operands; for few heads, the segmented layout)."""
+    lib = load_library()
+    d = make_desc(B, H, L, d_k, d_v, in_dtype, out_dtype, gamma, rotate, theta_base, pos_offset)
+    return int(lib.ret_chunkwise_fast_size(ctypes.byref(d), int(chunk)))
 
 
 def ret_chunkwise_prepare(Q, K, gamma, chunk, workspace, rotate=False, theta_base=10000.0,
@@ -511,7 +523,7 @@ def ret_chunkwise(Q, K, V, gamma, chunk, O=None, state_in=None, state_out=None, 
     need = int(lib.ret_workspace_size(ctypes.byref(d), int(chunk), int(O is not None),
                                       int(Y is not None)))
     if prep:
-        need = max(need, int(lib.ret_chunkwise_prep_size(ctypes.byref(d), int(chunk))))
+        need = max(need, int(lib.ret_chunkwise_fast_size(ctypes.byref(d), int(chunk))))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

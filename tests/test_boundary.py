@@ -292,8 +292,8 @@ def test_chunkwise_segmented_arguments(lib):
     assert call(seg=3) == S("RET_ERR_SHAPE") and size(seg=3) == 0          # L % segments
     assert call(seg=64) == S("RET_ERR_SHAPE")                                # H * segments > 128
     assert call(chunk=96) == S("RET_ERR_SHAPE")                              # not a tensor-core chunk
-    assert call(dd=desc(B=1, H=4, L=1024, d_k=64, d_v=256,
-                        gamma=[0.9] * 4)) == S("RET_ERR_SHAPE")              # no segment states at d_k 64
+    assert call(dd=desc(B=1, H=4, L=1024, d_k=32, d_v=256,
+                        gamma=[0.9] * 4)) == S("RET_ERR_SHAPE")              # not a tensor-core d_k
     assert call(dd=desc(B=1, H=4, L=1024, d_k=128, d_v=256, in_dtype=R.RET_F32,
                         gamma=[0.9] * 4)) == S("RET_ERR_DTYPE")
     assert call(O=None) == S("RET_ERR_NULL")
@@ -319,6 +319,32 @@ def test_static_entry_checks_arguments_before_its_scratch_limit(lib):
     assert call(d, chunk=0) == S("RET_ERR_ARG")
     assert call(desc(gamma=[1.5, 0.9])) == S("RET_ERR_ARG")
     assert call(d) == S("RET_ERR_WORKSPACE")
+
+
+def test_fast_size(lib):
+    """ret_chunkwise_fast_size: the streaming pass's room for shapes with
+    enough heads, the segmented layout (segments keeping one wave of CTAs,
+    at least 512 rows each) for few heads, 0 off the tensor-core path."""
+    bf = R.RET_BF16
+    fast = lambda d, chunk=128: lib.ret_chunkwise_fast_size(ctypes.byref(d), chunk)  # noqa: E731
+    prep = lambda d, chunk=128: lib.ret_chunkwise_prep_size(ctypes.byref(d), chunk)  # noqa: E731
+    seg = lambda d, n, chunk=128: lib.ret_chunkwise_segmented_workspace_size(  # noqa: E731
+        ctypes.byref(d), chunk, n)
+    many = desc(B=8, H=8, L=1024, d_k=256, d_v=512, in_dtype=bf, out_dtype=bf, gamma=[0.9] * 8)
+    assert fast(many) == prep(many) > 0                                  # 256 CTAs: no segments
+    # 2 heads x 1 value tile: 8 segments of 256 rows would be too short, 4 of 512 qualify
+    few = desc(B=1, H=2, L=2048, d_k=128, d_v=128, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
+    assert fast(few) == seg(few, 4) > prep(few) > 0
+    # msr_small's shape: 32 heads of d_v 64, 4 segments of 512 rows (128 CTAs)
+    small = desc(B=4, H=8, L=2048, d_k=64, d_v=64, in_dtype=bf, out_dtype=bf,
+                 gamma=[0.9] * 8, rotate=False)
+    assert fast(small, 64) == seg(small, 4, 64) > 0
+    # rows that do not split into segments of 512: the streaming pass only
+    odd = desc(B=1, H=2, L=1000, d_k=128, d_v=128, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
+    assert fast(odd) == prep(odd) > 0
+    f32 = desc(B=1, H=2, L=2048, d_k=128, d_v=128, in_dtype=R.RET_F32, out_dtype=R.RET_F32,
+               gamma=[0.9, 0.99])
+    assert fast(f32) == 0
 
 
 def test_workspace_size_of_tensor_core_shapes(lib):

@@ -7,6 +7,8 @@ uncut run: outputs, the fused GroupNorm + gate, and the final state; and
 ret_chunkwise_segmented, which runs all segments of a sequence at once.
 
 "Retentive Network" paper summary, section 2.1, chunkwise form (3)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -139,3 +141,48 @@ def test_segmented_matches_oracle(L, S, dk, dv, with_in, rotate):
     for h in range(H):
         assert rel_l2(O[0, h], O_ref[0, h]) <= TOL_BF16, h
         assert rel_l2(St[0, h], S_ref[0, h]) <= TOL_BF16, h
+
+
+@pytest.mark.parametrize("L,dk,dv,rotate,segs", [
+    (2048, 128, 128, True, 4),     # 2 heads x 1 value tile: 4 segments of 512 rows
+    (2048, 64, 64, False, 4),      # msr_small's head shape, without rotation
+    (1536, 256, 256, True, 2),     # 1536 = 3 x 512: two segments of 768 rows
+])
+def test_chunkwise_takes_segments_for_few_heads(L, dk, dv, rotate, segs):
+    """ret_chunkwise with ret_chunkwise_fast_size bytes of workspace on few
+    heads: every sequence cut into segments that run at once, the fused
+    GroupNorm + gate on each segment's own rows, O and the final state from
+    a carried state; against the oracle's uncut run, and against the plain
+    loop (no workspace) up to rounding."""
+    B, H = 1, 2
+    g = [0.96875, 0.999]
+    Q, K, V = _qkv(B, H, L, dk, dv, 150)
+    G = random_tensor((B, L, H * dv), 155).bfloat16()
+    S0 = random_tensor((B, H, dk, dv), 156, 0.1)
+    O_ref, S_ref = orc.recurrent(Q, K, V, g, rotate=rotate, pos_offset=9, state_in=S0)
+    Y_ref = orc.gate_groupnorm(O_ref, G)
+    desc = R.make_desc(B, H, L, dk, dv, R.RET_BF16, R.RET_BF16, g, rotate, 10000.0, 9)
+    lib = R.load_library()
+    assert lib.ret_chunkwise_fast_size(ctypes.byref(desc), 128) == \
+        lib.ret_chunkwise_segmented_workspace_size(ctypes.byref(desc), 128, segs)
+    Qd, Kd, Vd, Gd, S0d = Q.cuda(), K.cuda(), V.cuda(), G.cuda(), S0.cuda()
+    O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
+    Y = torch.empty(B, L, H * dv, device="cuda", dtype=torch.bfloat16)
+    St = torch.empty(B, H, dk, dv, device="cuda")
+    n0 = R.ret_kernel_launches()
+    R.ret_chunkwise(Qd, Kd, Vd, g, 128, O=O, state_in=S0d, state_out=St, G=Gd, Y=Y,
+                    rotate=rotate, pos_offset=9)
+    # the streaming pass, the segment states, the scan, the chunk loop
+    assert R.ret_kernel_launches() - n0 == 4
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    for h in range(H):
+        assert rel_l2(O[0, h], O_ref[0, h]) <= TOL_BF16, h
+        assert rel_l2(Y[0, :, h * dv:(h + 1) * dv], Y_ref[0, :, h * dv:(h + 1) * dv]) <= TOL_BF16, h
+        assert rel_l2(St[0, h], S_ref[0, h]) <= TOL_BF16, h
+    # the plain loop on the same call, without the workspace
+    O2, Y2, S2 = torch.empty_like(O), torch.empty_like(Y), torch.empty_like(St)
+    R.ret_chunkwise(Qd, Kd, Vd, g, 128, O=O2, state_in=S0d, state_out=S2, G=Gd, Y=Y2,
+                    rotate=rotate, pos_offset=9, prep=False)
+    torch.cuda.synchronize()
+    assert rel_l2(O2, O) <= TOL_BF16 and rel_l2(Y2, Y) <= TOL_BF16 and rel_l2(S2, St) <= TOL_BF16
