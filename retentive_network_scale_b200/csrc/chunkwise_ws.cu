@@ -6,20 +6,22 @@
 // the chunk of n rows after state R, with xPos-rotated rows q^_j, k^_j:
 //   o_j = sum_{j'<=j} gamma^{j-j'} (q^_j.k^_j') v_j' + gamma^{j+1} q^_j R
 //   R  <- gamma^n R + sum_j' gamma^{n-1-j'} k^_j'^T v_j'
-// As in chunkwise_tc.cu the tensor cores see plain products only:
+// The tensor cores see plain products only:
 //   Rbar = bf16(gamma^n R),  O'' = Q^ Rbar + mask(Q^ K'^T) V',
 //   o_j = gamma^{j+1-n} O''_j,  R <- gamma^n R + K'^T V'
 // where the row weight zeta_j = gamma^{n-1-j} sits either on the key rows
-// (K' = diag(zeta) K^, V' = V: rows prepared by the streaming pass) or on
-// the value rows (K' = K^, V' = diag(zeta) V, applied here in shared memory;
+// (K' = diag(zeta) K^, V' = V: rows prepared by the streaming pass, or
+// turned and weighted here in shared memory as their tiles land) or on the
+// value rows (K' = K^, V' = diag(zeta) V, applied here in shared memory;
 // this needs no pass over Q and K at all when there is no rotation).  Both
-// give gamma^{j+1-n} gamma^{n-1-j'} = gamma^{j-j'} term by term.
+// give gamma^{j+1-n} gamma^{n-1-j'} = gamma^{j-j'} term by term.  All
+// factors stay in range while gamma^128 >= 2^-60.
 //
 // One CTA owns one (b, h) and 128 value columns (d_v = 64: one CTA with 64,
 // the rest of its V tile zero); the CTAs of a head form a cluster.  d_k is
-// 64, 128 or 256.  Unlike chunkwise_tc.cu, no role waits for a whole chunk
-// to finish: every hand-over is an mbarrier, so the epilogue of chunk c runs
-// while the tensor cores work on chunk c+1.  Roles (16 warps):
+// 64, 128 or 256.  No role waits for a whole chunk to finish: every
+// hand-over is an mbarrier, so the epilogue of chunk c runs while the
+// tensor cores work on chunk c+1.  Roles (16 warps):
 //   warp 0      issues the MMAs (one thread), chunk by chunk:
 //               S = Q^ K'^T -> O'' = Q^ Rbar -> R^T += V'^T K' -> O'' += P V'
 //   warp 1      issues the TMA loads of Q^, K', V as each buffer is released
@@ -32,7 +34,9 @@
 //               epilogue's global loads and stores in flight)
 //   warps 4-7   P = bf16(mask(S)) into tensor memory; then the state pass
 //               (R^T <- gamma^{n'} R^T in TMEM and its bf16 copy Rbar^T in
-//               shared memory for the next chunk, or state_out after the last)
+//               shared memory for the next chunk, or state_out after the last);
+//               with the rotation in the loop, then the xPos turn (and key
+//               weights) of the next chunk's Q and K tiles
 //   warps 8-15  the epilogue: O'' leaves tensor memory for registers at once
 //               (the next chunk's O'' may then start), row statistics merged
 //               across the cluster through distributed shared memory and
@@ -81,7 +85,8 @@ constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
 // Rbar^T and the decayed R^T ready); OF: O'' copied out by the epilogue;
 // SL: this CTA's GroupNorm partials written; GX0/GX1: the partials of every
 // CTA of the head published (by chunk parity).
-enum { QF = 0, KF, VF, VR, SSD, SOD, UD, PVD, PR, RBL, RB, OF, SL, GX0, GX1, kNumBars };
+// QR/KR: Q^ / K~ turned in shared memory (rotation in the loop only).
+enum { QF = 0, KF, VF, VR, SSD, SOD, UD, PVD, PR, RBL, RB, OF, SL, GX0, GX1, QR, KR, kNumBars };
 
 template <int DK>
 struct Layout {
@@ -97,9 +102,9 @@ struct Layout {
     static constexpr uint32_t kAbort = kTmemSlot + 4;
     // per row (mean, centred sum of squares) of this CTA's 128 columns, by
     // chunk parity; the peers read it remotely
-    static constexpr uint32_t kSlot = kSmall + 128;
+    static constexpr uint32_t kSlot = kSmall + 256;
     static constexpr uint32_t kBytes = kSlot + 2 * 128 * 8;
-    static_assert(8 * kNumBars + 8 <= 128, "small area");
+    static_assert(8 * kNumBars + 8 <= 256, "small area");
     static __device__ __forceinline__ uint32_t k_blk(int kb) { return kKR + kb * 32768; }
     static __device__ __forceinline__ uint32_t rbar_blk(int kb) { return kKR + kb * 32768 + 16384; }
 };
@@ -190,6 +195,76 @@ __device__ __forceinline__ void st_rbarT_row(uint8_t *smem, int c, int d0, const
         w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
         w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
         *reinterpret_cast<uint4 *>(blk + (((ch0 + q) ^ (c & 7)) << 4)) = w;
+    }
+}
+
+// The xPos turn of one landed 128-row tile in shared memory (128-byte
+// swizzle, d_k/64 blocks of 64 columns `blk_stride` bytes apart): row r
+// (position pos0 + r) has each pair (x_2j, x_2j+1) turned by
+// (pos0 + r) theta_j and, for keys, scaled by zeta_r = gamma^{n-1-r}, the
+// weight of the state update.  `nthr` threads, this one `ti`: a thread
+// takes one 16-byte column chunk (4 pairs) and the rows r0, r0+RS, ...,
+// two rows at a time in the lanes of packed fp32 pairs.  The angles start
+// from an fp64 reduction and advance by 2 RS theta_j per step.  Rows at or
+// past n are zeros from the load and stay as they are.
+template <int DK>
+__device__ __forceinline__ void turn_tile(uint8_t *smem, uint32_t blk0, uint32_t blk_stride,
+                                          const Params &p, long long pos0, int n, bool keys,
+                                          float lg, int ti, int nthr) {
+    constexpr int NCH = DK / 8;  // 16-byte chunks per row
+    const int RS = nthr / NCH;
+    const int c16 = ti % NCH, r0 = ti / NCH;
+    uint8_t *base = smem + blk0 + (c16 >> 3) * blk_stride;
+    const int cw = c16 & 7;
+    uint64_t C[4], NS[4], c2[4], s2[4], ns2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const double th = p.theta[c16 * 4 + e];
+        float ca, sa, cb, sb, cs, ss;
+        rot_cs_fast(pos0 + r0, th, &ca, &sa);
+        rot_cs_fast(pos0 + r0 + RS, th, &cb, &sb);
+        rot_cs_fast(2 * RS, th, &cs, &ss);
+        C[e] = f2_make(ca, cb);
+        NS[e] = f2_make(-sa, -sb);
+        c2[e] = f2_make(cs, cs);
+        s2[e] = f2_make(ss, ss);
+        ns2[e] = f2_make(-ss, -ss);
+    }
+    auto turn_pair = [&](uint4 &wa, uint4 &wb, int ra, int rb) {
+        const float za = keys ? (ra < n ? decay_pow(lg, n - 1 - ra) : 0.f) : 1.f;
+        const float zb = keys ? (rb < n ? decay_pow(lg, n - 1 - rb) : 0.f) : 1.f;
+        const uint64_t Z = f2_make(za, zb);
+        uint32_t *ua = reinterpret_cast<uint32_t *>(&wa);
+        uint32_t *ub = reinterpret_cast<uint32_t *>(&wb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            // x0 = low bf16, x1 = high bf16 of each row's pair
+            const uint64_t X0 = (static_cast<uint64_t>(ub[e] << 16) << 32) | (ua[e] << 16);
+            const uint64_t X1 = (static_cast<uint64_t>(ub[e] & 0xffff0000u) << 32) | (ua[e] & 0xffff0000u);
+            const uint64_t NX0 = X0 ^ 0x8000000080000000ull;
+            const uint64_t ZC = keys ? f2_mul(C[e], Z) : C[e];
+            const uint64_t ZNS = keys ? f2_mul(NS[e], Z) : NS[e];
+            const uint64_t Y0 = f2_fma(X1, ZNS, f2_mul(X0, ZC));   // x0 c - x1 s
+            const uint64_t Y1 = f2_fma(X1, ZC, f2_mul(NX0, ZNS));  // x0 s + x1 c
+            ua[e] = pack_bf16(f2_lo(Y0), f2_lo(Y1));
+            ub[e] = pack_bf16(f2_hi(Y0), f2_hi(Y1));
+            const uint64_t Cn = f2_fma(C[e], c2[e], f2_mul(NS[e], s2[e]));
+            NS[e] = f2_fma(NS[e], c2[e], f2_mul(C[e], ns2[e]));
+            C[e] = Cn;
+        }
+    };
+    auto at = [&](int r) { return reinterpret_cast<uint4 *>(base + r * 128 + ((cw ^ (r & 7)) << 4)); };
+    // rows r0 + RS k, four per step (the two rows of a packed pair RS apart)
+#pragma unroll 1
+    for (int ra = r0; ra < n; ra += 4 * RS) {
+        const int rb = ra + RS, rc = ra + 2 * RS, rd = ra + 3 * RS;
+        uint4 wa = *at(ra), wb = *at(rb), wc = *at(rc), wd = *at(rd);
+        turn_pair(wa, wb, ra, rb);
+        turn_pair(wc, wd, rc, rd);
+        *at(ra) = wa;
+        *at(rb) = wb;
+        *at(rc) = wc;
+        *at(rd) = wd;
     }
 }
 
@@ -316,7 +391,7 @@ __device__ __forceinline__ void store_row32(Pair pair, int m, int col0, Dst dst,
     }
 }
 
-template <int DK, typename TO, bool FUSE, bool REV>
+template <int DK, typename TO, bool FUSE, bool REV, bool ROT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p,
@@ -357,7 +432,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             uint32_t count = 1;
             // one arrival per warp of the role (lane 0, after the warp has met)
             if (i == VR) count = 1;
-            if (i == PR || i == RBL || i == RB) count = 4;
+            if (i == PR || i == RBL || i == RB || i == QR || i == KR) count = 4;
             if (i == OF) count = 8;
             if (i == GX0 || i == GX1) count = nr;
             mbar_init(bar(i), count);
@@ -414,7 +489,9 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1, prv = par ^ 1;
             // S: the tiles of chunk c, and P of chunk c-1 consumed
-            if (!(wait_all(QF, par) && wait_all(KF, par) && (c == 0 || wait_all(PVD, prv)))) break;
+            if (!(wait_all(ROT ? QR : QF, par) && wait_all(ROT ? KR : KF, par) &&
+                  (c == 0 || wait_all(PVD, prv))))
+                break;
             tc_fence_after();
             if (lane == 0) {
 #pragma unroll
@@ -565,8 +642,27 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             warp_arrive(RBL);
             warp_arrive(RB);
         }
+        // With the rotation in the loop: Q^ and K~ of step c turned in shared
+        // memory once their tiles land (the products wait on QR / KR)
+        auto turn = [&](int c) {
+            if constexpr (ROT) {
+                const uint32_t par = c & 1;
+                const int t0 = blk(c) * kC, n = min(kC, L - t0);
+                const long long pos0 = p.pos_offset + t0;
+                if (!wait_all(QF, par)) return false;
+                turn_tile<DK>(smem, Ly::kQ, 16384, p, pos0, n, false, lg, tid - 128, 128);
+                fence_proxy_async_smem();
+                warp_arrive(QR);
+                if (!wait_all(KF, par)) return false;
+                turn_tile<DK>(smem, Ly::kKR, 32768, p, pos0, n, true, lg, tid - 128, 128);
+                fence_proxy_async_smem();
+                warp_arrive(KR);
+            }
+            return true;
+        };
+        bool turned = turn(0);
 #pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < nchunks && turned; ++c) {
             const uint32_t par = c & 1;
             const bool last = c + 1 == nchunks;
             const int n_next = last ? 0 : min(kC, L - (rev ? blk(c + 1) : c + 1) * kC);
@@ -629,6 +725,7 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             if constexpr (DK < 128) warp_arrive(RBL);
             warp_arrive(RB);
+            if (!last && !(turned = turn(c + 1))) break;
         }
     } else {
         // ============================================ epilogue (warps 8-15)
@@ -819,12 +916,12 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 }
 
-template <int DK, typename TO, bool FUSE, bool REV = false>
+template <int DK, typename TO, bool FUSE, bool REV = false, bool ROT = false>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                      const void *G, RowLayout g, void *Y, float eps, int zeta_v,
                      int v_head_major, int *status, cudaStream_t st) {
-    auto kern = chunkwise_ws_kernel<DK, TO, FUSE, REV>;
+    auto kern = chunkwise_ws_kernel<DK, TO, FUSE, REV, ROT>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -850,14 +947,25 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
 template <int DK>
 cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, const CUtensorMap &mk,
                       const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
-                      const void *G, RowLayout g, void *Y, float eps, int zeta_v, int vhm,
+                      const void *G, RowLayout g, void *Y, float eps, int zeta_v, int vhm, bool rot,
                       int *status, cudaStream_t st) {
     const bool fuse = Y != nullptr;
     if (p.reverse) {
         // the anti-causal products of the backward pass: fp32 O, no gate
         if constexpr (DK >= 128) {
-            if (!out_bf16 && !fuse)
+            if (!out_bf16 && !fuse && !rot)
                 return launch_t<DK, float, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
+        }
+        return cudaErrorInvalidValue;
+    }
+    if (rot) {
+        // xPos turn of the landed tiles inside the loop (d_k 128 and 256)
+        if constexpr (DK >= 128) {
+            if (out_bf16)
+                return fuse ? launch_t<DK, __nv_bfloat16, true, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st)
+                            : launch_t<DK, __nv_bfloat16, false, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
+            return fuse ? launch_t<DK, float, true, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st)
+                        : launch_t<DK, float, false, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
         }
         return cudaErrorInvalidValue;
     }
@@ -874,7 +982,8 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
                                 const void *K, const void *V, RowLayout v_layout,
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
-                                bool zeta_on_v, int *status, cudaStream_t st) {
+                                bool zeta_on_v, bool rotate_in_loop, int *status,
+                                cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16_strided(&mq, Q, p.dk, p.L, bh, q_layout.row, q_layout.head, kC) ||
@@ -887,10 +996,10 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
     if (!ok) return cudaErrorInvalidValue;
     const int zv = zeta_on_v ? 1 : 0, vhm = v_head_major ? 1 : 0;
     if (p.dk == 256)
-        return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
+        return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
     if (p.dk == 64)
-        return launch_dk<64>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, status, st);
+        return launch_dk<64>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
 }
 
 }  // namespace ret

@@ -94,13 +94,16 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
 // v_head_major, else rows of H*d_v columns), G through `g_layout` (rows of
 // H*d_v columns).  zeta_on_v: K' is K^ itself and the kernel weights the
 // value rows by gamma^{n-1-j}; otherwise K' already carries that weight
-// (the streaming pass).  Writes Y ([B][L][H*d_v], with G) and/or O
-// ([B][H][L][d_v]) in the output dtype.
+// (the streaming pass).  rotate_in_loop: Q and K are the raw rows and the
+// kernel turns the landed tiles (and weights the keys) in shared memory
+// itself (d_k 128 or 256, plain heads).  Writes Y ([B][L][H*d_v], with G)
+// and/or O ([B][H][L][d_v]) in the output dtype.
 cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, RowLayout q_layout,
                                 const void *K, const void *V, RowLayout v_layout,
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
-                                bool zeta_on_v, int *status, cudaStream_t st);
+                                bool zeta_on_v, bool rotate_in_loop, int *status,
+                                cudaStream_t st);
 
 // The streaming pass reading Q and K through a layout; with always_q it
 // writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),

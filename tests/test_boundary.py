@@ -349,14 +349,15 @@ def test_fast_size(lib):
 
 def test_workspace_size_of_tensor_core_shapes(lib):
     """The tensor-core path needs no workspace, except for rotated shapes
-    that only the prepared-rows loop serves (d_k 64, d_v 64, chunks of 64
-    rows): there ret_workspace_size asks for the streaming pass's room."""
+    of d_k 64, which only the prepared-rows loop serves (the loop turns
+    tiles of d_k 128 and 256 itself): there ret_workspace_size asks for the
+    streaming pass's room."""
     bf = R.RET_BF16
     ws = lambda d, chunk=128, o=0, y=1: lib.ret_workspace_size(ctypes.byref(d), chunk, o, y)  # noqa: E731
     prep = lambda d, chunk=128: lib.ret_chunkwise_prep_size(ctypes.byref(d), chunk)  # noqa: E731
     big = dict(B=1, H=2, L=300, d_k=256, d_v=512, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
     assert ws(desc(**big)) == 0 and ws(desc(**big), chunk=256) == 0
-    assert ws(desc(**big), chunk=64) == prep(desc(**big), chunk=64) > 0
+    assert ws(desc(**big), chunk=64) == 0 and prep(desc(**big), chunk=64) > 0
     small = {**big, "d_k": 64, "d_v": 64}
     assert ws(desc(**small), chunk=64) == prep(desc(**small), chunk=64) > 0
     assert ws(desc(**small), chunk=64, o=1, y=0) == prep(desc(**small), chunk=64)
