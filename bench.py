@@ -566,7 +566,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
-    if args.only in ("decode", "parallel", "long_ctx", "msr_small"):
+    if args.only in ("decode", "parallel", "long_ctx", "msr_small", "backward"):
         if args.only == "decode":
             out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
         elif args.only == "long_ctx":
@@ -578,7 +578,10 @@ def run_ours(args, world, rank, local):
             if args.batch:
                 w = dataclasses.replace(w, B=args.batch)
             d = {k: v.cuda() for k, v in make_inputs(w).items()}
-            out = bench_parallel(R, w, d, pk, reps=max(1, args.steps))
+            if args.only == "backward":
+                out = bench_backward(R, w, d, pk, reps=max(1, args.steps))
+            else:
+                out = bench_parallel(R, w, d, pk, reps=max(1, args.steps))
         if rank == 0:
             print(json.dumps({"only": args.only, **out}), flush=True)
         return
@@ -739,7 +742,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
-    ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx", "msr_small"],
+    ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx", "msr_small",
+                                       "backward"],
                     default=None,
                     help="run one measurement alone (profiler captures)")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -340,7 +340,10 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
     float *partA = reinterpret_cast<float *>(ws + z.part_dk);
     const size_t part_stride = round_up(rows * dk * 4) / 4;      // floats between partials
     float *partB = partA + part_stride * z.nsplit;
-    float *partC = reinterpret_cast<float *>(ws + z.part_dv);
+    // dV needs neither a second partial nor a turn: in fp32 the product
+    // writes it in place
+    const bool dv_direct = desc->out_dtype == RET_F32;
+    float *partC = dv_direct ? static_cast<float *>(dV) : reinterpret_cast<float *>(ws + z.part_dv);
 
     cudaError_t e = cudaSuccess;
     auto run = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
@@ -374,7 +377,7 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
     } else {
         run(unturn_sum<float>(p, dk, partA, a1, false, rot, dQ, st));
         run(unturn_sum<float>(p, dk, partB, b1, false, rot, dK, st));
-        run(unturn_sum<float>(p, dv, partC, nullptr, false, false, dV, st));
+        if (!dv_direct) run(unturn_sum<float>(p, dv, partC, nullptr, false, false, dV, st));
     }
     return e == cudaSuccess ? RET_OK : RET_ERR_CUDA;
 }

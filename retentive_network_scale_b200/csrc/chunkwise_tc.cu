@@ -70,7 +70,7 @@ cudaError_t launch_tc_rows(const Params &p, bool out_bf16, const void *Q, const 
     // G [B][L][H d_v] of the real heads (segment heads: H = real heads x
     // seg_heads, L = rows of one segment; the batch stride is the same)
     const RowLayout gl{(long long)(p.H / p.seg_heads) * p.dv, 0, (long long)p.L * p.H * p.dv};
-    return launch_chunkwise_ws(p, out_bf16, Q, hm, K, V, vl, true, s_in, s_out, O, G, gl, Y, eps,
+    return launch_chunkwise_ws(p, out_bf16, Q, hm, K, hm, V, vl, true, s_in, s_out, O, G, gl, Y, eps,
                                !pre && !rot, rot, status, st);
 }
 
@@ -202,7 +202,7 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
                                          RowLayout v_layout, bool v_head_major, const void *G,
                                          RowLayout g_layout, void *Y, void *O, float eps,
                                          int *status, cudaStream_t st) {
-    return launch_chunkwise_ws(p, out_bf16, Qh, q_layout, Kt, V, v_layout, v_head_major, nullptr,
+    return launch_chunkwise_ws(p, out_bf16, Qh, q_layout, Kt, bhld_layout(p, p.dk), V, v_layout, v_head_major, nullptr,
                                nullptr, O, G, g_layout, Y, eps, false, false, status, st);
 }
 

@@ -979,7 +979,7 @@ cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, con
 }  // namespace
 
 cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, RowLayout q_layout,
-                                const void *K, const void *V, RowLayout v_layout,
+                                const void *K, RowLayout k_layout, const void *V, RowLayout v_layout,
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
                                 bool zeta_on_v, bool rotate_in_loop, int *status,
@@ -987,7 +987,7 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16_strided(&mq, Q, p.dk, p.L, bh, q_layout.row, q_layout.head, kC) ||
-        !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kC))
+        !make_tma_map_bf16_strided(&mk, K, p.dk, p.L, bh, k_layout.row, k_layout.head, kC))
         return cudaErrorInvalidValue;
     const bool ok = v_head_major
                         ? make_tma_map_bf16_strided(&mv, V, p.dv, p.L, bh, v_layout.row, v_layout.head, kC)

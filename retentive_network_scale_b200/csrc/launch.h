@@ -89,8 +89,8 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
                                          RowLayout g_layout, void *Y, void *O, float eps,
                                          int *status, cudaStream_t st);
 // Warp-specialised tensor-core chunk loop (chunkwise_ws.cu): the same
-// shapes as the kernel above.  Q^ is read through `q_layout` (head-major),
-// K' as [B][H][L][d_k], V through `v_layout` (head-major rows when
+// shapes as the kernel above.  Q^ and K' are read through `q_layout` and
+// `k_layout` (head-major), V through `v_layout` (head-major rows when
 // v_head_major, else rows of H*d_v columns), G through `g_layout` (rows of
 // H*d_v columns).  zeta_on_v: K' is K^ itself and the kernel weights the
 // value rows by gamma^{n-1-j}; otherwise K' already carries that weight
@@ -99,7 +99,7 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
 // itself (d_k 128 or 256, plain heads).  Writes Y ([B][L][H*d_v], with G)
 // and/or O ([B][H][L][d_v]) in the output dtype.
 cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, RowLayout q_layout,
-                                const void *K, const void *V, RowLayout v_layout,
+                                const void *K, RowLayout k_layout, const void *V, RowLayout v_layout,
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
                                 bool zeta_on_v, bool rotate_in_loop, int *status,
