@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -98,6 +99,7 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        self.lines, self.first = [], 0
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -105,19 +107,33 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        if self.proc is not None:
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            # nvidia-smi's start-up (NVML) is over before the timed region
+            # opens: wait for its first sample, then keep only later ones
+            t0 = time.time()
+            while not self.lines and self.proc.poll() is None and time.time() - t0 < 20:
+                time.sleep(0.02)
+            self.first = len(self.lines)
         return self
 
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
     def __exit__(self, *a):
-        self.out = ""
         if self.proc is not None:
             time.sleep(0.2)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+            self.reader.join(timeout=5)
+        taken = self.lines[self.first:] or self.lines
+        self.out = "".join(taken)
 
     def summary(self):
         rows = []
@@ -551,11 +567,27 @@ def bench_layer(R, w, pk, reps=5):
     flops = (2 * rows * dm * n_proj + 2 * rows * w.H * w.d_v * dm
              + w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v))
     tf = flops / (ms * 1e-3) / 1e12
+    # the two projections alone, on the library's tensor-core GEMM
+    gemms = {}
+    Xr = X.view(rows, dm)
+    Yb = torch.empty(rows, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
+    P = torch.empty(rows, n_proj, device="cuda", dtype=torch.bfloat16)
+    for name, (a, b, c) in (("X W_qkvg", (Xr, W, P)), ("Y W_o", (Yb, Wo, out.view(rows, dm)))):
+        g_fn = lambda a=a, b=b, c=c: R.ret_gemm_bf16(a, b, c)  # noqa: E731
+        g_fn()
+        g_ms = time_launches(g_fn, reps, torch.cuda.current_stream())
+        g_fl = 2.0 * a.shape[0] * a.shape[1] * b.shape[1]
+        g_tf = g_fl / (g_ms * 1e-3) / 1e12
+        gemms[name] = {"shape": [a.shape[0], b.shape[1], a.shape[1]], "ms": g_ms, "achieved": g_tf,
+                       "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": g_tf / pk["bf16_tflops"]}
+    del P, Yb
     return {"workload": f"MSR layer: B={w.B} L={w.L} d_model={dm} H={w.H} d_k={w.d_k} d_v={w.d_v}, "
-                        f"X W_qkvg (cuBLAS) + prep + fused chunkwise/GroupNorm/gate + Y W_o (cuBLAS)",
+                        f"X W_qkvg (tensor-core GEMM, CTA pairs) + prep + fused chunkwise/GroupNorm/gate "
+                        f"+ Y W_o (the same GEMM)",
             "ms": ms, "tokens_per_s": rows / (ms * 1e-3),
             "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops},
+            "gemm": gemms}
 
 
 def run_ours(args, world, rank, local):
@@ -566,7 +598,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
-    if args.only in ("decode", "parallel", "long_ctx", "msr_small", "backward"):
+    if args.only in ("decode", "parallel", "long_ctx", "msr_small", "backward", "layer"):
         if args.only == "decode":
             out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
         elif args.only == "long_ctx":
@@ -580,6 +612,8 @@ def run_ours(args, world, rank, local):
             d = {k: v.cuda() for k, v in make_inputs(w).items()}
             if args.only == "backward":
                 out = bench_backward(R, w, d, pk, reps=max(1, args.steps))
+            elif args.only == "layer":
+                out = bench_layer(R, w, pk, reps=max(1, args.steps))
             else:
                 out = bench_parallel(R, w, d, pk, reps=max(1, args.steps))
         if rank == 0:
@@ -622,6 +656,11 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     launches = R.ret_kernel_launches() - n0
+    # a bounded wait that ran out inside a kernel latches a status: such a
+    # run measured nothing
+    status = R.ret_last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
     ms_local = start.elapsed_time(end) / args.steps
     ms = max_over_ranks(ms_local, world)
     tokens_step = w.B * w.L
@@ -743,7 +782,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
     ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx", "msr_small",
-                                       "backward"],
+                                       "backward", "layer"],
                     default=None,
                     help="run one measurement alone (profiler captures)")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -20,7 +20,8 @@
  *    named as host pointers are read during the call only.
  *  - The caller owns every buffer and the stream.  The library allocates no
  *    device memory (cuBLAS allocates its own when the library first makes a
- *    handle on a device, for ret_msr_layer and ret_segment_state), keeps no
+ *    handle on a device, for the shapes of ret_segment_state off its
+ *    tensor-core kernel), keeps no
  *    per-call state, and never synchronises unless a function says so.
  *    `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.
@@ -288,13 +289,12 @@ size_t ret_chunkwise_host_workspace_size(const ret_desc *desc, int chunk,
  *   out     device bf16 [B][L][d_model]
  *   workspace  device, 256-byte aligned, at least
  *           ret_msr_layer_workspace_size() bytes (it holds P, the prepared
- *           Q and K, Y and the GEMM library's scratch).
+ *           Q and K, and Y).
  * desc->in_dtype and out_dtype are RET_BF16; d_model is a multiple of 8.
  * The layer runs on the tensor-core chunkwise path only (chunk a multiple of
  * 64, d_k 128 or 256, d_v a multiple of 128 up to 512, gamma_h^128 >=
- * 2^-60).  The two projections are cuBLAS GEMMs with fp32 accumulation; P
- * and Y are held in bf16.  Not safe to call from two host threads at once
- * on one device.
+ * 2^-60).  The two projections run on ret_gemm_bf16's tensor-core product
+ * (fp32 accumulation); P and Y are held in bf16.
  * Errors: those of ret_chunkwise; RET_ERR_SHAPE off the tensor-core path.
  */
 ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk,
@@ -306,6 +306,28 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk,
  * reject by their arguments and for empty problems.  Never fails. */
 size_t ret_msr_layer_workspace_size(const ret_desc *desc, int d_model,
                                     int chunk);
+
+/*
+ * ret_gemm_bf16 -- C = A B, the dense product the layer's projections are
+ * (paper summary, section 2.2: X W_Q, X W_K, X W_V, X W_G and the product
+ * with W_O), on the tensor cores: bf16 operands, fp32 accumulation, bf16
+ * result rounded to nearest even.
+ *   A  device bf16, M rows of K values, row r at A + r*lda
+ *   B  device bf16, K rows of N values, row k at B + k*ldb
+ *   C  device bf16, M rows of N values, row r at C + r*ldc (written)
+ * lda, ldb, ldc are in elements, multiples of 8, with lda >= K, ldb >= N,
+ * ldc >= N; N is a multiple of 8; M, N, K fit in 32 bits.  C must not
+ * overlap A or B.  M == 0 or N == 0 is an empty problem (RET_OK, nothing
+ * launched).
+ * Errors: RET_ERR_ARG (a negative size), RET_ERR_NULL, RET_ERR_SHAPE (K ==
+ * 0, N not a multiple of 8, leading dimensions as above), RET_ERR_ALIGN
+ * (a pointer not 16-byte aligned), RET_ERR_UNSUPPORTED (not an sm_100
+ * device), RET_ERR_CUDA (launch failure).  A bounded wait that runs out
+ * latches RET_ERR_TIMEOUT for ret_last_device_status.
+ */
+ret_status ret_gemm_bf16(long long M, long long N, long long K, const void *A,
+                         long long lda, const void *B, long long ldb, void *C,
+                         long long ldc, void *stream);
 
 /*
  * ret_backward -- the gradients of the retention output O (as computed by

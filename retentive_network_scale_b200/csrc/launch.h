@@ -118,6 +118,15 @@ cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void
 cudaError_t launch_key_prep(const Params &p, int chunk, const void *K, void *kt,
                             cudaStream_t st);
 
+// C[M x N] = A[M x K] B[K x N] on the tensor cores (gemm_tc.cu): bf16
+// row-major operands with leading dimensions lda, ldb, ldc (elements,
+// multiples of 8), fp32 accumulation, bf16 C.  N a multiple of 8.
+bool gemm_tc_supported(long long M, long long N, long long K, long long lda, long long ldb,
+                       long long ldc);
+cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A, long long lda,
+                           const void *B, long long ldb, void *C, long long ldc, int *status,
+                           cudaStream_t st);
+
 // The current device's cuBLAS handle, bound to `st` and to kBlasWorkspace
 // bytes of `workspace`; the caller holds blas_mutex() for as long as it
 // uses the handle (a handle is not safe to share between host threads).

@@ -11,13 +11,9 @@
 //                                            V and G read from P through
 //                                            strided tensor maps
 //   out = Y W_O                              one bf16 GEMM, fp32 accumulate
-// The two GEMMs are plain dense products and go to cuBLAS; everything
-// between them is this library's kernels, and nothing between them
-// round-trips through a separate layout pass.
-#include <cublas_v2.h>
-
-#include <mutex>
-
+// The two products run on this library's own tensor-core GEMM (gemm_tc.cu);
+// everything between them is this library's kernels, and nothing between
+// them round-trips through a separate layout pass.
 #include "launch.h"
 #include "retention.h"
 
@@ -28,13 +24,10 @@ constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-std::mutex g_mu;
-cublasHandle_t g_handle[kMaxDevices];
-
 struct LayerSizes {
     long long rows;   // B*L
     long long n_proj; // H*(2 d_k + 2 d_v)
-    size_t proj, prep, y, off_prep, off_y, off_blas, bytes;
+    size_t proj, prep, y, off_prep, off_y, bytes;
 };
 
 LayerSizes sizes_of(const ret_desc *d) {
@@ -46,45 +39,12 @@ LayerSizes sizes_of(const ret_desc *d) {
     s.y = (size_t)s.rows * d->H * d->d_v * 2;
     s.off_prep = round_up(s.proj);
     s.off_y = s.off_prep + round_up(s.prep);
-    s.off_blas = s.off_y + round_up(s.y);
-    s.bytes = s.off_blas + ret::kBlasWorkspace;
+    s.bytes = s.off_y + round_up(s.y);
     return s;
-}
-
-// Row-major C[M x N] = A[M x K] B[K x N] (bf16, fp32 accumulate), i.e. the
-// column-major product C^T = B^T A^T.
-cublasStatus_t gemm_rm(cublasHandle_t h, long long M, long long N, long long K, const void *A,
-                       const void *B, void *C) {
-    const float one = 1.f, zero = 0.f;
-    return cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, (int)N, (int)M, (int)K, &one, B, CUDA_R_16BF,
-                        (int)N, A, CUDA_R_16BF, (int)K, &zero, C, CUDA_R_16BF, (int)N,
-                        CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
 }
 
 }  // namespace
 
-namespace ret {
-
-std::mutex &blas_mutex() { return g_mu; }
-
-cublasHandle_t blas_handle(cudaStream_t st, void *workspace) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        cudaGetLastError();
-        return nullptr;
-    }
-    if (!g_handle[dev] && cublasCreate(&g_handle[dev]) != CUBLAS_STATUS_SUCCESS) {
-        g_handle[dev] = nullptr;
-        return nullptr;
-    }
-    cublasHandle_t h = g_handle[dev];
-    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS ||
-        cublasSetWorkspace(h, workspace, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
-        return nullptr;
-    return h;
-}
-
-}  // namespace ret
 
 extern "C" {
 
@@ -128,17 +88,14 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
     int *status = ret::device_status_word();
     if (!status) return RET_ERR_CUDA;
 
-    // one cuBLAS handle per device, used under the lock
-    std::lock_guard<std::mutex> lock(ret::blas_mutex());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    cublasHandle_t h = ret::blas_handle(st, ws + z.off_blas);
-    if (!h) return RET_ERR_CUDA;
 
     const int H = desc->H, dk = desc->d_k, dv = desc->d_v;
     const auto *P = reinterpret_cast<const __nv_bfloat16 *>(ws);
     // 1. the four projections in one product
-    if (gemm_rm(h, z.rows, z.n_proj, d_model, X, W_qkvg, ws) != CUBLAS_STATUS_SUCCESS)
+    if (ret::launch_gemm_tc(z.rows, z.n_proj, d_model, X, d_model, W_qkvg, z.n_proj, ws, z.n_proj,
+                            status, st) != cudaSuccess)
         return RET_ERR_CUDA;
     // 2. Q^ and K~ from the projection rows: row t of head h of batch b sits
     //    at (b L + t) n_proj + h d_k in the Q block (the K block follows)
@@ -156,8 +113,9 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
                                           ws + z.off_y, nullptr, gn_eps, status, st);
     if (e != cudaSuccess) return RET_ERR_CUDA;
     // 4. the output projection
-    if (gemm_rm(h, z.rows, d_model, (long long)H * dv, ws + z.off_y, W_o, out) !=
-        CUBLAS_STATUS_SUCCESS)
+    const long long hdv = (long long)H * dv;
+    if (ret::launch_gemm_tc(z.rows, d_model, hdv, ws + z.off_y, hdv, W_o, d_model, out, d_model,
+                            status, st) != cudaSuccess)
         return RET_ERR_CUDA;
     return RET_OK;
 }

@@ -24,6 +24,34 @@
 #include "retention.h"
 
 namespace ret {
+
+// One cuBLAS handle per device for the batched GEMM fallback of the segment
+// states (shapes off the tensor-core kernel), made on first use.
+namespace {
+constexpr int kBlasDevices = 64;
+std::mutex g_blas_mu;
+cublasHandle_t g_blas[kBlasDevices];
+}  // namespace
+
+std::mutex &blas_mutex() { return g_blas_mu; }
+
+cublasHandle_t blas_handle(cudaStream_t st, void *workspace) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kBlasDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
+        g_blas[dev] = nullptr;
+        return nullptr;
+    }
+    cublasHandle_t h = g_blas[dev];
+    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS ||
+        cublasSetWorkspace(h, workspace, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
+        return nullptr;
+    return h;
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;

@@ -32,6 +32,7 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_chunkwise_fast_size",
            "ret_chunkwise_prepare", "ret_chunkwise_prepared", "ret_chunkwise_host", "ret_chunkwise_host_workspace_size",
            "ret_selftest_wait_timeout", "ret_msr_layer", "ret_msr_layer_workspace_size",
+           "ret_gemm_bf16",
            "ret_backward", "ret_backward_workspace_size",
            "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
            "ret_chunkwise_segmented", "ret_chunkwise_segmented_workspace_size",
@@ -100,6 +101,8 @@ def load_library(path: str = LIB_PATH):
                                   st, vp]
     lib.ret_msr_layer_workspace_size.argtypes = [D, ctypes.c_int, ctypes.c_int]
     lib.ret_msr_layer_workspace_size.restype = st
+    ll = ctypes.c_longlong
+    lib.ret_gemm_bf16.argtypes = [ll, ll, ll, vp, ll, vp, ll, vp, ll, vp]
     lib.ret_backward.argtypes = [D, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, st, vp]
     lib.ret_backward_workspace_size.argtypes = [D, ctypes.c_int]
     lib.ret_backward_workspace_size.restype = st
@@ -354,6 +357,29 @@ def ret_msr_layer(X, W_qkvg, W_o, gamma, chunk, d_k, d_v, out=None, gn_eps=1e-5,
                              float(gn_eps), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
            "ret_msr_layer")
     return out
+
+
+def ret_gemm_bf16(A, B, C=None, stream=None):
+    """C = A B (bf16 [M, K] times bf16 [K, N], fp32 accumulation, bf16 C
+    [M, N]) on the library's tensor-core product; 2-D tensors whose rows
+    may be strided (unit stride along a row).  Returns C."""
+    lib = load_library()
+    for t, n in ((A, "A"), (B, "B")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dim() != 2 or t.stride(1) != 1 \
+                or t.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be a 2-D bf16 CUDA tensor with unit row stride")
+    M, K = A.shape
+    K2, N = B.shape
+    if K2 != K:
+        raise ValueError("inner sizes differ")
+    if C is None:
+        C = torch.empty(M, N, device=A.device, dtype=torch.bfloat16)
+    if not C.is_cuda or C.dim() != 2 or C.stride(1) != 1 or tuple(C.shape) != (M, N) \
+            or C.dtype != torch.bfloat16:
+        raise ValueError("C must be a 2-D bf16 CUDA tensor [M, N] with unit row stride")
+    _check(lib.ret_gemm_bf16(M, N, K, _ptr(A), A.stride(0), _ptr(B), B.stride(0), _ptr(C),
+                             C.stride(0), _stream(stream)), "ret_gemm_bf16")
+    return C
 
 
 def lib_msr_layer_workspace_size(B, H, L, d_k, d_v, gamma, d_model, chunk, rotate=False):

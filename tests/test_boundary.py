@@ -31,7 +31,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ret_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ret_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_lists_the_entry_points():
