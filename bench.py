@@ -567,10 +567,13 @@ def bench_layer(R, w, pk, reps=5):
     flops = (2 * rows * dm * n_proj + 2 * rows * w.H * w.d_v * dm
              + w.B * w.H * w.L * chunkwise_flops_per_token_head(w.chunk, w.d_k, w.d_v))
     tf = flops / (ms * 1e-3) / 1e12
-    # the two projections alone, on the library's tensor-core GEMM
+    # the two products alone, on the library's tensor-core GEMM (plain
+    # epilogue)
     gemms = {}
     Xr = X.view(rows, dm)
-    Yb = torch.empty(rows, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
+    # random operands (an all-zero one draws less power and would run above
+    # the power-capped peak)
+    Yb = (torch.randn(rows, w.H * w.d_v, device="cuda", generator=gen) * 0.5).bfloat16()
     P = torch.empty(rows, n_proj, device="cuda", dtype=torch.bfloat16)
     for name, (a, b, c) in (("X W_qkvg", (Xr, W, P)), ("Y W_o", (Yb, Wo, out.view(rows, dm)))):
         g_fn = lambda a=a, b=b, c=c: R.ret_gemm_bf16(a, b, c)  # noqa: E731
@@ -582,8 +585,8 @@ def bench_layer(R, w, pk, reps=5):
                        "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": g_tf / pk["bf16_tflops"]}
     del P, Yb
     return {"workload": f"MSR layer: B={w.B} L={w.L} d_model={dm} H={w.H} d_k={w.d_k} d_v={w.d_v}, "
-                        f"X W_qkvg (tensor-core GEMM, CTA pairs) + prep + fused chunkwise/GroupNorm/gate "
-                        f"+ Y W_o (the same GEMM)",
+                        f"X W_qkvg (tensor-core GEMM, CTA pairs; the xPos turn and key weights in its "
+                        f"epilogue) + fused chunkwise/GroupNorm/gate + Y W_o (the same GEMM)",
             "ms": ms, "tokens_per_s": rows / (ms * 1e-3),
             "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops},

@@ -59,6 +59,7 @@ constexpr int kThreads = 256;
 constexpr uint32_t kABytes = kBM * kBK * 2;  // 16 KB: this CTA's 128 rows x 64 k
 constexpr uint32_t kBBlock = kBK * 64 * 2;   // one 64-column block of B: 8 KB
 constexpr long long kTimeoutCycles = 4000000000LL;  // about 2 s
+constexpr int kProjBlock = 128;  // rows per block of the chunk loop the projection feeds
 
 // PAIR: two CTAs of a cluster share each 256 x 256 tile: each loads its own
 // 128 rows of A and its own 128 of the 256 columns of B, and the even CTA
@@ -138,10 +139,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
-template <bool PAIR>
+// PROJ: C is the layer's projection P = X [W_Q | W_K | W_V | W_G] and the
+// epilogue also does what the streaming pass would: the columns of the Q
+// block leave turned by the xPos angles of their row's position, the
+// columns of the K block turned and weighted by gamma_h^{n-1-j} (j the row's
+// place in its block of 128 rows, n that block's rows), each into its own
+// [B][H][L][d_k] array (qh, kt); only the V and G columns go to C.
+template <bool PAIR, bool PROJ>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               int M, int N, int K, __nv_bfloat16 *__restrict__ C, long long ldc, int *status) {
+               int M, int N, int K, __nv_bfloat16 *__restrict__ C, long long ldc, int *status,
+               const __grid_constant__ Params pp, __nv_bfloat16 *__restrict__ qh,
+               __nv_bfloat16 *__restrict__ kt) {
     using G = Cfg<PAIR>;
     constexpr int kStages = G::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -271,22 +280,59 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_fence_after();
             const int row = m0 + quad * 32 + lane;
             __nv_bfloat16 *crow = C + (size_t)row * ldc + n0;
+            // (PROJ) this row's sequence, position and place in its block
+            int pb = 0, pl = 0, pn = 0;
+            if constexpr (PROJ) {
+                pb = row / pp.L;
+                pl = row - pb * pp.L;
+                const int j0 = pl - pl % kProjBlock;
+                pn = min(kProjBlock, pp.L - j0);
+            }
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t x[32];
                 tmem_ld32(tmem + lane_base + b * kBN + 32 * c, x);
                 tmem_wait_ld(x);
+                const int col0 = n0 + 32 * c;
+                __nv_bfloat16 *dst = crow + 32 * c;
+                if constexpr (PROJ) {
+                    const int hdk = pp.H * pp.dk;
+                    if (col0 < 2 * hdk) {
+                        // a Q or K column chunk (32 columns of one head)
+                        const bool key = col0 >= hdk;
+                        const int cq = key ? col0 - hdk : col0;
+                        const int h = cq / pp.dk, d0 = cq - h * pp.dk;
+                        const float z = key ? decay_pow(pp.log2g[h], pn - 1 - (pl % kProjBlock)) : 1.f;
+                        if (pp.rotate) {
+                            const long long pos = pp.pos_offset + pl;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                float cs, sn;
+                                rot_cs_fast(pos, pp.theta[d0 / 2 + e], &cs, &sn);
+                                const float x0 = __uint_as_float(x[2 * e]), x1 = __uint_as_float(x[2 * e + 1]);
+                                x[2 * e] = __float_as_uint(z * (x0 * cs - x1 * sn));
+                                x[2 * e + 1] = __float_as_uint(z * (x0 * sn + x1 * cs));
+                            }
+                        } else if (key) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) x[e] = __float_as_uint(z * __uint_as_float(x[e]));
+                        }
+                        dst = (key ? kt : qh) + (((size_t)pb * pp.H + h) * pp.L + pl) * pp.dk + d0;
+                    } else {
+                        dst = crow + 32 * c;
+                    }
+                }
                 if (row < M) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int col = n0 + 32 * c + 8 * q;
+                        const int col = col0 + 8 * q;
                         if (col < N) {
                             uint4 w;
                             w.x = pack2(__uint_as_float(x[8 * q + 0]), __uint_as_float(x[8 * q + 1]));
                             w.y = pack2(__uint_as_float(x[8 * q + 2]), __uint_as_float(x[8 * q + 3]));
                             w.z = pack2(__uint_as_float(x[8 * q + 4]), __uint_as_float(x[8 * q + 5]));
                             w.w = pack2(__uint_as_float(x[8 * q + 6]), __uint_as_float(x[8 * q + 7]));
-                            *reinterpret_cast<uint4 *>(crow + 32 * c + 8 * q) = w;
+                            *reinterpret_cast<uint4 *>(dst + 8 * q) = w;
                         }
                     }
                 }
@@ -336,9 +382,12 @@ bool gemm_tc_supported(long long M, long long N, long long K, long long lda, lon
            ldc >= N;
 }
 
-cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A, long long lda,
-                           const void *B, long long ldb, void *C, long long ldc, int *status,
-                           cudaStream_t st) {
+namespace {
+
+template <bool PROJ>
+cudaError_t launch_gemm(long long M, long long N, long long K, const void *A, long long lda,
+                        const void *B, long long ldb, void *C, long long ldc, const Params &pp,
+                        void *qh, void *kt, int *status, cudaStream_t st) {
     if (!gemm_tc_supported(M, N, K, lda, ldb, ldc)) return cudaErrorInvalidValue;
     // CTA pairs (256-row tiles) once there are enough rows to fill them
     const bool pair = M > kBM;
@@ -351,10 +400,11 @@ cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A,
     if (sms < 2) return cudaErrorInvalidValue;
     const long long ntiles = ((M + tm - 1) / tm) * ((N + kBN - 1) / kBN);
     __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(C);
+    __nv_bfloat16 *q = static_cast<__nv_bfloat16 *>(qh), *k = static_cast<__nv_bfloat16 *>(kt);
     cudaError_t e;
     if (pair) {
         const uint32_t smem = Cfg<true>::kSmemBytes;
-        e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(gemm_tc_kernel<true, PROJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
@@ -369,18 +419,38 @@ cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A,
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<true>, ma, mb, (int)M, (int)N, (int)K, c, ldc, status);
+        e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<true, PROJ>, ma, mb, (int)M, (int)N, (int)K, c, ldc,
+                               status, pp, q, k);
     } else {
         const uint32_t smem = Cfg<false>::kSmemBytes;
-        e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(gemm_tc_kernel<false, PROJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
         const int grid = (int)std::min<long long>(ntiles, sms);
-        gemm_tc_kernel<false><<<grid, kThreads, smem, st>>>(ma, mb, (int)M, (int)N, (int)K, c, ldc, status);
+        gemm_tc_kernel<false, PROJ><<<grid, kThreads, smem, st>>>(ma, mb, (int)M, (int)N, (int)K, c, ldc,
+                                                                 status, pp, q, k);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) note_launches(1);
     return e;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A, long long lda,
+                           const void *B, long long ldb, void *C, long long ldc, int *status,
+                           cudaStream_t st) {
+    Params none{};
+    return launch_gemm<false>(M, N, K, A, lda, B, ldb, C, ldc, none, nullptr, nullptr, status, st);
+}
+
+cudaError_t launch_gemm_proj(const Params &p, int d_model, const void *X, const void *W, void *P,
+                             void *qh, void *kt, int *status, cudaStream_t st) {
+    // every 32-column chunk of a tile lies in one head of one block
+    if (p.dk % 32 != 0 || p.dv % 32 != 0 || !qh || !kt) return cudaErrorInvalidValue;
+    const long long n_proj = (long long)p.H * (2LL * p.dk + 2LL * p.dv);
+    return launch_gemm<true>((long long)p.B * p.L, n_proj, d_model, X, d_model, W, n_proj, P, n_proj,
+                             p, qh, kt, status, st);
 }
 
 }  // namespace ret

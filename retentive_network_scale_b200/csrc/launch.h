@@ -127,6 +127,14 @@ cudaError_t launch_gemm_tc(long long M, long long N, long long K, const void *A,
                            const void *B, long long ldb, void *C, long long ldc, int *status,
                            cudaStream_t st);
 
+// The layer's projection P = X [W_Q | W_K | W_V | W_G] (X [B*L][d_model],
+// P [B*L][H (2 d_k + 2 d_v)]) with the streaming pass folded into the
+// epilogue: the Q and K columns leave as Q^ and K~ (turned when p.rotate,
+// K~ weighted by gamma^{n-1-j} per block of 128 rows), bf16
+// [B][H][L][d_k] into qh and kt; only the V and G columns are written to P.
+cudaError_t launch_gemm_proj(const Params &p, int d_model, const void *X, const void *W, void *P,
+                             void *qh, void *kt, int *status, cudaStream_t st);
+
 // The current device's cuBLAS handle, bound to `st` and to kBlasWorkspace
 // bytes of `workspace`; the caller holds blas_mutex() for as long as it
 // uses the handle (a handle is not safe to share between host threads).

@@ -4,16 +4,16 @@
 // "Retentive Network" paper summary, section 2.1 (Q = (X W_Q) (.) Theta,
 // K = (X W_K) (.) conj(Theta), V = X W_V, one decay per head) and section
 // 2.2 (Y = GroupNorm_h(Concat(heads)); MSR(X) = (swish(X W_G) (.) Y) W_O):
-//   P   = X [W_Q | W_K | W_V | W_G]          one bf16 GEMM, fp32 accumulate
-//   Q^, K~ from P's first two column blocks  the streaming prep pass, reading
-//                                            the projection rows in place
+//   P   = X [W_Q | W_K | W_V | W_G]          one bf16 GEMM, fp32 accumulate,
+//                                            whose epilogue writes the Q and
+//                                            K columns as Q^ and K~ (turned,
+//                                            keys decay-weighted) per head
 //   Y   = swish(G) (.) GroupNorm_h(O)        the fused chunkwise kernel, with
 //                                            V and G read from P through
 //                                            strided tensor maps
 //   out = Y W_O                              one bf16 GEMM, fp32 accumulate
-// The two products run on this library's own tensor-core GEMM (gemm_tc.cu);
-// everything between them is this library's kernels, and nothing between
-// them round-trips through a separate layout pass.
+// Three launches, all this library's own kernels (the GEMM is gemm_tc.cu);
+// nothing between them round-trips through a separate layout pass.
 #include "launch.h"
 #include "retention.h"
 
@@ -93,26 +93,21 @@ ret_status ret_msr_layer(const ret_desc *desc, int d_model, int chunk, const voi
 
     const int H = desc->H, dk = desc->d_k, dv = desc->d_v;
     const auto *P = reinterpret_cast<const __nv_bfloat16 *>(ws);
-    // 1. the four projections in one product
-    if (ret::launch_gemm_tc(z.rows, z.n_proj, d_model, X, d_model, W_qkvg, z.n_proj, ws, z.n_proj,
-                            status, st) != cudaSuccess)
+    // 1. the four projections in one product, whose epilogue turns the Q
+    //    and K columns (and weights the keys) into [B][H][L][d_k] arrays
+    uint8_t *qh = ws + z.off_prep;
+    uint8_t *kt = qh + z.prep / 2;
+    if (ret::launch_gemm_proj(p, d_model, X, W_qkvg, ws, qh, kt, status, st) != cudaSuccess)
         return RET_ERR_CUDA;
-    // 2. Q^ and K~ from the projection rows: row t of head h of batch b sits
-    //    at (b L + t) n_proj + h d_k in the Q block (the K block follows)
-    const ret::RowLayout qk{z.n_proj, dk, (long long)desc->L * z.n_proj};
-    const void *qh = nullptr, *kt = nullptr;
-    cudaError_t e = ret::launch_chunkwise_prep_strided(p, 128, P, P + (size_t)H * dk, qk, true,
-                                                       ws + z.off_prep, &qh, &kt, st);
-    if (e != cudaSuccess) return RET_ERR_CUDA;
-    // 3. the chunk loop with the fused GroupNorm + gate; V and G are read as
+    // 2. the chunk loop with the fused GroupNorm + gate; V and G are read as
     //    rows of H d_v columns of the projection
     const ret::RowLayout vg{z.n_proj, 0, (long long)desc->L * z.n_proj};
-    e = ret::launch_chunkwise_tc_prepared(p, true, qh, ret::bhld_layout(p, dk), kt,
-                                          P + 2 * (size_t)H * dk, vg, false,
-                                          P + 2 * (size_t)H * dk + (size_t)H * dv, vg,
-                                          ws + z.off_y, nullptr, gn_eps, status, st);
+    cudaError_t e = ret::launch_chunkwise_tc_prepared(p, true, qh, ret::bhld_layout(p, dk), kt,
+                                                      P + 2 * (size_t)H * dk, vg, false,
+                                                      P + 2 * (size_t)H * dk + (size_t)H * dv, vg,
+                                                      ws + z.off_y, nullptr, gn_eps, status, st);
     if (e != cudaSuccess) return RET_ERR_CUDA;
-    // 4. the output projection
+    // 3. the output projection
     const long long hdv = (long long)H * dv;
     if (ret::launch_gemm_tc(z.rows, d_model, hdv, ws + z.off_y, hdv, W_o, d_model, out, d_model,
                             status, st) != cudaSuccess)

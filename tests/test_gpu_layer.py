@@ -1,8 +1,10 @@
 """ret_msr_layer (projections, retention with the fused GroupNorm + gate,
-output projection) against the fp64 layer oracle; the layer's kernels read
-the projection in place (strided Q/K for the prep pass, strided V and G
-tensor maps), so a small case with two heads, a ragged length and both
-tensor-core d_k checks that plumbing; plus argument refusals."""
+output projection) against the fp64 layer oracle; the projection's epilogue
+writes the turned / decay-weighted Q and K per head and the chunk loop reads
+V and G from the projection in place (strided tensor maps), so small cases
+with two or three heads, ragged lengths (blocks of 128 rows cut short, rows
+of one tile spanning two sequences) and both tensor-core d_k check that
+plumbing; plus argument refusals."""
 import pytest
 import torch
 
@@ -24,10 +26,12 @@ def _lib():
     assert R.ret_last_device_status() == 0
 
 
-@pytest.mark.parametrize("dk,dv,rotate", [(128, 128, True), (256, 256, False), (128, 384, True)])
-def test_msr_layer_matches_oracle(dk, dv, rotate):
-    B, L, H, dm = 2, 300, 2, 256
-    g = [0.96875, 0.999]
+@pytest.mark.parametrize("dk,dv,rotate,H", [(128, 128, True, 2), (256, 256, False, 2),
+                                            (128, 384, True, 2), (128, 128, True, 3),
+                                            (256, 128, True, 1)])
+def test_msr_layer_matches_oracle(dk, dv, rotate, H):
+    B, L, dm = 2, 300, 256
+    g = [0.96875, 0.999, 0.9921875][:H]
     n_proj = H * (2 * dk + 2 * dv)
     X = random_tensor((B, L, dm), 700).bfloat16()
     W = random_tensor((dm, n_proj), 701, dm ** -0.5).bfloat16()
@@ -36,7 +40,7 @@ def test_msr_layer_matches_oracle(dk, dv, rotate):
     n0 = R.ret_kernel_launches()
     out = R.ret_msr_layer(X.cuda(), W.cuda(), Wo.cuda(), g, 128, dk, dv, rotate=rotate,
                           pos_offset=5)
-    assert R.ret_kernel_launches() - n0 == 4          # projection, prep pass, chunk loop, W_o
+    assert R.ret_kernel_launches() - n0 == 3          # projection (+ turn), chunk loop, W_o
     torch.cuda.synchronize()
     assert R.ret_last_device_status() == 0
     assert rel_l2(out, ref) <= TOL_BF16
