@@ -33,7 +33,7 @@
 //            (an arrival on the even CTA's barrier)
 // Tensor memory holds two accumulators (2 x 256 columns), so the epilogue
 // of tile i runs while the tensor cores work on tile i+1.  Shared memory
-// holds six stages of 32 KB (four of 48 KB unpaired).
+// holds seven stages of 32 KB (four of 48 KB unpaired).
 //
 // Operands past M, N or K read as zeros from the TMA (so K needs no
 // multiple of 64); stores past M or N are skipped (N a multiple of 8).
@@ -68,11 +68,11 @@ constexpr int kProjBlock = 128;  // rows per block of the chunk loop the project
 // memory.  Alone: one CTA, a 128 x 256 tile, all of B's 256 columns.
 template <bool PAIR>
 struct Cfg {
-    static constexpr int kStages = PAIR ? 6 : 4;
+    static constexpr int kStages = PAIR ? 7 : 4;
     static constexpr int kBCols = PAIR ? kBN / 2 : kBN;            // B columns loaded by a CTA
     static constexpr uint32_t kBBytes = kBBlock * (kBCols / 64);   // 16 or 32 KB
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 32 or 48 KB
-    static constexpr uint32_t kData = kStages * kStageBytes;       // 192 KB
+    static constexpr uint32_t kData = kStages * kStageBytes;       // 224 or 192 KB
     // FULL[s]: stage s landed (the even CTA's barrier counts both CTAs'
     // bytes); EMPTY[s]: its products completed; ACCF[b]: accumulator b
     // final; ACCE[b]: accumulator b read out by the epilogue warps (of both
