@@ -16,10 +16,12 @@
 // nothing representable in fp32; the walk stops there.  Roles (12 warps):
 // one thread issues the MMAs -- S of tile t into one of two tensor-memory
 // buffers, then P V of tile t-1 -- so that the P pass of one tile runs while
-// the tensor cores multiply its neighbour; one thread issues the TMA loads
-// (the next K tile once S has read the current one, the next V tile once
-// P V has); warps 4-11 run the P pass and finally move the output tile out
-// through shared memory and TMA stores.  Every hand-over is an mbarrier with
+// the tensor cores multiply its neighbour; one thread issues the TMA loads of
+// Q and of the next K tile once S has read the current one; another loads V
+// in halves of 64 keys into a ring of three (so the next tile's first half
+// lands while the current tile's products run, and its second half as soon
+// as the current first half is consumed); warps 4-11 run the P pass and
+// finally move the output tile out through shared memory and TMA stores.  Every hand-over is an mbarrier with
 // a bounded wait.
 //
 // The rotation (xPos) is applied once per row by xpos_rotate_kernel into a
@@ -43,25 +45,33 @@ constexpr int kThreads = 384;   // three warpgroups
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr float kMinLog2GammaTimesT = -60.f;  // gamma^-127 stays below 2^60
 
-// BQ/BK/BV: tile landed; SD0/SD1: S of the tile in S buffer b done; PR0/PR1:
-// P of buffer b written; PV0/PV1: P V of buffer b's tile done (the buffer,
-// and the V tile, free again).  The buffer barriers complete once every two
-// key tiles, so no waiter can fall two phases behind.
-enum { BQ = 0, BK, BV, SD0, SD1, PR0, PR1, PV0, PV1, kNumBars };
+// BQ/BK: tile landed; VF0-2: V half in ring slot s landed; VE0-2: the
+// products that read ring slot s done (slot free); SD0/SD1: S of the tile in
+// S buffer b done; PR0/PR1: P of buffer b written; PV0/PV1: P V of buffer
+// b's tile done (the buffer free again).  The buffer barriers complete once
+// every two key tiles and the ring's once every three halves, so no waiter
+// can fall two phases behind.
+enum { BQ = 0, BK, VF0, VF1, VF2, VE0, VE1, VE2, SD0, SD1, PR0, PR1, PV0, PV1, kNumBars };
+constexpr int kRing = 3;  // V half tiles (64 keys) in flight
 
 template <int DK, int TV>
 struct PLayout {
     static constexpr uint32_t kQ = 0;                     // Q^: DK/64 blocks of 16 KB
     static constexpr uint32_t kQBytes = kT * DK * 2;
     static constexpr uint32_t kK = kQ + kQBytes;          // K^_k
-    static constexpr uint32_t kV = kK + kQBytes;          // V_k: TV/64 blocks of 16 KB
-    static constexpr uint32_t kVBytes = kT * TV * 2;
-    static constexpr uint32_t kSmall = kV + kVBytes;
+    // V: a ring of kRing half tiles (64 keys x TV columns, TV/64 blocks of
+    // 8 KB); at the end the first 2 slots stage the bf16 output tile
+    static constexpr uint32_t kV = kK + kQBytes;
+    static constexpr uint32_t kVBlock = (kT / 2) * 64 * 2;
+    static constexpr uint32_t kVSlot = kVBlock * (TV / 64);
+    static constexpr uint32_t kSmall = kV + kRing * kVSlot;
     static constexpr uint32_t kBar = kSmall;
     static constexpr uint32_t kTmemSlot = kSmall + 8 * kNumBars;
     static constexpr uint32_t kAbort = kTmemSlot + 4;
     static constexpr uint32_t kColScale = kSmall + 128;   // gamma^{-j'}, 128 floats
     static constexpr uint32_t kBytes = kColScale + 512;
+    static_assert(8 * kNumBars + 8 <= 128, "small area");
+    static_assert(kRing * kVSlot >= kT * TV * 2, "the output tile is staged in the V ring");
 };
 
 __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
@@ -135,19 +145,25 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // then P V of tile it-1 while the P pass works on tile it
         const uint64_t dQ = sdesc_sw128(sbase + Ly::kQ, 16, 1024);
         const uint64_t dK = sdesc_sw128(sbase + Ly::kK, 16, 1024);
-        const uint64_t dV = sdesc_sw128(sbase + Ly::kV, 16384, 1024);
-        auto pv = [&](int j) {  // P V of tile j (buffer j & 1)
+        auto pv = [&](int j) {  // P V of tile j (buffer j & 1), one V half (64 keys) at a time
             const int b = j & 1;
-            if (!(wait_all(PR0 + b, (j >> 1) & 1) && wait_all(BV, j & 1))) return false;
-            tc_fence_after();
-            if (lane == 0) {
+            if (!wait_all(PR0 + b, (j >> 1) & 1)) return false;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                const int hi = 2 * j + half, slot = hi % kRing;
+                if (!wait_all(VF0 + slot, (hi / kRing) & 1)) return false;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t dV = sdesc_sw128(sbase + Ly::kV + slot * Ly::kVSlot, Ly::kVBlock, 1024);
 #pragma unroll
-                for (int ks = 0; ks < kT / 16; ++ks)
-                    mma_ts(tO, tS(b) + (ks >> 2) * 64 + (ks & 3) * 8, dV + (uint64_t)((ks * 2048) >> 4),
-                           kIdescPV, (ks > 0 || j > 0) ? 1u : 0u);
-                mma_commit(bar(PV0 + b));
+                    for (int ks = 0; ks < kT / 32; ++ks)
+                        mma_ts(tO, tS(b) + half * 64 + ks * 8, dV + (uint64_t)((ks * 2048) >> 4), kIdescPV,
+                               (ks > 0 || half > 0 || j > 0) ? 1u : 0u);
+                    mma_commit(bar(VE0 + slot));
+                    if (half == 1) mma_commit(bar(PV0 + b));
+                }
+                __syncwarp();
             }
-            __syncwarp();
             return true;
         };
         bool ok = wait_all(BQ, 0);
@@ -171,32 +187,40 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         if (ok) pv(nit - 1);
     } else if (warp == 1) {
-        // ====== TMA loads: K of the next tile once S has read the current,
-        // V of the next tile once P V has read the current
+        // ====== TMA loads of Q and K: the next K tile as soon as S has read
+        // the current one
         auto load_k = [&](int kt) {
             mbar_expect_tx(bar(BK), Ly::kQBytes);
             for (int kb = 0; kb < KB; ++kb)
                 tma_load_3d(sbase + Ly::kK + kb * 16384, &tmK, bar(BK), kb * 64, kt * kT, bh);
-        };
-        auto load_v = [&](int kt) {
-            mbar_expect_tx(bar(BV), Ly::kVBytes);
-            for (int nb = 0; nb < VB; ++nb)
-                tma_load_3d(sbase + Ly::kV + nb * 16384, &tmV, bar(BV), v0 + nb * 64, kt * kT, bh);
         };
         if (lane == 0) {
             mbar_expect_tx(bar(BQ), Ly::kQBytes);
             for (int kb = 0; kb < KB; ++kb)
                 tma_load_3d(sbase + Ly::kQ + kb * 16384, &tmQ, bar(BQ), kb * 64, q0, bh);
             load_k(qt);
-            load_v(qt);
         }
 #pragma unroll 1
         for (int it = 0; it + 1 < nit; ++it) {
-            const int b = it & 1;
-            if (!wait_all(SD0 + b, (it >> 1) & 1)) break;
+            if (!wait_all(SD0 + (it & 1), (it >> 1) & 1)) break;
             if (lane == 0) load_k(qt - it - 1);
-            if (!wait_all(PV0 + b, (it >> 1) & 1)) break;
-            if (lane == 0) load_v(qt - it - 1);
+            __syncwarp();
+        }
+    } else if (warp == 2) {
+        // ====== TMA loads of V, half a key tile at a time into the ring, as
+        // soon as the products that read a slot's previous half are done
+        // (the next tile's halves land while the current tile's products run)
+#pragma unroll 1
+        for (int hi = 0; hi < 2 * nit; ++hi) {
+            const int slot = hi % kRing;
+            if (hi >= kRing && !wait_all(VE0 + slot, (hi / kRing - 1) & 1)) break;
+            if (lane == 0) {
+                const int kt = qt - (hi >> 1), r0 = kt * kT + (hi & 1) * (kT / 2);
+                const uint32_t dst = sbase + Ly::kV + slot * Ly::kVSlot;
+                mbar_expect_tx(bar(VF0 + slot), Ly::kVSlot);
+                for (int nb = 0; nb < VB; ++nb)
+                    tma_load_3d(dst + nb * Ly::kVBlock, &tmV, bar(VF0 + slot), v0 + nb * 64, r0, bh);
+            }
             __syncwarp();
         }
     } else if (warp >= 4) {
@@ -407,7 +431,7 @@ cudaError_t launch_parallel_tc(const Params &p, bool out_bf16, const void *Q, co
     std::memset(&mo, 0, sizeof(mo));
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16(&mq, Q, p.dk, p.L, bh, kT) || !make_tma_map_bf16(&mk, K, p.dk, p.L, bh, kT) ||
-        !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kT))
+        !make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kT / 2))
         return cudaErrorInvalidValue;
     if (out_bf16 && !make_tma_map_bf16(&mo, O, p.dv, p.L, bh, kT)) return cudaErrorInvalidValue;
     if (p.dk == 256)
