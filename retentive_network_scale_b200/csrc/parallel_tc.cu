@@ -79,6 +79,17 @@ __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile in
     return mbar_wait_bounded(bar, parity, abort_flag, status, kTimeoutCycles);
 }
 
+// Two consecutive 32-bit values of a tensor-memory load as a packed pair.
+__device__ __forceinline__ uint64_t f2_pair(const uint32_t *r) {
+    return (static_cast<uint64_t>(r[1]) << 32) | r[0];
+}
+// The pair with its low / high lane zeroed where asked.
+__device__ __forceinline__ uint64_t f2_mask(uint64_t x, bool lo_zero, bool hi_zero) {
+    if (lo_zero) x &= 0xffffffff00000000ull;
+    if (hi_zero) x &= 0x00000000ffffffffull;
+    return x;
+}
+
 __device__ __forceinline__ uint32_t pk_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -244,16 +255,29 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             tmem_wait_ld(a);
             tmem_wait_ld(c);
             const float aj = exp2f((float)(delta + row) * lg);  // gamma^{Delta + j}
-            const bool diag = delta == 0;
+            const uint64_t A2 = f2_make(aj, aj);
+            // the column weights gamma^{-j'} of this warpgroup's keys, four
+            // at a time (one address for the whole warp: a broadcast)
+            const float4 *cs4 = reinterpret_cast<const float4 *>(colscale + k0);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int j0 = k0 + 2 * i, j1 = k0 + 32 + 2 * i;
-                const float w00 = (diag && j0 > row) ? 0.f : aj * colscale[j0];
-                const float w01 = (diag && j0 + 1 > row) ? 0.f : aj * colscale[j0 + 1];
-                const float w10 = (diag && j1 > row) ? 0.f : aj * colscale[j1];
-                const float w11 = (diag && j1 + 1 > row) ? 0.f : aj * colscale[j1 + 1];
-                pk[i] = pk_bf16(__uint_as_float(a[2 * i]) * w00, __uint_as_float(a[2 * i + 1]) * w01);
-                pk[16 + i] = pk_bf16(__uint_as_float(c[2 * i]) * w10, __uint_as_float(c[2 * i + 1]) * w11);
+            for (int q = 0; q < 8; ++q) {
+                const float4 wa = cs4[q], wb = cs4[8 + q];  // keys k0 + 4q.., k0 + 32 + 4q..
+                const uint64_t w0 = f2_mul(A2, f2_make(wa.x, wa.y)), w1 = f2_mul(A2, f2_make(wa.z, wa.w));
+                const uint64_t w2 = f2_mul(A2, f2_make(wb.x, wb.y)), w3 = f2_mul(A2, f2_make(wb.z, wb.w));
+                uint64_t x0 = f2_mul(f2_pair(a + 4 * q), w0), x1 = f2_mul(f2_pair(a + 4 * q + 2), w1);
+                uint64_t x2 = f2_mul(f2_pair(c + 4 * q), w2), x3 = f2_mul(f2_pair(c + 4 * q + 2), w3);
+                if (delta == 0) {
+                    // the diagonal tile: keys after the row's own position are masked
+                    const int j = k0 + 4 * q;
+                    x0 = f2_mask(x0, j > row, j + 1 > row);
+                    x1 = f2_mask(x1, j + 2 > row, j + 3 > row);
+                    x2 = f2_mask(x2, j + 32 > row, j + 33 > row);
+                    x3 = f2_mask(x3, j + 34 > row, j + 35 > row);
+                }
+                pk[2 * q] = pk_bf16(f2_lo(x0), f2_hi(x0));
+                pk[2 * q + 1] = pk_bf16(f2_lo(x1), f2_hi(x1));
+                pk[16 + 2 * q] = pk_bf16(f2_lo(x2), f2_hi(x2));
+                pk[16 + 2 * q + 1] = pk_bf16(f2_lo(x3), f2_hi(x3));
             }
             // keys [64w, 64w+64) -> columns [64w, 64w+32) of the buffer
             tmem_st32(tS(b) + lane_base + k0, pk);
