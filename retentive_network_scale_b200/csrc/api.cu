@@ -2,6 +2,7 @@
 // parameter set-up and dispatch to the kernels.  Every check runs before
 // any CUDA call, so a rejected call touches no device state.
 #include <atomic>
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -151,13 +152,23 @@ size_t ret_workspace_size(const ret_desc *desc, int chunk, int want_O, int want_
     return 0;
 }
 
+namespace {
+// The chunk loop's CTAs (one per head and 128 value columns) would leave most
+// of the 148 SMs idle.
+bool few_heads(const ret::Params &p) { return (long long)p.B * p.H * ((p.dv + 127) / 128) < 64; }
+}  // namespace
+
 size_t ret_chunkwise_fast_size(const ret_desc *desc, int chunk) {
     if (check_desc(desc) != RET_OK || chunk < 1 || (long long)desc->B * desc->L == 0) return 0;
     Params p;
     make_params(desc, &p);
     if (!chunkwise_tc_supported(p, chunk, desc->in_dtype == RET_BF16)) return 0;
     const int S = auto_segments(p, chunk);
-    return S > 1 ? segmented_bytes(p, S) : chunkwise_prep_bytes(p);
+    size_t bytes = S > 1 ? segmented_bytes(p, S) : chunkwise_prep_bytes(p);
+    // few heads on the one-launch shapes: room for its block sums too (a call
+    // with a carried state takes the segments or the loop instead)
+    if (few_heads(p) && onepass_supported(p, true, false)) bytes = std::max(bytes, onepass_bytes(p));
+    return bytes;
 }
 
 size_t ret_chunkwise_prep_size(const ret_desc *desc, int chunk) {
@@ -254,8 +265,13 @@ ret_status ret_chunkwise(const ret_desc *desc, int chunk, const void *Q, const v
     if (chunkwise_tc_supported(p, chunk, in_bf16)) {
         int *status = device_status_word();
         if (!status) return RET_ERR_CUDA;
-        // few (b, h) heads and room for the segment states: every sequence
-        // cut into segments that run at once
+        // few (b, h) heads: every block of every sequence at once in one
+        // launch (the one-launch shapes, no carried state, room for the block
+        // sums), else every sequence cut into segments that run at once
+        if (few_heads(p) && onepass_supported(p, in_bf16, state_in || state_out) && workspace &&
+            workspace_bytes >= onepass_bytes(p))
+            return from_cuda(launch_onepass(p, out_bf16, Q, K, V, O, G, Y, gn_eps, workspace, status,
+                                            st));
         const int S = auto_segments(p, chunk);
         if (S > 1 && workspace && workspace_bytes >= segmented_bytes(p, S))
             return from_cuda(launch_segmented(p, S, out_bf16, Q, K, V, state_in, state_out, O, G,

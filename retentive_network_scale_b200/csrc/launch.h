@@ -169,6 +169,17 @@ cudaError_t launch_segmented(const Params &p, int S, bool out_bf16, const void *
                              const void *G, void *Y, float eps, void *workspace, int *status,
                              cudaStream_t st);
 
+// The chunkwise form in one launch for few heads (onepass.cu): one CTA per
+// block of 128 rows of every head, each taking its entering state from the
+// key-value sums the head's earlier blocks publish to the workspace
+// (onepass_bytes).  d_k and d_v 64 or 128, bf16, no rotation, no carried
+// state, at most 32 blocks per head; writes Y (with G) and/or O.
+bool onepass_supported(const Params &p, bool in_bf16, bool has_state);
+size_t onepass_bytes(const Params &p);
+cudaError_t launch_onepass(const Params &p, bool out_bf16, const void *Q, const void *K,
+                           const void *V, void *O, const void *G, void *Y, float eps,
+                           void *workspace, int *status, cudaStream_t st);
+
 // Tensor-core parallel form: bf16 inputs, d_k 64, 128 or 256, d_v 64 or a
 // multiple of 128, every gamma_h^127 >= 2^-60.  With rotation it first writes the turned
 // Q^ and K^ (bf16) into the workspace (parallel_tc_workspace bytes).

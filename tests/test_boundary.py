@@ -324,7 +324,8 @@ def test_static_entry_checks_arguments_before_its_scratch_limit(lib):
 def test_fast_size(lib):
     """ret_chunkwise_fast_size: the streaming pass's room for shapes with
     enough heads, the segmented layout (segments keeping one wave of CTAs,
-    at least 512 rows each) for few heads, 0 off the tensor-core path."""
+    at least 512 rows each) for few heads, or the one-launch path's block
+    sums where they are larger, 0 off the tensor-core path."""
     bf = R.RET_BF16
     fast = lambda d, chunk=128: lib.ret_chunkwise_fast_size(ctypes.byref(d), chunk)  # noqa: E731
     prep = lambda d, chunk=128: lib.ret_chunkwise_prep_size(ctypes.byref(d), chunk)  # noqa: E731
@@ -335,10 +336,17 @@ def test_fast_size(lib):
     # 2 heads x 1 value tile: 8 segments of 256 rows would be too short, 4 of 512 qualify
     few = desc(B=1, H=2, L=2048, d_k=128, d_v=128, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
     assert fast(few) == seg(few, 4) > prep(few) > 0
-    # msr_small's shape: 32 heads of d_v 64, 4 segments of 512 rows (128 CTAs)
+    # msr_small's shape: 32 heads of d_v 64, no rotation: room for the
+    # one-launch path's block sums (B*H*16 blocks of a 64 x 64 fp32 sum, then
+    # a flag per block) or for 4 segments of 512 rows, whichever is larger
     small = desc(B=4, H=8, L=2048, d_k=64, d_v=64, in_dtype=bf, out_dtype=bf,
                  gamma=[0.9] * 8, rotate=False)
-    assert fast(small, 64) == seg(small, 4, 64) > 0
+    onepass = 4 * 8 * 16 * 64 * 64 * 4 + 4 * 8 * 16 * 4
+    assert fast(small, 64) == max(seg(small, 4, 64), onepass) > 0
+    # the same with rotation: the segments only
+    small_rot = desc(B=4, H=8, L=2048, d_k=64, d_v=64, in_dtype=bf, out_dtype=bf,
+                     gamma=[0.9] * 8, rotate=True)
+    assert fast(small_rot, 64) == seg(small_rot, 4, 64) > 0
     # rows that do not split into segments of 512: the streaming pass only
     odd = desc(B=1, H=2, L=1000, d_k=128, d_v=128, in_dtype=bf, out_dtype=bf, gamma=[0.9, 0.99])
     assert fast(odd) == prep(odd) > 0

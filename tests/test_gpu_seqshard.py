@@ -163,7 +163,9 @@ def test_chunkwise_takes_segments_for_few_heads(L, dk, dv, rotate, segs):
     Y_ref = orc.gate_groupnorm(O_ref, G)
     desc = R.make_desc(B, H, L, dk, dv, R.RET_BF16, R.RET_BF16, g, rotate, 10000.0, 9)
     lib = R.load_library()
-    assert lib.ret_chunkwise_fast_size(ctypes.byref(desc), 128) == \
+    # (at least the segments' bytes: the one-launch path's block sums may
+    # need more, but a call with a carried state takes the segments)
+    assert lib.ret_chunkwise_fast_size(ctypes.byref(desc), 128) >= \
         lib.ret_chunkwise_segmented_workspace_size(ctypes.byref(desc), 128, segs)
     Qd, Kd, Vd, Gd, S0d = Q.cuda(), K.cuda(), V.cuda(), G.cuda(), S0.cuda()
     O = torch.empty(B, H, L, dv, device="cuda", dtype=torch.bfloat16)
