@@ -533,7 +533,8 @@ def bench_msr_small(R, pk, reps=50):
     tf_p = fl_p / (ms_p * 1e-3) / 1e12
     return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d_k={w.d_k} d_v={w.d_v} chunk={w.chunk}, "
                         f"no rotation, Y = swish(G) GroupNorm(O), bf16; L2 flushed before each call; "
-                        f"the chunkwise call in segments (fast-path workspace)",
+                        f"the chunkwise call in one launch, every 128-row block at once (fast-path "
+                        f"workspace)",
             "chunkwise_ms": ms_c, "tokens_per_s": w.B * w.L / (ms_c * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "bytes": alg_bytes,
