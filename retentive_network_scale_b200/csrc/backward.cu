@@ -264,10 +264,11 @@ cudaError_t unturn_sum(const Params &p, int d, const float *part0, const float *
 
 // One retention product on the tensor cores: query/key rows read through
 // `qk` (column offset already in the pointers), value rows [B][H][L][dv']
-// contiguous, fp32 output [B][H][L][dv'].
+// contiguous, fp32 output [B][H][L][dv'].  With acc_in the output is
+// acc_in + the product, turned back by the rows' angles when `unturn`.
 cudaError_t product(const Params &base, int dqk, int dval, const void *q, const void *k,
                     RowLayout qk, const void *v, bool anti, void *prep_ws, float *out, int *status,
-                    cudaStream_t st) {
+                    cudaStream_t st, const float *acc_in = nullptr, bool unturn = false) {
     Params p = base;
     p.dk = dqk;
     p.dv = dval;
@@ -277,8 +278,9 @@ cudaError_t product(const Params &base, int dqk, int dval, const void *q, const 
     const void *qh = nullptr, *kt = nullptr;
     cudaError_t e = launch_chunkwise_prep_strided(p, 128, q, k, qk, false, prep_ws, &qh, &kt, st);
     if (e != cudaSuccess) return e;
-    return launch_chunkwise_tc_prepared(p, false, qh, qk, kt, v, bhld_layout(p, dval), true,
-                                        nullptr, RowLayout{0, 0, 0}, nullptr, out, 0.f, status, st);
+    return launch_chunkwise_ws(p, false, qh, qk, kt, bhld_layout(p, dqk), v, bhld_layout(p, dval), true,
+                               nullptr, nullptr, out, nullptr, RowLayout{0, 0, 0}, nullptr, 0.f, false,
+                               false, status, st, acc_in, unturn ? 1 : 0);
 }
 
 bool dims_ok(const ret_desc *d) {
@@ -358,12 +360,19 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
     const int n = split_dv(dv, w);
     const RowLayout full_v = bhld_layout(p, dv);
     const auto *dO8 = static_cast<const uint8_t *>(dO), *V8 = static_cast<const uint8_t *>(V);
+    // In fp32 with two column blocks, the second block's products add the
+    // first block's partials and turn the sums back in their epilogue,
+    // writing dQ and dK themselves (no sum pass).
+    const bool fold = desc->out_dtype == RET_F32 && n == 2;
     for (int i = 0, c0 = 0; i < n && e == cudaSuccess; c0 += w[i], ++i) {
         const size_t off = (size_t)c0 * 2;
+        const bool last = fold && i == 1;
         run(product(p, w[i], dk, dO8 + off, V8 + off, full_v, Kh, false, prep,
-                    partA + i * part_stride, status, st));
+                    last ? static_cast<float *>(dQ) : partA + i * part_stride, status, st,
+                    last ? partA : nullptr, rot));
         run(product(p, w[i], dk, V8 + off, dO8 + off, full_v, Qh, true, prep,
-                    partB + i * part_stride, status, st));
+                    last ? static_cast<float *>(dK) : partB + i * part_stride, status, st,
+                    last ? partB : nullptr, rot));
     }
     // 3. dV (anti-causal: K^, Q^, dO)
     run(product(p, dk, dv, Kh, Qh, bhld_layout(p, dk), dO, true, prep, partC, status, st));
@@ -374,11 +383,11 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
         run(unturn_sum<__nv_bfloat16>(p, dk, partA, a1, false, rot, dQ, st));
         run(unturn_sum<__nv_bfloat16>(p, dk, partB, b1, false, rot, dK, st));
         run(unturn_sum<__nv_bfloat16>(p, dv, partC, nullptr, false, false, dV, st));
-    } else {
+    } else if (!fold) {
         run(unturn_sum<float>(p, dk, partA, a1, false, rot, dQ, st));
         run(unturn_sum<float>(p, dk, partB, b1, false, rot, dK, st));
-        if (!dv_direct) run(unturn_sum<float>(p, dv, partC, nullptr, false, false, dV, st));
     }
+    // (fp32 dV was written by its product)
     return e == cudaSuccess ? RET_OK : RET_ERR_CUDA;
 }
 

@@ -398,7 +398,8 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const float *__restrict__ state_in, float *__restrict__ state_out,
                     TO *__restrict__ O, const __nv_bfloat16 *__restrict__ G, long long g_row,
                     long long g_batch, TO *__restrict__ Y, float gn_eps, int zeta_v,
-                    int v_head_major, int *status) {
+                    int v_head_major, int *status, const float *__restrict__ acc_in,
+                    int acc_unturn) {
     using Ly = Layout<DK>;
     constexpr int KB = DK / 64;
     constexpr uint32_t kIdescU = idesc_bf16(128, DK, 1, 1);  // R^T += V'^T K' (both MN-major)
@@ -853,7 +854,44 @@ chunkwise_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     tc_fence_before();
                     warp_arrive(OF);  // the next chunk's O'' may overwrite tensor memory
                 }
-                if (O)
+                bool plain = O != nullptr;
+                if constexpr (!FUSE) {
+                    if (O && acc_in) {
+                        // O = acc_in + this product, turned back by the angles of
+                        // the row's position when acc_unturn (the second half of
+                        // a backward gradient: the partial sum, then Theta_t^T)
+                        plain = false;
+                        const int col0 = v0 + o0 + 32 * hf;
+                        float v[32];
+                        const bool mine = ocols && row < n;
+                        const float *ar = acc_in + ((size_t)bh * L + t0 + row) * dv + col0;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 a4 = mine ? *reinterpret_cast<const float4 *>(ar + 4 * q)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                            const uint64_t s0 = f2_mul(f2_of(x + 4 * q), A2), s1 = f2_mul(f2_of(x + 4 * q + 2), A2);
+                            v[4 * q] = a4.x + f2_lo(s0);
+                            v[4 * q + 1] = a4.y + f2_hi(s0);
+                            v[4 * q + 2] = a4.z + f2_lo(s1);
+                            v[4 * q + 3] = a4.w + f2_hi(s1);
+                        }
+                        if (acc_unturn) {
+                            const long long pos = p.pos_offset + t0 + row;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                float c, sn;
+                                rot_cs_fast(pos, p.theta[col0 / 2 + e], &c, &sn);
+                                const float a0 = v[2 * e], a1 = v[2 * e + 1];
+                                v[2 * e] = a0 * c + a1 * sn;
+                                v[2 * e + 1] = a1 * c - a0 * sn;
+                            }
+                        }
+                        store_row32<TO>([&](int k) { return f2_make(v[2 * k], v[2 * k + 1]); }, m4, 32 * hf,
+                                        [&](int i) { return O + ((size_t)bh * L + t0 + grow(i)) * dv + v0 + o0; },
+                                        row_ok);
+                    }
+                }
+                if (plain)
                     store_row32<TO>([&](int k) { return f2_mul(f2_of(x + 2 * k), A2); }, m4, 32 * hf,
                                     [&](int i) { return O + ((size_t)bh * L + t0 + grow(i)) * dv + v0 + o0; },
                                     row_ok);
@@ -920,7 +958,8 @@ template <int DK, typename TO, bool FUSE, bool REV = false, bool ROT = false>
 cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                      const void *G, RowLayout g, void *Y, float eps, int zeta_v,
-                     int v_head_major, int *status, cudaStream_t st) {
+                     int v_head_major, int *status, cudaStream_t st,
+                     const float *acc_in = nullptr, int acc_unturn = 0) {
     auto kern = chunkwise_ws_kernel<DK, TO, FUSE, REV, ROT>;
     const int smem = (int)Layout<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -939,7 +978,7 @@ cudaError_t launch_t(const Params &p, const CUtensorMap &mq, const CUtensorMap &
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p, s_in, s_out, (TO *)O,
                            (const __nv_bfloat16 *)G, g.row, g.batch, (TO *)Y, eps, zeta_v,
-                           v_head_major, status);
+                           v_head_major, status, acc_in, acc_unturn);
     if (e == cudaSuccess) note_launches(1);
     return e;
 }
@@ -948,16 +987,20 @@ template <int DK>
 cudaError_t launch_dk(const Params &p, bool out_bf16, const CUtensorMap &mq, const CUtensorMap &mk,
                       const CUtensorMap &mv, const float *s_in, float *s_out, void *O,
                       const void *G, RowLayout g, void *Y, float eps, int zeta_v, int vhm, bool rot,
-                      int *status, cudaStream_t st) {
+                      int *status, cudaStream_t st, const float *acc_in, int acc_unturn) {
     const bool fuse = Y != nullptr;
+    if (acc_in && (out_bf16 || fuse || rot)) return cudaErrorInvalidValue;
     if (p.reverse) {
         // the anti-causal products of the backward pass: fp32 O, no gate
         if constexpr (DK >= 128) {
             if (!out_bf16 && !fuse && !rot)
-                return launch_t<DK, float, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm, status, st);
+                return launch_t<DK, float, false, true>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm,
+                                                        status, st, acc_in, acc_unturn);
         }
         return cudaErrorInvalidValue;
     }
+    if (acc_in) return launch_t<DK, float, false>(p, mq, mk, mv, s_in, s_out, O, G, g, Y, eps, zeta_v, vhm,
+                                                  status, st, acc_in, acc_unturn);
     if (rot) {
         // xPos turn of the landed tiles inside the loop (d_k 128 and 256)
         if constexpr (DK >= 128) {
@@ -983,7 +1026,7 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
                                 bool zeta_on_v, bool rotate_in_loop, int *status,
-                                cudaStream_t st) {
+                                cudaStream_t st, const float *acc_in, int acc_unturn) {
     CUtensorMap mq, mk, mv;
     const int bh = p.B * p.H;
     if (!make_tma_map_bf16_strided(&mq, Q, p.dk, p.L, bh, q_layout.row, q_layout.head, kC) ||
@@ -996,10 +1039,10 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
     if (!ok) return cudaErrorInvalidValue;
     const int zv = zeta_on_v ? 1 : 0, vhm = v_head_major ? 1 : 0;
     if (p.dk == 256)
-        return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
+        return launch_dk<256>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st, acc_in, acc_unturn);
     if (p.dk == 64)
-        return launch_dk<64>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
-    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st);
+        return launch_dk<64>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st, acc_in, acc_unturn);
+    return launch_dk<128>(p, out_bf16, mq, mk, mv, s_in, s_out, O, G, g_layout, Y, eps, zv, vhm, rotate_in_loop, status, st, acc_in, acc_unturn);
 }
 
 }  // namespace ret

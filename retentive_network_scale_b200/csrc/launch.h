@@ -97,13 +97,16 @@ cudaError_t launch_chunkwise_tc_prepared(const Params &p, bool out_bf16, const v
 // (the streaming pass).  rotate_in_loop: Q and K are the raw rows and the
 // kernel turns the landed tiles (and weights the keys) in shared memory
 // itself (d_k 128 or 256, plain heads).  Writes Y ([B][L][H*d_v], with G)
-// and/or O ([B][H][L][d_v]) in the output dtype.
+// and/or O ([B][H][L][d_v]) in the output dtype.  acc_in (fp32 O only, no
+// gate, prepared rows): O = acc_in + the product, turned back by the angles
+// of each row's position (Theta_t^T) when acc_unturn.
 cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, RowLayout q_layout,
                                 const void *K, RowLayout k_layout, const void *V, RowLayout v_layout,
                                 bool v_head_major, const float *s_in, float *s_out, void *O,
                                 const void *G, RowLayout g_layout, void *Y, float eps,
                                 bool zeta_on_v, bool rotate_in_loop, int *status,
-                                cudaStream_t st);
+                                cudaStream_t st, const float *acc_in = nullptr,
+                                int acc_unturn = 0);
 
 // The streaming pass reading Q and K through a layout; with always_q it
 // writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),
