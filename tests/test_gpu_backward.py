@@ -28,6 +28,7 @@ def _lib():
     (128, 128, True, torch.float32),
     (256, 384, False, torch.float32),
     (128, 512, True, torch.bfloat16),
+    (256, 512, True, torch.float32),   # the second column block folds the sums and the turn in
 ])
 def test_backward_matches_oracle(dk, dv, rotate, out):
     B, H, L = 2, 2, 300
