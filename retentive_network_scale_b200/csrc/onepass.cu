@@ -13,7 +13,8 @@
 // gate, Y = swish(G) (.) GroupNorm_h(O) over the head's d_v columns (section
 // 2.2), all of which this CTA holds.
 //
-// One CTA of 8 warps per (b, h, block), blockIdx.x = block + blocks * (b, h):
+// One CTA per (b, h, block), blockIdx.x = block + blocks * (b, h) (4 warps
+// for d_v = 64, 8 for d_v = 128; see OCfg):
 //   1. TMA loads of the block's Q, K, V tiles; K scaled to K~ in shared memory
 //   2. U^T = V^T K~ on the tensor cores, read out and published to the
 //      workspace with a flag (release at GPU scope)
@@ -23,10 +24,10 @@
 //   5. O'' = Q Rbar + P V; the epilogue (decay scale, GroupNorm, gate) writes
 //      Y or O
 // A CTA waits only on CTAs of lower index of the same launch, which start
-// before it; shared memory is sized so at most two CTAs share an SM, and two
-// tensor-memory allocations of 256 columns fit in an SM's 512, so no
-// resident CTA waits for one that cannot start.  The flags are zeroed
-// (a memset on the stream) before each launch.
+// before it; the CTAs an SM can hold (by their registers: four of 128
+// threads, or two of 256) fit its 512 tensor-memory columns together (128 or
+// 256 each), so no resident CTA waits for one that cannot start.  The flags
+// are zeroed (a memset on the stream) before each launch.
 //
 // Shapes: d_k 64 or 128, d_v 64 or 128, bf16, no rotation, no carried state,
 // at most kMaxBlocks blocks per head.  Every wait is bounded (about 2 s of SM
