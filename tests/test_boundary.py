@@ -209,6 +209,24 @@ def test_host_pipeline_arguments(lib):
     assert call(ws=FAKE, ws_bytes=size(2) - 1) == S("RET_ERR_WORKSPACE")
 
 
+def test_gemm_arguments(lib):
+    """ret_gemm_bf16 checks its sizes, leading dimensions, pointers and
+    alignment before any CUDA call, and refuses a machine without sm_100."""
+    S = R.STATUS_NAMES.index
+    g = lambda M=256, N=256, K=64, A=FAKE, lda=64, B=FAKE, ldb=256, C=FAKE, ldc=256: \
+        lib.ret_gemm_bf16(M, N, K, A, lda, B, ldb, C, ldc, None)  # noqa: E731
+    assert g(M=-1) == S("RET_ERR_ARG")
+    assert g(M=0) == S("RET_OK") and g(N=0) == S("RET_OK")        # empty: nothing launched
+    assert g(N=12, ldb=16, ldc=16) == S("RET_ERR_SHAPE")           # N not a multiple of 8
+    assert g(K=0) == S("RET_ERR_SHAPE")
+    assert g(lda=32) == S("RET_ERR_SHAPE")                          # lda < K
+    assert g(ldb=260) == S("RET_ERR_SHAPE")                         # not a multiple of 8
+    assert g(A=None) == S("RET_ERR_NULL")
+    assert g(C=FAKE + 2) == S("RET_ERR_ALIGN")
+    if not torch.cuda.is_available():
+        assert g() == S("RET_ERR_UNSUPPORTED")
+
+
 def test_selftest_wait_timeout_arguments(lib):
     S = R.STATUS_NAMES.index
     assert lib.ret_selftest_wait_timeout(999, None) == S("RET_ERR_ARG")
