@@ -54,3 +54,24 @@ def test_msr_layer_refusals():
         R.ret_msr_layer(X, W, Wo, [0.9, 0.99], 96, 128, 128)
     with pytest.raises(R.RetentionError, match="RET_ERR_SHAPE"):   # gamma^128 below 2^-60
         R.ret_msr_layer(X, W, Wo, [0.5, 0.99], 128, 128, 128)
+
+
+def test_msr_layer_full_size_sampled():
+    """The RetNet-1.3B layer at full size (B=8 L=4096 d_model=2048 H=8
+    d_k=256 d_v=512, chunk 128, xPos: the benchmarked shapes, 128 x 48 tiles
+    of the projection GEMM, positions up to 4095 in its turn epilogue); batch
+    element 0, every row and column, against the fp64 layer oracle on that
+    element alone (a row of the layer depends only on its own sequence)."""
+    from retentive_network_scale_b200.synth import WORKLOADS
+    w = WORKLOADS["msr_1p3b"]
+    dm = w.H * w.d_k
+    n_proj = w.H * (2 * w.d_k + 2 * w.d_v)
+    X = random_tensor((w.B, w.L, dm), 710).bfloat16()
+    W = random_tensor((dm, n_proj), 711, dm ** -0.5).bfloat16()
+    Wo = random_tensor((w.H * w.d_v, dm), 712, (w.H * w.d_v) ** -0.5).bfloat16()
+    out = R.ret_msr_layer(X.cuda(), W.cuda(), Wo.cuda(), R.msr_gammas(w.H), w.chunk, w.d_k, w.d_v,
+                          rotate=True)
+    torch.cuda.synchronize()
+    assert R.ret_last_device_status() == 0
+    ref = orc.msr_layer(X[:1], W, Wo, orc.gammas(w.H), w.d_k, w.d_v, rotate=True)
+    assert rel_l2(out[0], ref[0]) <= TOL_BF16
