@@ -76,9 +76,11 @@ def _bind(lib):
         ctypes.POINTER(ctypes.c_longlong), d]
     lib.oracle_gate_groupnorm.argtypes = [ctypes.c_int] * 4 + [
         d, d, ctypes.c_double, d]
+    lib.oracle_gate_groupnorm_backward.argtypes = [ctypes.c_int] * 4 + [
+        d, d, d, ctypes.c_double, d, d]
     for f in ("oracle_retention_parallel", "oracle_retention_recurrent",
               "oracle_retention_chunkwise", "oracle_retention_rows",
-              "oracle_gate_groupnorm"):
+              "oracle_gate_groupnorm", "oracle_gate_groupnorm_backward"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -225,6 +227,18 @@ def gate_groupnorm(O, G, eps=1e-5, lib=None) -> np.ndarray:
     _check(lib.oracle_gate_groupnorm(B, L, H, dv, _ptr(O), _ptr(G), float(eps), _ptr(Y)),
            "gate_groupnorm")
     return Y
+
+
+def gate_groupnorm_backward(O, G, dY, eps=1e-5, lib=None):
+    """Gradients (dO, dG) of Y = gate_groupnorm(O, G) given dY.  O, dO
+    [B, H, L, dv]; G, dY, dG [B, L, H*dv]."""
+    lib = lib or load()
+    O, G, dY = _f64(O), _f64(G), _f64(dY)
+    B, H, L, dv = O.shape
+    dO, dG = np.zeros_like(O), np.zeros_like(G)
+    _check(lib.oracle_gate_groupnorm_backward(B, L, H, dv, _ptr(O), _ptr(G), _ptr(dY), float(eps),
+                                              _ptr(dO), _ptr(dG)), "gate_groupnorm_backward")
+    return dO, dG
 
 
 def msr_layer(X, W_qkvg, W_o, gamma, d_k, d_v, rotate=False, theta_base=10000.0, pos_offset=0,

@@ -392,3 +392,54 @@ int oracle_gate_groupnorm(int B, int L, int H, int dv, const double *O,
             }
     return 0;
 }
+
+/* Gradients of the section 2.2 output Y = swish(G) (.) GroupNorm_h(O) above,
+ * for a given dY, by the chain rule through its three steps, per (b, t, h)
+ * row of dv channels, fp64:
+ *   n_c = (o_c - mu) r with r = 1 / sqrt(var + eps)   (the normalised row)
+ *   Y_c = s(g_c) n_c, s(g) = g sigmoid(g)
+ *   dG_c = dY_c n_c s'(g_c), s'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)))
+ *   dn_c = dY_c s(g_c)
+ *   dO_c = r (dn_c - mean_j dn_j - n_c mean_j (dn_j n_j))
+ * The last line is the derivative of the normalisation: mu and var both
+ * depend on every o_j of the row (d mu / d o_j = 1/dv, d var / d o_j =
+ * 2 (o_j - mu) / dv).  Layouts as in oracle_gate_groupnorm; dY and dG share
+ * G's, dO shares O's. */
+int oracle_gate_groupnorm_backward(int B, int L, int H, int dv, const double *O,
+                                   const double *G, const double *dY, double eps,
+                                   double *dO, double *dG)
+{
+    if (B < 0 || L < 0 || H < 0 || dv < 1 || eps < 0.0) return 1;
+    double *n = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *dn = (double *)malloc(sizeof(double) * (size_t)dv);
+    if (!n || !dn) { free(n); free(dn); return 2; }
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < L; ++t)
+            for (int h = 0; h < H; ++h) {
+                size_t orow = (((size_t)b * H + h) * L + t) * dv;
+                size_t gy = ((size_t)b * L + t) * (size_t)H * dv + (size_t)h * dv;
+                const double *o = O + orow;
+                double mu = 0.0, var = 0.0;
+                for (int c = 0; c < dv; ++c) mu += o[c];
+                mu /= (double)dv;
+                for (int c = 0; c < dv; ++c) var += (o[c] - mu) * (o[c] - mu);
+                var /= (double)dv;
+                double r = 1.0 / sqrt(var + eps);
+                double mean_dn = 0.0, mean_dnn = 0.0;
+                for (int c = 0; c < dv; ++c) {
+                    double gv = G[gy + c];
+                    double sig = 1.0 / (1.0 + exp(-gv));
+                    n[c] = (o[c] - mu) * r;
+                    dn[c] = dY[gy + c] * gv * sig;
+                    dG[gy + c] = dY[gy + c] * n[c] * sig * (1.0 + gv * (1.0 - sig));
+                    mean_dn += dn[c];
+                    mean_dnn += dn[c] * n[c];
+                }
+                mean_dn /= dv;
+                mean_dnn /= dv;
+                for (int c = 0; c < dv; ++c)
+                    dO[orow + c] = r * (dn[c] - mean_dn - n[c] * mean_dnn);
+            }
+    free(n); free(dn);
+    return 0;
+}

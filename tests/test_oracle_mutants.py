@@ -35,6 +35,12 @@ MUTANTS = {
     "unbiased_var": ("var /= dv;", "var /= (dv - 1);"),
     # zeta applied as gamma^{j'} instead of gamma^{n-1-j'}
     "zeta_index": ("double zeta = pow(g, (double)(n - 1 - jj));", "double zeta = pow(g, (double)(jj));"),
+    # normalisation gradient without the variance term
+    "gn_grad_no_var_term": ("dO[orow + c] = r * (dn[c] - mean_dn - n[c] * mean_dnn);",
+                            "dO[orow + c] = r * (dn[c] - mean_dn);"),
+    # swish derivative taken as sigmoid(g) alone
+    "swish_grad": ("dG[gy + c] = dY[gy + c] * n[c] * sig * (1.0 + gv * (1.0 - sig));",
+                   "dG[gy + c] = dY[gy + c] * n[c] * sig;"),
     # gamma schedule 1 - 2^(-4-h)
     "gamma_schedule": ("gamma[h] = 1.0 - pow(2.0, -5.0 - (double)h);",
                        "gamma[h] = 1.0 - pow(2.0, -4.0 - (double)h);"),

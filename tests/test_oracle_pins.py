@@ -222,10 +222,42 @@ def pin_gate_groupnorm(lib):
     assert np.abs(Yn.var(-1) - var / (var + eps)).max() < 1e-10
 
 
+def pin_gate_groupnorm_backward(lib):
+    """Gradients of section 2.2's GroupNorm + swish gate against central
+    finite differences of the forward oracle along random directions:
+    d/de <dY, Y(O + e U, G + e W)> at 0 equals <dO, U> + <dG, W>.  This only
+    runs the forward, so it is independent of the gradient formulas.  Plus
+    what the mathematics fixes: every dO row sums to 0 (adding a constant to
+    a row leaves its normalisation unchanged), and at G = 0 dO is 0 and dG is
+    dY times the normalised row over 2 (swish'(0) = 1/2)."""
+    rng = _rng(21)
+    B, H, L, dv = 2, 3, 4, 8
+    O = rng.normal(size=(B, H, L, dv)) * 2 + 0.5
+    G = rng.normal(size=(B, L, H * dv)) * 1.5
+    dY = rng.normal(size=(B, L, H * dv))
+    eps = 1e-3
+    dO, dG = orc.gate_groupnorm_backward(O, G, dY, eps, lib=lib)
+    f = lambda o, g: float(np.sum(dY * orc.gate_groupnorm(o, g, eps, lib=lib)))  # noqa: E731
+    h = 1e-6
+    for _ in range(3):
+        U = rng.normal(size=O.shape)
+        W = rng.normal(size=G.shape)
+        for u, w in ((U, 0 * W), (0 * U, W), (U, W)):
+            fd = (f(O + h * u, G + h * w) - f(O - h * u, G - h * w)) / (2 * h)
+            an = float(np.sum(dO * u) + np.sum(dG * w))
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (fd, an)
+    assert np.abs(dO.sum(-1)).max() < 1e-12
+    dO0, dG0 = orc.gate_groupnorm_backward(O, np.zeros_like(G), dY, eps, lib=lib)
+    assert np.abs(dO0).max() == 0
+    mu = O.mean(-1, keepdims=True)
+    n = ((O - mu) / np.sqrt(O.var(-1, keepdims=True) + eps)).transpose(0, 2, 1, 3)
+    assert _normwise(dG0, 0.5 * dY * n.reshape(B, L, H * dv)) < 1e-13
+
+
 PINS = [pin_gamma_schedule, pin_three_forms_agree, pin_linear_attention,
         pin_gamma_zero, pin_single_token, pin_rotation_closed_forms,
         pin_offset_invariance, pin_state_closed_form, pin_state_handoff,
-        pin_gate_groupnorm]
+        pin_gate_groupnorm, pin_gate_groupnorm_backward]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
