@@ -400,10 +400,32 @@ def bench_backward(R, w, d, pk, reps=3):
     per = 2 * fl(w.d_v, w.d_k) + fl(w.d_k, w.d_v)   # dQ^, dK^ (over d_v), dV
     flops = w.B * w.H * w.L * per
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": f"retention backward (dQ, dK, dV fp32) on {w.name}", "ms": ms,
+    out = {"workload": f"retention backward (dQ, dK, dV fp32) on {w.name}", "ms": ms,
+           "tokens_per_s": w.B * w.L / (ms * 1e-3),
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
+    del dQ, dK, dV, ws
+    out["gate_norm_backward"] = bench_gate_backward(R, w, d, pk, gen, reps=max(5, reps))
+    return out
+
+
+def bench_gate_backward(R, w, d, pk, gen, reps=20):
+    """dO and dG of the GroupNorm + swish gate given dY (bf16 O, G, dY, dO,
+    dG): one streaming kernel, HBM-bound.  Its inputs (0.8 GB) exceed L2."""
+    O = torch.randn(w.B, w.H, w.L, w.d_v, device="cuda", generator=gen).bfloat16()
+    dY = torch.randn(w.B, w.L, w.H * w.d_v, device="cuda", generator=gen).bfloat16()
+    dO = torch.empty_like(O)
+    dG = torch.empty_like(dY)
+    fn = lambda: R.ret_gate_norm_backward(O, d["G"], dY, dO, dG, 1e-5)  # noqa: E731
+    for _ in range(3):
+        fn()
+    ms = time_launches(fn, reps, torch.cuda.current_stream())
+    nbytes = 5 * O.numel() * O.element_size()  # read O, G, dY; write dO, dG
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"GroupNorm + swish gate backward (dO, dG bf16) on {w.name}", "ms": ms,
             "tokens_per_s": w.B * w.L / (ms * 1e-3),
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "flops": flops}}
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": nbytes}}
 
 
 def bench_seqshard(R, w, d, pk, reps=5, parts=8):

@@ -490,6 +490,29 @@ ret_status ret_gate_norm(int B, int L, int H, int d_v, int o_dtype,
                          const void *O, int g_dtype, const void *G, float eps,
                          int y_dtype, void *Y, void *stream);
 
+/*
+ * ret_gate_norm_backward -- gradients of section 2.2's output
+ * Y = swish(G) (.) GroupNorm_h(O) (the computation of ret_gate_norm) with
+ * respect to O and G, given dY, by the chain rule through its three steps
+ * (per (b, t, h) row of d_v channels, n = (O - mu) / sqrt(var + eps)):
+ *     dG = dY (.) n (.) swish'(G),  swish'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)))
+ *     dn = dY (.) swish(G)
+ *     dO = (dn - mean(dn) - n mean(dn (.) n)) / sqrt(var + eps)
+ * The paper summary gives the forward only; this is its derivative, the
+ * step a training pass takes before the retention backward (ret_backward
+ * takes the dO written here).
+ *   O   device o_dtype [B][H][L][d_v], the retention output of the forward
+ *   G   device g_dtype [B][L][H*d_v];  dY  device g_dtype [B][L][H*d_v]
+ *   dO  device o_dtype [B][H][L][d_v];  dG  device g_dtype [B][L][H*d_v]
+ * Both outputs are fully overwritten and must not alias an input.  fp32
+ * arithmetic.  Errors: RET_ERR_NULL, _SHAPE (as ret_gate_norm), _DTYPE,
+ * _ALIGN, _ARG (eps < 0 or not finite), _UNSUPPORTED, _CUDA.
+ */
+ret_status ret_gate_norm_backward(int B, int L, int H, int d_v, int o_dtype,
+                                  const void *O, int g_dtype, const void *G,
+                                  const void *dY, float eps, void *dO, void *dG,
+                                  void *stream);
+
 /* Synchronises `stream`, then returns and clears the device status word
  * that bounded waits in the kernels latch (RET_ERR_TIMEOUT), or
  * RET_ERR_CUDA when the stream reports an error. */

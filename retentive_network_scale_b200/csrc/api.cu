@@ -324,6 +324,25 @@ ret_status ret_gate_norm(int B, int L, int H, int d_v, int o_dtype, const void *
                                       eps, y_dtype == RET_BF16, Y, (cudaStream_t)stream));
 }
 
+ret_status ret_gate_norm_backward(int B, int L, int H, int d_v, int o_dtype, const void *O,
+                                  int g_dtype, const void *G, const void *dY, float eps, void *dO,
+                                  void *dG, void *stream) {
+    if (B < 0 || L < 0 || H < 1 || H > RET_MAX_HEADS || d_v < 1 || d_v > kMaxDv || d_v % 4)
+        return RET_ERR_SHAPE;
+    if (!valid_dtype(o_dtype) || !valid_dtype(g_dtype)) return RET_ERR_DTYPE;
+    if (!(eps >= 0.0f && std::isfinite(eps))) return RET_ERR_ARG;
+    const bool empty = (long long)B * L == 0;
+    if (!empty && (!O || !G || !dY || !dO || !dG)) return RET_ERR_NULL;
+    if (!aligned16(O) || !aligned16(G) || !aligned16(dY) || !aligned16(dO) || !aligned16(dG))
+        return RET_ERR_ALIGN;
+    ret_status s = check_device();
+    if (s != RET_OK) return s;
+    if (empty) return RET_OK;
+    return from_cuda(launch_gate_norm_backward(B, L, H, d_v, o_dtype == RET_BF16, O,
+                                               g_dtype == RET_BF16, G, dY, eps, dO, dG,
+                                               (cudaStream_t)stream));
+}
+
 unsigned long long ret_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 ret_status ret_last_device_status(void *stream) {

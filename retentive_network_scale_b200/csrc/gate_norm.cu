@@ -6,6 +6,14 @@
 // lane holds up to 16 of the row's d_v <= 512 values in registers (4-wide
 // vector loads), so the mean and the centred variance are two register
 // passes and warp reductions with no second read of memory.
+//
+// The backward (gate_norm_backward_kernel) takes dY to dO and dG by the
+// chain rule through the same three steps, with the same row ownership:
+// n = (o - mu) r, r = 1/sqrt(var + eps); dG = dY n swish'(G) with
+// swish'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))); dn = dY swish(G);
+// dO = r (dn - mean(dn) - n mean(dn n)).  O, G and dY are each read once,
+// all three requested before the first reduction and held as loaded (dn
+// in fp32) between the reductions; dO and dG are written once.
 #include "common.cuh"
 #include "launch.h"
 
@@ -13,6 +21,7 @@ namespace ret {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kThreadsB = 128;  // backward: five blocks of four warps per SM
 constexpr int kPerLane = kMaxDv / 128;  // 4-vectors per lane
 
 __device__ __forceinline__ void load4(const float *p, float *x) {
@@ -123,7 +132,159 @@ cudaError_t launch_g(bool g_bf16, bool y_bf16, int B, int L, int H, int dv,
                   : launch_y<TO_, float>(y_bf16, B, L, H, dv, O, G, eps, Y, st);
 }
 
+// Four consecutive elements as loaded (16 bytes of fp32 or 8 of bf16), so
+// that a row's three inputs can all be in flight before any arithmetic.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+    float4 v;
+    __device__ __forceinline__ void load(const float *p) { v = *reinterpret_cast<const float4 *>(p); }
+    __device__ __forceinline__ void get(float *x) const { x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w; }
+};
+template <> struct Raw4<__nv_bfloat16> {
+    uint2 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = *reinterpret_cast<const uint2 *>(p); }
+    __device__ __forceinline__ void get(float *x) const {
+        float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.x));
+        float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.y));
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    }
+};
+
+// Offsets of row r = (b, t, h): into O / dO, and into G / dY / dG.
+__device__ __forceinline__ void row_offsets(long long r, int L, int H, int dv, size_t &orow,
+                                            size_t &gy) {
+    const int h = (int)(r % H);
+    const long long bt = r / H;
+    const int t = (int)(bt % L);
+    const long long b = bt / L;
+    orow = (((size_t)b * H + h) * L + t) * dv;
+    gy = (size_t)bt * H * dv + (size_t)h * dv;
+}
+
+template <typename TO_, typename TG>
+__device__ __forceinline__ void load_row(const TO_ *O, const TG *G, const TG *dY, size_t orow,
+                                         size_t gy, int dv, int lane, Raw4<TO_> *ro,
+                                         Raw4<TG> *rg, Raw4<TG> *rdy) {
+#pragma unroll
+    for (int it = 0; it < kPerLane; ++it) {
+        int e = 128 * it + 4 * lane;
+        if (e < dv) {
+            ro[it].load(O + orow + e);
+            rg[it].load(G + gy + e);
+            rdy[it].load(dY + gy + e);
+        }
+    }
+}
+
+template <typename TO_, typename TG>
+__global__ void __launch_bounds__(kThreadsB, 5)
+gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G, const TG *dY,
+                          float eps, TO_ *dO, TG *dG) {
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)B * L * H;
+    const long long warps = (long long)gridDim.x * (kThreadsB / 32);
+    for (long long r = (long long)blockIdx.x * (kThreadsB / 32) + threadIdx.x / 32; r < rows; r += warps) {
+        size_t orow, gy;
+        row_offsets(r, L, H, dv, orow, gy);
+        // the row's O, G and dY are requested together, before the
+        // reductions that only O feeds
+        Raw4<TO_> ro[kPerLane];
+        Raw4<TG> rg[kPerLane], rdy[kPerLane];
+        load_row(O, G, dY, orow, gy, dv, lane, ro, rg, rdy);
+        // O stays as loaded; each pass converts it again, which is cheaper
+        // than holding the centred row in fp32 registers
+        float sum = 0.f;
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                float x[4];
+                ro[it].get(x);
+                sum += (x[0] + x[1]) + (x[2] + x[3]);
+            }
+        }
+        const float mu = warp_sum(sum) / (float)dv;
+        float sq = 0.f;
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                float x[4];
+                ro[it].get(x);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    x[q] -= mu;
+                    sq = fmaf(x[q], x[q], sq);
+                }
+            }
+        }
+        const float rs = rsqrtf(warp_sum(sq) / (float)dv + eps);
+        const float nshift = -mu * rs;  // n = o rs + nshift
+        // dn = dY swish(G) kept; dG written here
+        float dn[kPerLane][4];
+        float s_dn = 0.f, s_dnn = 0.f;
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                float x[4], g[4], dy[4], dg[4];
+                ro[it].get(x);
+                rg[it].get(g);
+                rdy[it].get(dy);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float sig = 1.0f / (1.0f + expf(-g[q]));
+                    const float n = fmaf(x[q], rs, nshift);
+                    dn[it][q] = dy[q] * (g[q] * sig);
+                    dg[q] = dy[q] * n * (sig * fmaf(g[q], 1.0f - sig, 1.0f));
+                    s_dn += dn[it][q];
+                    s_dnn = fmaf(dn[it][q], n, s_dnn);
+                }
+                store4(dG + gy + e, dg);
+            }
+        }
+        const float m_dn = warp_sum(s_dn) / (float)dv;
+        const float m_dnn = warp_sum(s_dnn) / (float)dv;
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                float x[4], d[4];
+                ro[it].get(x);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    d[q] = rs * (dn[it][q] - m_dn - fmaf(x[q], rs, nshift) * m_dnn);
+                store4(dO + orow + e, d);
+            }
+        }
+    }
+}
+
+template <typename TO_, typename TG>
+cudaError_t launch_backward_t(int B, int L, int H, int dv, const void *O, const void *G,
+                              const void *dY, float eps, void *dO, void *dG, cudaStream_t st) {
+    long long rows = (long long)B * L * H;
+    long long blocks = (rows + (kThreadsB / 32) - 1) / (kThreadsB / 32);
+    if (blocks > 148LL * 128) blocks = 148LL * 128;
+    gate_norm_backward_kernel<TO_, TG><<<(unsigned)blocks, kThreadsB, 0, st>>>(
+        B, L, H, dv, (const TO_ *)O, (const TG *)G, (const TG *)dY, eps, (TO_ *)dO, (TG *)dG);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
 }  // namespace
+
+cudaError_t launch_gate_norm_backward(int B, int L, int H, int dv, bool o_bf16, const void *O,
+                                      bool g_bf16, const void *G, const void *dY, float eps,
+                                      void *dO, void *dG, cudaStream_t st) {
+    if ((long long)B * L * H == 0) return cudaSuccess;
+    if (o_bf16)
+        return g_bf16 ? launch_backward_t<__nv_bfloat16, __nv_bfloat16>(B, L, H, dv, O, G, dY, eps, dO, dG, st)
+                      : launch_backward_t<__nv_bfloat16, float>(B, L, H, dv, O, G, dY, eps, dO, dG, st);
+    return g_bf16 ? launch_backward_t<float, __nv_bfloat16>(B, L, H, dv, O, G, dY, eps, dO, dG, st)
+                  : launch_backward_t<float, float>(B, L, H, dv, O, G, dY, eps, dO, dG, st);
+}
 
 cudaError_t launch_gate_norm(int B, int L, int H, int dv, bool o_bf16,
                              const void *O, bool g_bf16, const void *G,

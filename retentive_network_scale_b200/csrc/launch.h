@@ -208,4 +208,10 @@ cudaError_t launch_gate_norm(int B, int L, int H, int dv, bool o_bf16,
                              const void *O, bool g_bf16, const void *G,
                              float eps, bool y_bf16, void *Y, cudaStream_t st);
 
+// dO (O's type) and dG (G's type) of Y = swish(G) GroupNorm_h(O) given dY
+// (G's type).
+cudaError_t launch_gate_norm_backward(int B, int L, int H, int dv, bool o_bf16, const void *O,
+                                      bool g_bf16, const void *G, const void *dY, float eps,
+                                      void *dO, void *dG, cudaStream_t st);
+
 }  // namespace ret

@@ -36,8 +36,8 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_backward", "ret_backward_workspace_size",
            "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
            "ret_chunkwise_segmented", "ret_chunkwise_segmented_workspace_size",
-           "ret_recurrent_step", "ret_gate_norm", "ret_last_device_status", "ret_kernel_launches",
-           "ret_status_string")
+           "ret_recurrent_step", "ret_gate_norm", "ret_gate_norm_backward", "ret_last_device_status",
+           "ret_kernel_launches", "ret_status_string")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
 RET_MAX_DECODE_STEPS = 16
 RET_MAX_SEGMENTS = 64
@@ -118,13 +118,15 @@ def load_library(path: str = LIB_PATH):
     lib.ret_recurrent_step.argtypes = [D, vp, vp, vp, vp, vp, vp]
     lib.ret_gate_norm.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, ctypes.c_float,
                                                        ctypes.c_int, vp, vp]
+    lib.ret_gate_norm_backward.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, vp,
+                                                                ctypes.c_float, vp, vp, vp]
     lib.ret_last_device_status.argtypes = [vp]
     lib.ret_kernel_launches.argtypes = []
     lib.ret_kernel_launches.restype = ctypes.c_ulonglong
     lib.ret_status_string.argtypes = [ctypes.c_int]
     lib.ret_status_string.restype = ctypes.c_char_p
     for f in ("ret_parallel", "ret_chunkwise", "ret_chunkwise_gate_static", "ret_recurrent_step",
-              "ret_gate_norm", "ret_last_device_status"):
+              "ret_gate_norm", "ret_gate_norm_backward", "ret_last_device_status"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -612,6 +614,21 @@ def ret_gate_norm(O, G, Y, eps=1e-5, stream=None):
                              float(eps), _dtype_code(Y), _ptr(Y), _stream(stream)),
            "ret_gate_norm")
     return Y
+
+
+def ret_gate_norm_backward(O, G, dY, dO, dG, eps=1e-5, stream=None):
+    """dO, dG of Y = swish(G) (.) GroupNorm_h(O) given dY: O, dO [B,H,L,dv]
+    (O's dtype); G, dY, dG [B,L,H*dv] (G's dtype)."""
+    lib = load_library()
+    B, H, L, dv = O.shape
+    _dev(O, "O"); _dev(dO, "dO", (B, H, L, dv)); _dev(G, "G", (B, L, H * dv))
+    _dev(dY, "dY", (B, L, H * dv)); _dev(dG, "dG", (B, L, H * dv))
+    if dO.dtype != O.dtype or dY.dtype != G.dtype or dG.dtype != G.dtype:
+        raise TypeError("dO takes O's dtype; dY and dG take G's")
+    _check(lib.ret_gate_norm_backward(B, L, H, dv, _dtype_code(O), _ptr(O), _dtype_code(G),
+                                      _ptr(G), _ptr(dY), float(eps), _ptr(dO), _ptr(dG),
+                                      _stream(stream)), "ret_gate_norm_backward")
+    return dO, dG
 
 
 def ret_last_device_status(stream=None) -> int:

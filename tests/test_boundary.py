@@ -170,6 +170,19 @@ def test_gate_norm_arguments(lib):
         R.STATUS_NAMES.index("RET_ERR_NULL")
 
 
+def test_gate_norm_backward_arguments(lib):
+    SHAPE, DT = R.STATUS_NAMES.index("RET_ERR_SHAPE"), R.STATUS_NAMES.index("RET_ERR_DTYPE")
+    f = lib.ret_gate_norm_backward
+    assert f(1, 4, 2, 18, 0, FAKE, 0, FAKE, FAKE, 1e-5, FAKE, FAKE, None) == SHAPE
+    assert f(1, 4, 2, 16, 0, FAKE, 2, FAKE, FAKE, 1e-5, FAKE, FAKE, None) == DT
+    assert f(1, 4, 2, 16, 0, FAKE, 0, FAKE, FAKE, float("nan"), FAKE, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_ARG")
+    assert f(1, 4, 2, 16, 0, FAKE, 0, FAKE, None, 1e-5, FAKE, FAKE, None) == \
+        R.STATUS_NAMES.index("RET_ERR_NULL")
+    assert f(1, 4, 2, 16, 0, FAKE, 0, FAKE, FAKE, 1e-5, FAKE, MISALIGNED, None) == \
+        R.STATUS_NAMES.index("RET_ERR_ALIGN")
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the refusal on a machine without sm_100")
 def test_valid_call_without_sm100_refuses(lib):
     # zero-length problem: valid arguments, nothing would be read

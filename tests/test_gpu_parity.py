@@ -173,6 +173,59 @@ def test_gate_norm_standalone(dtype):
     assert ok, err
 
 
+@pytest.mark.parametrize("o_dtype,g_dtype", [(torch.float32, torch.float32),
+                                             (torch.bfloat16, torch.bfloat16),
+                                             (torch.float32, torch.bfloat16)])
+@pytest.mark.parametrize("dv", [64, 20, 512])
+def test_gate_norm_backward(o_dtype, g_dtype, dv):
+    """dO and dG of the GroupNorm + swish gate against the fp64 oracle's
+    chain rule, with a ragged row count, d_v below, across and at the
+    kernel's 512-channel limit."""
+    B, H, L = 2, 3, 37
+    O = (random_tensor((B, H, L, dv), 71) * 2 + 0.5).to(o_dtype)
+    G = (random_tensor((B, L, H * dv), 72) * 1.5).to(g_dtype)
+    dY = random_tensor((B, L, H * dv), 73).to(g_dtype)
+    dO_ref, dG_ref = orc.gate_groupnorm_backward(O, G, dY, 1e-5)
+    dO = torch.full((B, H, L, dv), float("nan"), device="cuda", dtype=o_dtype)
+    dG = torch.full((B, L, H * dv), float("nan"), device="cuda", dtype=g_dtype)
+    n0 = R.ret_kernel_launches()
+    R.ret_gate_norm_backward(O.cuda(), G.cuda(), dY.cuda(), dO, dG, 1e-5)
+    assert R.ret_kernel_launches() - n0 == 1
+    ok, err = within(dO, dO_ref, o_dtype)
+    assert ok, ("dO", err)
+    ok, err = within(dG, dG_ref, g_dtype)
+    assert ok, ("dG", err)
+
+
+def test_gate_norm_backward_full_size_sampled():
+    """At the msr_1p3b size the bench times (B=8 H=8 L=4096 d_v=512, bf16
+    O, G and dY): rows sampled across the batch, the sequence and the tail
+    are checked against the oracle (rows are independent), and every row of
+    dO sums to zero up to bf16 rounding."""
+    w = WORKLOADS["msr_1p3b"]
+    B, H, L, dv = w.B, w.H, w.L, w.d_v
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    O = torch.randn(B, H, L, dv, device="cuda", generator=gen).bfloat16()
+    G = torch.randn(B, L, H * dv, device="cuda", generator=gen).bfloat16()
+    dY = torch.randn(B, L, H * dv, device="cuda", generator=gen).bfloat16()
+    dO = torch.empty_like(O)
+    dG = torch.empty_like(G)
+    R.ret_gate_norm_backward(O, G, dY, dO, dG, 1e-5)
+    torch.cuda.synchronize()
+    rows = [(0, 0), (0, 1), (3, 2047), (5, 100), (7, L - 2), (7, L - 1)]
+    for b, t in rows:
+        o = O[b, :, t:t + 1, :].unsqueeze(0).cpu()
+        g = G[b, t:t + 1, :].unsqueeze(0).cpu()
+        dy = dY[b, t:t + 1, :].unsqueeze(0).cpu()
+        dO_ref, dG_ref = orc.gate_groupnorm_backward(o, g, dy, 1e-5)
+        assert rel_l2(dO[b, :, t:t + 1, :].unsqueeze(0), dO_ref) <= TOL_BF16, (b, t)
+        assert rel_l2(dG[b, t:t + 1, :].unsqueeze(0), dG_ref) <= TOL_BF16, (b, t)
+    # bf16 rounding leaves each row sum about 2^-9/sqrt(3) of the row's norm
+    f = dO.float()
+    assert bool((f.sum(-1).abs() <= 0.02 * f.norm(dim=-1) + 1e-6).all())
+
+
 # ------------------------------------------------------------------ workloads
 def test_msr_small_bf16():
     """B=4 H=8 L=2048 d=64, chunk 64, GroupNorm + swish gate: every output."""
