@@ -17,9 +17,12 @@
 //     gamma^{n - 128 b - m}, which makes up the rest of gamma^{n-1-t}.  One CTA
 // owns one (b, h) and 128 value columns (d_v = 64: the 64, the rest of its
 // V tile held at zero; d_k 64, 128 or 256) and accumulates U^T = V^T K~ in
-// tensor memory over blocks of 128 rows, which TMA brings through a ring
-// of stages; its one MMA thread also reissues each stage's loads once the
-// product that read it has completed.  The eight warps then move U^T out
+// tensor memory over blocks of rows, which TMA brings through a ring of
+// stages; its one MMA thread also reissues each stage's loads once the
+// product that read it has completed.  A stage holds 128 rows at d_k 256
+// and 64 rows at d_k 64 or 128, so that there two CTAs share an SM (96 KB
+// or less of shared memory each) and a launch of up to 296 CTAs runs as
+// one wave.  The eight warps then move U^T out
 // of tensor memory into U [d_k][d_v] (fp32), one value column per lane.
 //
 // Every wait is bounded (about 2 s): on expiry RET_ERR_TIMEOUT is latched in
@@ -36,7 +39,6 @@ namespace {
 
 using namespace tc;
 
-constexpr int kRows = 128;  // rows per block (the MMA's K extent, 8 steps of 16)
 constexpr int kTV = 128;    // value columns per CTA (MMA M)
 constexpr int kThreads = 256;                // warp 0 issues, warps 1-7 scale value rows
 constexpr int kScalers = kThreads - 32;
@@ -44,6 +46,8 @@ constexpr long long kTimeoutCycles = 4000000000LL;
 
 template <int DK>
 struct SLayout {
+    static constexpr int kRows = DK == 256 ? 128 : 64;    // rows per stage (the MMA's K extent)
+    static constexpr uint32_t kBlk = kRows * 128;         // one 64-column block of a stage
     static constexpr int kStages = DK == 256 ? 2 : DK == 128 ? 3 : 4;
     static constexpr uint32_t kVBytes = kRows * kTV * 2;  // 2 blocks of 64 columns
     static constexpr uint32_t kKBytes = kRows * DK * 2;   // DK/64 blocks of 64 columns
@@ -60,6 +64,8 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
                      const Params p, int zeta_v, float *__restrict__ U, int *status) {
     using Ly = SLayout<DK>;
     constexpr int NS = Ly::kStages;
+    constexpr int kRows = Ly::kRows;
+    constexpr uint32_t kBlk = Ly::kBlk;
     constexpr int KB = DK / 64;
     constexpr uint32_t kIdesc = idesc_bf16(128, DK, 1, 1);  // U^T += V^T K~ (both MN-major)
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -94,8 +100,8 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
         // d_v = 64: the second 64-column block of every stage's V tile is
         // never loaded and stays zero
         for (int s = 0; s < NS; ++s)
-            for (int i = tid; i < 16384 / 16; i += kThreads)
-                reinterpret_cast<uint4 *>(smem + s * Ly::kStage + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = tid; i < (int)kBlk / 16; i += kThreads)
+                reinterpret_cast<uint4 *>(smem + s * Ly::kStage + kBlk)[i] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -108,9 +114,9 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
             const uint32_t st = sbase + s * Ly::kStage;
             mbar_expect_tx(full(s), dvr * kRows * 2 + Ly::kKBytes);
             for (int nb = 0; nb < dvr / 64; ++nb)
-                tma_load_3d(st + nb * 16384, &tmV, full(s), v0 + nb * 64, blk * kRows, bh);
+                tma_load_3d(st + nb * kBlk, &tmV, full(s), v0 + nb * 64, blk * kRows, bh);
             for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(st + Ly::kVBytes + kb * 16384, &tmK, full(s), kb * 64, blk * kRows, bh);
+                tma_load_3d(st + Ly::kVBytes + kb * kBlk, &tmK, full(s), kb * 64, blk * kRows, bh);
         };
         for (int s = 0; s < NS && s < nblk; ++s) load(s, s);
         bool ok = true;
@@ -122,8 +128,8 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
             if (!ok) break;
             tc_fence_after();
             const uint32_t st = sbase + s * Ly::kStage;
-            const uint64_t dA = sdesc_sw128(st, 16384, 1024);                  // V, MN-major
-            const uint64_t dB = sdesc_sw128(st + Ly::kVBytes, 16384, 1024);    // K~, MN-major
+            const uint64_t dA = sdesc_sw128(st, kBlk, 1024);                   // V, MN-major
+            const uint64_t dB = sdesc_sw128(st + Ly::kVBytes, kBlk, 1024);     // K~, MN-major
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks) {
                 const uint64_t off = (uint64_t)((ks * 2048) >> 4);
@@ -138,9 +144,11 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
         }
         mma_commit(done);
     } else if (zeta_v && warp > 0) {
-        // V' = diag(zeta) V as each block lands, zeta_t = gamma^{L-1-t}
-        // (mode 1) or gamma^{L - 128 blk - m} for the block's m rows (mode
-        // 2): warps 1-7, one row per thread and pass (rows past L are zeros)
+        // V' = diag(zeta) V as each stage lands, zeta_t = gamma^{L-1-t}
+        // (mode 1) or gamma^{L - 128 c - m} for row t of the c-th block of
+        // 128 rows, which has m rows (mode 2, the blocks the keys were
+        // weighted in): warps 1-7, one row per thread and pass (rows past L
+        // are zeros)
         const int t = tid - 32;
         const int lane = tid & 31;
 #pragma unroll 1
@@ -154,9 +162,10 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
 #pragma unroll 1
             for (int r = t; r < kRows; r += kScalers) {
                 const int row = blk * kRows + r;
-                const int m = min(kRows, L - blk * kRows);
+                const int c0 = row - row % kChunkBlock;
+                const int m = min(kChunkBlock, L - c0);
                 const float z = row >= L ? 0.f
-                                         : decay_pow(lg, zeta_v == 1 ? L - 1 - row : L - blk * kRows - m);
+                                         : decay_pow(lg, zeta_v == 1 ? L - 1 - row : L - c0 - m);
                 const uint64_t Z = f2_make(z, z);
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb)
@@ -164,7 +173,7 @@ segment_state_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_const
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
                         // rows of a phase start at different 16-byte pieces: no bank conflicts
-                        uint4 *ptr = reinterpret_cast<uint4 *>(vt + nb * 16384 + r * 128 + (((ch + r) & 7) << 4));
+                        uint4 *ptr = reinterpret_cast<uint4 *>(vt + nb * kBlk + r * 128 + (((ch + r) & 7) << 4));
                         uint4 w = *ptr;
                         uint32_t *u = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
@@ -239,7 +248,8 @@ cudaError_t launch_segment_state_tc(const Params &p, const void *V, const void *
                                     float *U, int *status, cudaStream_t st) {
     CUtensorMap mv, mk;
     const int bh = p.B * p.H;
-    if (!make_tma_map_bf16(&mv, V, p.dv, p.L, bh, kRows) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, kRows))
+    const int rows = p.dk == 256 ? SLayout<256>::kRows : SLayout<128>::kRows;
+    if (!make_tma_map_bf16(&mv, V, p.dv, p.L, bh, rows) || !make_tma_map_bf16(&mk, Kt, p.dk, p.L, bh, rows))
         return cudaErrorInvalidValue;
     if (p.dk == 256) return launch_dk<256>(p, mv, mk, zeta_v, U, status, st);
     if (p.dk == 64) return launch_dk<64>(p, mv, mk, zeta_v, U, status, st);
