@@ -13,7 +13,9 @@
 // swish'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))); dn = dY swish(G);
 // dO = r (dn - mean(dn) - n mean(dn n)).  O, G and dY are each read once,
 // all three requested before the first reduction and held as loaded (dn
-// in fp32) between the reductions; dO and dG are written once.
+// in fp32) between the reductions; dO and dG are written once.  The kernel
+// is bound by instruction issue, so the row statistics take one shifted
+// pass and the sigmoid the fast exponential and reciprocal.
 #include "common.cuh"
 #include "launch.h"
 
@@ -191,20 +193,17 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
         Raw4<TO_> ro[kPerLane];
         Raw4<TG> rg[kPerLane], rdy[kPerLane];
         load_row(O, G, dY, orow, gy, dv, lane, ro, rg, rdy);
-        // O stays as loaded; each pass converts it again, which is cheaper
-        // than holding the centred row in fp32 registers
-        float sum = 0.f;
-#pragma unroll
-        for (int it = 0; it < kPerLane; ++it) {
-            int e = 128 * it + 4 * lane;
-            if (e < dv) {
-                float x[4];
-                ro[it].get(x);
-                sum += (x[0] + x[1]) + (x[2] + x[3]);
-            }
-        }
-        const float mu = warp_sum(sum) / (float)dv;
-        float sq = 0.f;
+        // O stays as loaded and is converted again where it is used, which
+        // is cheaper than holding the row in fp32 registers.  Its mean and
+        // variance come from one pass of sums shifted by the row's first
+        // value (so that a large mean does not cancel the variance), and
+        // both sums reduce together.
+        const float shift = __shfl_sync(0xffffffffu, [&] {
+            float x[4];
+            ro[0].get(x);
+            return x[0];
+        }(), 0);
+        float s1 = 0.f, s2 = 0.f;
 #pragma unroll
         for (int it = 0; it < kPerLane; ++it) {
             int e = 128 * it + 4 * lane;
@@ -213,13 +212,20 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
                 ro[it].get(x);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    x[q] -= mu;
-                    sq = fmaf(x[q], x[q], sq);
+                    const float c = x[q] - shift;
+                    s1 += c;
+                    s2 = fmaf(c, c, s2);
                 }
             }
         }
-        const float rs = rsqrtf(warp_sum(sq) / (float)dv + eps);
-        const float nshift = -mu * rs;  // n = o rs + nshift
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            s1 += __shfl_xor_sync(0xffffffffu, s1, m);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, m);
+        }
+        const float m1 = s1 / (float)dv;
+        const float rs = rsqrtf(fmaxf(s2 / (float)dv - m1 * m1, 0.f) + eps);
+        const float nshift = -m1 * rs;  // n = (o - shift) rs + nshift
         // dn = dY swish(G) kept; dG written here
         float dn[kPerLane][4];
         float s_dn = 0.f, s_dnn = 0.f;
@@ -233,8 +239,10 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
                 rdy[it].get(dy);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float sig = 1.0f / (1.0f + expf(-g[q]));
-                    const float n = fmaf(x[q], rs, nshift);
+                    // sigmoid by the fast exponential and reciprocal (a few
+                    // units in the last place; the sum saturates to 0 or 1)
+                    const float sig = __fdividef(1.0f, 1.0f + __expf(-g[q]));
+                    const float n = fmaf(x[q] - shift, rs, nshift);
                     dn[it][q] = dy[q] * (g[q] * sig);
                     dg[q] = dy[q] * n * (sig * fmaf(g[q], 1.0f - sig, 1.0f));
                     s_dn += dn[it][q];
@@ -243,8 +251,13 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
                 store4(dG + gy + e, dg);
             }
         }
-        const float m_dn = warp_sum(s_dn) / (float)dv;
-        const float m_dnn = warp_sum(s_dnn) / (float)dv;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            s_dn += __shfl_xor_sync(0xffffffffu, s_dn, m);
+            s_dnn += __shfl_xor_sync(0xffffffffu, s_dnn, m);
+        }
+        const float m_dn = s_dn / (float)dv;
+        const float m_dnn = s_dnn / (float)dv;
 #pragma unroll
         for (int it = 0; it < kPerLane; ++it) {
             int e = 128 * it + 4 * lane;
@@ -253,7 +266,7 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
                 ro[it].get(x);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    d[q] = rs * (dn[it][q] - m_dn - fmaf(x[q], rs, nshift) * m_dnn);
+                    d[q] = rs * (dn[it][q] - m_dn - fmaf(x[q] - shift, rs, nshift) * m_dnn);
                 store4(dO + orow + e, d);
             }
         }

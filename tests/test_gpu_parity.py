@@ -197,6 +197,21 @@ def test_gate_norm_backward(o_dtype, g_dtype, dv):
     assert ok, ("dG", err)
 
 
+def test_gate_norm_backward_large_mean():
+    """Rows whose mean is far above their spread (O around 300 with a
+    spread of 0.5): the statistics must not lose the variance to the mean."""
+    B, H, L, dv = 1, 2, 9, 128
+    O = random_tensor((B, H, L, dv), 74) * 0.5 + 300.0
+    G = random_tensor((B, L, H * dv), 75)
+    dY = random_tensor((B, L, H * dv), 76)
+    dO_ref, dG_ref = orc.gate_groupnorm_backward(O, G, dY, 1e-5)
+    dO = torch.empty(B, H, L, dv, device="cuda")
+    dG = torch.empty(B, L, H * dv, device="cuda")
+    R.ret_gate_norm_backward(O.cuda(), G.cuda(), dY.cuda(), dO, dG, 1e-5)
+    assert normwise(dO, dO_ref) <= TOL_F32
+    assert normwise(dG, dG_ref) <= TOL_F32
+
+
 def test_gate_norm_backward_full_size_sampled():
     """At the msr_1p3b size the bench times (B=8 H=8 L=4096 d_v=512, bf16
     O, G and dY): rows sampled across the batch, the sequence and the tail
