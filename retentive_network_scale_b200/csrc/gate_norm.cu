@@ -15,7 +15,8 @@
 // all three requested before the first reduction and held as loaded (dn
 // in fp32) between the reductions; dO and dG are written once.  The kernel
 // is bound by instruction issue, so the row statistics take one shifted
-// pass and the sigmoid the fast exponential and reciprocal.
+// pass, the sigmoid the fast exponential and reciprocal, and the rest runs
+// on pairs of fp32 values (the paired add, mul and fma).
 #include "common.cuh"
 #include "launch.h"
 
@@ -136,15 +137,47 @@ cudaError_t launch_g(bool g_bf16, bool y_bf16, int B, int L, int H, int dv,
 
 // Four consecutive elements as loaded (16 bytes of fp32 or 8 of bf16), so
 // that a row's three inputs can all be in flight before any arithmetic.
+// Two fp32 values in one 64-bit register pair (lo, hi), for the paired
+// fp32 instructions (add, mul, fma on .f32x2).
+__device__ __forceinline__ uint64_t p2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ float p2_lo(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a)); }
+__device__ __forceinline__ float p2_hi(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a >> 32)); }
+__device__ __forceinline__ uint64_t p2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t p2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t p2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 template <typename T> struct Raw4;
 template <> struct Raw4<float> {
     float4 v;
+    // elements (2k, 2k+1) as a pair
+    __device__ __forceinline__ uint64_t pair(int k) const { return k ? p2(v.z, v.w) : p2(v.x, v.y); }
     __device__ __forceinline__ void load(const float *p) { v = *reinterpret_cast<const float4 *>(p); }
     __device__ __forceinline__ void get(float *x) const { x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w; }
 };
 template <> struct Raw4<__nv_bfloat16> {
     uint2 v;
     __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = *reinterpret_cast<const uint2 *>(p); }
+    // elements (2k, 2k+1) as a pair: a bf16 is the high half of its fp32
+    __device__ __forceinline__ uint64_t pair(int k) const {
+        const uint32_t u = k ? v.y : v.x;
+        return p2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
     __device__ __forceinline__ void get(float *x) const {
         float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.x));
         float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.y));
@@ -203,70 +236,80 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
             ro[0].get(x);
             return x[0];
         }(), 0);
-        float s1 = 0.f, s2 = 0.f;
+        const uint64_t nshift2 = p2(-shift, -shift);
+        uint64_t s1 = 0, s2 = 0;  // (+0, +0) pairs
 #pragma unroll
         for (int it = 0; it < kPerLane; ++it) {
             int e = 128 * it + 4 * lane;
             if (e < dv) {
-                float x[4];
-                ro[it].get(x);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float c = x[q] - shift;
-                    s1 += c;
-                    s2 = fmaf(c, c, s2);
+                for (int k = 0; k < 2; ++k) {
+                    const uint64_t c = p2_add(ro[it].pair(k), nshift2);
+                    s1 = p2_add(s1, c);
+                    s2 = p2_fma(c, c, s2);
                 }
             }
         }
+        float t1 = p2_lo(s1) + p2_hi(s1), t2 = p2_lo(s2) + p2_hi(s2);
 #pragma unroll
         for (int m = 16; m > 0; m >>= 1) {
-            s1 += __shfl_xor_sync(0xffffffffu, s1, m);
-            s2 += __shfl_xor_sync(0xffffffffu, s2, m);
+            t1 += __shfl_xor_sync(0xffffffffu, t1, m);
+            t2 += __shfl_xor_sync(0xffffffffu, t2, m);
         }
-        const float m1 = s1 / (float)dv;
-        const float rs = rsqrtf(fmaxf(s2 / (float)dv - m1 * m1, 0.f) + eps);
-        const float nshift = -m1 * rs;  // n = (o - shift) rs + nshift
+        const float m1 = t1 / (float)dv;
+        const float rs = rsqrtf(fmaxf(t2 / (float)dv - m1 * m1, 0.f) + eps);
+        // n = (o - shift) rs - m1 rs
+        const uint64_t rs2 = p2(rs, rs), nb2 = p2(-m1 * rs, -m1 * rs);
+        const uint64_t one2 = p2(1.f, 1.f), mone2 = p2(-1.f, -1.f);
         // dn = dY swish(G) kept; dG written here
-        float dn[kPerLane][4];
-        float s_dn = 0.f, s_dnn = 0.f;
+        uint64_t dn[kPerLane][2];
+        uint64_t a_dn = 0, a_dnn = 0;
 #pragma unroll
         for (int it = 0; it < kPerLane; ++it) {
             int e = 128 * it + 4 * lane;
             if (e < dv) {
-                float x[4], g[4], dy[4], dg[4];
-                ro[it].get(x);
-                rg[it].get(g);
-                rdy[it].get(dy);
+                float dg[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int k = 0; k < 2; ++k) {
+                    const uint64_t g = rg[it].pair(k), dy = rdy[it].pair(k);
                     // sigmoid by the fast exponential and reciprocal (a few
-                    // units in the last place; the sum saturates to 0 or 1)
-                    const float sig = __fdividef(1.0f, 1.0f + __expf(-g[q]));
-                    const float n = fmaf(x[q] - shift, rs, nshift);
-                    dn[it][q] = dy[q] * (g[q] * sig);
-                    dg[q] = dy[q] * n * (sig * fmaf(g[q], 1.0f - sig, 1.0f));
-                    s_dn += dn[it][q];
-                    s_dnn = fmaf(dn[it][q], n, s_dnn);
+                    // units in the last place; it saturates to 0 or 1)
+                    const uint64_t sig = p2(__fdividef(1.0f, 1.0f + __expf(-p2_lo(g))),
+                                            __fdividef(1.0f, 1.0f + __expf(-p2_hi(g))));
+                    const uint64_t n = p2_fma(p2_add(ro[it].pair(k), nshift2), rs2, nb2);
+                    dn[it][k] = p2_mul(dy, p2_mul(g, sig));
+                    // swish'(g) = sig (1 + g (1 - sig))
+                    const uint64_t ds = p2_mul(sig, p2_fma(g, p2_fma(sig, mone2, one2), one2));
+                    const uint64_t d = p2_mul(p2_mul(dy, n), ds);
+                    dg[2 * k] = p2_lo(d);
+                    dg[2 * k + 1] = p2_hi(d);
+                    a_dn = p2_add(a_dn, dn[it][k]);
+                    a_dnn = p2_fma(dn[it][k], n, a_dnn);
                 }
                 store4(dG + gy + e, dg);
             }
         }
+        float s_dn = p2_lo(a_dn) + p2_hi(a_dn), s_dnn = p2_lo(a_dnn) + p2_hi(a_dnn);
 #pragma unroll
         for (int m = 16; m > 0; m >>= 1) {
             s_dn += __shfl_xor_sync(0xffffffffu, s_dn, m);
             s_dnn += __shfl_xor_sync(0xffffffffu, s_dnn, m);
         }
-        const float m_dn = s_dn / (float)dv;
-        const float m_dnn = s_dnn / (float)dv;
+        // dO = rs (dn - mean(dn) - n mean(dn n)) = rs dn + (C n + Bc)
+        const float m_dn = s_dn / (float)dv, m_dnn = s_dnn / (float)dv;
+        const uint64_t C2 = p2(-rs * m_dnn, -rs * m_dnn), B2 = p2(-rs * m_dn, -rs * m_dn);
 #pragma unroll
         for (int it = 0; it < kPerLane; ++it) {
             int e = 128 * it + 4 * lane;
             if (e < dv) {
-                float x[4], d[4];
-                ro[it].get(x);
+                float d[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    d[q] = rs * (dn[it][q] - m_dn - fmaf(x[q] - shift, rs, nshift) * m_dnn);
+                for (int k = 0; k < 2; ++k) {
+                    const uint64_t n = p2_fma(p2_add(ro[it].pair(k), nshift2), rs2, nb2);
+                    const uint64_t r = p2_fma(dn[it][k], rs2, p2_fma(n, C2, B2));
+                    d[2 * k] = p2_lo(r);
+                    d[2 * k + 1] = p2_hi(r);
+                }
                 store4(dO + orow + e, d);
             }
         }
