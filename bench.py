@@ -409,6 +409,26 @@ def bench_backward(R, w, d, pk, reps=3):
     return out
 
 
+def bench_gate_norm(R, w, d, pk, reps=20):
+    """The standalone GroupNorm + swish gate, Y from a bf16 O and G (the
+    form used when the chunk loop writes O): one streaming kernel,
+    HBM-bound.  Its inputs (0.54 GB) exceed L2."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed + 9)
+    O = torch.randn(w.B, w.H, w.L, w.d_v, device="cuda", generator=gen).bfloat16()
+    Y = torch.empty(w.B, w.L, w.H * w.d_v, device="cuda", dtype=torch.bfloat16)
+    fn = lambda: R.ret_gate_norm(O, d["G"], Y, 1e-5)  # noqa: E731
+    for _ in range(3):
+        fn()
+    ms = time_launches(fn, reps, torch.cuda.current_stream())
+    nbytes = 3 * O.numel() * O.element_size()  # read O, G; write Y
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"GroupNorm + swish gate alone (bf16 O, G -> Y) on {w.name}", "ms": ms,
+            "tokens_per_s": w.B * w.L / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": nbytes}}
+
+
 def bench_gate_backward(R, w, d, pk, gen, reps=20):
     """dO and dG of the GroupNorm + swish gate given dY (bf16 O, G, dY, dO,
     dG): one streaming kernel, HBM-bound.  Its inputs (0.8 GB) exceed L2."""
@@ -624,7 +644,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     R.load_library()
     pk, pk_src = peaks()
-    if args.only in ("decode", "parallel", "long_ctx", "msr_small", "backward", "layer"):
+    if args.only in ("decode", "parallel", "long_ctx", "msr_small", "backward", "layer",
+                     "gate_norm"):
         if args.only == "decode":
             out = bench_decode(R, pk, warm=args.warmup, reps=max(1, args.steps), batch=args.decode_batch)
         elif args.only == "long_ctx":
@@ -638,6 +659,8 @@ def run_ours(args, world, rank, local):
             d = {k: v.cuda() for k, v in make_inputs(w).items()}
             if args.only == "backward":
                 out = bench_backward(R, w, d, pk, reps=max(1, args.steps))
+            elif args.only == "gate_norm":
+                out = bench_gate_norm(R, w, d, pk, reps=max(1, args.steps))
             elif args.only == "layer":
                 out = bench_layer(R, w, pk, reps=max(1, args.steps))
             else:
@@ -761,6 +784,7 @@ def run_ours(args, world, rank, local):
     if not args.skip_extra:
         extra["parallel"] = bench_parallel(R, w, d, pk)
         extra["backward"] = bench_backward(R, w, d, pk)
+        extra["gate_norm"] = bench_gate_norm(R, w, d, pk)
         extra["sequence_shard"] = bench_seqshard(R, w, d, pk)
         del d
         torch.cuda.empty_cache()
@@ -808,7 +832,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the MSR workload's batch (small cases for profiler captures)")
     ap.add_argument("--only", choices=["main", "parallel", "decode", "long_ctx", "msr_small",
-                                       "backward", "layer"],
+                                       "backward", "layer", "gate_norm"],
                     default=None,
                     help="run one measurement alone (profiler captures)")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -3,9 +3,12 @@
 // section 2.2, the MSR equation; population variance, no affine terms).
 //
 // Bound by HBM (read O and G, write Y).  One warp per (b, t, h) row: each
-// lane holds up to 16 of the row's d_v <= 512 values in registers (4-wide
-// vector loads), so the mean and the centred variance are two register
-// passes and warp reductions with no second read of memory.
+// lane holds up to 16 of the row's d_v <= 512 values in registers as
+// loaded (4-wide vector loads, O and G requested together), so the mean and
+// variance (one pass of shifted sums) need no second read of memory.  The
+// arithmetic runs on pairs of fp32 values and the sigmoid on the fast
+// exponential and reciprocal, since a plain version is bound by instruction
+// issue rather than by memory.
 //
 // The backward (gate_norm_backward_kernel) takes dY to dO and dG by the
 // chain rule through the same three steps, with the same row ownership:
@@ -23,20 +26,9 @@
 namespace ret {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kThreadsB = 128;  // backward: five blocks of four warps per SM
+constexpr int kThreadsB = 128;  // blocks of four warps, five per SM
 constexpr int kPerLane = kMaxDv / 128;  // 4-vectors per lane
 
-__device__ __forceinline__ void load4(const float *p, float *x) {
-    float4 v = *reinterpret_cast<const float4 *>(p);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-}
-__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float *x) {
-    uint2 u = *reinterpret_cast<const uint2 *>(p);
-    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u.x));
-    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
 __device__ __forceinline__ void store4(float *p, const float *x) {
     *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
 }
@@ -49,94 +41,6 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float *x) {
     *reinterpret_cast<uint2 *>(p) = u;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-    return v;
-}
-
-template <typename TO_, typename TG, typename TY>
-__global__ void __launch_bounds__(kThreads)
-gate_norm_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G,
-                 float eps, TY *Y) {
-    const int lane = threadIdx.x & 31;
-    const long long rows = (long long)B * L * H;
-    const long long warps = (long long)gridDim.x * (kThreads / 32);
-    for (long long r = (long long)blockIdx.x * (kThreads / 32) + threadIdx.x / 32; r < rows; r += warps) {
-        const int h = (int)(r % H);
-        const long long bt = r / H;
-        const int t = (int)(bt % L);
-        const long long b = bt / L;
-        const TO_ *o = O + (((size_t)b * H + h) * L + t) * dv;
-        const size_t gy = (size_t)bt * H * dv + (size_t)h * dv;
-
-        float x[kPerLane][4];
-        float sum = 0.f;
-#pragma unroll
-        for (int it = 0; it < kPerLane; ++it) {
-            int e = 128 * it + 4 * lane;
-            if (e < dv) {
-                load4(o + e, x[it]);
-                sum += (x[it][0] + x[it][1]) + (x[it][2] + x[it][3]);
-            }
-        }
-        const float mu = warp_sum(sum) / (float)dv;
-        float sq = 0.f;
-#pragma unroll
-        for (int it = 0; it < kPerLane; ++it) {
-            int e = 128 * it + 4 * lane;
-            if (e < dv) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    x[it][q] -= mu;
-                    sq = fmaf(x[it][q], x[it][q], sq);
-                }
-            }
-        }
-        const float inv = rsqrtf(warp_sum(sq) / (float)dv + eps);
-#pragma unroll
-        for (int it = 0; it < kPerLane; ++it) {
-            int e = 128 * it + 4 * lane;
-            if (e < dv) {
-                float g[4], y[4];
-                load4(G + gy + e, g);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) y[q] = g[q] / (1.0f + expf(-g[q])) * (x[it][q] * inv);
-                store4(Y + gy + e, y);
-            }
-        }
-    }
-}
-
-template <typename TO_, typename TG, typename TY>
-cudaError_t launch_t(int B, int L, int H, int dv, const void *O, const void *G,
-                     float eps, void *Y, cudaStream_t st) {
-    long long rows = (long long)B * L * H;
-    long long blocks = (rows + (kThreads / 32) - 1) / (kThreads / 32);
-    if (blocks > 148LL * 64) blocks = 148LL * 64;
-    gate_norm_kernel<TO_, TG, TY><<<(unsigned)blocks, kThreads, 0, st>>>(
-        B, L, H, dv, (const TO_ *)O, (const TG *)G, eps, (TY *)Y);
-    cudaError_t err = cudaGetLastError();
-    if (err == cudaSuccess) note_launches(1);
-    return err;
-}
-
-template <typename TO_, typename TG>
-cudaError_t launch_y(bool y_bf16, int B, int L, int H, int dv, const void *O,
-                     const void *G, float eps, void *Y, cudaStream_t st) {
-    return y_bf16 ? launch_t<TO_, TG, __nv_bfloat16>(B, L, H, dv, O, G, eps, Y, st)
-                  : launch_t<TO_, TG, float>(B, L, H, dv, O, G, eps, Y, st);
-}
-
-template <typename TO_>
-cudaError_t launch_g(bool g_bf16, bool y_bf16, int B, int L, int H, int dv,
-                     const void *O, const void *G, float eps, void *Y, cudaStream_t st) {
-    return g_bf16 ? launch_y<TO_, __nv_bfloat16>(y_bf16, B, L, H, dv, O, G, eps, Y, st)
-                  : launch_y<TO_, float>(y_bf16, B, L, H, dv, O, G, eps, Y, st);
-}
-
-// Four consecutive elements as loaded (16 bytes of fp32 or 8 of bf16), so
-// that a row's three inputs can all be in flight before any arithmetic.
 // Two fp32 values in one 64-bit register pair (lo, hi), for the paired
 // fp32 instructions (add, mul, fma on .f32x2).
 __device__ __forceinline__ uint64_t p2(float lo, float hi) {
@@ -162,6 +66,8 @@ __device__ __forceinline__ uint64_t p2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
+// Four consecutive elements as loaded (16 bytes of fp32 or 8 of bf16), so
+// that a row's three inputs can all be in flight before any arithmetic.
 template <typename T> struct Raw4;
 template <> struct Raw4<float> {
     float4 v;
@@ -211,6 +117,118 @@ __device__ __forceinline__ void load_row(const TO_ *O, const TG *G, const TG *dY
     }
 }
 
+// The row statistics shared by both directions: mean and variance of the
+// row's O (held as loaded) from one pass of sums shifted by the row's first
+// value, so that a large mean does not cancel the variance.  Returns the
+// pairs (shift'), rs and nb with n = (o + shift') rs + nb the normalised
+// row.
+template <typename TO_>
+__device__ __forceinline__ void row_stats(const Raw4<TO_> *ro, int dv, int lane, float eps,
+                                          uint64_t &nshift2, uint64_t &rs2, uint64_t &nb2) {
+    float x0[4];
+    ro[0].get(x0);
+    const float shift = __shfl_sync(0xffffffffu, x0[0], 0);
+    nshift2 = p2(-shift, -shift);
+    uint64_t s1 = 0, s2 = 0;  // (+0, +0) pairs
+#pragma unroll
+    for (int it = 0; it < kPerLane; ++it) {
+        int e = 128 * it + 4 * lane;
+        if (e < dv) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint64_t c = p2_add(ro[it].pair(k), nshift2);
+                s1 = p2_add(s1, c);
+                s2 = p2_fma(c, c, s2);
+            }
+        }
+    }
+    float t1 = p2_lo(s1) + p2_hi(s1), t2 = p2_lo(s2) + p2_hi(s2);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) {
+        t1 += __shfl_xor_sync(0xffffffffu, t1, m);
+        t2 += __shfl_xor_sync(0xffffffffu, t2, m);
+    }
+    const float m1 = t1 / (float)dv;
+    const float rs = rsqrtf(fmaxf(t2 / (float)dv - m1 * m1, 0.f) + eps);
+    rs2 = p2(rs, rs);
+    nb2 = p2(-m1 * rs, -m1 * rs);
+}
+
+// sigmoid of both values of a pair, by the fast exponential and reciprocal
+// (a few units in the last place; it saturates to 0 or 1)
+__device__ __forceinline__ uint64_t sigmoid2(uint64_t g) {
+    return p2(__fdividef(1.0f, 1.0f + __expf(-p2_lo(g))), __fdividef(1.0f, 1.0f + __expf(-p2_hi(g))));
+}
+
+template <typename TO_, typename TG, typename TY>
+__global__ void __launch_bounds__(kThreadsB, 5)
+gate_norm_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G,
+                 float eps, TY *Y) {
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)B * L * H;
+    const long long warps = (long long)gridDim.x * (kThreadsB / 32);
+    for (long long r = (long long)blockIdx.x * (kThreadsB / 32) + threadIdx.x / 32; r < rows; r += warps) {
+        size_t orow, gy;
+        row_offsets(r, L, H, dv, orow, gy);
+        // the row's O and G are requested together; O stays as loaded
+        Raw4<TO_> ro[kPerLane];
+        Raw4<TG> rg[kPerLane];
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                ro[it].load(O + orow + e);
+                rg[it].load(G + gy + e);
+            }
+        }
+        uint64_t nshift2, rs2, nb2;
+        row_stats(ro, dv, lane, eps, nshift2, rs2, nb2);
+#pragma unroll
+        for (int it = 0; it < kPerLane; ++it) {
+            int e = 128 * it + 4 * lane;
+            if (e < dv) {
+                float y[4];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const uint64_t g = rg[it].pair(k);
+                    const uint64_t n = p2_fma(p2_add(ro[it].pair(k), nshift2), rs2, nb2);
+                    const uint64_t v = p2_mul(p2_mul(g, sigmoid2(g)), n);
+                    y[2 * k] = p2_lo(v);
+                    y[2 * k + 1] = p2_hi(v);
+                }
+                store4(Y + gy + e, y);
+            }
+        }
+    }
+}
+
+template <typename TO_, typename TG, typename TY>
+cudaError_t launch_t(int B, int L, int H, int dv, const void *O, const void *G,
+                     float eps, void *Y, cudaStream_t st) {
+    long long rows = (long long)B * L * H;
+    long long blocks = (rows + (kThreadsB / 32) - 1) / (kThreadsB / 32);
+    if (blocks > 148LL * 128) blocks = 148LL * 128;
+    gate_norm_kernel<TO_, TG, TY><<<(unsigned)blocks, kThreadsB, 0, st>>>(
+        B, L, H, dv, (const TO_ *)O, (const TG *)G, eps, (TY *)Y);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+template <typename TO_, typename TG>
+cudaError_t launch_y(bool y_bf16, int B, int L, int H, int dv, const void *O,
+                     const void *G, float eps, void *Y, cudaStream_t st) {
+    return y_bf16 ? launch_t<TO_, TG, __nv_bfloat16>(B, L, H, dv, O, G, eps, Y, st)
+                  : launch_t<TO_, TG, float>(B, L, H, dv, O, G, eps, Y, st);
+}
+
+template <typename TO_>
+cudaError_t launch_g(bool g_bf16, bool y_bf16, int B, int L, int H, int dv,
+                     const void *O, const void *G, float eps, void *Y, cudaStream_t st) {
+    return g_bf16 ? launch_y<TO_, __nv_bfloat16>(y_bf16, B, L, H, dv, O, G, eps, Y, st)
+                  : launch_y<TO_, float>(y_bf16, B, L, H, dv, O, G, eps, Y, st);
+}
+
 template <typename TO_, typename TG>
 __global__ void __launch_bounds__(kThreadsB, 5)
 gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G, const TG *dY,
@@ -227,39 +245,10 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
         Raw4<TG> rg[kPerLane], rdy[kPerLane];
         load_row(O, G, dY, orow, gy, dv, lane, ro, rg, rdy);
         // O stays as loaded and is converted again where it is used, which
-        // is cheaper than holding the row in fp32 registers.  Its mean and
-        // variance come from one pass of sums shifted by the row's first
-        // value (so that a large mean does not cancel the variance), and
-        // both sums reduce together.
-        const float shift = __shfl_sync(0xffffffffu, [&] {
-            float x[4];
-            ro[0].get(x);
-            return x[0];
-        }(), 0);
-        const uint64_t nshift2 = p2(-shift, -shift);
-        uint64_t s1 = 0, s2 = 0;  // (+0, +0) pairs
-#pragma unroll
-        for (int it = 0; it < kPerLane; ++it) {
-            int e = 128 * it + 4 * lane;
-            if (e < dv) {
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const uint64_t c = p2_add(ro[it].pair(k), nshift2);
-                    s1 = p2_add(s1, c);
-                    s2 = p2_fma(c, c, s2);
-                }
-            }
-        }
-        float t1 = p2_lo(s1) + p2_hi(s1), t2 = p2_lo(s2) + p2_hi(s2);
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) {
-            t1 += __shfl_xor_sync(0xffffffffu, t1, m);
-            t2 += __shfl_xor_sync(0xffffffffu, t2, m);
-        }
-        const float m1 = t1 / (float)dv;
-        const float rs = rsqrtf(fmaxf(t2 / (float)dv - m1 * m1, 0.f) + eps);
-        // n = (o - shift) rs - m1 rs
-        const uint64_t rs2 = p2(rs, rs), nb2 = p2(-m1 * rs, -m1 * rs);
+        // is cheaper than holding the row in fp32 registers
+        uint64_t nshift2, rs2, nb2;
+        row_stats(ro, dv, lane, eps, nshift2, rs2, nb2);
+        const float rs = p2_lo(rs2);
         const uint64_t one2 = p2(1.f, 1.f), mone2 = p2(-1.f, -1.f);
         // dn = dY swish(G) kept; dG written here
         uint64_t dn[kPerLane][2];
@@ -272,10 +261,7 @@ gate_norm_backward_kernel(int B, int L, int H, int dv, const TO_ *O, const TG *G
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     const uint64_t g = rg[it].pair(k), dy = rdy[it].pair(k);
-                    // sigmoid by the fast exponential and reciprocal (a few
-                    // units in the last place; it saturates to 0 or 1)
-                    const uint64_t sig = p2(__fdividef(1.0f, 1.0f + __expf(-p2_lo(g))),
-                                            __fdividef(1.0f, 1.0f + __expf(-p2_hi(g))));
+                    const uint64_t sig = sigmoid2(g);
                     const uint64_t n = p2_fma(p2_add(ro[it].pair(k), nshift2), rs2, nb2);
                     dn[it][k] = p2_mul(dy, p2_mul(g, sig));
                     // swish'(g) = sig (1 + g (1 - sig))

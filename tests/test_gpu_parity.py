@@ -162,8 +162,9 @@ def test_limits_max_dims_and_heads():
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_gate_norm_standalone(dtype):
-    B, H, L, dv = 2, 3, 33, 64
+@pytest.mark.parametrize("dv", [64, 20, 512])
+def test_gate_norm_standalone(dtype, dv):
+    B, H, L = 2, 3, 33
     O = (random_tensor((B, H, L, dv), 51) * 2 + 0.5).to(dtype)
     G = random_tensor((B, L, H * dv), 52).to(dtype)
     ref = orc.gate_groupnorm(O, G, 1e-5)
@@ -171,6 +172,17 @@ def test_gate_norm_standalone(dtype):
     R.ret_gate_norm(O.cuda(), G.cuda(), Y, 1e-5)
     ok, err = within(Y, ref, dtype)
     assert ok, err
+
+
+def test_gate_norm_large_mean():
+    """Rows far from zero mean (around 300, spread 0.5): the shifted sums
+    keep the variance."""
+    B, H, L, dv = 1, 2, 9, 128
+    O = random_tensor((B, H, L, dv), 53) * 0.5 + 300.0
+    G = random_tensor((B, L, H * dv), 54)
+    Y = torch.empty(B, L, H * dv, device="cuda")
+    R.ret_gate_norm(O.cuda(), G.cuda(), Y, 1e-5)
+    assert normwise(Y, orc.gate_groupnorm(O, G, 1e-5)) <= TOL_F32
 
 
 @pytest.mark.parametrize("o_dtype,g_dtype", [(torch.float32, torch.float32),
