@@ -204,7 +204,7 @@ int split_dv(int dv, int *w) {  // at most two blocks for d_v <= 512
 }
 
 struct BwdLayout {
-    size_t kh, qh, prep, part_dk, part_dv;  // offsets
+    size_t kh, qh, prep, part_dk, part_dv;  // offsets (prep: two buffers)
     size_t bytes;
     int nsplit;
 };
@@ -219,7 +219,7 @@ BwdLayout bwd_layout(const ret_desc *d) {
     (void)bv;
     z.kh = o; o += d->rotate ? round_up(bk) : 0;  // turned K and Q
     z.qh = o; o += d->rotate ? round_up(bk) : 0;
-    z.prep = o; o += round_up(2 * rows * 256 * 2);            // prepared Q^, K~ of one call
+    z.prep = o; o += round_up(2 * rows * 256 * 2) * 2;  // weighted keys of two products
     z.part_dk = o; o += round_up(rows * d->d_k * 4) * 2 * z.nsplit;  // dQ^, dK^ partials
     z.part_dv = o; o += round_up(rows * d->d_v * 4);
     z.bytes = o;
@@ -266,19 +266,29 @@ cudaError_t unturn_sum(const Params &p, int d, const float *part0, const float *
 // `qk` (column offset already in the pointers), value rows [B][H][L][dv']
 // contiguous, fp32 output [B][H][L][dv'].  With acc_in the output is
 // acc_in + the product, turned back by the rows' angles when `unturn`.
-cudaError_t product(const Params &base, int dqk, int dval, const void *q, const void *k,
-                    RowLayout qk, const void *v, bool anti, void *prep_ws, float *out, int *status,
-                    cudaStream_t st, const float *acc_in = nullptr, bool unturn = false) {
+// It is two launches: the streaming pass that writes the weighted key rows
+// K~ into prep_ws (product_keys), then the chunk loop (product_loop), so
+// that the pass of the next product can run beside this one's loop.
+Params product_params(const Params &base, int dqk, int dval, bool anti) {
     Params p = base;
     p.dk = dqk;
     p.dv = dval;
     p.rotate = 0;  // the operands come turned already
     p.reverse = anti ? 1 : 0;
+    return p;
+}
+
+cudaError_t product_keys(const Params &p, const void *q, const void *k, RowLayout qk,
+                         void *prep_ws, const void **kt, cudaStream_t st) {
     // only K~ is written: the query rows are read in place through `qk`
-    const void *qh = nullptr, *kt = nullptr;
-    cudaError_t e = launch_chunkwise_prep_strided(p, 128, q, k, qk, false, prep_ws, &qh, &kt, st);
-    if (e != cudaSuccess) return e;
-    return launch_chunkwise_ws(p, false, qh, qk, kt, bhld_layout(p, dqk), v, bhld_layout(p, dval), true,
+    const void *qh = nullptr;
+    return launch_chunkwise_prep_strided(p, 128, q, k, qk, false, prep_ws, &qh, kt, st);
+}
+
+cudaError_t product_loop(const Params &p, const void *q, RowLayout qk, const void *kt,
+                         const void *v, float *out, int *status, cudaStream_t st,
+                         const float *acc_in = nullptr, bool unturn = false) {
+    return launch_chunkwise_ws(p, false, q, qk, kt, bhld_layout(p, p.dk), v, bhld_layout(p, p.dv), true,
                                nullptr, nullptr, out, nullptr, RowLayout{0, 0, 0}, nullptr, 0.f, false,
                                false, status, st, acc_in, unturn ? 1 : 0);
 }
@@ -349,33 +359,83 @@ ret_status ret_backward(const ret_desc *desc, int chunk, const void *Q, const vo
 
     cudaError_t e = cudaSuccess;
     auto run = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
-    // 1. turned bf16 copies of K and Q
-    if (rot) {
-        run(flip_turn(p, dk, K, ws + z.kh, true, false, st));
-        run(flip_turn(p, dk, Q, ws + z.qh, true, false, st));
-    }
-    // 2. dQ^ (causal: dO, V, K^) and dK^ (anti-causal: V, dO, Q^), per
-    //    column block of d_v
+    // The products, in order: dQ^ (causal: dO, V, K^) and dK^ (anti-causal:
+    // V, dO, Q^) per column block of d_v, then dV (anti-causal: K^, Q^, dO).
+    // In fp32 with two column blocks, the second block's products add the
+    // first block's partials and turn the sums back in their epilogue,
+    // writing dQ and dK themselves (no sum pass).
+    struct Prod {
+        Params p;
+        const void *q, *k, *v;
+        RowLayout qk;
+        float *out;
+        const float *acc_in;
+        bool unturn, needs_qh;
+    };
+    Prod prods[2 * 8 + 1];
+    int np = 0;
     int w[8];
     const int n = split_dv(dv, w);
     const RowLayout full_v = bhld_layout(p, dv);
     const auto *dO8 = static_cast<const uint8_t *>(dO), *V8 = static_cast<const uint8_t *>(V);
-    // In fp32 with two column blocks, the second block's products add the
-    // first block's partials and turn the sums back in their epilogue,
-    // writing dQ and dK themselves (no sum pass).
     const bool fold = desc->out_dtype == RET_F32 && n == 2;
-    for (int i = 0, c0 = 0; i < n && e == cudaSuccess; c0 += w[i], ++i) {
+    for (int i = 0, c0 = 0; i < n; c0 += w[i], ++i) {
         const size_t off = (size_t)c0 * 2;
         const bool last = fold && i == 1;
-        run(product(p, w[i], dk, dO8 + off, V8 + off, full_v, Kh, false, prep,
-                    last ? static_cast<float *>(dQ) : partA + i * part_stride, status, st,
-                    last ? partA : nullptr, rot));
-        run(product(p, w[i], dk, V8 + off, dO8 + off, full_v, Qh, true, prep,
-                    last ? static_cast<float *>(dK) : partB + i * part_stride, status, st,
-                    last ? partB : nullptr, rot));
+        prods[np++] = Prod{product_params(p, w[i], dk, false), dO8 + off, V8 + off, Kh, full_v,
+                           last ? static_cast<float *>(dQ) : partA + i * part_stride,
+                           last ? partA : nullptr, rot, false};
+        prods[np++] = Prod{product_params(p, w[i], dk, true), V8 + off, dO8 + off, Qh, full_v,
+                           last ? static_cast<float *>(dK) : partB + i * part_stride,
+                           last ? partB : nullptr, rot, false};
     }
-    // 3. dV (anti-causal: K^, Q^, dO)
-    run(product(p, dk, dv, Kh, Qh, bhld_layout(p, dk), dO, true, prep, partC, status, st));
+    prods[np++] = Prod{product_params(p, dk, dv, true), Kh, Qh, dO, bhld_layout(p, dk), partC,
+                       nullptr, false, true};
+    const size_t prep_b = round_up(2 * rows * 256 * 2);
+    void *prep_buf[2] = {prep, static_cast<uint8_t *>(prep) + prep_b};
+    const void *kt[2 * 8 + 1] = {};
+
+    SideStreamRef side{};
+    if (side_stream_ref(&side)) {
+        // The weighting passes run on the side stream, each ahead of its
+        // product, in two buffers used in turn: the pass of product j+1
+        // fills the SMs that product j's loop (one wave or less) leaves
+        // free, so only the first pass is exposed.  Events: ready = a pass
+        // is done; aux[0..1] = the loop that read buffer 0 / 1 is done;
+        // aux[2] = the turned copies are written.
+        std::lock_guard<std::mutex> lock(*side.mu);
+        run(cudaEventRecord(side.start, st));
+        run(cudaStreamWaitEvent(side.s, side.start, 0));
+        // 1. turned bf16 copies of K and Q, beside the first passes (which
+        //    read V and dO only)
+        if (rot) {
+            run(flip_turn(p, dk, K, ws + z.kh, true, false, st));
+            run(flip_turn(p, dk, Q, ws + z.qh, true, false, st));
+        }
+        run(cudaEventRecord(side.aux[2], st));
+        // 2. the products
+        for (int j = 0; j < np && e == cudaSuccess; ++j) {
+            const Prod &r = prods[j];
+            if (j >= 2) run(cudaStreamWaitEvent(side.s, side.aux[j % 2], 0));
+            if (r.needs_qh) run(cudaStreamWaitEvent(side.s, side.aux[2], 0));
+            run(product_keys(r.p, r.q, r.k, r.qk, prep_buf[j % 2], &kt[j], side.s));
+            run(cudaEventRecord(side.ready, side.s));
+            run(cudaStreamWaitEvent(st, side.ready, 0));
+            run(product_loop(r.p, r.q, r.qk, kt[j], r.v, r.out, status, st, r.acc_in, r.unturn));
+            run(cudaEventRecord(side.aux[j % 2], st));
+        }
+    } else {
+        // no side stream: everything in order on the caller's stream
+        if (rot) {
+            run(flip_turn(p, dk, K, ws + z.kh, true, false, st));
+            run(flip_turn(p, dk, Q, ws + z.qh, true, false, st));
+        }
+        for (int j = 0; j < np && e == cudaSuccess; ++j) {
+            const Prod &r = prods[j];
+            run(product_keys(r.p, r.q, r.k, r.qk, prep_buf[0], &kt[j], st));
+            run(product_loop(r.p, r.q, r.qk, kt[j], r.v, r.out, status, st, r.acc_in, r.unturn));
+        }
+    }
     // 4. sums and the opposite turn
     const float *a1 = n > 1 ? partA + part_stride : nullptr;
     const float *b1 = n > 1 ? partB + part_stride : nullptr;

@@ -83,6 +83,7 @@ struct SideStream {
     bool made = false, ok = false;
     cudaStream_t s = nullptr;
     cudaEvent_t start = nullptr, ready = nullptr;
+    cudaEvent_t aux[kSideAuxEvents] = {};  // for other users of the stream
     int sms = 0;
 };
 constexpr int kMaxDevices = 64;
@@ -107,12 +108,26 @@ SideStream *side_stream() {
                 cudaEventCreateWithFlags(&ss.ready, cudaEventDisableTiming) == cudaSuccess &&
                 cudaDeviceGetAttribute(&ss.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
                 ss.sms > 0;
+        for (int i = 0; i < kSideAuxEvents && ss.ok; ++i)
+            ss.ok = cudaEventCreateWithFlags(&ss.aux[i], cudaEventDisableTiming) == cudaSuccess;
         if (!ss.ok) cudaGetLastError();
     }
     return ss.ok ? &ss : nullptr;
 }
 
 }  // namespace
+
+bool side_stream_ref(SideStreamRef *r) {
+    SideStream *ss = side_stream();
+    if (!ss) return false;
+    r->mu = &ss->mu;
+    r->s = ss->s;
+    r->start = ss->start;
+    r->ready = ss->ready;
+    for (int i = 0; i < kSideAuxEvents; ++i) r->aux[i] = ss->aux[i];
+    r->sms = ss->sms;
+    return true;
+}
 
 // With room for them, the turned Q^ and scaled K~ are written once by a
 // streaming pass and the kernel only loads them.  When the chunk loop needs

@@ -111,6 +111,20 @@ cudaError_t launch_chunkwise_ws(const Params &p, bool out_bf16, const void *Q, R
 // The streaming pass reading Q and K through a layout; with always_q it
 // writes Q^ even without rotation (then a plain copy into [B][H][L][d_k]),
 // so the workspace holds 2*B*H*L*d_k values.
+// The per-device side stream (lowest priority: kernels on it fill the SMs
+// that a one-wave launch on the caller's stream leaves free) and events to
+// join it to the caller's stream.  Made once per device; whoever enqueues
+// on it holds *mu for the whole enqueue sequence.  False when it could not
+// be made (the caller then queues everything on its own stream).
+constexpr int kSideAuxEvents = 3;
+struct SideStreamRef {
+    std::mutex *mu;
+    cudaStream_t s;
+    cudaEvent_t start, ready, aux[kSideAuxEvents];
+    int sms;
+};
+bool side_stream_ref(SideStreamRef *r);
+
 cudaError_t launch_chunkwise_prep_strided(const Params &p, int chunk, const void *Q, const void *K,
                                           RowLayout src, bool always_q, void *workspace,
                                           const void **q_used, const void **k_used,
