@@ -525,6 +525,16 @@ unsigned long long ret_kernel_launches(void);
 /* Static, NUL-terminated description of a status code. */
 const char *ret_status_string(ret_status status);
 
+/*
+ * ret_msr_gammas -- section 2.2: the decay of head h of the multi-scale
+ * retention layer, gamma_h = 1 - 2^(-5-h) for h = 0 .. H-1 (short windows
+ * for the first heads, long ones for the last).  A host function: it writes
+ * the H doubles of `gamma` (HOST memory, caller-owned), ready to be the
+ * `gamma` array of a ret_desc.  Errors: RET_ERR_NULL, RET_ERR_SHAPE for H
+ * outside 1..RET_MAX_HEADS.
+ */
+ret_status ret_msr_gammas(int H, double *gamma);
+
 #ifdef __cplusplus
 }
 #endif

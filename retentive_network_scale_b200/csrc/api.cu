@@ -92,6 +92,13 @@ using namespace ret;
 
 extern "C" {
 
+ret_status ret_msr_gammas(int H, double *gamma) {
+    if (H < 1 || H > RET_MAX_HEADS) return RET_ERR_SHAPE;
+    if (!gamma) return RET_ERR_NULL;
+    for (int h = 0; h < H; ++h) gamma[h] = 1.0 - std::ldexp(1.0, -5 - h);
+    return RET_OK;
+}
+
 const char *ret_status_string(ret_status s) {
     switch (s) {
         case RET_OK: return "ok";

@@ -37,7 +37,7 @@ EXPORTS = ("ret_parallel", "ret_parallel_workspace_size", "ret_chunkwise",
            "ret_segment_state", "ret_segment_state_workspace_size", "ret_state_scan",
            "ret_chunkwise_segmented", "ret_chunkwise_segmented_workspace_size",
            "ret_recurrent_step", "ret_gate_norm", "ret_gate_norm_backward", "ret_last_device_status",
-           "ret_kernel_launches", "ret_status_string")
+           "ret_kernel_launches", "ret_status_string", "ret_msr_gammas")
 RET_STATIC_SCRATCH_FLOATS = 4 << 20
 RET_MAX_DECODE_STEPS = 16
 RET_MAX_SEGMENTS = 64
@@ -121,6 +121,8 @@ def load_library(path: str = LIB_PATH):
     lib.ret_gate_norm_backward.argtypes = [ctypes.c_int] * 5 + [vp, ctypes.c_int, vp, vp,
                                                                 ctypes.c_float, vp, vp, vp]
     lib.ret_last_device_status.argtypes = [vp]
+    lib.ret_msr_gammas.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    lib.ret_msr_gammas.restype = ctypes.c_int
     lib.ret_kernel_launches.argtypes = []
     lib.ret_kernel_launches.restype = ctypes.c_ulonglong
     lib.ret_status_string.argtypes = [ctypes.c_int]
@@ -142,8 +144,11 @@ def _status_text(status: int) -> str:
 
 def msr_gammas(H: int) -> list:
     """Decay schedule gamma_h = 1 - 2^(-5-h) of the multi-scale retention
-    layer ("Retentive Network" paper summary, section 2.2)."""
-    return [1.0 - 2.0 ** (-5 - h) for h in range(H)]
+    layer ("Retentive Network" paper summary, section 2.2), from the
+    library's ret_msr_gammas."""
+    out = (ctypes.c_double * max(int(H), 1))()
+    _check(load_library().ret_msr_gammas(int(H), out), "ret_msr_gammas")
+    return list(out)[:H]
 
 
 # ---------------------------------------------------------------- marshalling

@@ -170,6 +170,27 @@ def test_gate_norm_arguments(lib):
         R.STATUS_NAMES.index("RET_ERR_NULL")
 
 
+def test_msr_gammas_schedule(lib):
+    """ret_msr_gammas (a host function) against the hand-worked binary
+    fractions of section 2.2's schedule, and its refusals."""
+    import os
+    from fractions import Fraction
+    want = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "gamma_schedule.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                h, frac = line.split()
+                want[int(h)] = Fraction(frac)
+    got = R.msr_gammas(16)
+    assert len(got) == 16
+    for h, fr in want.items():
+        assert Fraction(got[h]) == fr, (h, got[h], fr)
+    out = (ctypes.c_double * 4)()
+    assert lib.ret_msr_gammas(0, out) == R.STATUS_NAMES.index("RET_ERR_SHAPE")
+    assert lib.ret_msr_gammas(R.RET_MAX_HEADS + 1, out) == R.STATUS_NAMES.index("RET_ERR_SHAPE")
+    assert lib.ret_msr_gammas(4, None) == R.STATUS_NAMES.index("RET_ERR_NULL")
+
+
 def test_gate_norm_backward_arguments(lib):
     SHAPE, DT = R.STATUS_NAMES.index("RET_ERR_SHAPE"), R.STATUS_NAMES.index("RET_ERR_DTYPE")
     f = lib.ret_gate_norm_backward
