@@ -27,8 +27,9 @@
  *    stream.
  *  - Process-level objects, made once per device under a lock: the device
  *    status word of the bounded waits (a __device__ variable), the cuBLAS
- *    handle, and the side stream with two events on which ret_chunkwise runs
- *    the streaming pass of its next batch slice.  Calls from several host
+ *    handle, and the side stream with five events on which ret_chunkwise
+ *    runs the streaming pass of its next batch slice and ret_backward the
+ *    key-weighting pass of its next product.  Calls from several host
  *    threads are safe; on one device they take those locks in turn while
  *    they enqueue work.
  *  - Arguments are checked before any launch.  A call that returns an error
@@ -341,6 +342,8 @@ ret_status ret_gemm_bf16(long long M, long long N, long long K, const void *A,
  * Each is evaluated as a chunkwise retention of rearranged operands on the
  * tensor cores (the two anti-causal ones by the chunk loop's reverse mode,
  * on the operands in place; with rotation Q and K are first copied turned).
+ * The key-weighting pass of each product runs on the library's side stream
+ * (joined to `stream` by events), beside the previous product's loop.
  *   Q, K    device bf16 [B][H][L][d_k];  V, dO device bf16 [B][H][L][d_v]
  *   dQ, dK  device out_dtype [B][H][L][d_k];  dV device out_dtype
  *           [B][H][L][d_v]; all fully overwritten
